@@ -1,0 +1,237 @@
+"""Seeded synthetic inputs shaped like the long-context prefill workloads.
+
+This module only draws random numbers and lays them out: it holds none of
+the attention method's arithmetic, so both the CUDA path (tests, bench) and
+the float64 oracle read the same canonical tensors from it.
+
+All tensors are float32 arrays whose values are exactly representable in
+bfloat16 (rounded to nearest-even from the float32 draw); ``bf16_bits``
+turns them into the uint16 bit patterns the device receives.
+
+Recipes (the pages measure on needle-in-a-haystack RULER prompts of real
+models, which are not available; these stand in for them):
+
+* ``needles``  -- Q, K, V ~ N(0, 1) plus planted needles: a random unit
+  direction u, a query block b and a key position p in an earlier,
+  non-sink block; K[p] is set to 4u and 4u is added to every query row of
+  block b in the heads of that kv-head group.
+* ``lowrank``  -- Q, K = N(0, 1) + z W_g with W_g in R^{4 x d} ~ N(0, 1)
+  per kv-head, shared by the keys of kv-head g and the queries of its
+  group, and z ~ N(0, I_4) drawn per token and head (per-entry std of the
+  shared part about 2).  The keys of the first 4 tokens of every sequence
+  are scaled by 8 (attention sinks).  V ~ N(0, 1).
+* ``lowrank+needles`` -- ``lowrank`` plus needles at uniform positions.
+
+A paged layout places every sequence's 64-token pages at a seeded random
+permutation of a larger pool.  Whole pages that no sequence uses are filled
+with NaN (a stray page read shows up as NaN), and the slots after the end
+of a sequence in its last page hold the finite sentinel 100.0.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+
+# ----------------------------------------------------------------------------
+# bfloat16 canonicalisation
+# ----------------------------------------------------------------------------
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest bfloat16 (ties to even), in place
+    when possible; returns float32 holding bf16-exact values."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32)
+    lsb = (u >> np.uint32(16)) & np.uint32(1)
+    u += np.uint32(0x7FFF) + lsb
+    u &= np.uint32(0xFFFF0000)
+    return x
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """uint16 bit patterns of a float32 array of bf16-exact values."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    return (x.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+def bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """float32 values of uint16 bf16 bit patterns."""
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+# ----------------------------------------------------------------------------
+# Problem description
+# ----------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    seqlens: List[int]
+    Hq: int
+    Hkv: int
+    d: int
+    B: int
+    tau: float
+    generator: str = "lowrank"
+    n_needles: int = 0
+    page_size: int = 0          # 0 = contiguous K/V, else paged
+    pool_pages: int = 0         # pages in the pool when paged
+    dtype: str = "bf16"
+    seed: int = 0
+
+    @property
+    def T(self) -> int:
+        return int(sum(self.seqlens))
+
+
+def workloads() -> Dict[str, Workload]:
+    """The named workloads: a small reference case, two single-layer shapes
+    (32K and 128K), a paged continuous-batching mix and a length sweep."""
+    w = {
+        "pr1_ref_1k": Workload("pr1_ref_1k", [1024], 4, 1, 64, 64, 0.3, "needles", 8, seed=1000),
+        "llama_32k": Workload("llama_32k", [32768], 32, 8, 128, 128, 0.1, "lowrank", 0, seed=1001),
+        "qwen_128k": Workload("qwen_128k", [131072], 32, 8, 128, 128, 0.05, "lowrank+needles", 64,
+                              seed=1002),
+        "paged_mix": Workload("paged_mix", [4096, 9000, 16384, 30000, 65536, 1500], 32, 8, 128, 128,
+                              0.1, "lowrank", 0, page_size=64, pool_pages=2048, seed=1003),
+    }
+    for li, L in enumerate([4096, 8192, 16384, 32768, 65536, 131072]):
+        for ti, tau in enumerate([0.0, 0.05, 0.2]):
+            name = f"sweep_{L // 1024}k_tau{tau:g}"
+            w[name] = Workload(name, [L], 32, 8, 128, 128, tau, "lowrank", 0,
+                               seed=1004 + 10 * li + ti)
+    return w
+
+
+# ----------------------------------------------------------------------------
+# Generators
+# ----------------------------------------------------------------------------
+
+def _normal(rng: np.random.Generator, shape) -> np.ndarray:
+    return rng.standard_normal(size=shape, dtype=np.float32)
+
+
+def _lowrank_into(rng, out: np.ndarray, W: np.ndarray, group: int) -> None:
+    """out[T, H, d] = N(0,1) + z W_{h // group}, head by head."""
+    T, H, d = out.shape
+    for h in range(H):
+        z = _normal(rng, (T, W.shape[1]))
+        out[:, h, :] = _normal(rng, (T, d))
+        out[:, h, :] += z @ W[h // group]
+
+
+def _plant_needles(rng, q, k, seqlens, Hkv, B, n_needles, first_qblock=2) -> List[tuple]:
+    """Plant needles; returns (seq, kv_head, q_block, key_pos) tuples."""
+    Hq, d = q.shape[1], q.shape[2]
+    G = Hq // Hkv
+    cu = np.concatenate([[0], np.cumsum(seqlens)])
+    planted = []
+    for _ in range(n_needles):
+        s = int(rng.integers(0, len(seqlens)))
+        nb = (int(seqlens[s]) + B - 1) // B
+        if nb <= first_qblock:
+            continue
+        b = int(rng.integers(first_qblock, nb))
+        p = int(rng.integers(B, b * B))
+        g = int(rng.integers(0, Hkv))
+        u = _normal(rng, (d,)).astype(np.float64)
+        u /= np.linalg.norm(u)
+        u4 = (4.0 * u).astype(np.float32)
+        k[cu[s] + p, g, :] = u4
+        lo, hi = cu[s] + b * B, cu[s] + min((b + 1) * B, int(seqlens[s]))
+        q[lo:hi, g * G:(g + 1) * G, :] += u4[None, None, :]
+        planted.append((s, g, b, p))
+    return planted
+
+
+def generate(wl: Workload) -> Dict[str, object]:
+    """Canonical inputs for a workload.
+
+    Returns q [T, Hq, d], k, v [T, Hkv, d] (float32, bf16-exact), the
+    contiguous cu_seqlens, and for paged workloads k_pool / v_pool
+    [P, page, Hkv, d] and page_table [n, max_pages] (int32, unused = -1).
+    """
+    rng = np.random.Generator(np.random.PCG64(wl.seed))
+    T, Hq, Hkv, d = wl.T, wl.Hq, wl.Hkv, wl.d
+    q = np.empty((T, Hq, d), dtype=np.float32)
+    k = np.empty((T, Hkv, d), dtype=np.float32)
+    if wl.generator.startswith("lowrank"):
+        W = _normal(rng, (Hkv, 4, d))
+        _lowrank_into(rng, q, W, Hq // Hkv)
+        _lowrank_into(rng, k, W, 1)
+        t0 = 0
+        for L in wl.seqlens:
+            k[t0:t0 + min(4, L)] *= 8.0
+            t0 += L
+    elif wl.generator == "needles" or wl.generator == "normal":
+        q[...] = _normal(rng, q.shape)
+        k[...] = _normal(rng, k.shape)
+    else:
+        raise ValueError(wl.generator)
+    v = _normal(rng, (T, Hkv, d))
+    planted = []
+    if wl.n_needles:
+        planted = _plant_needles(rng, q, k, wl.seqlens, Hkv, wl.B, wl.n_needles)
+    bf16_round(q)
+    bf16_round(k)
+    bf16_round(v)
+    out = {"q": q, "k": k, "v": v, "needles": planted,
+           "cu_seqlens": np.concatenate([[0], np.cumsum(wl.seqlens)]).astype(np.int32)}
+    if wl.page_size:
+        out.update(make_paged(rng, k, v, wl.seqlens, wl.page_size, wl.pool_pages))
+    return out
+
+
+def make_paged(rng, k: np.ndarray, v: np.ndarray, seqlens: Sequence[int], page: int,
+               pool_pages: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """Scatter contiguous k, v into a shuffled page pool.
+
+    NaN fills unused pages; 100.0 fills the slots past a sequence's end in
+    its last page.
+    """
+    n_pages = [(int(L) + page - 1) // page for L in seqlens]
+    total = int(sum(n_pages))
+    P = int(pool_pages) if pool_pages else total
+    assert P >= total
+    perm = rng.permutation(P)[:total]
+    Hkv, d = k.shape[1], k.shape[2]
+    k_pool = np.full((P, page, Hkv, d), np.nan, dtype=np.float32)
+    v_pool = np.full((P, page, Hkv, d), np.nan, dtype=np.float32)
+    table = np.full((len(seqlens), max(n_pages) if n_pages else 1), -1, dtype=np.int32)
+    t0 = 0
+    c = 0
+    for s, L in enumerate(seqlens):
+        L = int(L)
+        for pg in range(n_pages[s]):
+            pid = int(perm[c])
+            c += 1
+            table[s, pg] = pid
+            lo = pg * page
+            n = min(page, L - lo)
+            k_pool[pid, :n] = k[t0 + lo:t0 + lo + n]
+            v_pool[pid, :n] = v[t0 + lo:t0 + lo + n]
+            if n < page:
+                k_pool[pid, n:] = 100.0
+                v_pool[pid, n:] = 100.0
+        t0 += L
+    return {"k_pool": k_pool, "v_pool": v_pool, "page_table": table}
+
+
+def small_workload(seqlens, Hq, Hkv, d, B, tau, seed, generator="lowrank", n_needles=0,
+                   page_size=0, pool_pages=0) -> Workload:
+    """A test-sized workload with the same generators."""
+    return Workload(f"small_{seed}", list(seqlens), Hq, Hkv, d, B, tau, generator, n_needles,
+                    page_size=page_size, pool_pages=pool_pages, seed=seed)
+
+
+def sample_qblocks(nb: int, count: int, seed: int) -> List[int]:
+    """Seeded sample of query blocks of one sequence, always holding the
+    first and the last block."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    if nb <= count:
+        return list(range(nb))
+    mid = rng.choice(np.arange(1, nb - 1), size=count - 2, replace=False)
+    return sorted([0, nb - 1] + [int(x) for x in mid])
