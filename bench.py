@@ -1,0 +1,366 @@
+"""Benchmark of the block-sparse prefill hot path (plan + prefill) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole path over one attention layer of synthetic
+input: stage 1 (pooling, scoring, thresholding, CSR) and stage 2 (sparse
+attention with mean correction).  The default workload is the 128K-token
+Qwen3-4B-shaped layer (32 query / 8 kv heads, head dim 128, block 128,
+tau 0.05, low-rank + needle generator).
+
+Prints one JSON line.  `value` is dense-equivalent TFLOP/s of the whole job
+(sum over ranks of 2*d*Hq*sum L(L+1) per step, divided by the max over ranks
+of the device time), inputs resident in HBM.  Each rank runs an independent
+layer (weak scaling, no collective on the data path); torch.distributed only
+provides the barrier and the max over ranks.
+
+--impl reference runs the float64 CPU oracle on a bounded sample of the same
+workload (rank 0 only) and prints the same metric for it.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from block_sparse_long_fp2_b200 import synth  # noqa: E402
+
+METRIC = "ms/layer & dense-equiv TFLOPS at 128K prefill; tensor-pipe % of B200 peak"
+UNIT = "dense-equiv TFLOP/s"
+
+
+def dense_equiv_flop(wl) -> float:
+    """Causal attention FLOP of the dense layer: 2 * d * Hq * sum L (L + 1)."""
+    return float(sum(2.0 * wl.d * wl.Hq * L * (L + 1) for L in wl.seqlens))
+
+
+def kept_tile_flop(wl) -> float:
+    """Tensor-core FLOP of one kept (row, key block) pair: QK^T + PV for the
+    G heads x B tokens of the row = 4 * d * G * B^2."""
+    G = wl.Hq // wl.Hkv
+    return 4.0 * wl.d * G * wl.B * wl.B
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16": p["bf16_tflops"],
+                "bf16_sustained": p["bf16_tflops_sustained"], "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.f = None
+
+    def __enter__(self):
+        try:
+            self.f = tempfile.TemporaryFile(mode="w+")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.f is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.f.seek(0)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from block_sparse_long_fp2_b200 import binding as fb
+    from block_sparse_long_fp2_b200 import build as fbuild
+
+    fbuild.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = synth.workloads()[args.workload]
+    wl.seed += 7919 * rank            # each rank: an independent layer
+    x = synth.generate(wl)
+    stream = torch.cuda.current_stream()
+
+    def dev_bf16(a):
+        return torch.from_numpy(a).to(torch.bfloat16).to(dev)
+
+    q = dev_bf16(x["q"])
+    if wl.page_size:
+        k, v = dev_bf16(x["k_pool"]), dev_bf16(x["v_pool"])
+        pt = torch.from_numpy(x["page_table"]).to(dev)
+    else:
+        k, v = dev_bf16(x["k"]), dev_bf16(x["v"])
+        pt = None
+    cu = torch.from_numpy(x["cu_seqlens"]).to(dev)
+    prob = fb.Problem(wl.seqlens, cu, wl.Hq, wl.Hkv, wl.d, wl.B, wl.tau,
+                      page_size=wl.page_size, page_table=pt,
+                      num_pages=int(x["k_pool"].shape[0]) if wl.page_size else 0)
+    lay, plan, ws = fb.allocate(prob, dev)
+    o = torch.empty((wl.T, wl.Hq, wl.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.Hq, wl.T), dtype=torch.float32, device=dev)
+    in_bytes = (q.numel() + k.numel() + v.numel()) * 2
+
+    def step():
+        fb.fp2_plan(prob, q, k, v, plan, ws, stream)
+        fb.fp2_prefill(prob, plan, q, k, v, o, lse, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    rc, st = fb.fp2_status_check(plan, stream)
+    if rc != 0:
+        raise RuntimeError(f"device status {st:#x} ({fb.strerror(rc)})")
+    nnz = int(fb.PlanView(plan, lay, wl.Hkv, wl.d).row_ptr[-1].item())
+
+    # timed region: K steps, per-stage events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                      int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])) as clk:
+        t0.record(stream)
+        for s in range(args.steps):
+            ev[s][0].record(stream)
+            fb.fp2_plan(prob, q, k, v, plan, ws, stream)
+            ev[s][1].record(stream)
+            fb.fp2_prefill(prob, plan, q, k, v, o, lse, stream=stream)
+            ev[s][2].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = t0.elapsed_time(t1)
+    plan_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    launches_per_step = (6 if wl.tau > 0 else 5) + 1
+
+    # end to end through the C ABI with host buffers (pinned), copies inside
+    qh = torch.from_numpy(x["q"]).to(torch.bfloat16).pin_memory()
+    kh = (torch.from_numpy(x["k_pool"] if wl.page_size else x["k"]).to(torch.bfloat16)
+          .pin_memory())
+    vh = (torch.from_numpy(x["v_pool"] if wl.page_size else x["v"]).to(torch.bfloat16)
+          .pin_memory())
+    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 3))
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        step()
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    # max over ranks
+    vals = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = float(vals[0]), float(vals[1])
+    ms_step = total_ms / args.steps
+    flop = dense_equiv_flop(wl)
+    value = world * flop / (ms_step * 1e-3) / 1e12
+    pk = peaks()
+    attn_avg = statistics.mean(attn_ms)
+    plan_avg = statistics.mean(plan_ms)
+    executed = nnz * kept_tile_flop(wl)
+    achieved = executed / (attn_avg * 1e-3) / 1e12
+    G = wl.Hq // wl.Hkv
+    R = int(lay.num_rows)
+    density = nnz / float(lay.nnz_cap)
+    plan_bytes = in_bytes + int(lay.num_blocks) * wl.Hkv * wl.d * (4 + 4 + 2 + 2)
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded low-rank + needles generator; no model weights)",
+        "config": {"workload": wl.name, "seqlens": wl.seqlens, "Hq": wl.Hq, "Hkv": wl.Hkv,
+                   "head_dim": wl.d, "block": wl.B, "tau": wl.tau, "paged": bool(wl.page_size),
+                   "parallelism": f"independent layer per GPU x{world}",
+                   "l2": "inputs (%.2f GB) larger than L2 (126 MB), no flush" % (in_bytes / 1e9)},
+        "ms_per_layer": round(ms_step, 4), "ms_plan": round(plan_avg, 4),
+        "ms_attention": round(attn_avg, 4), "density": round(density, 5), "nnz": nnz,
+        "dense_equiv_tflop": round(flop / 1e12, 3),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
+                     "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                     "frac": round(achieved / pk["bf16_sustained"], 4), "traffic": None,
+                     "kernel": "k_attn (sparse attention + correction)",
+                     "peak_kind": f"bf16 sustained ({pk['source']})",
+                     "frac_of_burst_peak": round(achieved / pk["bf16"], 4)},
+        "planning": {"achieved_gbs": round(plan_bytes / (plan_avg * 1e-3) / 1e9, 1),
+                     "peak_gbs": pk["hbm_gbs"],
+                     "frac": round(plan_bytes / (plan_avg * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
+        "e2e": {"value": round(world * flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(in_bytes),
+                "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "rows": R, "G": G,
+    }
+    return out, x
+
+
+def oracle_sample(wl, x, budget_s: float = 20.0):
+    """Times the oracle on a bounded sample of the workload: block means of
+    the whole layer plus scoring and attention of a few query blocks per
+    kv-head, reported as dense-equivalent FLOP of the sampled rows / s."""
+    import oracle
+    t_start = time.perf_counter()
+    nb = [(L + wl.B - 1) // wl.B for L in wl.seqlens]
+    s_last = int(np.argmax(wl.seqlens))
+    rng = np.random.default_rng(0)
+    cand = sorted(rng.choice(np.arange(nb[s_last]), size=min(nb[s_last], 64), replace=False),
+                  reverse=True)
+    q, k, v = x["q"], x.get("k"), x.get("v")
+    if wl.page_size:
+        k = oracle.gather_paged(x["k_pool"], x["page_table"], wl.seqlens, wl.page_size)
+        v = oracle.gather_paged(x["v_pool"], x["page_table"], wl.seqlens, wl.page_size)
+    sample = [(s_last, int(i)) for i in cand]
+    pl = oracle.plan(q, k, v, wl.seqlens, wl.B, wl.tau, rows=sample)
+    rows, flop = [], 0.0
+    for (s_, i) in sample:
+        oracle.attend(q, k, v, pl, rows=[(s_, i)])
+        rows.append((s_, i))
+        n_i = min(wl.B, wl.seqlens[s_] - i * wl.B)
+        p0 = i * wl.B
+        flop += 2.0 * 2.0 * wl.d * wl.Hq * sum(p0 + u + 1 for u in range(n_i))
+        if time.perf_counter() - t_start > budget_s:
+            break
+    el = time.perf_counter() - t_start
+    return flop / el / 1e12, el, rows
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    os.environ.setdefault("OMP_NUM_THREADS", str(len(os.sched_getaffinity(0))))
+    wl = synth.workloads()[args.workload]
+    x = synth.generate(wl)
+    cores = len(os.sched_getaffinity(0))
+    per_step = []
+    rows = []
+    budget = max(5.0, 120.0 / max(1, args.steps + args.warmup))
+    for s in range(args.warmup + args.steps):
+        val, el, rows = oracle_sample(wl, x, budget)
+        if s >= args.warmup:
+            per_step.append((val, el))
+    value = statistics.mean(v for v, _ in per_step)
+    ms = statistics.mean(e for _, e in per_step) * 1e3
+    sample = (f"block means of the full layer + scoring and attention of {len(rows)} "
+              f"query blocks (all kv-heads) of the {wl.seqlens[0]}-token layer, float64 NumPy")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "seqlens": wl.seqlens, "Hq": wl.Hq, "Hkv": wl.Hkv,
+                       "head_dim": wl.d, "block": wl.B, "tau": wl.tau},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="qwen_128k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    out, x = run_ours(args, rank, world, local_rank)
+    if rank == 0 and not args.no_cpu_baseline:
+        wl = synth.workloads()[args.workload]
+        val, el, rows = oracle_sample(wl, x, 20.0)
+        out["cpu_baseline"] = {
+            "value": val, "unit": UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"block means of the whole layer + scoring/attention of {len(rows)} query "
+                      f"blocks (all kv-heads), {el:.1f} s"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,284 @@
+// C ABI of libfp2: argument validation, plan/workspace layout and dispatch.
+//
+// Everything here runs on the host.  No entry point allocates or frees
+// device memory or synchronises, except fp2_status_check (which
+// synchronises the stream and reads the 4-byte status word).
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "fp2_internal.h"
+
+namespace fp2 {
+
+namespace {
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Carver {
+    size_t off = 0;
+    size_t take(size_t bytes) {
+        size_t o = align_up(off, 256);
+        off = o + bytes;
+        return o;
+    }
+};
+
+}  // namespace
+
+int compute_layout(const fp2_problem* p, Layout* out) {
+    if (!p || !out) return FP2_ERR_INVALID_ARG;
+    if (p->num_seqs < 1 || !p->seqlens || !p->cu_seqlens) return FP2_ERR_INVALID_ARG;
+    if (p->num_q_heads < 1 || p->num_kv_heads < 1) return FP2_ERR_INVALID_ARG;
+    if (p->num_q_heads % p->num_kv_heads != 0) return FP2_ERR_INVALID_ARG;
+    if (!(p->tau >= 0.0) || p->tau > 1e30) return FP2_ERR_INVALID_ARG;
+    if (p->head_dim != 64 && p->head_dim != 128) return FP2_ERR_UNSUPPORTED;
+    if (p->block_size != 64 && p->block_size != 128) return FP2_ERR_UNSUPPORTED;
+    const int G = p->num_q_heads / p->num_kv_heads;
+    if (G > kScoreQV) return FP2_ERR_UNSUPPORTED;
+    if ((G * p->block_size) % kTileM != 0) return FP2_ERR_UNSUPPORTED;
+    if (p->page_size != 0 && p->page_size != 64) return FP2_ERR_UNSUPPORTED;
+
+    Dims d{};
+    d.n_seqs = p->num_seqs;
+    d.Hq = p->num_q_heads;
+    d.Hkv = p->num_kv_heads;
+    d.G = G;
+    d.d = p->head_dim;
+    d.B = p->block_size;
+    d.page_size = p->page_size;
+    d.num_pages = p->num_pages;
+    d.pt_stride = p->page_table_stride;
+    d.tau = p->tau;
+    d.rows_per_group = kScoreQV / G;
+
+    int64_t T = 0, NB = 0, tri = 0, groups = 0;
+    int max_nb = 0, max_pages = 0;
+    for (int s = 0; s < p->num_seqs; ++s) {
+        const int64_t L = p->seqlens[s];
+        if (L < 1 || L > (int64_t)1 << 30) return FP2_ERR_INVALID_ARG;
+        const int64_t nb = (L + d.B - 1) / d.B;
+        T += L;
+        NB += nb;
+        tri += nb * (nb + 1) / 2;
+        groups += (nb + d.rows_per_group - 1) / d.rows_per_group;
+        max_nb = std::max<int>(max_nb, (int)nb);
+        max_pages = std::max<int>(max_pages, (int)((L + 63) / 64));
+    }
+    if (T > ((int64_t)1 << 31) - 1) return FP2_ERR_UNSUPPORTED;
+    if (p->page_size == 64) {
+        if (!p->page_table || p->num_pages < 1) return FP2_ERR_INVALID_ARG;
+        if (p->page_table_stride < max_pages) return FP2_ERR_INVALID_ARG;
+    }
+    d.T = T;
+    d.NB = NB;
+    d.R = NB * d.Hkv;
+    d.tri_total = tri;
+    d.nnz_cap = tri * d.Hkv;
+    if (d.nnz_cap > ((int64_t)1 << 31) - 1) return FP2_ERR_UNSUPPORTED;
+    d.max_nb = max_nb;
+    d.mask_words = (max_nb + 31) / 32;
+    d.n_groups_cap = (int)groups;
+
+    Layout& L = *out;
+    std::memset(&L, 0, sizeof(L));
+    L.dims = d;
+    fp2_plan_layout& pub = L.pub;
+    pub.num_tokens = T;
+    pub.num_blocks = NB;
+    pub.num_rows = d.R;
+    pub.nnz_cap = d.nnz_cap;
+    pub.mask_words = d.mask_words;
+    pub.max_blocks_per_seq = max_nb;
+
+    const size_t n = (size_t)p->num_seqs;
+    const size_t mean_elems = (size_t)NB * d.Hkv * d.d;
+    Carver c;
+    pub.off_status = c.take(sizeof(int32_t));
+    L.off_meta_valid = c.take(sizeof(int32_t));
+    pub.off_meta = L.off_meta_valid;
+    pub.off_row_ptr = c.take(sizeof(int32_t) * (size_t)(d.R + 1));
+    pub.off_col_idx = c.take(sizeof(int32_t) * (size_t)d.nnz_cap);
+    pub.off_kept_mask = c.take(sizeof(uint32_t) * (size_t)d.R * d.mask_words);
+    pub.off_kbar = c.take(sizeof(float) * mean_elems);
+    pub.off_vbar = c.take(sizeof(float) * mean_elems);
+    pub.off_kbar_bf16 = c.take(sizeof(uint16_t) * mean_elems);
+    pub.off_vbar_bf16 = c.take(sizeof(uint16_t) * mean_elems);
+    pub.off_kbar_e4m3 = c.take(mean_elems);
+    pub.off_vbar_e4m3 = c.take(mean_elems);
+    pub.off_kbar_scale = c.take(sizeof(float) * (size_t)NB * d.Hkv);
+    pub.off_vbar_scale = c.take(sizeof(float) * (size_t)NB * d.Hkv);
+    L.off_cu_blocks = c.take(sizeof(int32_t) * (n + 1));
+    L.off_block_seq = c.take(sizeof(int32_t) * (size_t)NB);
+    L.off_tri_off = c.take(sizeof(int64_t) * (n + 1));
+    L.off_group_cu = c.take(sizeof(int32_t) * (n + 1));
+    L.off_group_seq = c.take(sizeof(int32_t) * (size_t)std::max<int64_t>(1, groups));
+    pub.plan_bytes = align_up(c.off, 256);
+
+    Carver w;
+    L.ws_qbar64 = w.take(sizeof(double) * (size_t)NB * d.Hq * d.d);
+    L.ws_kbar64 = w.take(sizeof(double) * mean_elems);
+    L.ws_qnorm = w.take(sizeof(float) * (size_t)NB * d.Hkv);
+    L.ws_knorm = w.take(sizeof(float) * (size_t)NB * d.Hkv);
+    L.ws_scores = w.take(sizeof(float) * (size_t)d.nnz_cap);
+    L.ws_counts = w.take(sizeof(int32_t) * (size_t)d.R);
+    pub.workspace_bytes = align_up(w.off, 256);
+    return FP2_OK;
+}
+
+PlanPtrs plan_ptrs(const Layout& L, void* plan) {
+    char* b = static_cast<char*>(plan);
+    const fp2_plan_layout& u = L.pub;
+    PlanPtrs p;
+    p.row_ptr = reinterpret_cast<int32_t*>(b + u.off_row_ptr);
+    p.col_idx = reinterpret_cast<int32_t*>(b + u.off_col_idx);
+    p.kept_mask = reinterpret_cast<uint32_t*>(b + u.off_kept_mask);
+    p.kbar = reinterpret_cast<float*>(b + u.off_kbar);
+    p.vbar = reinterpret_cast<float*>(b + u.off_vbar);
+    p.kbar16 = reinterpret_cast<uint16_t*>(b + u.off_kbar_bf16);
+    p.vbar16 = reinterpret_cast<uint16_t*>(b + u.off_vbar_bf16);
+    p.kbar8 = reinterpret_cast<uint8_t*>(b + u.off_kbar_e4m3);
+    p.vbar8 = reinterpret_cast<uint8_t*>(b + u.off_vbar_e4m3);
+    p.kbar_scale = reinterpret_cast<float*>(b + u.off_kbar_scale);
+    p.vbar_scale = reinterpret_cast<float*>(b + u.off_vbar_scale);
+    p.status = reinterpret_cast<int32_t*>(b + u.off_status);
+    p.meta_valid = reinterpret_cast<int32_t*>(b + L.off_meta_valid);
+    p.cu_blocks = reinterpret_cast<int32_t*>(b + L.off_cu_blocks);
+    p.block_seq = reinterpret_cast<int32_t*>(b + L.off_block_seq);
+    p.tri_off = reinterpret_cast<int64_t*>(b + L.off_tri_off);
+    p.group_cu = reinterpret_cast<int32_t*>(b + L.off_group_cu);
+    p.group_seq = reinterpret_cast<int32_t*>(b + L.off_group_seq);
+    return p;
+}
+
+WsPtrs ws_ptrs(const Layout& L, void* ws) {
+    char* b = static_cast<char*>(ws);
+    WsPtrs w;
+    w.qbar64 = reinterpret_cast<double*>(b + L.ws_qbar64);
+    w.kbar64 = reinterpret_cast<double*>(b + L.ws_kbar64);
+    w.qnorm = reinterpret_cast<float*>(b + L.ws_qnorm);
+    w.knorm = reinterpret_cast<float*>(b + L.ws_knorm);
+    w.scores = reinterpret_cast<float*>(b + L.ws_scores);
+    w.counts = reinterpret_cast<int32_t*>(b + L.ws_counts);
+    return w;
+}
+
+int sm_count() {
+    static std::mutex mu;
+    static std::vector<int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+}  // namespace fp2
+
+using namespace fp2;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int fp2_version(void) { return FP2_VERSION; }
+
+const char* fp2_strerror(int code) {
+    switch (code) {
+        case FP2_OK: return "ok";
+        case FP2_ERR_INVALID_ARG: return "invalid argument";
+        case FP2_ERR_UNSUPPORTED: return "unsupported configuration";
+        case FP2_ERR_CAPACITY: return "caller buffer too small";
+        case FP2_ERR_CUDA: return "CUDA error";
+        case FP2_ERR_TIMEOUT: return "device-side wait timed out";
+        case FP2_ERR_DEVICE_CHECK: return "device-side consistency check failed";
+        default: return "unknown error";
+    }
+}
+
+int fp2_plan_sizes(const fp2_problem* problem, fp2_plan_layout* layout) {
+    if (!layout) return FP2_ERR_INVALID_ARG;
+    Layout L;
+    int rc = compute_layout(problem, &L);
+    if (rc != FP2_OK) return rc;
+    *layout = L.pub;
+    return FP2_OK;
+}
+
+int fp2_plan(const fp2_problem* problem, const void* q, const void* k, const void* v, void* plan,
+             size_t plan_bytes, void* workspace, size_t workspace_bytes, void* stream) {
+    Layout L;
+    int rc = compute_layout(problem, &L);
+    if (rc != FP2_OK) return rc;
+    if (!q || !k || !v || !plan || !workspace) return FP2_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return FP2_ERR_INVALID_ARG;
+    if (!aligned(plan, 256) || !aligned(workspace, 256)) return FP2_ERR_INVALID_ARG;
+    if (plan_bytes < L.pub.plan_bytes || workspace_bytes < L.pub.workspace_bytes)
+        return FP2_ERR_CAPACITY;
+    return launch_plan(L, problem, q, k, v, plan_ptrs(L, plan), ws_ptrs(L, workspace),
+                       static_cast<cudaStream_t>(stream));
+}
+
+int fp2_quantize_fp8(const fp2_problem* problem, const void* plan, size_t plan_bytes, const void* x,
+                     int32_t which, void* x_e4m3, float* scales, void* stream) {
+    Layout L;
+    int rc = compute_layout(problem, &L);
+    if (rc != FP2_OK) return rc;
+    if (!plan || !x || !x_e4m3 || !scales || which < 0 || which > 2) return FP2_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(x_e4m3, 16) || !aligned(scales, 4) || !aligned(plan, 256))
+        return FP2_ERR_INVALID_ARG;
+    if (plan_bytes < L.pub.plan_bytes) return FP2_ERR_CAPACITY;
+    return launch_quantize(L, problem, plan_ptrs(L, const_cast<void*>(plan)), x, which, x_e4m3,
+                           scales, static_cast<cudaStream_t>(stream));
+}
+
+int fp2_prefill(const fp2_problem* problem, const void* plan, size_t plan_bytes, const void* q,
+                const void* k, const void* v, const float* q_scale, const float* k_scale,
+                const float* v_scale, int32_t dtype, void* o, float* lse, uint32_t flags,
+                void* stream) {
+    Layout L;
+    int rc = compute_layout(problem, &L);
+    if (rc != FP2_OK) return rc;
+    if (!plan || !q || !k || !v || !o || !lse) return FP2_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(lse, 4) || !aligned(plan, 256))
+        return FP2_ERR_INVALID_ARG;
+    if (plan_bytes < L.pub.plan_bytes) return FP2_ERR_CAPACITY;
+    if (dtype == FP2_DTYPE_BF16) {
+        if (q_scale || k_scale || v_scale) return FP2_ERR_INVALID_ARG;
+    } else if (dtype == FP2_DTYPE_E4M3) {
+        if (!q_scale || !k_scale || !v_scale) return FP2_ERR_INVALID_ARG;
+        return FP2_ERR_UNSUPPORTED;
+    } else {
+        return FP2_ERR_INVALID_ARG;
+    }
+    const uint32_t known = FP2_NO_CORRECTION | FP2_DEBUG_DROP_Q_LOAD;
+    if (flags & ~known) return FP2_ERR_INVALID_ARG;
+    return launch_prefill(L, problem, plan_ptrs(L, const_cast<void*>(plan)), q, k, v, q_scale,
+                          k_scale, v_scale, dtype, o, lse, flags,
+                          static_cast<cudaStream_t>(stream));
+}
+
+int fp2_status_check(const void* plan, size_t plan_bytes, void* stream, int32_t* device_status) {
+    if (!plan || plan_bytes < 4) return FP2_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP2_ERR_CUDA;
+    int32_t st = 0;
+    // The status word is the first field of the plan buffer (offset 0).
+    if (cudaMemcpy(&st, plan, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return FP2_ERR_CUDA;
+    if (device_status) *device_status = st;
+    if (st == 0) return FP2_OK;
+    if (st & FP2_STATUS_TIMEOUT) return FP2_ERR_TIMEOUT;
+    return FP2_ERR_DEVICE_CHECK;
+}
+
+}  // extern "C"

@@ -1,0 +1,93 @@
+// Internal declarations shared by the libfp2 translation units.
+//
+// Layout of the plan buffer and of fp2_plan's workspace, the derived
+// problem sizes every kernel needs, and the kernel launchers.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "../../include/fp2.h"
+
+namespace fp2 {
+
+// Query rows of one PackGQA tile (M of one tcgen05 MMA).
+constexpr int kTileM = 128;
+// Query vectors scored together by one CTA of the scoring kernel.
+constexpr int kScoreQV = 128;
+
+// Derived sizes of one problem (host computed, passed to kernels by value).
+struct Dims {
+    int n_seqs;
+    int Hq, Hkv, G, d, B;
+    int page_size, num_pages, pt_stride;
+    int mask_words;       // 32-bit words per kept-mask row
+    int max_nb;           // largest nb_s
+    int rows_per_group;   // query blocks per scoring CTA (kScoreQV / G)
+    int n_groups_cap;     // upper bound of scoring CTAs per kv-head
+    int64_t T, NB, R, tri_total, nnz_cap;
+    double tau;
+};
+
+// Device pointers into the plan buffer.
+struct PlanPtrs {
+    int32_t* row_ptr;
+    int32_t* col_idx;
+    uint32_t* kept_mask;
+    float* kbar;
+    float* vbar;
+    uint16_t* kbar16;
+    uint16_t* vbar16;
+    uint8_t* kbar8;
+    uint8_t* vbar8;
+    float* kbar_scale;
+    float* vbar_scale;
+    int32_t* status;
+    // private meta
+    int32_t* meta_valid;   // [1]  1 when cu_seqlens passed the device checks
+    int32_t* cu_blocks;    // [n+1]
+    int32_t* block_seq;    // [NB]
+    int64_t* tri_off;      // [n+1] prefix of nb (nb + 1) / 2
+    int32_t* group_cu;     // [n+1] prefix of scoring CTAs per sequence
+    int32_t* group_seq;    // [n_groups_cap]
+};
+
+// Device pointers into fp2_plan's workspace.
+struct WsPtrs {
+    double* qbar64;   // [NB, Hq, d]
+    double* kbar64;   // [NB, Hkv, d]
+    float* qnorm;     // [NB, Hkv]  max over the group's heads of |Qbar|_2 (rounded up)
+    float* knorm;     // [NB, Hkv]  |Kbar|_2 (rounded up)
+    float* scores;    // [Hkv, tri_total] fp32 block scores, row (s,g,i) at
+                      //   g * tri_total + tri_off[s] + i (i + 1) / 2 + j
+    int32_t* counts;  // [R] kept blocks per row
+};
+
+struct Layout {
+    Dims dims;
+    fp2_plan_layout pub;
+    size_t off_meta_valid, off_cu_blocks, off_block_seq, off_tri_off, off_group_cu, off_group_seq;
+    size_t ws_qbar64, ws_kbar64, ws_qnorm, ws_knorm, ws_scores, ws_counts;
+};
+
+// Validates the problem on the host and computes sizes and offsets.
+int compute_layout(const fp2_problem* p, Layout* out);
+PlanPtrs plan_ptrs(const Layout& L, void* plan);
+WsPtrs ws_ptrs(const Layout& L, void* ws);
+
+// Launchers (return FP2_OK or FP2_ERR_CUDA).
+int launch_plan(const Layout& L, const fp2_problem* p, const void* q, const void* k,
+                const void* v, const PlanPtrs& pp, const WsPtrs& ws, cudaStream_t st);
+int launch_quantize(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, const void* x,
+                    int which, void* x8, float* scales, cudaStream_t st);
+int launch_prefill(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, const void* q,
+                   const void* k, const void* v, const float* qs, const float* ks,
+                   const float* vs, int dtype, void* o, float* lse, uint32_t flags,
+                   cudaStream_t st);
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+}  // namespace fp2

@@ -15,6 +15,9 @@ models, which are not available; these stand in for them):
   direction u, a query block b and a key position p in an earlier,
   non-sink block; K[p] is set to 4u and 4u is added to every query row of
   block b in the heads of that kv-head group.
+Every head draws from its own generator spawned from the workload seed.
+
+* ``normal``   -- Q, K, V ~ N(0, 1).
 * ``lowrank``  -- Q, K = N(0, 1) + z W_g with W_g in R^{4 x d} ~ N(0, 1)
   per kv-head, shared by the keys of kv-head g and the queries of its
   group, and z ~ N(0, I_4) drawn per token and head (per-entry std of the
@@ -44,10 +47,14 @@ def bf16_round(x: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bfloat16 (ties to even), in place
     when possible; returns float32 holding bf16-exact values."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32)
-    lsb = (u >> np.uint32(16)) & np.uint32(1)
-    u += np.uint32(0x7FFF) + lsb
-    u &= np.uint32(0xFFFF0000)
+    flat = x.reshape(-1).view(np.uint32)
+    chunk = 1 << 20
+    for lo in range(0, flat.size, chunk):
+        u = flat[lo:lo + chunk]
+        lsb = (u >> np.uint32(16)) & np.uint32(1)
+        lsb += np.uint32(0x7FFF)
+        u += lsb
+        u &= np.uint32(0xFFFF0000)
     return x
 
 
@@ -114,13 +121,24 @@ def _normal(rng: np.random.Generator, shape) -> np.ndarray:
     return rng.standard_normal(size=shape, dtype=np.float32)
 
 
-def _lowrank_into(rng, out: np.ndarray, W: np.ndarray, group: int) -> None:
-    """out[T, H, d] = N(0,1) + z W_{h // group}, head by head."""
-    T, H, d = out.shape
-    for h in range(H):
-        z = _normal(rng, (T, W.shape[1]))
+def _fill_head(seed_seq, out: np.ndarray, h: int, W: Optional[np.ndarray]) -> None:
+    """out[:, h, :] = N(0, 1) (+ z W when W is given), from the head's own
+    generator so the result does not depend on thread scheduling."""
+    rng = np.random.Generator(np.random.PCG64(seed_seq))
+    T, _, d = out.shape
+    if W is None:
         out[:, h, :] = _normal(rng, (T, d))
-        out[:, h, :] += z @ W[h // group]
+        return
+    z = _normal(rng, (T, W.shape[0]))
+    out[:, h, :] = _normal(rng, (T, d))
+    out[:, h, :] += z @ W
+
+
+def _fill_heads(children, out: np.ndarray, Ws) -> None:
+    import concurrent.futures
+    import os
+    with concurrent.futures.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
+        list(ex.map(lambda h: _fill_head(children[h], out, h, Ws[h]), range(out.shape[1])))
 
 
 def _plant_needles(rng, q, k, seqlens, Hkv, B, n_needles, first_qblock=2) -> List[tuple]:
@@ -154,24 +172,28 @@ def generate(wl: Workload) -> Dict[str, object]:
     contiguous cu_seqlens, and for paged workloads k_pool / v_pool
     [P, page, Hkv, d] and page_table [n, max_pages] (int32, unused = -1).
     """
-    rng = np.random.Generator(np.random.PCG64(wl.seed))
+    ss = np.random.SeedSequence(wl.seed)
+    kids = ss.spawn(wl.Hq + 2 * wl.Hkv + 1)
+    rng = np.random.Generator(np.random.PCG64(kids[-1]))      # W, needles, pages
     T, Hq, Hkv, d = wl.T, wl.Hq, wl.Hkv, wl.d
+    G = Hq // Hkv
     q = np.empty((T, Hq, d), dtype=np.float32)
     k = np.empty((T, Hkv, d), dtype=np.float32)
+    v = np.empty((T, Hkv, d), dtype=np.float32)
     if wl.generator.startswith("lowrank"):
         W = _normal(rng, (Hkv, 4, d))
-        _lowrank_into(rng, q, W, Hq // Hkv)
-        _lowrank_into(rng, k, W, 1)
+        _fill_heads(kids[:Hq], q, [W[h // G] for h in range(Hq)])
+        _fill_heads(kids[Hq:Hq + Hkv], k, [W[g] for g in range(Hkv)])
         t0 = 0
         for L in wl.seqlens:
             k[t0:t0 + min(4, L)] *= 8.0
             t0 += L
     elif wl.generator == "needles" or wl.generator == "normal":
-        q[...] = _normal(rng, q.shape)
-        k[...] = _normal(rng, k.shape)
+        _fill_heads(kids[:Hq], q, [None] * Hq)
+        _fill_heads(kids[Hq:Hq + Hkv], k, [None] * Hkv)
     else:
         raise ValueError(wl.generator)
-    v = _normal(rng, (T, Hkv, d))
+    _fill_heads(kids[Hq + Hkv:Hq + 2 * Hkv], v, [None] * Hkv)
     planted = []
     if wl.n_needles:
         planted = _plant_needles(rng, q, k, wl.seqlens, Hkv, wl.B, wl.n_needles)

@@ -1,0 +1,237 @@
+/*
+ * fp2.h -- C ABI of libfp2: FlashPrefill V2 block-sparse prefill attention
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the one described in "FlashPrefill V2: Block-Sparse
+ * Prefill Attention for Long-Context LLM Serving" (metallab.ai summary of
+ * arXiv 2608.19758):
+ *   - Figure 3: stage 1 ("pattern discovery") pools block-mean statistics
+ *     under PackGQA and emits a CSR index of the selected key blocks;
+ *     stage 2 runs sparse attention over the selected blocks while the
+ *     unselected ones go through the mean-correction path, and both merge
+ *     inside one online softmax.
+ *   - Figure 4: a pruned block J contributes the surrogate
+ *     |B_J| e^{s_J} (v_J, 1) to the softmax numerator and denominator.
+ *   - Abstract: "max-based dynamic thresholding" (Table 9: alpha, here tau).
+ *   - Table 7: CSR of selected blocks, per KV head, int32.
+ *   - Figure 1 / Table 7: paged KV cache and continuous batching (varlen).
+ *   - Table 1 footnote: FP8 by direct online quantisation.
+ *
+ * Formulas.  Hq query heads, Hkv kv-heads, G = Hq / Hkv (query head h reads
+ * kv-head h / G), head dim d, block size B.  Sequence s of length L_s has
+ * nb_s = ceil(L_s / B) blocks; NB = sum_s nb_s.  For the row (s, g, i):
+ *   sc_j = max_{h in group g} mean(Q_block i, h) . mean(K_block j, g) / sqrt(d)
+ *   tau == 0 keeps every block j <= i; otherwise block j is kept when
+ *   sc_j >= tau * max_{j' <= i} sc_j', and blocks 0 and i are always kept.
+ *   Attention covers the kept blocks exactly (causal inside block i) and
+ *   adds, for every skipped block j (always a full block, n_j = B), one
+ *   pseudo-token with logit q . Kbar_j / sqrt(d) + ln n_j and value Vbar_j.
+ *   O = numerator / denominator; LSE = ln(denominator) in the 1/sqrt(d)-
+ *   scaled logit units, pseudo-tokens included.
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are CUDA global-memory addresses on the current
+ *     device; host pointers are ordinary process memory.  Every buffer is
+ *     owned by the caller.  The library allocates no memory, never frees,
+ *     and never synchronises except inside fp2_status_check.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously in stream order; inputs must
+ *     stay unchanged until the enqueued work has completed.
+ *   - Return value: FP2_OK (0) or a negative FP2_ERR_* code.  Argument
+ *     errors are detected on the host before anything is enqueued.
+ *     Inconsistencies that can only be seen on the device (cu_seqlens that
+ *     disagree with seqlens, page ids out of range, a wait that timed out)
+ *     are recorded in the plan's status word and reported by
+ *     fp2_status_check; kernels that see a bad plan do no work.
+ *   - Calls that use distinct plan and workspace buffers may run
+ *     concurrently from several host threads.
+ */
+#ifndef FP2_H_
+#define FP2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FP2_VERSION 1
+
+/* ---- error codes -------------------------------------------------------- */
+#define FP2_OK 0
+#define FP2_ERR_INVALID_ARG -1   /* a host-visible argument is wrong                 */
+#define FP2_ERR_UNSUPPORTED -2   /* a valid configuration this build does not handle */
+#define FP2_ERR_CAPACITY -3      /* a caller buffer is smaller than fp2_plan_sizes asks */
+#define FP2_ERR_CUDA -4          /* a CUDA call or kernel launch failed              */
+#define FP2_ERR_TIMEOUT -5       /* a device-side wait gave up (status word)         */
+#define FP2_ERR_DEVICE_CHECK -6  /* a device-side consistency check failed (status)  */
+
+/* ---- status word bits (fp2_status_check *device_status) ------------------ */
+#define FP2_STATUS_BAD_SEQLENS 0x1u   /* cu_seqlens not consistent with the problem sizes */
+#define FP2_STATUS_BAD_PAGE 0x2u      /* a page id outside [0, num_pages)                 */
+#define FP2_STATUS_TIMEOUT 0x4u       /* a bounded wait inside a kernel ran out           */
+
+/* ---- element types -------------------------------------------------------- */
+#define FP2_DTYPE_BF16 0   /* bfloat16 Q, K, V                                     */
+#define FP2_DTYPE_E4M3 1   /* float8 e4m3 Q, K, V with per-(block, head) fp32 scales */
+
+/* ---- fp2_prefill flags ---------------------------------------------------- */
+#define FP2_NO_CORRECTION 0x1u     /* skipped blocks are dropped (no pseudo-tokens)   */
+#define FP2_DEBUG_DROP_Q_LOAD 0x100u /* fault injection: never load Q, so the first
+                                        wait on it runs out; the kernel records
+                                        FP2_STATUS_TIMEOUT and returns */
+
+/*
+ * One prefill problem: a varlen batch of num_seqs causal sequences packed
+ * along the token axis (T = sum of seqlens tokens).
+ *
+ *   seqlens      HOST int32 [num_seqs], each >= 1.  Used for validation and
+ *                sizing on the host.
+ *   cu_seqlens   DEVICE int32 [num_seqs + 1]; cu_seqlens[0] = 0 and
+ *                cu_seqlens[s+1] - cu_seqlens[s] = seqlens[s].  Checked on the
+ *                device (FP2_STATUS_BAD_SEQLENS).
+ *   num_q_heads, num_kv_heads   Hq, Hkv with Hq % Hkv == 0 and
+ *                (Hq / Hkv) * block_size a multiple of 128 (PackGQA tiles of
+ *                128 query rows).
+ *   head_dim     d in {64, 128}.   block_size   B in {64, 128}.
+ *   tau          threshold >= 0 (0 = dense: every causal block kept).
+ *   page_size    0: K and V are contiguous [T, Hkv, d].  64: K and V are page
+ *                pools [num_pages, 64, Hkv, d]; token t of sequence s is in
+ *                page page_table[s * page_table_stride + t / 64], slot t % 64.
+ *   num_pages, page_table (DEVICE int32), page_table_stride
+ *                describe the pool when page_size == 64; the stride must be
+ *                >= ceil(max L_s / 64).  Page ids are checked on the device
+ *                (FP2_STATUS_BAD_PAGE; such a page reads as zeros).
+ */
+typedef struct fp2_problem {
+    int32_t num_seqs;
+    const int32_t* seqlens;
+    const int32_t* cu_seqlens;
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int32_t head_dim;
+    int32_t block_size;
+    double tau;
+    int32_t page_size;
+    int32_t num_pages;
+    const int32_t* page_table;
+    int32_t page_table_stride;
+} fp2_problem;
+
+/*
+ * Sizes and the layout of the plan buffer, all in bytes from its start
+ * (every offset is 256-byte aligned).  Filled by fp2_plan_sizes.
+ *
+ *   row_ptr     int32 [num_rows + 1]      CSR row pointers.  Row r is the
+ *               (sequence s, kv-head g, query block i) with
+ *               r = g * num_blocks + (blocks of sequences before s) + i.
+ *   col_idx     int32 [nnz_cap]           kept key-block ids, local to the
+ *               sequence, ascending within a row (0 first, i last).
+ *   kept_mask   uint32 [num_rows, mask_words]  bit j of row r set iff block j
+ *               is kept (same information as the CSR row).
+ *   kbar, vbar  float [num_blocks, Hkv, d] block means of K and V.
+ *   kbar_bf16, vbar_bf16  the same means rounded to bfloat16 (operands of the
+ *               correction's tensor-core products).
+ *   kbar_e4m3, vbar_e4m3  uint8 [num_blocks, Hkv, d] e4m3 codes of the means,
+ *   kbar_scale, vbar_scale float [num_blocks, Hkv] their per-(block, head)
+ *               scales (absmax / 448); used by the FP8 path.
+ *   status      int32 [1] status word (FP2_STATUS_* bits), cleared by fp2_plan.
+ *   (the rest is private to the library)
+ */
+typedef struct fp2_plan_layout {
+    int64_t num_tokens;
+    int64_t num_blocks;
+    int64_t num_rows;
+    int64_t nnz_cap;
+    int32_t mask_words;
+    int32_t max_blocks_per_seq;
+    size_t off_row_ptr;
+    size_t off_col_idx;
+    size_t off_kept_mask;
+    size_t off_kbar;
+    size_t off_vbar;
+    size_t off_kbar_bf16;
+    size_t off_vbar_bf16;
+    size_t off_kbar_e4m3;
+    size_t off_vbar_e4m3;
+    size_t off_kbar_scale;
+    size_t off_vbar_scale;
+    size_t off_status;
+    size_t off_meta;
+    size_t plan_bytes;        /* bytes the plan buffer must have      */
+    size_t workspace_bytes;   /* bytes fp2_plan's scratch must have    */
+} fp2_plan_layout;
+
+/* Library version (FP2_VERSION of the build). */
+int fp2_version(void);
+
+/* Static description of an error code; never NULL. */
+const char* fp2_strerror(int code);
+
+/*
+ * Host-only and pure: validates *problem (device pointers are not
+ * dereferenced) and fills *layout.  nnz_cap is the dense count
+ * Hkv * sum_s nb_s (nb_s + 1) / 2, so the CSR can never overflow.
+ */
+int fp2_plan_sizes(const fp2_problem* problem, fp2_plan_layout* layout);
+
+/*
+ * Stage 1, pattern discovery (Figure 3).  Reads bf16 q [T, Hq, d] and bf16
+ * k, v (contiguous or paged, per problem->page_size) once, and writes into
+ * `plan` (plan_bytes >= layout.plan_bytes) the CSR index, the kept-block
+ * masks, the K/V block means (fp32, bf16 and e4m3 + scales) and a cleared
+ * status word.  `workspace` (workspace_bytes >= layout.workspace_bytes,
+ * device memory, 256-byte aligned) is scratch, free again once the enqueued
+ * work completes.  Block lists are decided as if every score were computed in
+ * float64: scores are computed in float32 and any block within the float32
+ * error bound of the threshold (or of the row maximum) is re-scored in
+ * float64.
+ */
+int fp2_plan(const fp2_problem* problem, const void* q, const void* k, const void* v,
+             void* plan, size_t plan_bytes, void* workspace, size_t workspace_bytes,
+             void* stream);
+
+/*
+ * Direct online FP8 quantisation (Table 1 footnote): for every (block, head)
+ * of x, scale = absmax / 448 (1 for an all-zero block) and
+ * x_e4m3 = round-to-nearest-even-saturating(x / scale), both in fp32.
+ *   which = 0: x is q [T, Hq, d];  scales [num_blocks, Hq].
+ *   which = 1 or 2: x is k or v in the problem's K/V layout (contiguous or
+ *                   paged); x_e4m3 has the same layout; scales [num_blocks, Hkv].
+ *                   In a paged pool only the slots of real tokens are written.
+ * `plan` must come from fp2_plan on the same problem (it holds the block map).
+ */
+int fp2_quantize_fp8(const fp2_problem* problem, const void* plan, size_t plan_bytes,
+                     const void* x, int32_t which, void* x_e4m3, float* scales, void* stream);
+
+/*
+ * Stage 2, sparse attention with mean correction (Figure 3 / Figure 4).
+ *   dtype FP2_DTYPE_BF16: q, k, v are the bf16 tensors given to fp2_plan and
+ *     q_scale, k_scale, v_scale must be NULL.
+ *   dtype FP2_DTYPE_E4M3: q, k, v are e4m3 tensors from fp2_quantize_fp8 and
+ *     the three scale arrays are the ones it produced.
+ *   o    DEVICE bf16 [T, Hq, d]   attention output.
+ *   lse  DEVICE float [Hq, T]     natural-log softmax denominator.
+ *   flags  FP2_NO_CORRECTION and FP2_DEBUG_* bits.
+ * Work is spread over one persistent CTA per SM; each CTA takes PackGQA
+ * tiles (two 128-row query tiles of one kv-head) longest row first.
+ */
+int fp2_prefill(const fp2_problem* problem, const void* plan, size_t plan_bytes,
+                const void* q, const void* k, const void* v,
+                const float* q_scale, const float* k_scale, const float* v_scale,
+                int32_t dtype, void* o, float* lse, uint32_t flags, void* stream);
+
+/*
+ * Synchronises `stream`, then reads the plan's status word into
+ * *device_status (may be NULL).  Returns FP2_OK when it is zero,
+ * FP2_ERR_TIMEOUT when FP2_STATUS_TIMEOUT is set, otherwise
+ * FP2_ERR_DEVICE_CHECK; FP2_ERR_CUDA when the synchronisation itself fails.
+ */
+int fp2_status_check(const void* plan, size_t plan_bytes, void* stream, int32_t* device_status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP2_H_ */

@@ -92,7 +92,7 @@ def block_means(x, seqlens: Sequence[int], B: int):
     x: [T, H, d] packed varlen tensor.  Returns (means [NB, H, d] float64,
     counts [NB] int64), blocks ordered sequence by sequence.
     """
-    x = _as64(x)
+    x = np.asarray(x)
     lay = block_layout(seqlens, B)
     T, H, d = x.shape
     NB = int(lay["cu_blocks"][-1])
@@ -104,7 +104,7 @@ def block_means(x, seqlens: Sequence[int], B: int):
         for i in range(int(lay["nb"][s])):
             lo = t0 + i * B
             hi = t0 + min((i + 1) * B, int(L))
-            means[b0 + i] = x[lo:hi].mean(axis=0)
+            means[b0 + i] = _as64(x[lo:hi]).mean(axis=0)
             counts[b0 + i] = hi - lo
     return means, counts
 
@@ -144,7 +144,8 @@ def select_blocks(sc: np.ndarray, tau: float) -> np.ndarray:
     return np.nonzero(keep)[0].astype(np.int64)
 
 
-def plan(q, k, v, seqlens: Sequence[int], B: int, tau: float) -> Dict[str, object]:
+def plan(q, k, v, seqlens: Sequence[int], B: int, tau: float,
+         rows: Optional[Sequence[tuple]] = None) -> Dict[str, object]:
     """Stage 1 of the pipeline: means, scores, kept lists, CSR and K/V means.
 
     q [T, Hq, d], k and v [T, Hkv, d] (contiguous; use gather_paged first for
@@ -154,10 +155,10 @@ def plan(q, k, v, seqlens: Sequence[int], B: int, tau: float) -> Dict[str, objec
       thresh  list over rows of tau * m (None for tau == 0),
       kept    list over rows of ascending kept block ids (local to the sequence),
       row_ptr [R+1] int64, col_idx [nnz] int64, with R = Hkv * NB.
+    rows: optional list of (s, i) query blocks; only their rows (all
+      kv-heads) are scored and selected, the others stay None and the CSR is
+      not built.
     """
-    q = _as64(q)
-    k = _as64(k)
-    v = _as64(v)
     Hq, Hkv = q.shape[1], k.shape[1]
     assert Hq % Hkv == 0
     G = Hq // Hkv
@@ -171,22 +172,25 @@ def plan(q, k, v, seqlens: Sequence[int], B: int, tau: float) -> Dict[str, objec
     scores: List[Optional[np.ndarray]] = [None] * R
     thresh: List[Optional[float]] = [None] * R
     kept: List[Optional[np.ndarray]] = [None] * R
+    if rows is None:
+        rows = [(s, i) for s in range(len(lay["seqlens"])) for i in range(int(lay["nb"][s]))]
     for g in range(Hkv):
         heads = list(range(g * G, (g + 1) * G))
-        for s in range(len(lay["seqlens"])):
+        for (s, i) in rows:
             b0 = int(lay["cu_blocks"][s])
             nbs = int(lay["nb"][s])
             kb = kbar[b0:b0 + nbs, g, :]
-            for i in range(nbs):
-                r = g * NB + b0 + i
-                sc = block_scores(qbar[b0 + i][heads], kb, i)
-                scores[r] = sc
-                thresh[r] = None if tau == 0.0 else float(tau * sc.max())
-                kept[r] = select_blocks(sc, tau)
-    row_ptr = np.zeros(R + 1, dtype=np.int64)
-    for r in range(R):
-        row_ptr[r + 1] = row_ptr[r] + len(kept[r])
-    col_idx = np.concatenate(kept) if R else np.zeros(0, dtype=np.int64)
+            r = g * NB + b0 + i
+            sc = block_scores(qbar[b0 + i][heads], kb, i)
+            scores[r] = sc
+            thresh[r] = None if tau == 0.0 else float(tau * sc.max())
+            kept[r] = select_blocks(sc, tau)
+    row_ptr = col_idx = None
+    if all(x is not None for x in kept):
+        row_ptr = np.zeros(R + 1, dtype=np.int64)
+        for r in range(R):
+            row_ptr[r + 1] = row_ptr[r] + len(kept[r])
+        col_idx = np.concatenate(kept) if R else np.zeros(0, dtype=np.int64)
     return {
         "B": B, "tau": tau, "Hq": Hq, "Hkv": Hkv, "G": G, "layout": lay,
         "qbar": qbar, "kbar": kbar, "vbar": vbar, "counts": counts,
@@ -211,9 +215,9 @@ def attend(q, k, v, pl: Dict[str, object], correction: bool = True,
       left NaN.  kept_override: optional {(s, g, i): kept ids} replacing the
       plan's selection for those rows.
     """
-    q = _as64(q)
-    k = _as64(k)
-    v = _as64(v)
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
     B = int(pl["B"])
     G = int(pl["G"])
     Hq, Hkv = int(pl["Hq"]), int(pl["Hkv"])
@@ -242,9 +246,9 @@ def attend(q, k, v, pl: Dict[str, object], correction: bool = True,
             # exact keys of the kept blocks
             kidx = np.concatenate([np.arange(t0 + j * B, t0 + min((j + 1) * B, L)) for j in kept])
             kpos = kidx - t0
-            Kk, Vk = k[kidx, g, :], v[kidx, g, :]
+            Kk, Vk = _as64(k[kidx, g, :]), _as64(v[kidx, g, :])
             for h in range(g * G, (g + 1) * G):
-                Qh = q[qlo:qhi, h, :]                          # [n_i, d]
+                Qh = _as64(q[qlo:qhi, h, :])                   # [n_i, d]
                 s_exact = (Qh @ Kk.T) * inv_sqrt_d               # [n_i, nk]
                 s_exact = np.where(kpos[None, :] <= qpos[:, None], s_exact, -np.inf)
                 if correction and skipped:

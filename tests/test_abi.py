@@ -1,0 +1,140 @@
+"""The C-ABI library loads, exports what include/fp2.h declares, and its
+host-only entry points validate arguments (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from block_sparse_long_fp2_b200 import binding as fb
+from block_sparse_long_fp2_b200 import build as fbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fbuild.build()
+    return fb.lib()
+
+
+def _declared():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            text = open(os.path.join(inc, f)).read()
+            names |= set(re.findall(r"^\s*(?:int|const char\*)\s+(fp2_\w+)\s*\(", text, re.M))
+    return names
+
+
+def test_header_declares_the_entry_points():
+    assert {"fp2_version", "fp2_strerror", "fp2_plan_sizes", "fp2_plan", "fp2_quantize_fp8",
+            "fp2_prefill", "fp2_status_check"} <= _declared()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_version_and_strerror(lib):
+    assert fb.fp2_version() == 1
+    assert fb.strerror(0) == "ok"
+    for code in [-1, -2, -3, -4, -5, -6]:
+        assert fb.strerror(code) not in ("", "unknown error")
+    assert fb.strerror(-99) == "unknown error"
+
+
+def _problem(seqlens=(1000, 37), Hq=32, Hkv=8, d=128, B=128, tau=0.1, page_size=0,
+             page_table=None, num_pages=0):
+    # device pointers are never dereferenced by fp2_plan_sizes: fake non-null values
+    p = fb.Problem(seqlens, 0x1000, Hq, Hkv, d, B, tau)
+    p.c.page_size = page_size
+    p.c.num_pages = num_pages
+    if page_table is not None:
+        p.c.page_table = 0x2000
+        p.c.page_table_stride = page_table
+    return p
+
+
+def test_plan_sizes_counts(lib):
+    lay = fb.fp2_plan_sizes(_problem())
+    nb = [8, 1]
+    assert lay.num_tokens == 1037 and lay.num_blocks == 9 and lay.num_rows == 72
+    assert lay.nnz_cap == 8 * (8 * 9 // 2 + 1)
+    assert lay.mask_words == 1 and lay.max_blocks_per_seq == 8
+    offs = [lay.off_status, lay.off_row_ptr, lay.off_col_idx, lay.off_kept_mask, lay.off_kbar,
+            lay.off_vbar, lay.off_kbar_bf16, lay.off_vbar_bf16, lay.off_kbar_e4m3,
+            lay.off_vbar_e4m3, lay.off_kbar_scale, lay.off_vbar_scale]
+    assert lay.off_status == 0
+    assert all(o % 256 == 0 for o in offs)
+    assert len(set(offs)) == len(offs) and max(offs) < lay.plan_bytes
+    assert lay.off_col_idx - lay.off_row_ptr >= 4 * 73
+    assert lay.workspace_bytes >= 8 * 9 * 32 * 128 + 4 * lay.nnz_cap
+    assert sum(n * (n + 1) // 2 for n in nb) * 8 == lay.nnz_cap
+
+
+def test_plan_sizes_128k_index_memory(lib):
+    # the CSR of a 128K prefill with 8 kv-heads is at most the dense count
+    lay = fb.fp2_plan_sizes(_problem(seqlens=(131072,), tau=0.05))
+    assert lay.nnz_cap == 8 * 1024 * 1025 // 2
+    assert lay.mask_words == 32
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=30, Hkv=8), fb.FP2_ERR_INVALID_ARG),          # Hq % Hkv
+    (dict(d=96), fb.FP2_ERR_UNSUPPORTED),
+    (dict(B=32), fb.FP2_ERR_UNSUPPORTED),
+    (dict(Hq=8, Hkv=8, B=64), fb.FP2_ERR_UNSUPPORTED),     # G * B not a multiple of 128
+    (dict(tau=-0.1), fb.FP2_ERR_INVALID_ARG),
+    (dict(tau=float("nan")), fb.FP2_ERR_INVALID_ARG),
+    (dict(seqlens=(10, 0)), fb.FP2_ERR_INVALID_ARG),
+    (dict(page_size=32), fb.FP2_ERR_UNSUPPORTED),
+    (dict(page_size=64, page_table=None, num_pages=4), fb.FP2_ERR_INVALID_ARG),
+    (dict(page_size=64, page_table=15, num_pages=40), fb.FP2_ERR_INVALID_ARG),  # stride < 16 pages
+])
+def test_plan_sizes_rejects(lib, kw, code):
+    with pytest.raises(fb.Fp2Error) as e:
+        fb.fp2_plan_sizes(_problem(**kw))
+    assert e.value.code == code
+
+
+def test_paged_problem_accepted(lib):
+    lay = fb.fp2_plan_sizes(_problem(page_size=64, page_table=16, num_pages=40))
+    assert lay.num_blocks == 9
+
+
+def test_null_problem_and_buffers_rejected(lib):
+    L = fb.lib()
+    assert L.fp2_plan_sizes(None, None) == fb.FP2_ERR_INVALID_ARG
+    p = _problem()
+    assert L.fp2_plan(p.ref, None, None, None, None, 0, None, 0, None) == fb.FP2_ERR_INVALID_ARG
+    lay = fb.fp2_plan_sizes(p)
+    # capacity is checked before anything is enqueued
+    rc = L.fp2_plan(p.ref, 0x10000, 0x10000, 0x10000, 0x100000, lay.plan_bytes - 256, 0x200000,
+                    lay.workspace_bytes, None)
+    assert rc == fb.FP2_ERR_CAPACITY
+    rc = L.fp2_prefill(p.ref, 0x100000, lay.plan_bytes, 0x10000, 0x10000, 0x10000, None, None,
+                       None, 7, 0x10000, 0x10000, 0, None)
+    assert rc == fb.FP2_ERR_INVALID_ARG   # unknown dtype
+    rc = L.fp2_prefill(p.ref, 0x100000, lay.plan_bytes, 0x10008, 0x10000, 0x10000, None, None,
+                       None, 0, 0x10000, 0x10000, 0, None)
+    assert rc == fb.FP2_ERR_INVALID_ARG   # q not 16-byte aligned
+    rc = L.fp2_prefill(p.ref, 0x100000, lay.plan_bytes, 0x10000, 0x10000, 0x10000, None, None,
+                       None, 0, 0x10000, 0x10000, 0x8000, None)
+    assert rc == fb.FP2_ERR_INVALID_ARG   # unknown flag
+    rc = L.fp2_quantize_fp8(p.ref, 0x100000, lay.plan_bytes, 0x10000, 3, 0x10000, 0x10000, None)
+    assert rc == fb.FP2_ERR_INVALID_ARG   # which out of range
+
+
+def test_no_cpu_fallback_in_product_path():
+    # the package never imports the oracle
+    pkg = os.path.join(ROOT, "block_sparse_long_fp2_b200")
+    for f in os.listdir(pkg):
+        if f.endswith(".py"):
+            src = open(os.path.join(pkg, f)).read()
+            assert "import oracle" not in src and "from oracle" not in src, f

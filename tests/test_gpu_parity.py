@@ -1,0 +1,188 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle.
+
+Block lists must match bit-exactly outside the 1e-5 threshold band; O within
+rel-L2 1e-2 and LSE within 1e-3 (BF16).  Small cases are checked on every
+row; they span several tiles, ragged tails, one and several query-tile
+pairs per row, several pseudo tiles per row, varlen and paged layouts.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from block_sparse_long_fp2_b200 import binding as fb
+from block_sparse_long_fp2_b200 import synth
+
+from fp2_harness import (LSE_ABS, REL_L2_BF16, GpuRun, check_attention, compare_plan,
+                         oracle_inputs)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from block_sparse_long_fp2_b200 import build
+    build.build()
+    fb.lib()
+
+
+SMALL = {
+    # name: (seqlens, Hq, Hkv, d, B, tau, generator, needles, page_size, pool_pages)
+    "pr1_ref_1k": ([1024], 4, 1, 64, 64, 0.3, "needles", 8, 0, 0),
+    "ragged_d128": ([700, 333, 1100], 8, 2, 128, 128, 0.1, "lowrank", 0, 0, 0),
+    "one_tile_G2_B64": ([513], 2, 1, 64, 64, 0.05, "lowrank", 0, 0, 0),
+    "one_tile_G1_B128": ([640, 200], 4, 4, 128, 128, 0.3, "lowrank", 0, 0, 0),
+    "G8_d64_B128_tau1": ([900], 16, 2, 64, 128, 1.0, "lowrank", 0, 0, 0),
+    "G3_odd_tiles": ([1000, 129], 6, 2, 64, 128, 0.2, "lowrank", 0, 0, 0),
+    "B64_d128": ([777], 8, 2, 128, 64, 0.1, "lowrank", 0, 0, 0),
+    "dense_tau0": ([1000, 300], 8, 2, 128, 128, 0.0, "lowrank", 0, 0, 0),
+    "paged_mix_small": ([1500, 640, 97], 8, 2, 128, 128, 0.1, "lowrank", 0, 64, 60),
+    "two_pseudo_tiles": ([9000], 2, 1, 64, 64, 0.2, "lowrank", 0, 0, 0),
+}
+
+
+def _case(name, seed_base=500):
+    seqlens, Hq, Hkv, d, B, tau, gen, nn, page, pool = SMALL[name]
+    wl = synth.small_workload(seqlens, Hq, Hkv, d, B, tau, seed=seed_base + sorted(SMALL).index(name),
+                              generator=gen, n_needles=nn, page_size=page, pool_pages=pool)
+    if name == "pr1_ref_1k":
+        wl = synth.workloads()["pr1_ref_1k"]
+    return wl, synth.generate(wl)
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_plan_matches_oracle(name):
+    wl, x = _case(name)
+    run = GpuRun(wl, x).plan()
+    rc, st = run.status()
+    assert rc == fb.FP2_OK and st == 0
+    q, k, v = oracle_inputs(x, wl)
+    pl = oracle.plan(q, k, v, wl.seqlens, wl.B, wl.tau)
+    res = compare_plan(pl, run.kept_lists())
+    assert res["outside_band"] == 0, res
+    # the CSR is exactly the kept lists: row_ptr consistent, nnz <= cap
+    rp = run.view.row_ptr.cpu().numpy()
+    assert rp[0] == 0 and np.all(np.diff(rp) >= 1) and rp[-1] <= run.lay.nnz_cap
+    # block means of K and V (fp32 of the exact means)
+    kb = run.view.kbar.cpu().numpy()
+    vb = run.view.vbar.cpu().numpy()
+    assert np.allclose(kb, pl["kbar"], rtol=2e-7, atol=1e-7)
+    assert np.allclose(vb, pl["vbar"], rtol=2e-7, atol=1e-7)
+    kb16 = run.view.kbar_bf16.float().cpu().numpy()
+    assert np.allclose(kb16, pl["kbar"], rtol=2 ** -8, atol=1e-6)
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_prefill_matches_oracle(name):
+    wl, x = _case(name)
+    run = GpuRun(wl, x).plan().prefill()
+    rc, st = run.status()
+    assert rc == fb.FP2_OK and st == 0
+    q, k, v = oracle_inputs(x, wl)
+    pl = oracle.plan(q, k, v, wl.seqlens, wl.B, wl.tau)
+    res = check_attention(wl, x, run, pl)
+    assert res["finite"], res
+    assert res["rel_l2"] <= REL_L2_BF16, res
+    assert res["lse_max_abs"] <= LSE_ABS, res
+
+
+def test_no_correction_flag_drops_the_surrogate():
+    # N(0, 1) inputs keep the logits O(1), so the skipped mass is visible
+    wl = synth.small_workload([700, 333, 1100], 8, 2, 128, 128, 0.3, seed=91, generator="normal")
+    x = synth.generate(wl)
+    run = GpuRun(wl, x).plan().prefill(flags=fb.FP2_NO_CORRECTION)
+    q, k, v = oracle_inputs(x, wl)
+    pl = oracle.plan(q, k, v, wl.seqlens, wl.B, wl.tau)
+    res = check_attention(wl, x, run, pl, correction=False)
+    assert res["rel_l2"] <= REL_L2_BF16 and res["lse_max_abs"] <= LSE_ABS, res
+    # and the corrected run is measurably different (something was skipped)
+    run2 = GpuRun(wl, x).plan().prefill()
+    assert len(run2.kept_lists()[0]) >= 1
+    assert float((run2.lse - run.lse).abs().max()) > 1e-2
+
+
+def test_dense_tau0_equals_brute_force_dense():
+    wl, x = _case("dense_tau0")
+    run = GpuRun(wl, x).plan().prefill()
+    O, LSE = run.outputs()
+    Od, Ld = oracle.dense_attention(x["q"], x["k"], x["v"], wl.seqlens)
+    from fp2_harness import rel_l2
+    assert rel_l2(O, Od) <= REL_L2_BF16
+    assert np.max(np.abs(LSE - Ld)) <= LSE_ABS
+
+
+def test_paged_layout_is_bit_identical_to_contiguous():
+    # equal-length batch, shuffled pages vs the packed contiguous layout
+    seqlens = [1536, 1536, 1536]
+    wl = synth.small_workload(seqlens, 8, 2, 128, 128, 0.1, seed=77, page_size=64, pool_pages=90)
+    x = synth.generate(wl)
+    a = GpuRun(wl, x, paged=True).plan().prefill()
+    b = GpuRun(wl, x, paged=False).plan().prefill()
+    assert a.kept_lists() == b.kept_lists()
+    Oa, La = a.outputs()
+    Ob, Lb = b.outputs()
+    assert np.array_equal(Oa, Ob) and np.array_equal(La, Lb)
+
+
+def test_repeat_calls_are_deterministic():
+    wl, x = _case("ragged_d128")
+    run = GpuRun(wl, x).plan().prefill()
+    O1, L1 = run.outputs()
+    run.plan().prefill()
+    O2, L2 = run.outputs()
+    assert np.array_equal(O1, O2) and np.array_equal(L1, L2)
+
+
+@pytest.mark.parametrize("edit", ["empty_sequence", "total_mismatch", "nonzero_start"])
+def test_device_check_bad_cu_seqlens_does_no_work(edit):
+    # cu_seqlens whose sizes disagree with the host seqlens: every kernel
+    # returns without touching memory and the status word says why.  (A
+    # permutation of lengths that keeps every total is consistent, and is
+    # simply the problem the device was given.)
+    import torch
+    wl, x = _case("ragged_d128")
+    run = GpuRun(wl, x)
+    if edit == "empty_sequence":
+        run.cu[2] = run.cu[1]
+    elif edit == "total_mismatch":
+        run.cu[3] += 1
+    else:
+        run.cu[0] = 1
+    run.plan().prefill()
+    rc, st = run.status()
+    assert rc == fb.FP2_ERR_DEVICE_CHECK and st & fb.FP2_STATUS_BAD_SEQLENS
+    assert torch.isnan(run.o.float()).all()   # prefill did not write
+
+
+def test_device_check_bad_page_id_is_recorded():
+    wl, x = _case("paged_mix_small")
+    x = dict(x)
+    pt = x["page_table"].copy()
+    pt[1, 3] = 10_000                # out of the pool
+    x["page_table"] = pt
+    run = GpuRun(wl, x).plan().prefill()
+    rc, st = run.status()
+    assert rc == fb.FP2_ERR_DEVICE_CHECK and st & fb.FP2_STATUS_BAD_PAGE
+    # a fresh, valid plan on the same context works again
+    wl2, x2 = _case("paged_mix_small")
+    run2 = GpuRun(wl2, x2).plan().prefill()
+    assert run2.status() == (fb.FP2_OK, 0)
+
+
+def test_quantize_fp8_matches_oracle_codes():
+    import torch
+    wl, x = _case("ragged_d128")
+    run = GpuRun(wl, x).plan()
+    NB = int(run.lay.num_blocks)
+    for which, name, H in [(0, "q", wl.Hq), (1, "k", wl.Hkv), (2, "v", wl.Hkv)]:
+        src = {0: run.q, 1: run.k, 2: run.v}[which]
+        codes = torch.zeros(src.shape, dtype=torch.uint8, device="cuda")
+        scales = torch.zeros((NB, H), dtype=torch.float32, device="cuda")
+        fb.fp2_quantize_fp8(run.prob, run.plan_buf, src, which, codes, scales)
+        got = codes.view(torch.float8_e4m3fn).to(torch.float64).cpu().numpy()
+        ref, ref_s = oracle.quantize_e4m3(x[name], wl.seqlens, wl.B)
+        assert np.array_equal(scales.cpu().numpy().astype(np.float64), ref_s)
+        assert np.array_equal(got, ref)
