@@ -1,0 +1,71 @@
+// fp2_plan_static: fp2_plan for callers that cannot allocate device memory.
+//
+// fp2_plan needs a caller-provided scratch workspace.  Some callers have no
+// way to provide one: a serving process that has already handed (nearly)
+// all device memory to its own KV-cache pool or caching allocator, so a
+// further cudaMalloc would fail or fragment that pool; or a host program
+// that only receives device pointers from another runtime and owns no
+// device allocator at all.  This entry point runs the same planning
+// kernels with their scratch placed in a fixed-size array that lives in
+// the library's device image (kStaticWorkspaceBytes below).  The array is
+// created when the library is loaded onto a device and is held by every
+// device that loads the library until the process exits.
+#include <mutex>
+#include <vector>
+
+#include "fp2_internal.h"
+
+namespace fp2 {
+
+namespace {
+
+constexpr size_t kStaticWorkspaceBytes = FP2_STATIC_WORKSPACE_BYTES;
+
+// The scratch array.  In host code this name is only a host-side stand-in
+// for the symbol, not a device address: the device address is obtained with
+// cudaGetSymbolAddress below and only that address is handed to kernels.
+static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+
+std::mutex g_mu;
+std::vector<void*> g_addr;   // per device: device address of g_static_workspace
+
+// Device address of the array on the current device, looked up once per
+// device (with that device current).  nullptr on failure.
+void* static_workspace_address() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if ((int)g_addr.size() <= dev) g_addr.resize(dev + 1, nullptr);
+    if (!g_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess) return nullptr;
+        g_addr[dev] = p;
+    }
+    return g_addr[dev];
+}
+
+}  // namespace
+
+}  // namespace fp2
+
+using namespace fp2;
+
+extern "C" int fp2_plan_static(const fp2_problem* problem, const void* q, const void* k,
+                               const void* v, void* plan, size_t plan_bytes, void* stream) {
+    Layout L;
+    int rc = compute_layout(problem, &L);
+    if (rc != FP2_OK) return rc;
+    if (!q || !k || !v || !plan) return FP2_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+         reinterpret_cast<uintptr_t>(v)) % 16 != 0 ||
+        reinterpret_cast<uintptr_t>(plan) % 256 != 0)
+        return FP2_ERR_INVALID_ARG;
+    if (plan_bytes < L.pub.plan_bytes) return FP2_ERR_CAPACITY;
+    if (L.pub.workspace_bytes > kStaticWorkspaceBytes) return FP2_ERR_CAPACITY;
+    void* ws = static_workspace_address();
+    if (!ws) return FP2_ERR_CUDA;
+    // No part of the workspace has to start at zero: every kernel writes the
+    // scratch entries it reads later in the same call.
+    return launch_plan(L, problem, q, k, v, plan_ptrs(L, plan), ws_ptrs(L, ws),
+                       static_cast<cudaStream_t>(stream));
+}

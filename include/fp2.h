@@ -223,6 +223,31 @@ int fp2_prefill(const fp2_problem* problem, const void* plan, size_t plan_bytes,
                 int32_t dtype, void* o, float* lse, uint32_t flags, void* stream);
 
 /*
+ * fp2_plan_static -- the same stage 1 as fp2_plan, for callers that cannot
+ * allocate device memory for a workspace (for example a serving process
+ * whose KV-cache pool or caching allocator already holds the device
+ * memory, or a host that only receives device pointers from another
+ * runtime and has no allocator of its own).  The paper has no counterpart:
+ * this is an interface convenience of this library.
+ *
+ * The scratch lives in one fixed array of FP2_STATIC_WORKSPACE_BYTES inside
+ * the library's device image, which every device that loads the library
+ * holds until the process exits.  Problems whose layout.workspace_bytes
+ * exceed it are rejected with FP2_ERR_CAPACITY (16 MiB covers, e.g., one
+ * 32K-token layer with 32 query / 8 kv heads of dim 128).  The call
+ * allocates and frees nothing.  Its first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  Every call shares the
+ * one array and leaves the last call's scratch in it (no entry needs to
+ * start at zero), so calls whose work overlaps on the GPU -- on two streams,
+ * or from two threads -- race; order them on one stream.  Arguments,
+ * outputs and errors are otherwise those of fp2_plan.
+ */
+#define FP2_STATIC_WORKSPACE_BYTES ((size_t)16 << 20)
+int fp2_plan_static(const fp2_problem* problem, const void* q, const void* k, const void* v,
+                    void* plan, size_t plan_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then reads the plan's status word into
  * *device_status (may be NULL).  Returns FP2_OK when it is zero,
  * FP2_ERR_TIMEOUT when FP2_STATUS_TIMEOUT is set, otherwise
