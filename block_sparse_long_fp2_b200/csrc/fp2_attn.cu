@@ -431,6 +431,107 @@ drain:
     mbar_wait_drain(&B.drain, 0, P.status);
 }
 
+// Row maximum of the raw (unscaled) scores of the masked-in columns of this
+// thread's row of S.  Two 32-column TMEM loads in flight.
+template <int BLK, bool MASKED>
+__device__ __forceinline__ void max16(const uint32_t (&r)[16], uint32_t vb, float& mx) {
+    if (MASKED) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            if ((vb >> e) & 1u) mx = fmaxf(mx, __uint_as_float(r[e]));
+    } else {
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) mx = fmax3(mx, __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+    }
+}
+
+template <int BLK, bool MASKED>
+__device__ __forceinline__ uint32_t chunk_bits(int kind, int tok, const TileWalk<BLK>& walk, int j,
+                                               int c16) {
+    return MASKED ? (col_bits(kind, tok, walk, j, c16 / 2) >> (16 * (c16 & 1))) : 0xFFFFu;
+}
+
+// Row maximum of the raw (unscaled) scores of the masked-in columns of this
+// thread's row of S; one 16-column TMEM load always in flight.
+template <int BLK, bool MASKED>
+__device__ __forceinline__ float tile_max(uint32_t t_s, int kind, int tok, const TileWalk<BLK>& walk,
+                                          int j) {
+    float mx = -INFINITY;
+    uint32_t ra[16], rb[16];
+    tmem_ld16(t_s, ra);
+#pragma unroll 1
+    for (int c = 0; c < BLK / 16; c += 2) {
+        tmem_ld_wait();
+        tmem_ld16(t_s + 16 * (c + 1), rb);
+        max16<BLK, MASKED>(ra, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c), mx);
+        tmem_ld_wait();
+        if (c + 2 < BLK / 16) tmem_ld16(t_s + 16 * (c + 2), ra);
+        max16<BLK, MASKED>(rb, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c + 1), mx);
+    }
+    return mx;
+}
+
+// 16 columns (two 8-column chunks) of P: 2^(s * scale + shift), bf16, into
+// the 128B-swizzled K-major P tile.
+template <bool MASKED>
+__device__ __forceinline__ void p16(const uint32_t (&r)[16], uint32_t vb, int c16, uint8_t* pbuf,
+                                    int prow, uint64_t scale2, uint64_t shift2, uint64_t& sum2,
+                                    float& mx) {
+#pragma unroll
+    for (int q8 = 0; q8 < 2; ++q8) {
+        uint32_t packed[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+            const int e = 8 * q8 + 2 * e2;
+            float s0 = __uint_as_float(r[e]), s1 = __uint_as_float(r[e + 1]);
+            if (MASKED) {
+                s0 = ((vb >> e) & 1u) ? s0 : -INFINITY;
+                s1 = ((vb >> (e + 1)) & 1u) ? s1 : -INFINITY;
+            }
+            mx = fmax3(mx, s0, s1);
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(s0, s1), scale2, shift2), x0, x1);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            sum2 = f2_add(sum2, f2_pack(p0, p1));
+            packed[e2] = pack_bf16x2(p0, p1);
+        }
+        const int cc = 2 * c16 + q8;                 // 8-column chunk of the row
+        const int atom = cc >> 3, chunk = cc & 7;
+        uint8_t* dst = pbuf + atom * (kTileM * 128) + prow * 128 + ((chunk ^ (prow & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    }
+}
+
+// P = 2^(s * scale + shift) for this thread's row of S (zero where masked
+// out), written as bf16 into the P tile; returns the fp32 row sum and the
+// row maximum of the raw masked-in scores.
+template <int BLK, bool MASKED>
+__device__ __forceinline__ float tile_p(uint32_t t_s, uint8_t* pbuf, int prow, int kind, int tok,
+                                        const TileWalk<BLK>& walk, int j, float scale, float shift,
+                                        float& rmax_raw) {
+    const uint64_t scale2 = f2_pack(scale, scale);
+    const uint64_t shift2 = f2_pack(shift, shift);
+    uint64_t sum2 = f2_pack(0.f, 0.f);
+    float mx = -INFINITY;
+    uint32_t ra[16], rb[16];
+    tmem_ld16(t_s, ra);
+#pragma unroll 1
+    for (int c = 0; c < BLK / 16; c += 2) {
+        tmem_ld_wait();
+        tmem_ld16(t_s + 16 * (c + 1), rb);
+        p16<MASKED>(ra, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c), c, pbuf, prow, scale2,
+                    shift2, sum2, mx);
+        tmem_ld_wait();
+        if (c + 2 < BLK / 16) tmem_ld16(t_s + 16 * (c + 2), ra);
+        p16<MASKED>(rb, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c + 1), c + 1, pbuf, prow,
+                    scale2, shift2, sum2, mx);
+    }
+    rmax_raw = mx;
+    float a, b;
+    f2_unpack(sum2, a, b);
+    return a + b;
+}
+
 // ---------------------------------------------------------------------------
 // softmax + correction + epilogue (warps 0-7)
 // ---------------------------------------------------------------------------
@@ -469,82 +570,49 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
             if (!warp_wait(&B.s_full[m], scnt & 1, B, P.status)) return;
             ++scnt;
             tc_fence_after();
+            const bool masked = kind != kFull;
             const float bias = kind == kPseudo ? pseudo_bias : 0.f;
-
-            // pass 1: row maximum of the masked raw scores
-            float rmax_raw = -INFINITY;
-#pragma unroll 1
-            for (int c = 0; c < BLK / 32; ++c) {
-                const uint32_t vb = col_bits(kind, tok, walk, j, c);
-                uint32_t r[32];
-                tmem_ld32(t_s + 32 * c, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    if ((vb >> e) & 1u) rmax_raw = fmaxf(rmax_raw, __uint_as_float(r[e]));
-            }
-            const float rmax = fmaf(rmax_raw, scale, bias);   // -inf stays -inf
-
+            float rmax_raw, rsum = 0.f;
             if (n == 0) {
-                m_ref = rmax;
-            } else {
-                const float m_new = fmaxf(m_ref, rmax);
-                const bool need = m_new > m_ref + 8.0f;
-                if (__any_sync(0xffffffffu, need)) {
-                    const float alpha = need ? ex2_approx(m_ref - m_new) : 1.0f;
-                    if (need) m_ref = m_new;
-                    l *= alpha;
-#pragma unroll
-                    for (int c = 0; c < HD / 32; ++c) {
-                        uint32_t r[32];
-                        tmem_ld32(t_o + 32 * c, r);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                        tmem_st32(t_o + 32 * c, r);
-                    }
-                    tmem_st_wait();
-                }
+                // first tile of the row: its maximum becomes the reference
+                rmax_raw = masked ? tile_max<BLK, true>(t_s, kind, tok, walk, j)
+                                  : tile_max<BLK, false>(t_s, kind, tok, walk, j);
+                m_ref = fmaf(rmax_raw, scale, bias);
             }
-
-            // pass 2: P = 2^(s * scale + bias - m_ref) as bf16 into the
-            // 128B-swizzled K-major P tile
-            const float shift = bias - m_ref;
-            float rsum = 0.f;
+            // one pass against the running maximum; redone only when the row
+            // maximum grew by more than 2^8 (then O and l are rescaled first)
 #pragma unroll 1
-            for (int c = 0; c < BLK / 32; ++c) {
-                const uint32_t vb = col_bits(kind, tok, walk, j, c);
-                uint32_t r[32];
-                tmem_ld32(t_s + 32 * c, r);
-                tmem_ld_wait();
+            for (int pass = 0; pass < 2; ++pass) {
+                rsum = masked ? tile_p<BLK, true>(t_s, pbuf, prow, kind, tok, walk, j, scale,
+                                                  bias - m_ref, rmax_raw)
+                              : tile_p<BLK, false>(t_s, pbuf, prow, kind, tok, walk, j, scale,
+                                                   bias - m_ref, rmax_raw);
+                const float rmax = fmaf(rmax_raw, scale, bias);
+                const bool need = rmax > m_ref + 8.0f;
+                if (!__any_sync(0xffffffffu, need)) break;
+                const float m_new = fmaxf(m_ref, rmax);
+                const float alpha = ex2_approx(m_ref - m_new);
+                m_ref = m_new;
+                l *= alpha;
+#pragma unroll 1
+                for (int c = 0; c < HD / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(t_o + 32 * c, r);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    float p[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int ce = 8 * q8 + e;
-                        p[e] = ((vb >> ce) & 1u)
-                                   ? ex2_approx(fmaf(__uint_as_float(r[ce]), scale, shift))
-                                   : 0.f;
-                        rsum += p[e];
-                    }
-                    uint4 v;
-                    v.x = pack_bf16x2(p[0], p[1]);
-                    v.y = pack_bf16x2(p[2], p[3]);
-                    v.z = pack_bf16x2(p[4], p[5]);
-                    v.w = pack_bf16x2(p[6], p[7]);
-                    const int cc = 4 * c + q8;                 // 8-column chunk of the row
-                    const int atom = cc / 8, chunk = cc % 8;
-                    uint8_t* dst = pbuf + atom * C::kAtomQ + prow * 128 + ((chunk ^ (prow & 7)) << 4);
-                    *reinterpret_cast<uint4*>(dst) = v;
+                    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                    tmem_st32(t_o + 32 * c, r);
                 }
+                tmem_st_wait();
             }
             l += rsum;
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&B.s_free[m]);
-            mbar_arrive(&B.p_full[m]);
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&B.s_free[m]);
+                mbar_arrive(&B.p_full[m]);
+            }
             ++n;
         }
 
@@ -573,7 +641,8 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
         }
         if (row_valid) P.lse[(int64_t)h * D.T + it.tok0 + pos] = (m_ref + log2f(l)) * 0.6931471805599453f;
         tc_fence_before();
-        mbar_arrive(&B.o_free[m]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.o_free[m]);
     }
 }
 
@@ -596,10 +665,10 @@ k_attn(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap
             mbar_init(&B.q_full[m], 1);
             mbar_init(&B.q_empty[m], 1);
             mbar_init(&B.s_full[m], 1);
-            mbar_init(&B.s_free[m], kTileM);
-            mbar_init(&B.p_full[m], kTileM);
+            mbar_init(&B.s_free[m], kTileM / 32);
+            mbar_init(&B.p_full[m], kTileM / 32);
             mbar_init(&B.o_full[m], 1);
-            mbar_init(&B.o_free[m], kTileM);
+            mbar_init(&B.o_free[m], kTileM / 32);
         }
         for (int s = 0; s < kSlots; ++s) {
             mbar_init(&B.kv_full[s], 1);

@@ -186,3 +186,25 @@ def test_quantize_fp8_matches_oracle_codes():
         ref, ref_s = oracle.quantize_e4m3(x[name], wl.seqlens, wl.B)
         assert np.array_equal(scales.cpu().numpy().astype(np.float64), ref_s)
         assert np.array_equal(got, ref)
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    # Fault injection on the host side of the contract: a flag makes the
+    # producer never load Q, so the MMA warp's first wait can never complete.
+    # Every wait is bounded (~1 s): the kernel must record FP2_STATUS_TIMEOUT,
+    # drain its in-flight copies, free tensor memory and return, leaving the
+    # context usable for the next call.
+    import time
+    wl, x = _case("pr1_ref_1k")
+    run = GpuRun(wl, x).plan()
+    t0 = time.time()
+    run.prefill(flags=fb.FP2_DEBUG_DROP_Q_LOAD)
+    rc, st = run.status()
+    assert rc == fb.FP2_ERR_TIMEOUT and st & fb.FP2_STATUS_TIMEOUT
+    assert time.time() - t0 < 30
+    run.plan().prefill()
+    assert run.status() == (fb.FP2_OK, 0)
+    q, k, v = oracle_inputs(x, wl)
+    pl = oracle.plan(q, k, v, wl.seqlens, wl.B, wl.tau)
+    res = check_attention(wl, x, run, pl)
+    assert res["rel_l2"] <= REL_L2_BF16 and res["lse_max_abs"] <= LSE_ABS, res
