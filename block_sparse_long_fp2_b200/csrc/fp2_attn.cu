@@ -54,18 +54,16 @@ template <int HD, int BLK>
 struct Cfg {
     static constexpr int kQBytes = kTileM * HD * 2;      // one 128-row query tile (bf16)
     static constexpr int kSlotBytes = BLK * HD * 2;      // one K or V tile (bf16)
-    static constexpr int kPBytes = kTileM * BLK * 2;     // one P tile (bf16)
     static constexpr int kOffQ = 0;
     static constexpr int kOffSlot = 2 * kQBytes;
-    static constexpr int kOffP = kOffSlot + kSlots * kSlotBytes;
-    static constexpr int kOffBar = kOffP + 2 * kPBytes;
+    static constexpr int kOffBar = kOffSlot + kSlots * kSlotBytes;
     static constexpr int kSmemBytes = kOffBar + 512 + 1024;   // barriers + alignment slack
     static constexpr int kColS0 = 0;
     static constexpr int kColS1 = BLK;
     static constexpr int kColO0 = 2 * BLK;
     static constexpr int kColO1 = 2 * BLK + HD;
     static constexpr int kTmemCols = pow2_ceil(2 * (BLK + HD));
-    static constexpr int kAtomQ = kTileM * 128;          // bytes between 64-column atoms of Q / P
+    static constexpr int kAtomQ = kTileM * 128;          // bytes between 64-column atoms of Q
     static constexpr int kAtomKV = BLK * 128;            // bytes between 64-column atoms of K / V
 };
 
@@ -310,16 +308,15 @@ __device__ __forceinline__ void issue_s(uint32_t tmem_s, uint32_t q_addr, uint32
 }
 
 template <int HD, int BLK>
-__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t p_addr, uint32_t v_addr,
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_addr,
                                          bool accumulate) {
     using C = Cfg<HD, BLK>;
     constexpr uint32_t idesc = idesc_bf16(kTileM, HD, true);
 #pragma unroll
     for (int kk = 0; kk < BLK / 16; ++kk) {
-        const uint32_t a = p_addr + (kk / 4) * C::kAtomQ + (kk % 4) * 32;
         const uint32_t b = v_addr + kk * 16 * 128;
-        umma_f16(tmem_o, smem_desc_sw128(a, 16, 1024), smem_desc_sw128(b, C::kAtomKV, 1024), idesc,
-                 (accumulate || kk > 0) ? 1u : 0u);
+        umma_f16_ts(tmem_o, tmem_p + kk * 8, smem_desc_sw128(b, C::kAtomKV, 1024), idesc,
+                    (accumulate || kk > 0) ? 1u : 0u);
     }
 }
 
@@ -334,7 +331,6 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
     const uint32_t tb = B.tmem_base;
     const uint32_t s_base = smem_u32(smem);
     const uint32_t q_addr[2] = {s_base + C::kOffQ, s_base + C::kOffQ + C::kQBytes};
-    const uint32_t p_addr[2] = {s_base + C::kOffP, s_base + C::kOffP + C::kPBytes};
     const uint32_t t_s[2] = {tb + C::kColS0, tb + C::kColS1};
     const uint32_t t_o[2] = {tb + C::kColO0, tb + C::kColO1};
     uint32_t qcnt[2] = {0, 0}, scnt[2] = {0, 0}, pcnt[2] = {0, 0}, ocnt[2] = {0, 0};
@@ -346,7 +342,7 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
         ++pcnt[1];
         if (pt.first && !mbar_wait(&B.o_free[1], (ocnt[1] & 1) ^ 1, &B.abort, P.status)) return false;
         tc_fence_after();
-        issue_pv<HD, BLK>(t_o[1], p_addr[1], s_base + C::kOffSlot + pt.vslot * C::kSlotBytes,
+        issue_pv<HD, BLK>(t_o[1], t_s[1], s_base + C::kOffSlot + pt.vslot * C::kSlotBytes,
                           !pt.first);
         umma_commit(&B.kv_empty[pt.vslot]);
         if (pt.last) {
@@ -414,7 +410,7 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
             ++pcnt[0];
             if (first && !mbar_wait(&B.o_free[0], (ocnt[0] & 1) ^ 1, &B.abort, P.status)) goto drain;
             tc_fence_after();
-            issue_pv<HD, BLK>(t_o[0], p_addr[0], v_addr, !first);
+            issue_pv<HD, BLK>(t_o[0], t_s[0], v_addr, !first);
             if (!it.has_m1) umma_commit(&B.kv_empty[vs]);
             if (last) {
                 umma_commit(&B.o_full[0]);
@@ -434,99 +430,97 @@ drain:
 // Row maximum of the raw (unscaled) scores of the masked-in columns of this
 // thread's row of S.  Two 32-column TMEM loads in flight.
 template <int BLK, bool MASKED>
-__device__ __forceinline__ void max16(const uint32_t (&r)[16], uint32_t vb, float& mx) {
+__device__ __forceinline__ uint32_t chunk_bits(int kind, int tok, const TileWalk<BLK>& walk, int j,
+                                               int c32) {
+    return MASKED ? col_bits(kind, tok, walk, j, c32) : 0xFFFFFFFFu;
+}
+
+template <bool MASKED>
+__device__ __forceinline__ void max32(const uint32_t (&r)[32], uint32_t vb, float& mx) {
     if (MASKED) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
+        for (int e = 0; e < 32; ++e)
             if ((vb >> e) & 1u) mx = fmaxf(mx, __uint_as_float(r[e]));
     } else {
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) mx = fmax3(mx, __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+        for (int e = 0; e < 32; e += 2) mx = fmax3(mx, __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
     }
 }
 
-template <int BLK, bool MASKED>
-__device__ __forceinline__ uint32_t chunk_bits(int kind, int tok, const TileWalk<BLK>& walk, int j,
-                                               int c16) {
-    return MASKED ? (col_bits(kind, tok, walk, j, c16 / 2) >> (16 * (c16 & 1))) : 0xFFFFu;
-}
-
 // Row maximum of the raw (unscaled) scores of the masked-in columns of this
-// thread's row of S; one 16-column TMEM load always in flight.
+// thread's row of S.  32-column TMEM loads, two in flight.
 template <int BLK, bool MASKED>
 __device__ __forceinline__ float tile_max(uint32_t t_s, int kind, int tok, const TileWalk<BLK>& walk,
                                           int j) {
+    constexpr int NC = BLK / 32;
     float mx = -INFINITY;
-    uint32_t ra[16], rb[16];
-    tmem_ld16(t_s, ra);
+    uint32_t ra[32], rb[32];
+    tmem_ld32(t_s, ra);
+    tmem_ld32(t_s + 32, rb);
 #pragma unroll 1
-    for (int c = 0; c < BLK / 16; c += 2) {
+    for (int c = 0; c < NC; c += 2) {
         tmem_ld_wait();
-        tmem_ld16(t_s + 16 * (c + 1), rb);
-        max16<BLK, MASKED>(ra, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c), mx);
-        tmem_ld_wait();
-        if (c + 2 < BLK / 16) tmem_ld16(t_s + 16 * (c + 2), ra);
-        max16<BLK, MASKED>(rb, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c + 1), mx);
+        max32<MASKED>(ra, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c), mx);
+        if (c + 2 < NC) tmem_ld32(t_s + 32 * (c + 2), ra);
+        max32<MASKED>(rb, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c + 1), mx);
+        if (c + 3 < NC) tmem_ld32(t_s + 32 * (c + 3), rb);
     }
     return mx;
 }
 
-// 16 columns (two 8-column chunks) of P: 2^(s * scale + shift), bf16, into
-// the 128B-swizzled K-major P tile.
+// 32 columns of P = 2^(s * scale + shift) as 16 packed bf16 pairs, written
+// into tensor memory over the first half of the 32 S columns just read
+// (P of keys 2c and 2c+1 in column c): the A operand of the P.V MMA.
 template <bool MASKED>
-__device__ __forceinline__ void p16(const uint32_t (&r)[16], uint32_t vb, int c16, uint8_t* pbuf,
-                                    int prow, uint64_t scale2, uint64_t shift2, uint64_t& sum2,
-                                    float& mx) {
+__device__ __forceinline__ void p32(const uint32_t (&r)[32], uint32_t vb, uint32_t t_p,
+                                    uint64_t scale2, uint64_t shift2, uint64_t& sum2) {
 #pragma unroll
-    for (int q8 = 0; q8 < 2; ++q8) {
-        uint32_t packed[4];
+    for (int h = 0; h < 2; ++h) {
+        uint32_t packed[8];
 #pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-            const int e = 8 * q8 + 2 * e2;
+        for (int e2 = 0; e2 < 8; ++e2) {
+            const int e = 16 * h + 2 * e2;
             float s0 = __uint_as_float(r[e]), s1 = __uint_as_float(r[e + 1]);
             if (MASKED) {
                 s0 = ((vb >> e) & 1u) ? s0 : -INFINITY;
                 s1 = ((vb >> (e + 1)) & 1u) ? s1 : -INFINITY;
             }
-            mx = fmax3(mx, s0, s1);
             float x0, x1;
             f2_unpack(f2_fma(f2_pack(s0, s1), scale2, shift2), x0, x1);
             const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
             sum2 = f2_add(sum2, f2_pack(p0, p1));
             packed[e2] = pack_bf16x2(p0, p1);
         }
-        const int cc = 2 * c16 + q8;                 // 8-column chunk of the row
-        const int atom = cc >> 3, chunk = cc & 7;
-        uint8_t* dst = pbuf + atom * (kTileM * 128) + prow * 128 + ((chunk ^ (prow & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        tmem_st8(t_p + 8 * h, packed);
     }
 }
 
 // P = 2^(s * scale + shift) for this thread's row of S (zero where masked
-// out), written as bf16 into the P tile; returns the fp32 row sum and the
-// row maximum of the raw masked-in scores.
+// out), written as bf16 pairs in place over S in tensor memory (column c of
+// the P operand holds keys 2c, 2c+1 and lies inside S columns already read:
+// the P of chunk c goes to columns [16c, 16c+16) while the only loads in
+// flight cover [32(c+1), 32(c+2))).  Returns the fp32 row sum.
 template <int BLK, bool MASKED>
-__device__ __forceinline__ float tile_p(uint32_t t_s, uint8_t* pbuf, int prow, int kind, int tok,
-                                        const TileWalk<BLK>& walk, int j, float scale, float shift,
-                                        float& rmax_raw) {
+__device__ __forceinline__ float tile_p(uint32_t t_s, int kind, int tok, const TileWalk<BLK>& walk,
+                                        int j, float scale, float shift) {
+    constexpr int NC = BLK / 32;
     const uint64_t scale2 = f2_pack(scale, scale);
     const uint64_t shift2 = f2_pack(shift, shift);
     uint64_t sum2 = f2_pack(0.f, 0.f);
-    float mx = -INFINITY;
-    uint32_t ra[16], rb[16];
-    tmem_ld16(t_s, ra);
+    uint32_t ra[32], rb[32];
+    tmem_ld32(t_s, ra);
+    tmem_ld32(t_s + 32, rb);
 #pragma unroll 1
-    for (int c = 0; c < BLK / 16; c += 2) {
+    for (int c = 0; c < NC; c += 2) {
         tmem_ld_wait();
-        tmem_ld16(t_s + 16 * (c + 1), rb);
-        p16<MASKED>(ra, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c), c, pbuf, prow, scale2,
-                    shift2, sum2, mx);
-        tmem_ld_wait();
-        if (c + 2 < BLK / 16) tmem_ld16(t_s + 16 * (c + 2), ra);
-        p16<MASKED>(rb, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c + 1), c + 1, pbuf, prow,
-                    scale2, shift2, sum2, mx);
+        p32<MASKED>(ra, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c), t_s + 16 * c, scale2, shift2,
+                    sum2);
+        if (c + 2 < NC) tmem_ld32(t_s + 32 * (c + 2), ra);
+        p32<MASKED>(rb, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c + 1), t_s + 16 * (c + 1), scale2,
+                    shift2, sum2);
+        if (c + 3 < NC) tmem_ld32(t_s + 32 * (c + 3), rb);
     }
-    rmax_raw = mx;
+    tmem_st_wait();
     float a, b;
     f2_unpack(sum2, a, b);
     return a + b;
@@ -546,7 +540,6 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
     const uint32_t lane_off = static_cast<uint32_t>(32 * q4) << 16;
     const uint32_t t_s = B.tmem_base + lane_off + (m == 0 ? C::kColS0 : C::kColS1);
     const uint32_t t_o = B.tmem_base + lane_off + (m == 0 ? C::kColO0 : C::kColO1);
-    uint8_t* pbuf = smem + C::kOffP + m * C::kPBytes;
     const float scale = 1.4426950408889634f / sqrtf((float)HD);   // log2(e) / sqrt(d)
     const float pseudo_bias = log2f((float)BLK);                   // ln n_j in log2 units
     uint32_t scnt = 0, ocnt = 0;
@@ -572,41 +565,38 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
             tc_fence_after();
             const bool masked = kind != kFull;
             const float bias = kind == kPseudo ? pseudo_bias : 0.f;
-            float rmax_raw, rsum = 0.f;
+            // pass 1: row maximum of the masked scores
+            const float rmax_raw = masked ? tile_max<BLK, true>(t_s, kind, tok, walk, j)
+                                          : tile_max<BLK, false>(t_s, kind, tok, walk, j);
+            const float rmax = fmaf(rmax_raw, scale, bias);   // -inf stays -inf
             if (n == 0) {
-                // first tile of the row: its maximum becomes the reference
-                rmax_raw = masked ? tile_max<BLK, true>(t_s, kind, tok, walk, j)
-                                  : tile_max<BLK, false>(t_s, kind, tok, walk, j);
-                m_ref = fmaf(rmax_raw, scale, bias);
-            }
-            // one pass against the running maximum; redone only when the row
-            // maximum grew by more than 2^8 (then O and l are rescaled first)
-#pragma unroll 1
-            for (int pass = 0; pass < 2; ++pass) {
-                rsum = masked ? tile_p<BLK, true>(t_s, pbuf, prow, kind, tok, walk, j, scale,
-                                                  bias - m_ref, rmax_raw)
-                              : tile_p<BLK, false>(t_s, pbuf, prow, kind, tok, walk, j, scale,
-                                                   bias - m_ref, rmax_raw);
-                const float rmax = fmaf(rmax_raw, scale, bias);
+                m_ref = rmax;
+            } else {
+                // lazy rescale: O and l move to a new reference only when the
+                // row maximum grew by more than 2^8
                 const bool need = rmax > m_ref + 8.0f;
-                if (!__any_sync(0xffffffffu, need)) break;
-                const float m_new = fmaxf(m_ref, rmax);
-                const float alpha = ex2_approx(m_ref - m_new);
-                m_ref = m_new;
-                l *= alpha;
+                if (__any_sync(0xffffffffu, need)) {
+                    const float m_new = fmaxf(m_ref, rmax);
+                    const float alpha = ex2_approx(m_ref - m_new);
+                    m_ref = m_new;
+                    l *= alpha;
 #pragma unroll 1
-                for (int c = 0; c < HD / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(t_o + 32 * c, r);
-                    tmem_ld_wait();
+                    for (int c = 0; c < HD / 32; ++c) {
+                        uint32_t r[32];
+                        tmem_ld32(t_o + 32 * c, r);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                    tmem_st32(t_o + 32 * c, r);
+                        for (int e = 0; e < 32; ++e)
+                            r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                        tmem_st32(t_o + 32 * c, r);
+                    }
+                    tmem_st_wait();
                 }
-                tmem_st_wait();
             }
+            // pass 2: P in place over S
+            const float rsum = masked ? tile_p<BLK, true>(t_s, kind, tok, walk, j, scale, bias - m_ref)
+                                      : tile_p<BLK, false>(t_s, kind, tok, walk, j, scale, bias - m_ref);
             l += rsum;
-            fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {

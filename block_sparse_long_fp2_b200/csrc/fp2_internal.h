@@ -9,7 +9,7 @@
 
 #include <cuda_runtime.h>
 
-#include "../../include/fp2.h"
+#include "fp2.h"
 
 namespace fp2 {
 
