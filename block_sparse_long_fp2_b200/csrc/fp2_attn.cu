@@ -13,13 +13,16 @@
 //   warps 4-7   softmax warpgroup of query tile 1
 //   warp 8      TMA producer: Q tiles, then per kept block its K and V tiles
 //               (through the page table when paged), then per pseudo tile
-//               up to B bf16 block means Kbar/Vbar; a ring of 3 K-or-V slots.
-//   warp 9      allocates tensor memory and issues tcgen05 MMAs:
-//               S_m = Q_m K^T into TMEM, O_m += P_m V into TMEM.
-// Issue order for K/V tile n:  S0(n), PV1(n-1), S1(n), PV0(n).  Every commit
-// that publishes S_m(n) therefore also covers PV_m(n-1), so the softmax
-// warps may rescale O_m and overwrite their P buffer as soon as S_m(n) is
-// visible.
+//               up to B bf16 block means Kbar/Vbar; a ring of K-or-V slots
+//               (as many as shared memory holds, 5 at d = B = 128).
+//   warp 9      allocates tensor memory and issues every tcgen05 MMA:
+//               S_m = Q_m K^T into TMEM, O_m += P_m V with P_m read from TMEM
+//               (P overwrites its own S columns).  Issue order for K/V tile n:
+//               S0(n), P1(n-1).V, S1(n), P0(n).V.  Every commit that publishes
+//               S_m(n) therefore also covers P_m(n-1).V, so the softmax warps
+//               may rescale O_m and overwrite the P_m columns as soon as S_m(n)
+//               is visible; and S_m(n+1) is issued only after the issuer saw
+//               P_m(n) published, i.e. after the softmax finished reading S_m(n).
 //
 // Mean correction (Figure 4): each skipped, fully visible block j adds one
 // pseudo-key with key Kbar_j, value Vbar_j and logit bias ln n_j = ln B.
@@ -41,8 +44,16 @@ namespace {
 
 constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kSlots = 3;
+constexpr int kMmaWarp = 9;     // issues every MMA; owns the tensor memory
+// Ring slots for K / V tiles: as many as fit beside the two query tiles in
+// the 227 KiB of shared memory a CTA may use (at most 8).
+constexpr int kMaxSmem = 232448;
+constexpr int kMaxSlots = 8;
+template <int HD, int BLK>
+constexpr int ring_slots() {
+    const int avail = (kMaxSmem - 512 - 1024 - 2 * kTileM * HD * 2) / (BLK * HD * 2);
+    return avail < kMaxSlots ? avail : kMaxSlots;
+}
 
 constexpr int pow2_ceil(int x) {
     int p = 32;
@@ -52,12 +63,15 @@ constexpr int pow2_ceil(int x) {
 
 template <int HD, int BLK>
 struct Cfg {
+    static constexpr int kSlots = ring_slots<HD, BLK>();
     static constexpr int kQBytes = kTileM * HD * 2;      // one 128-row query tile (bf16)
     static constexpr int kSlotBytes = BLK * HD * 2;      // one K or V tile (bf16)
     static constexpr int kOffQ = 0;
     static constexpr int kOffSlot = 2 * kQBytes;
     static constexpr int kOffBar = kOffSlot + kSlots * kSlotBytes;
+    static_assert(kSlots >= 3, "the K/V ring needs at least three slots");
     static constexpr int kSmemBytes = kOffBar + 512 + 1024;   // barriers + alignment slack
+    static_assert(kSmemBytes <= kMaxSmem, "shared memory budget");
     static constexpr int kColS0 = 0;
     static constexpr int kColS1 = BLK;
     static constexpr int kColO0 = 2 * BLK;
@@ -69,8 +83,8 @@ struct Cfg {
 
 struct Bars {
     uint64_t q_full[2], q_empty[2];
-    uint64_t kv_full[kSlots], kv_empty[kSlots];
-    uint64_t s_full[2], s_free[2];
+    uint64_t kv_full[kMaxSlots], kv_empty[kMaxSlots];
+    uint64_t s_full[2];
     uint64_t p_full[2];
     uint64_t o_full[2], o_free[2];
     uint64_t drain;
@@ -129,13 +143,17 @@ enum TileKind { kFull = 0, kDiag = 1, kPseudo = 2 };
 
 // Walks the tiles of an item: the kept blocks in CSR order, then the pseudo
 // tiles that contain at least one skipped block.  Every role runs the same
-// walk, so they agree on the sequence without exchanging it.
+// walk, so they agree on the sequence without exchanging it.  The next
+// column id is loaded one step ahead and the non-empty pseudo tiles are
+// found once per item, so advancing never waits on a global load.
 template <int BLK>
 struct TileWalk {
     static constexpr int W = BLK / 32;
     const int32_t* cols;
     const uint32_t* mask;
     int n_kept, t, i, pt, n_pt, mask_words;
+    int j_next;          // col_idx[t] (valid when t < n_kept)
+    uint32_t pt_bits;    // bit p set: pseudo tile p (p < 32) holds a skipped block
 
     __device__ __forceinline__ void init(const AttnParams& P, const Item& it) {
         cols = P.col_idx + it.kbeg;
@@ -146,6 +164,10 @@ struct TileWalk {
         mask_words = P.D.mask_words;
         pt = 0;
         n_pt = (P.flags & FP2_NO_CORRECTION) ? 0 : (it.i + BLK - 1) / BLK;
+        j_next = n_kept > 0 ? __ldg(cols) : 0;
+        pt_bits = 0;
+        const int n_small = n_pt < 32 ? n_pt : 32;
+        for (int p = 0; p < n_small; ++p) pt_bits |= has_skip(p) ? (1u << p) : 0u;
     }
     // skip bits of blocks BLK*pt + 32*w .. +31 (skipped = visible, j < i, not kept)
     __device__ __forceinline__ uint32_t skip_word(int p, int w) const {
@@ -153,7 +175,7 @@ struct TileWalk {
         if (j0 >= i) return 0u;
         const uint32_t valid = (j0 + 32 <= i) ? 0xFFFFFFFFu : ((1u << (i - j0)) - 1u);
         const int widx = j0 / 32;
-        const uint32_t kept = widx < mask_words ? mask[widx] : 0xFFFFFFFFu;
+        const uint32_t kept = widx < mask_words ? __ldg(mask + widx) : 0xFFFFFFFFu;
         return ~kept & valid;
     }
     __device__ __forceinline__ bool has_skip(int p) const {
@@ -162,23 +184,28 @@ struct TileWalk {
         for (int w = 0; w < W; ++w) any |= skip_word(p, w);
         return any != 0;
     }
+    __device__ __forceinline__ bool pt_nonempty(int p) const {
+        return p < 32 ? ((pt_bits >> p) & 1u) != 0 : has_skip(p);
+    }
     // Advances to the next tile; returns false at the end.
     __device__ __forceinline__ bool next(int& kind, int& j) {
         if (t < n_kept) {
-            j = cols[t++];
+            j = j_next;
+            ++t;
+            if (t < n_kept) j_next = __ldg(cols + t);
             kind = (j == i) ? kDiag : kFull;
             return true;
         }
-        while (pt < n_pt && !has_skip(pt)) ++pt;
+        while (pt < n_pt && !pt_nonempty(pt)) ++pt;
         if (pt >= n_pt) return false;
         j = pt++;
         kind = kPseudo;
         return true;
     }
-    __device__ __forceinline__ bool is_last() {
+    __device__ __forceinline__ bool is_last() const {
         if (t < n_kept) return false;
         int p = pt;
-        while (p < n_pt && !has_skip(p)) ++p;
+        while (p < n_pt && !pt_nonempty(p)) ++p;
         return p >= n_pt;
     }
 };
@@ -215,7 +242,8 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
     const Dims& D = P.D;
     uint32_t qcnt[2] = {0, 0}, qloaded[2] = {0, 0};
     uint32_t ld = 0;                 // K/V loads issued (slot = ld % 3)
-    uint32_t issued[kSlots] = {0, 0, 0};
+    constexpr int kSlots = C::kSlots;
+    uint32_t issued[kMaxSlots] = {0, 0, 0, 0, 0, 0, 0, 0};
     const bool paged = D.page_size != 0;
     for (int64_t w = blockIdx.x; w < P.n_items; w += gridDim.x) {
         const Item it = decode_item(P, w);
@@ -294,30 +322,33 @@ drain:
 // MMA issuer (warp 9, one lane)
 // ---------------------------------------------------------------------------
 
+// The shared-memory descriptors of one operand tile differ between K-steps
+// only in the start-address field (bits 0-13, address / 16); the tiles never
+// cross 256 KiB, so the field never carries and a K-step is one add of a
+// compile-time constant to a descriptor built once per kernel.
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) {
+    return d + static_cast<uint64_t>(bytes >> 4);
+}
+
 template <int HD, int BLK>
-__device__ __forceinline__ void issue_s(uint32_t tmem_s, uint32_t q_addr, uint32_t k_addr) {
+__device__ __forceinline__ void issue_s(uint32_t tmem_s, uint64_t q_desc, uint64_t k_desc) {
     using C = Cfg<HD, BLK>;
     constexpr uint32_t idesc = idesc_bf16(kTileM, BLK, false);
 #pragma unroll
     for (int kk = 0; kk < HD / 16; ++kk) {
-        const uint32_t a = q_addr + (kk / 4) * C::kAtomQ + (kk % 4) * 32;
-        const uint32_t b = k_addr + (kk / 4) * C::kAtomKV + (kk % 4) * 32;
-        umma_f16(tmem_s, smem_desc_sw128(a, 16, 1024), smem_desc_sw128(b, 16, 1024), idesc,
-                 kk > 0 ? 1u : 0u);
+        umma_f16(tmem_s, desc_add(q_desc, (kk / 4) * C::kAtomQ + (kk % 4) * 32),
+                 desc_add(k_desc, (kk / 4) * C::kAtomKV + (kk % 4) * 32), idesc, kk > 0 ? 1u : 0u);
     }
 }
 
 template <int HD, int BLK>
-__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_addr,
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint64_t v_desc,
                                          bool accumulate) {
-    using C = Cfg<HD, BLK>;
     constexpr uint32_t idesc = idesc_bf16(kTileM, HD, true);
 #pragma unroll
-    for (int kk = 0; kk < BLK / 16; ++kk) {
-        const uint32_t b = v_addr + kk * 16 * 128;
-        umma_f16_ts(tmem_o, tmem_p + kk * 8, smem_desc_sw128(b, C::kAtomKV, 1024), idesc,
+    for (int kk = 0; kk < BLK / 16; ++kk)
+        umma_f16_ts(tmem_o, tmem_p + kk * 8, desc_add(v_desc, kk * 16 * 128), idesc,
                     (accumulate || kk > 0) ? 1u : 0u);
-    }
 }
 
 struct PrevTile {
@@ -325,15 +356,24 @@ struct PrevTile {
     int vslot;
 };
 
+// The MMA issuer (one lane of warp kMmaWarp).  A tcgen05.mma costs its
+// issuing thread ~50 cycles, about its 64-cycle execution time, so a single
+// thread issues every MMA in the order S0(n), P1(n-1).V, S1(n), P0(n).V
+// that keeps the two query tiles' chains interleaved.
 template <int HD, int BLK>
 __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
     using C = Cfg<HD, BLK>;
+    constexpr int kSlots = C::kSlots;
     const uint32_t tb = B.tmem_base;
     const uint32_t s_base = smem_u32(smem);
-    const uint32_t q_addr[2] = {s_base + C::kOffQ, s_base + C::kOffQ + C::kQBytes};
+    const uint64_t q_desc[2] = {smem_desc_sw128(s_base + C::kOffQ, 16, 1024),
+                                smem_desc_sw128(s_base + C::kOffQ + C::kQBytes, 16, 1024)};
+    // descriptors of ring slot 0 as a K (K-major) and as a V (MN-major) operand
+    const uint64_t k_desc0 = smem_desc_sw128(s_base + C::kOffSlot, 16, 1024);
+    const uint64_t v_desc0 = smem_desc_sw128(s_base + C::kOffSlot, C::kAtomKV, 1024);
     const uint32_t t_s[2] = {tb + C::kColS0, tb + C::kColS1};
     const uint32_t t_o[2] = {tb + C::kColO0, tb + C::kColO1};
-    uint32_t qcnt[2] = {0, 0}, scnt[2] = {0, 0}, pcnt[2] = {0, 0}, ocnt[2] = {0, 0};
+    uint32_t qcnt[2] = {0, 0}, pcnt[2] = {0, 0}, ocnt[2] = {0, 0};
     uint32_t ld = 0;
     PrevTile prev{false, false, false, false, 0};
 
@@ -342,8 +382,7 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
         ++pcnt[1];
         if (pt.first && !mbar_wait(&B.o_free[1], (ocnt[1] & 1) ^ 1, &B.abort, P.status)) return false;
         tc_fence_after();
-        issue_pv<HD, BLK>(t_o[1], t_s[1], s_base + C::kOffSlot + pt.vslot * C::kSlotBytes,
-                          !pt.first);
+        issue_pv<HD, BLK>(t_o[1], t_s[1], desc_add(v_desc0, pt.vslot * C::kSlotBytes), !pt.first);
         umma_commit(&B.kv_empty[pt.vslot]);
         if (pt.last) {
             umma_commit(&B.o_full[1]);
@@ -366,24 +405,22 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
             const int vs = ld % kSlots;
             const uint32_t vuse = ld / kSlots;
             ++ld;
-            const uint32_t k_addr = s_base + C::kOffSlot + ks * C::kSlotBytes;
-            const uint32_t v_addr = s_base + C::kOffSlot + vs * C::kSlotBytes;
+            const uint64_t kd = desc_add(k_desc0, ks * C::kSlotBytes);
+            const uint64_t vd = desc_add(v_desc0, vs * C::kSlotBytes);
             // S0 = Q0 K^T
             if (first) {
                 if (!mbar_wait(&B.q_full[0], qcnt[0] & 1, &B.abort, P.status)) goto drain;
                 ++qcnt[0];
             }
             if (!mbar_wait(&B.kv_full[ks], kuse & 1, &B.abort, P.status)) goto drain;
-            if (!mbar_wait(&B.s_free[0], (scnt[0] & 1) ^ 1, &B.abort, P.status)) goto drain;
             tc_fence_after();
-            issue_s<HD, BLK>(t_s[0], q_addr[0], k_addr);
+            issue_s<HD, BLK>(t_s[0], q_desc[0], kd);
             umma_commit(&B.s_full[0]);
-            ++scnt[0];
             if (!it.has_m1) {
                 umma_commit(&B.kv_empty[ks]);
                 if (last) umma_commit(&B.q_empty[0]);
             }
-            // PV1 of the previous tile
+            // P1.V of the previous tile
             if (prev.valid && prev.has_m1) {
                 if (!pv1(prev)) goto drain;
             }
@@ -393,24 +430,22 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
                     if (!mbar_wait(&B.q_full[1], qcnt[1] & 1, &B.abort, P.status)) goto drain;
                     ++qcnt[1];
                 }
-                if (!mbar_wait(&B.s_free[1], (scnt[1] & 1) ^ 1, &B.abort, P.status)) goto drain;
                 tc_fence_after();
-                issue_s<HD, BLK>(t_s[1], q_addr[1], k_addr);
+                issue_s<HD, BLK>(t_s[1], q_desc[1], kd);
                 umma_commit(&B.s_full[1]);
-                ++scnt[1];
                 umma_commit(&B.kv_empty[ks]);
                 if (last) {
                     umma_commit(&B.q_empty[0]);
                     umma_commit(&B.q_empty[1]);
                 }
             }
-            // PV0 of this tile
+            // P0.V of this tile
             if (!mbar_wait(&B.kv_full[vs], vuse & 1, &B.abort, P.status)) goto drain;
             if (!mbar_wait(&B.p_full[0], pcnt[0] & 1, &B.abort, P.status)) goto drain;
             ++pcnt[0];
             if (first && !mbar_wait(&B.o_free[0], (ocnt[0] & 1) ^ 1, &B.abort, P.status)) goto drain;
             tc_fence_after();
-            issue_pv<HD, BLK>(t_o[0], t_s[0], v_addr, !first);
+            issue_pv<HD, BLK>(t_o[0], t_s[0], vd, !first);
             if (!it.has_m1) umma_commit(&B.kv_empty[vs]);
             if (last) {
                 umma_commit(&B.o_full[0]);
@@ -427,46 +462,16 @@ drain:
     mbar_wait_drain(&B.drain, 0, P.status);
 }
 
-// Row maximum of the raw (unscaled) scores of the masked-in columns of this
-// thread's row of S.  Two 32-column TMEM loads in flight.
 template <int BLK, bool MASKED>
 __device__ __forceinline__ uint32_t chunk_bits(int kind, int tok, const TileWalk<BLK>& walk, int j,
                                                int c32) {
     return MASKED ? col_bits(kind, tok, walk, j, c32) : 0xFFFFFFFFu;
 }
 
-template <bool MASKED>
-__device__ __forceinline__ void max32(const uint32_t (&r)[32], uint32_t vb, float& mx) {
-    if (MASKED) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-            if ((vb >> e) & 1u) mx = fmaxf(mx, __uint_as_float(r[e]));
-    } else {
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) mx = fmax3(mx, __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
-    }
-}
-
-// Row maximum of the raw (unscaled) scores of the masked-in columns of this
-// thread's row of S.  32-column TMEM loads, two in flight.
-template <int BLK, bool MASKED>
-__device__ __forceinline__ float tile_max(uint32_t t_s, int kind, int tok, const TileWalk<BLK>& walk,
-                                          int j) {
-    constexpr int NC = BLK / 32;
-    float mx = -INFINITY;
-    uint32_t ra[32], rb[32];
-    tmem_ld32(t_s, ra);
-    tmem_ld32(t_s + 32, rb);
-#pragma unroll 1
-    for (int c = 0; c < NC; c += 2) {
-        tmem_ld_wait();
-        max32<MASKED>(ra, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c), mx);
-        if (c + 2 < NC) tmem_ld32(t_s + 32 * (c + 2), ra);
-        max32<MASKED>(rb, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c + 1), mx);
-        if (c + 3 < NC) tmem_ld32(t_s + 32 * (c + 3), rb);
-    }
-    return mx;
-}
+// exp2 headroom of the running row maximum: P = 2^(x - m_ref) may reach
+// 2^kHeadroom before the reference is moved (bf16 P, fp32 row sums and fp32
+// O accumulators stay far from overflow).
+constexpr float kHeadroom = 64.0f;
 
 // 32 columns of P = 2^(s * scale + shift) as 16 packed bf16 pairs, written
 // into tensor memory over the first half of the 32 S columns just read
@@ -495,17 +500,80 @@ __device__ __forceinline__ void p32(const uint32_t (&r)[32], uint32_t vb, uint32
     }
 }
 
-// P = 2^(s * scale + shift) for this thread's row of S (zero where masked
-// out), written as bf16 pairs in place over S in tensor memory (column c of
-// the P operand holds keys 2c, 2c+1 and lies inside S columns already read:
-// the P of chunk c goes to columns [16c, 16c+16) while the only loads in
-// flight cover [32(c+1), 32(c+2))).  Returns the fp32 row sum.
-template <int BLK, bool MASKED>
-__device__ __forceinline__ float tile_p(uint32_t t_s, int kind, int tok, const TileWalk<BLK>& walk,
-                                        int j, float scale, float shift) {
+template <bool MASKED>
+__device__ __forceinline__ float max32(const uint32_t (&r)[32], uint32_t vb) {
+    float mx = -INFINITY;
+    if (MASKED) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+            if ((vb >> e) & 1u) mx = fmaxf(mx, __uint_as_float(r[e]));
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) mx = fmax3(mx, __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+    }
+    return mx;
+}
+
+// Softmax state of one query row (one thread): the running reference
+// maximum (log2 units), the fp32 row sum, the row's O accumulator columns.
+struct RowState {
+    float m_ref, l;
+    uint32_t t_o;
+    bool o_valid;   // O holds data (false before the first P.V of the row)
+};
+
+// Moves the reference maximum of this thread's row to m_new (>= m_ref):
+// O, l, the partial sum of the current tile and the P columns already
+// written for it (cols [t_p0, t_p0 + n_pcols)) are scaled by 2^(m_ref - m_new).
+// Warp-collective (tensor memory accesses); lanes whose reference does not
+// move use the factor 1.
+template <int HD>
+__device__ __forceinline__ void move_reference(RowState& st, float m_new, uint64_t& sum2, uint32_t t_p0,
+                                            int n_pcols) {
+    const float alpha = m_new > st.m_ref ? ex2_approx(st.m_ref - m_new) : 1.0f;
+    if (m_new > st.m_ref) st.m_ref = m_new;
+    st.l *= alpha;
+    sum2 = f2_fma(sum2, f2_pack(alpha, alpha), f2_pack(0.f, 0.f));
+    if (st.o_valid) {
+#pragma unroll 1
+        for (int c = 0; c < HD / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(st.t_o + 32 * c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st32(st.t_o + 32 * c, r);
+        }
+    }
+#pragma unroll 1
+    for (int c = 0; c < n_pcols; c += 16) {
+        uint32_t r[16];
+        tmem_ld16(t_p0 + c, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float lo = __uint_as_float(r[e] << 16) * alpha;
+            const float hi = __uint_as_float(r[e] & 0xFFFF0000u) * alpha;
+            r[e] = pack_bf16x2(lo, hi);
+        }
+        tmem_st16(t_p0 + c, r);
+    }
+    tmem_st_wait();
+}
+
+// One pass over this thread's row of S: P = 2^(s * scale + bias - m_ref)
+// (zero where masked out) as bf16 pairs in place over S in tensor memory
+// (the P of chunk c goes to columns [16c, 16c+16) while the only loads in
+// flight cover [32(c+1), 32(c+2))).  Before a chunk is written its maximum
+// is checked against the reference; if it exceeds it by more than the
+// headroom the reference moves first.  Returns the fp32 row sum of the tile.
+template <int BLK, int HD, bool MASKED>
+__device__ __forceinline__ float tile_softmax(uint32_t t_s, int kind, int tok,
+                                              const TileWalk<BLK>& walk, int j, float scale,
+                                              float bias, RowState& st) {
     constexpr int NC = BLK / 32;
     const uint64_t scale2 = f2_pack(scale, scale);
-    const uint64_t shift2 = f2_pack(shift, shift);
+    uint64_t shift2 = f2_pack(bias - st.m_ref, bias - st.m_ref);
     uint64_t sum2 = f2_pack(0.f, 0.f);
     uint32_t ra[32], rb[32];
     tmem_ld32(t_s, ra);
@@ -513,12 +581,20 @@ __device__ __forceinline__ float tile_p(uint32_t t_s, int kind, int tok, const T
 #pragma unroll 1
     for (int c = 0; c < NC; c += 2) {
         tmem_ld_wait();
-        p32<MASKED>(ra, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c), t_s + 16 * c, scale2, shift2,
-                    sum2);
-        if (c + 2 < NC) tmem_ld32(t_s + 32 * (c + 2), ra);
-        p32<MASKED>(rb, chunk_bits<BLK, MASKED>(kind, tok, walk, j, c + 1), t_s + 16 * (c + 1), scale2,
-                    shift2, sum2);
-        if (c + 3 < NC) tmem_ld32(t_s + 32 * (c + 3), rb);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            uint32_t(&r)[32] = half ? rb : ra;
+            const int cc = c + half;
+            const uint32_t vb = chunk_bits<BLK, MASKED>(kind, tok, walk, j, cc);
+            const float cm = fmaf(max32<MASKED>(r, vb), scale, bias);
+            const bool need = cm > st.m_ref + kHeadroom;
+            if (__any_sync(0xffffffffu, need)) {
+                move_reference<HD>(st, need ? cm : st.m_ref, sum2, t_s, 16 * cc);
+                shift2 = f2_pack(bias - st.m_ref, bias - st.m_ref);
+            }
+            p32<MASKED>(r, vb, t_s + 16 * cc, scale2, shift2, sum2);
+            if (cc + 2 < NC) tmem_ld32(t_s + 32 * (cc + 2), r);
+        }
     }
     tmem_st_wait();
     float a, b;
@@ -554,7 +630,7 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
         const int h = it.g * D.G + hl;
         const int pos = it.i * BLK + tok;
         const bool row_valid = pos < it.L;
-        float m_ref = -INFINITY, l = 0.f;
+        RowState st{-INFINITY, 0.f, t_o, false};
 
         TileWalk<BLK> walk;
         walk.init(P, it);
@@ -565,44 +641,14 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
             tc_fence_after();
             const bool masked = kind != kFull;
             const float bias = kind == kPseudo ? pseudo_bias : 0.f;
-            // pass 1: row maximum of the masked scores
-            const float rmax_raw = masked ? tile_max<BLK, true>(t_s, kind, tok, walk, j)
-                                          : tile_max<BLK, false>(t_s, kind, tok, walk, j);
-            const float rmax = fmaf(rmax_raw, scale, bias);   // -inf stays -inf
-            if (n == 0) {
-                m_ref = rmax;
-            } else {
-                // lazy rescale: O and l move to a new reference only when the
-                // row maximum grew by more than 2^8
-                const bool need = rmax > m_ref + 8.0f;
-                if (__any_sync(0xffffffffu, need)) {
-                    const float m_new = fmaxf(m_ref, rmax);
-                    const float alpha = ex2_approx(m_ref - m_new);
-                    m_ref = m_new;
-                    l *= alpha;
-#pragma unroll 1
-                    for (int c = 0; c < HD / 32; ++c) {
-                        uint32_t r[32];
-                        tmem_ld32(t_o + 32 * c, r);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                        tmem_st32(t_o + 32 * c, r);
-                    }
-                    tmem_st_wait();
-                }
-            }
-            // pass 2: P in place over S
-            const float rsum = masked ? tile_p<BLK, true>(t_s, kind, tok, walk, j, scale, bias - m_ref)
-                                      : tile_p<BLK, false>(t_s, kind, tok, walk, j, scale, bias - m_ref);
-            l += rsum;
+            const float rsum =
+                masked ? tile_softmax<BLK, HD, true>(t_s, kind, tok, walk, j, scale, bias, st)
+                       : tile_softmax<BLK, HD, false>(t_s, kind, tok, walk, j, scale, bias, st);
+            st.o_valid = true;
+            st.l += rsum;
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&B.s_free[m]);
-                mbar_arrive(&B.p_full[m]);
-            }
+            if (lane == 0) mbar_arrive(&B.p_full[m]);
             ++n;
         }
 
@@ -610,7 +656,7 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
         if (!warp_wait(&B.o_full[m], ocnt & 1, B, P.status)) return;
         ++ocnt;
         tc_fence_after();
-        const float inv_l = 1.0f / l;
+        const float inv_l = 1.0f / st.l;
         uint16_t* orow = P.o + ((int64_t)(it.tok0 + pos) * D.Hq + h) * HD;
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
@@ -629,7 +675,7 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
                 }
             }
         }
-        if (row_valid) P.lse[(int64_t)h * D.T + it.tok0 + pos] = (m_ref + log2f(l)) * 0.6931471805599453f;
+        if (row_valid) P.lse[(int64_t)h * D.T + it.tok0 + pos] = (st.m_ref + log2f(st.l)) * 0.6931471805599453f;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.o_free[m]);
@@ -655,12 +701,11 @@ k_attn(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap
             mbar_init(&B.q_full[m], 1);
             mbar_init(&B.q_empty[m], 1);
             mbar_init(&B.s_full[m], 1);
-            mbar_init(&B.s_free[m], kTileM / 32);
             mbar_init(&B.p_full[m], kTileM / 32);
             mbar_init(&B.o_full[m], 1);
             mbar_init(&B.o_free[m], kTileM / 32);
         }
-        for (int s = 0; s < kSlots; ++s) {
+        for (int s = 0; s < C::kSlots; ++s) {
             mbar_init(&B.kv_full[s], 1);
             mbar_init(&B.kv_empty[s], 1);
         }

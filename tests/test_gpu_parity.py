@@ -208,3 +208,24 @@ def test_bounded_wait_times_out_and_context_survives():
     pl = oracle.plan(q, k, v, wl.seqlens, wl.B, wl.tau)
     res = check_attention(wl, x, run, pl)
     assert res["rel_l2"] <= REL_L2_BF16 and res["lse_max_abs"] <= LSE_ABS, res
+
+
+@pytest.mark.parametrize("pos", [2 * 128 + 40, 5 * 128 + 100, 3 * 128 + 5])
+def test_row_maximum_jump_inside_a_tile(pos):
+    # One key far larger than every other, in the middle of a later block:
+    # rows whose score jumps by far more than the exp2 headroom must move
+    # their reference inside the tile (rescaling O, l and the P columns
+    # already written for that tile) and still match the oracle.
+    wl = synth.small_workload([1100, 900], 8, 2, 128, 128, 0.0, seed=123, generator="normal")
+    x = synth.generate(wl)
+    x = dict(x)
+    k = x["k"].copy()
+    k[pos, 0, :] *= 100.0
+    x["k"] = synth.bf16_round(k)
+    run = GpuRun(wl, x).plan().prefill()
+    assert run.status() == (fb.FP2_OK, 0)
+    q, kk, v = oracle_inputs(x, wl)
+    pl = oracle.plan(q, kk, v, wl.seqlens, wl.B, wl.tau)
+    res = check_attention(wl, x, run, pl)
+    assert res["finite"], res
+    assert res["rel_l2"] <= REL_L2_BF16 and res["lse_max_abs"] <= LSE_ABS, res
