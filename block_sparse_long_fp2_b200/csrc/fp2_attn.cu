@@ -490,9 +490,10 @@ __device__ __forceinline__ void p32(const uint32_t (&r)[32], uint32_t vb, uint32
                 s0 = ((vb >> e) & 1u) ? s0 : -INFINITY;
                 s1 = ((vb >> (e + 1)) & 1u) ? s1 : -INFINITY;
             }
-            float x0, x1;
+            float x0, x1, p0, p1;
             f2_unpack(f2_fma(f2_pack(s0, s1), scale2, shift2), x0, x1);
-            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
             sum2 = f2_add(sum2, f2_pack(p0, p1));
             packed[e2] = pack_bf16x2(p0, p1);
         }
@@ -508,8 +509,15 @@ __device__ __forceinline__ float max32(const uint32_t (&r)[32], uint32_t vb) {
         for (int e = 0; e < 32; ++e)
             if ((vb >> e) & 1u) mx = fmaxf(mx, __uint_as_float(r[e]));
     } else {
+        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) mx = fmax3(mx, __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+        for (int e = 0; e < 32; e += 8) {
+            m0 = fmax3(m0, __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+            m1 = fmax3(m1, __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+            m2 = fmax3(m2, __uint_as_float(r[e + 4]), __uint_as_float(r[e + 5]));
+            m3 = fmax3(m3, __uint_as_float(r[e + 6]), __uint_as_float(r[e + 7]));
+        }
+        mx = fmaxf(fmax3(m0, m1, m2), m3);
     }
     return mx;
 }
@@ -564,9 +572,10 @@ __device__ __forceinline__ void move_reference(RowState& st, float m_new, uint64
 // One pass over this thread's row of S: P = 2^(s * scale + bias - m_ref)
 // (zero where masked out) as bf16 pairs in place over S in tensor memory
 // (the P of chunk c goes to columns [16c, 16c+16) while the only loads in
-// flight cover [32(c+1), 32(c+2))).  Before a chunk is written its maximum
-// is checked against the reference; if it exceeds it by more than the
-// headroom the reference moves first.  Returns the fp32 row sum of the tile.
+// flight cover [32(c+1), 32(c+3))).  Before a pair of 32-column chunks is
+// written its maximum is checked against the reference; if it exceeds it by
+// more than the headroom the reference moves first.  Returns the fp32 row
+// sum of the tile.
 template <int BLK, int HD, bool MASKED>
 __device__ __forceinline__ float tile_softmax(uint32_t t_s, int kind, int tok,
                                               const TileWalk<BLK>& walk, int j, float scale,
@@ -581,20 +590,18 @@ __device__ __forceinline__ float tile_softmax(uint32_t t_s, int kind, int tok,
 #pragma unroll 1
     for (int c = 0; c < NC; c += 2) {
         tmem_ld_wait();
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            uint32_t(&r)[32] = half ? rb : ra;
-            const int cc = c + half;
-            const uint32_t vb = chunk_bits<BLK, MASKED>(kind, tok, walk, j, cc);
-            const float cm = fmaf(max32<MASKED>(r, vb), scale, bias);
-            const bool need = cm > st.m_ref + kHeadroom;
-            if (__any_sync(0xffffffffu, need)) {
-                move_reference<HD>(st, need ? cm : st.m_ref, sum2, t_s, 16 * cc);
-                shift2 = f2_pack(bias - st.m_ref, bias - st.m_ref);
-            }
-            p32<MASKED>(r, vb, t_s + 16 * cc, scale2, shift2, sum2);
-            if (cc + 2 < NC) tmem_ld32(t_s + 32 * (cc + 2), r);
+        const uint32_t vba = chunk_bits<BLK, MASKED>(kind, tok, walk, j, c);
+        const uint32_t vbb = chunk_bits<BLK, MASKED>(kind, tok, walk, j, c + 1);
+        const float cm = fmaf(fmaxf(max32<MASKED>(ra, vba), max32<MASKED>(rb, vbb)), scale, bias);
+        const bool need = cm > st.m_ref + kHeadroom;
+        if (__any_sync(0xffffffffu, need)) {
+            move_reference<HD>(st, need ? cm : st.m_ref, sum2, t_s, 16 * c);
+            shift2 = f2_pack(bias - st.m_ref, bias - st.m_ref);
         }
+        p32<MASKED>(ra, vba, t_s + 16 * c, scale2, shift2, sum2);
+        if (c + 2 < NC) tmem_ld32(t_s + 32 * (c + 2), ra);
+        p32<MASKED>(rb, vbb, t_s + 16 * (c + 1), scale2, shift2, sum2);
+        if (c + 3 < NC) tmem_ld32(t_s + 32 * (c + 3), rb);
     }
     tmem_st_wait();
     float a, b;
