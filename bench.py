@@ -278,7 +278,7 @@ def oracle_sample(wl, x, budget_s: float = 20.0):
     pl = oracle.plan(q, k, v, wl.seqlens, wl.B, wl.tau, rows=sample)
     rows, flop = [], 0.0
     for (s_, i) in sample:
-        oracle.attend(q, k, v, pl, rows=[(s_, i)])
+        oracle.attend_rows(q, k, v, pl, [(s_, i)])
         rows.append((s_, i))
         n_i = min(wl.B, wl.seqlens[s_] - i * wl.B)
         p0 = i * wl.B

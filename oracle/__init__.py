@@ -33,9 +33,11 @@ from .fp2_oracle import (  # noqa: F401
     select_blocks,
     plan,
     attend,
+    attend_rows,
     dense_attention,
     gather_paged,
     e4m3_round,
     quantize_e4m3,
     dequantize_e4m3,
+    quantize_means_e4m3,
 )

@@ -203,17 +203,19 @@ def plan(q, k, v, seqlens: Sequence[int], B: int, tau: float,
 # Steps 4-5: attention over kept blocks with mean correction
 # ----------------------------------------------------------------------------
 
-def attend(q, k, v, pl: Dict[str, object], correction: bool = True,
-           rows: Optional[Sequence[tuple]] = None, kept_override=None):
-    """Stage 2: O [T, Hq, d] and LSE [Hq, T] (natural log of the softmax
-    denominator in 1/sqrt(d)-scaled logits, pseudo-tokens included).
+def attend_rows(q, k, v, pl: Dict[str, object], rows: Sequence[tuple],
+                correction: bool = True, kept_override=None):
+    """Stage 2 for the query blocks `rows` = [(s, i), ...] only.
 
-    pl: output of plan() (block means and kept lists).
+    Returns (toks, O, LSE): toks the packed token indices of those blocks in
+    order, O [len(toks), Hq, d] and LSE [Hq, len(toks)] (natural log of the
+    softmax denominator in 1/sqrt(d)-scaled logits, pseudo-tokens included).
+
+    pl: output of plan() (block means and kept lists of these rows).
     correction: add one pseudo-token per skipped block (Figure 4); False
       drops skipped blocks entirely.
-    rows: optional list of (s, i) query blocks to compute; the others are
-      left NaN.  kept_override: optional {(s, g, i): kept ids} replacing the
-      plan's selection for those rows.
+    kept_override: optional {(s, g, i): kept ids} replacing the plan's
+      selection for those rows.
     """
     q = np.asarray(q)
     k = np.asarray(k)
@@ -225,18 +227,17 @@ def attend(q, k, v, pl: Dict[str, object], correction: bool = True,
     NB = int(lay["cu_blocks"][-1])
     kbar, vbar = pl["kbar"], pl["vbar"]
     counts = pl["counts"]
-    T, _, d = q.shape
+    d = q.shape[2]
     inv_sqrt_d = 1.0 / math.sqrt(d)
-    O = np.full((T, Hq, d), np.nan)
-    LSE = np.full((Hq, T), np.nan)
-    if rows is None:
-        rows = [(s, i) for s in range(len(lay["seqlens"])) for i in range(int(lay["nb"][s]))]
+    toks, O_parts, L_parts = [], [], []
     for (s, i) in rows:
         t0 = int(lay["cu_seqlens"][s])
         L = int(lay["seqlens"][s])
         b0 = int(lay["cu_blocks"][s])
         qlo, qhi = t0 + i * B, t0 + min((i + 1) * B, L)
         qpos = np.arange(qlo, qhi) - t0                      # positions in the sequence
+        O_blk = np.zeros((qhi - qlo, Hq, d))
+        L_blk = np.zeros((Hq, qhi - qlo))
         for g in range(Hkv):
             r = g * NB + b0 + i
             kept = pl["kept"][r] if kept_override is None or (s, g, i) not in kept_override \
@@ -264,8 +265,29 @@ def attend(q, k, v, pl: Dict[str, object], correction: bool = True,
                 w_pseudo = np.exp(s_pseudo - M[:, None])
                 den = w_exact.sum(axis=1) + w_pseudo.sum(axis=1)
                 num = w_exact @ Vk + w_pseudo @ V_pseudo
-                O[qlo:qhi, h, :] = num / den[:, None]
-                LSE[h, qlo:qhi] = M + np.log(den)
+                O_blk[:, h, :] = num / den[:, None]
+                L_blk[h, :] = M + np.log(den)
+        toks.append(np.arange(qlo, qhi))
+        O_parts.append(O_blk)
+        L_parts.append(L_blk)
+    if not toks:
+        return np.zeros(0, dtype=np.int64), np.zeros((0, Hq, d)), np.zeros((Hq, 0))
+    return np.concatenate(toks), np.concatenate(O_parts, axis=0), np.concatenate(L_parts, axis=1)
+
+
+def attend(q, k, v, pl: Dict[str, object], correction: bool = True,
+           rows: Optional[Sequence[tuple]] = None, kept_override=None):
+    """Stage 2 for the whole batch (or the query blocks `rows`): O [T, Hq, d]
+    and LSE [Hq, T], entries outside `rows` left NaN.  See attend_rows."""
+    lay = pl["layout"]
+    T, Hq, d = np.shape(q)
+    if rows is None:
+        rows = [(s, i) for s in range(len(lay["seqlens"])) for i in range(int(lay["nb"][s]))]
+    toks, O_r, L_r = attend_rows(q, k, v, pl, rows, correction, kept_override)
+    O = np.full((T, Hq, d), np.nan)
+    LSE = np.full((Hq, T), np.nan)
+    O[toks] = O_r
+    LSE[:, toks] = L_r
     return O, LSE
 
 
@@ -385,3 +407,34 @@ def dequantize_e4m3(codes, scales, seqlens: Sequence[int], B: int) -> np.ndarray
             lo, hi = t0 + i * B, t0 + min((i + 1) * B, int(L))
             out[lo:hi] = codes[lo:hi] * scales[b0 + i][None, :, None]
     return out
+
+
+def quantize_means_e4m3(means, seqlens: Sequence[int], B: int):
+    """e4m3 codes of block means for the FP8 correction path.
+
+    means [NB, H, d] (float64 block means).  They are stored as float32, and
+    every chunk of B consecutive blocks of a sequence (the blocks one
+    pseudo-key tile covers) shares one scale per head: scale = absmax / 448
+    over the chunk (1 when all zero), code = e4m3_round(mean / scale), the
+    scale and the quotient rounded to float32 as the kernel computes them.
+    Returns (codes [NB, H, d] float64, scales [NB, H] float64 with the chunk's
+    scale at its first block and NaN elsewhere).
+    """
+    m32 = np.asarray(means, dtype=np.float32)
+    lay = block_layout(seqlens, B)
+    NB, H, d = m32.shape
+    codes = np.zeros((NB, H, d))
+    scales = np.full((NB, H), np.nan)
+    for s in range(len(lay["seqlens"])):
+        b0 = int(lay["cu_blocks"][s])
+        nb = int(lay["nb"][s])
+        for c0 in range(0, nb, B):
+            lo, hi = b0 + c0, b0 + min(c0 + B, nb)
+            for h in range(H):
+                blk = m32[lo:hi, h, :]
+                amax = np.float32(np.abs(blk).max())
+                sc = amax / np.float32(E4M3_MAX) if amax > 0 else np.float32(1.0)
+                scales[lo, h] = sc
+                codes[lo:hi, h, :] = e4m3_round(blk / sc)
+    return codes, scales
+

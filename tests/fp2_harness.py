@@ -168,11 +168,11 @@ def check_attention(wl, x, run: GpuRun, pl, rows_si=None, correction=True):
             r = g * NB + int(cu_b[s]) + i
             if list(pl["kept"][r]) != gk[r]:
                 override[(s, g, i)] = gk[r]
-    O_ref, L_ref = oracle.attend(q, k, v, pl, correction=correction, rows=rows_si,
-                                 kept_override=override)
+    toks, O_ref, L_ref = oracle.attend_rows(q, k, v, pl, rows_si, correction=correction,
+                                            kept_override=override)
     O, LSE = run.outputs()
-    toks = token_rows(wl, rows_si)
-    e_o = rel_l2(O[toks], O_ref[toks])
-    e_l = float(np.max(np.abs(LSE[:, toks] - L_ref[:, toks])))
+    assert np.array_equal(toks, token_rows(wl, rows_si))
+    e_o = rel_l2(O[toks], O_ref)
+    e_l = float(np.max(np.abs(LSE[:, toks] - L_ref)))
     return {"rel_l2": e_o, "lse_max_abs": e_l, "n_override": len(override),
             "finite": bool(np.isfinite(O[toks]).all() and np.isfinite(LSE[:, toks]).all())}
