@@ -114,10 +114,12 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     L.off_tri_off = c.take(sizeof(int64_t) * (n + 1));
     L.off_group_cu = c.take(sizeof(int32_t) * (n + 1));
     L.off_group_seq = c.take(sizeof(int32_t) * (size_t)std::max<int64_t>(1, groups));
+    L.off_vmax = c.take(sizeof(float) * n * (size_t)d.Hkv);
     pub.plan_bytes = align_up(c.off, 256);
 
     Carver w;
     L.ws_qbar64 = w.take(sizeof(double) * (size_t)NB * d.Hq * d.d);
+    L.ws_qbar32 = w.take(sizeof(float) * (size_t)NB * d.Hq * d.d);
     L.ws_kbar64 = w.take(sizeof(double) * mean_elems);
     L.ws_qnorm = w.take(sizeof(float) * (size_t)NB * d.Hkv);
     L.ws_knorm = w.take(sizeof(float) * (size_t)NB * d.Hkv);
@@ -149,6 +151,7 @@ PlanPtrs plan_ptrs(const Layout& L, void* plan) {
     p.tri_off = reinterpret_cast<int64_t*>(b + L.off_tri_off);
     p.group_cu = reinterpret_cast<int32_t*>(b + L.off_group_cu);
     p.group_seq = reinterpret_cast<int32_t*>(b + L.off_group_seq);
+    p.vmax = reinterpret_cast<float*>(b + L.off_vmax);
     return p;
 }
 
@@ -156,6 +159,7 @@ WsPtrs ws_ptrs(const Layout& L, void* ws) {
     char* b = static_cast<char*>(ws);
     WsPtrs w;
     w.qbar64 = reinterpret_cast<double*>(b + L.ws_qbar64);
+    w.qbar32 = reinterpret_cast<float*>(b + L.ws_qbar32);
     w.kbar64 = reinterpret_cast<double*>(b + L.ws_kbar64);
     w.qnorm = reinterpret_cast<float*>(b + L.ws_qnorm);
     w.knorm = reinterpret_cast<float*>(b + L.ws_knorm);

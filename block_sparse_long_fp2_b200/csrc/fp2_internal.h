@@ -26,7 +26,7 @@ struct Dims {
     int mask_words;       // 32-bit words per kept-mask row
     int max_nb;           // largest nb_s
     int rows_per_group;   // query blocks per scoring CTA (kScoreQV / G)
-    int n_groups_cap;     // upper bound of scoring CTAs per kv-head
+    int n_groups_cap;     // upper bound of scoring row groups per kv-head
     int64_t T, NB, R, tri_total, nnz_cap;
     double tau;
 };
@@ -52,11 +52,13 @@ struct PlanPtrs {
     int64_t* tri_off;      // [n+1] prefix of nb (nb + 1) / 2
     int32_t* group_cu;     // [n+1] prefix of scoring CTAs per sequence
     int32_t* group_seq;    // [n_groups_cap]
+    float* vmax;           // [n, Hkv]  largest V scale of each sequence and kv-head (FP8)
 };
 
 // Device pointers into fp2_plan's workspace.
 struct WsPtrs {
     double* qbar64;   // [NB, Hq, d]
+    float* qbar32;    // [NB, Hq, d]  the same means rounded to fp32
     double* kbar64;   // [NB, Hkv, d]
     float* qnorm;     // [NB, Hkv]  max over the group's heads of |Qbar|_2 (rounded up)
     float* knorm;     // [NB, Hkv]  |Kbar|_2 (rounded up)
@@ -68,8 +70,9 @@ struct WsPtrs {
 struct Layout {
     Dims dims;
     fp2_plan_layout pub;
-    size_t off_meta_valid, off_cu_blocks, off_block_seq, off_tri_off, off_group_cu, off_group_seq;
-    size_t ws_qbar64, ws_kbar64, ws_qnorm, ws_knorm, ws_scores, ws_counts;
+    size_t off_meta_valid, off_cu_blocks, off_block_seq, off_tri_off, off_group_cu, off_group_seq,
+        off_vmax;
+    size_t ws_qbar64, ws_qbar32, ws_kbar64, ws_qnorm, ws_knorm, ws_scores, ws_counts;
 };
 
 // Validates the problem on the host and computes sizes and offsets.

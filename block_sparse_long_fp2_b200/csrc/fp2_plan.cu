@@ -8,13 +8,16 @@
 //            accumulates each block's sum in float64 (exact for bf16 inputs),
 //            writing Qbar (fp64 workspace) and Kbar/Vbar (fp32, bf16, fp64).
 //   norms    |Qbar|, |Kbar| per block and kv-head (for the score error bound).
-//   score    per (sequence, kv-head, group of query blocks): float32 scores
-//            of every visible key block, then the threshold decision per row.
-//            A block whose float32 score lies within the float32 rounding
-//            bound of the threshold, and every candidate for the row maximum,
-//            is re-scored in float64, so the kept set is the one float64
-//            scores give.
+//   score    one CTA per tile of the causal triangle (128 query vectors of a
+//            group of query blocks x 64 key blocks, one kv-head): float32
+//            block scores, max over the group's heads, to a scratch array.
+//   threshold  one warp per row: the threshold decision.  A block whose
+//            float32 score lies within the float32 rounding bound of the
+//            threshold, and every candidate for the row maximum, is re-scored
+//            in float64, so the kept set is the one float64 scores give.
 //   scan     row_ptr = exclusive prefix sum of kept counts.
+//   quant_means  e4m3 codes of Kbar / Vbar with one scale per pseudo-tile
+//            chunk (used by the FP8 correction).
 //   compact  col_idx from the kept-block bit masks, ascending per row.
 #include <cfloat>
 #include <cmath>
@@ -174,6 +177,9 @@ k_pool(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict
         double* dst = W.qbar64 + (b * D.Hq + head) * d + e0;
 #pragma unroll
         for (int e = 0; e < 8; e += 2) *reinterpret_cast<double2*>(dst + e) = make_double2(m[e], m[e + 1]);
+        float* d32 = W.qbar32 + (b * D.Hq + head) * d + e0;
+        *reinterpret_cast<float4*>(d32) = make_float4((float)m[0], (float)m[1], (float)m[2], (float)m[3]);
+        *reinterpret_cast<float4*>(d32 + 4) = make_float4((float)m[4], (float)m[5], (float)m[6], (float)m[7]);
     } else {
         const int64_t off = (b * D.Hkv + head) * d + e0;
         float* f32 = (which == 1 ? P.kbar : P.vbar) + off;
@@ -240,20 +246,117 @@ __global__ void k_norms(Dims D, PlanPtrs P, WsPtrs W) {
 }
 
 // ---------------------------------------------------------------------------
-// score: float32 scores + exact-decision thresholding
+// score: float32 scores of every (row, visible key block), triangle-tiled
 // ---------------------------------------------------------------------------
 
 constexpr int kScoreThreads = 256;
-constexpr int kScoreKC = 32;   // key blocks per chunk
+constexpr int kScoreKC = 64;   // key blocks per tile
 
 template <int HD>
 struct ScoreSmem {
-    float q[kScoreQV][HD + 4];
-    float k[kScoreKC][HD + 4];
-    float dots[kScoreQV][kScoreKC + 1];
+    float q[kScoreQV][HD + 4];        // query block means of the tile's rows (padded rows)
+    union {
+        float k[kScoreKC][HD + 4];    // key block means of the tile's columns
+        float dots[kScoreQV][kScoreKC + 1];
+    };
 };
 
-// float64 score of key block j for row (b_i, g): max over the group's heads.
+// One CTA per (sequence, kv-head, group of rows_per_group query blocks,
+// chunk of kScoreKC key blocks) inside the causal triangle: 128 x 64 dot
+// products of length d from padded shared memory (4 query x 8 key register
+// tile per thread, conflict-free float4 loads), then the max over the
+// group's heads, written to the fp32 score scratch.
+template <int HD>
+__global__ void __launch_bounds__(kScoreThreads)
+k_score(Dims D, PlanPtrs P, WsPtrs W, int max_chunks) {
+    if (!*P.meta_valid) return;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    ScoreSmem<HD>& S = *reinterpret_cast<ScoreSmem<HD>*>(smem_raw);
+
+    const int gi = blockIdx.x / max_chunks;
+    const int jc = blockIdx.x % max_chunks;
+    const int g = blockIdx.y;
+    if (gi >= P.group_cu[D.n_seqs]) return;
+    const int s = P.group_seq[gi];
+    const int RI = D.rows_per_group;
+    const int G = D.G;
+    const int b0 = P.cu_blocks[s];
+    const int nb = P.cu_blocks[s + 1] - b0;
+    const int i0 = (gi - P.group_cu[s]) * RI;
+    const int i1 = min(i0 + RI, nb);
+    const int j0 = jc * kScoreKC;
+    if (j0 > i1 - 1) return;                       // above the causal triangle
+    const int j1 = min(j0 + kScoreKC, i1);
+    const int nrows = i1 - i0;
+    const int nqv = nrows * G;
+    const int tid = threadIdx.x;
+
+    for (int idx = tid; idx < kScoreQV * (HD / 4); idx += kScoreThreads) {
+        const int qv = idx / (HD / 4), e = (idx % (HD / 4)) * 4;
+        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (qv < nqv) {
+            const int ri = qv / G, hl = qv % G;
+            f = *reinterpret_cast<const float4*>(
+                W.qbar32 + ((int64_t)(b0 + i0 + ri) * D.Hq + g * G + hl) * HD + e);
+        }
+        *reinterpret_cast<float4*>(&S.q[qv][e]) = f;
+    }
+    for (int idx = tid; idx < kScoreKC * (HD / 4); idx += kScoreThreads) {
+        const int kv = idx / (HD / 4), e = (idx % (HD / 4)) * 4;
+        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j0 + kv < j1)
+            f = *reinterpret_cast<const float4*>(P.kbar + ((int64_t)(b0 + j0 + kv) * D.Hkv + g) * HD + e);
+        *reinterpret_cast<float4*>(&S.k[kv][e]) = f;
+    }
+    __syncthreads();
+    // Thread (tq, tk) owns query vectors tq + 32a and key blocks tk + 8c: a warp
+    // reads 4 consecutive query rows and 8 consecutive key rows per load, which
+    // the 4-float row padding spreads over distinct banks.
+    const int tq = tid >> 3;   // 0..31
+    const int tk = tid & 7;    // 0..7
+    float acc[4][8];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
+#pragma unroll 2
+    for (int e = 0; e < HD; e += 4) {
+        float4 qa[4], kb[8];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) qa[a] = *reinterpret_cast<const float4*>(&S.q[tq + 32 * a][e]);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) kb[c] = *reinterpret_cast<const float4*>(&S.k[tk + 8 * c][e]);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                acc[a][c] = fmaf(qa[a].x, kb[c].x, acc[a][c]);
+                acc[a][c] = fmaf(qa[a].y, kb[c].y, acc[a][c]);
+                acc[a][c] = fmaf(qa[a].z, kb[c].z, acc[a][c]);
+                acc[a][c] = fmaf(qa[a].w, kb[c].w, acc[a][c]);
+            }
+    }
+    __syncthreads();                               // S.k is reused as S.dots
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) S.dots[tq + 32 * a][tk + 8 * c] = acc[a][c];
+    __syncthreads();
+    const float inv_sqrt_d = 1.0f / sqrtf((float)HD);
+    float* scores = W.scores + (int64_t)g * D.tri_total + P.tri_off[s];
+    for (int idx = tid; idx < nrows * kScoreKC; idx += kScoreThreads) {
+        const int ri = idx / kScoreKC, jj = idx % kScoreKC;
+        const int i = i0 + ri, j = j0 + jj;
+        if (j <= i && j < j1) {
+            float best = S.dots[ri * G][jj];
+            for (int hl = 1; hl < G; ++hl) best = fmaxf(best, S.dots[ri * G + hl][jj]);
+            scores[(int64_t)i * (i + 1) / 2 + j] = best * inv_sqrt_d;
+        }
+    }
+}
+
+// float64 score of key block j for row (b_i, g): max over the group's heads
+// (warp-collective).
 template <int HD>
 __device__ double score64(const Dims& D, const WsPtrs& W, int64_t b_i, int64_t b_j, int g) {
     const int lane = threadIdx.x & 31;
@@ -270,168 +373,156 @@ __device__ double score64(const Dims& D, const WsPtrs& W, int64_t b_i, int64_t b
     return best / sqrt((double)HD);
 }
 
+// ---------------------------------------------------------------------------
+// threshold: one warp per row, decisions equal to the float64 ones
+// ---------------------------------------------------------------------------
+//
+// The float32 score of a block differs from the exact one by at most
+//   e_j = 2 (d + 8) 2^-24 max_h|Qbar_{i,h}| |Kbar_j| / sqrt(d)
+// (rounding of the means to fp32, the fp32 dot product, the scaling; with a
+// factor 2 of margin).  Every block whose score could be the row maximum and
+// every block whose score lies within e_j of tau * m is re-scored in float64.
 template <int HD>
-__global__ void __launch_bounds__(kScoreThreads)
-k_score(Dims D, PlanPtrs P, WsPtrs W) {
+__global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W) {
     if (!*P.meta_valid) return;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    ScoreSmem<HD>& S = *reinterpret_cast<ScoreSmem<HD>*>(smem_raw);
-
-    const int gi = blockIdx.x;
-    const int g = blockIdx.y;
-    const int s = P.group_seq[gi];
-    if (gi >= P.group_cu[D.n_seqs]) return;
-    const int RI = D.rows_per_group;
-    const int G = D.G;
+    const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (r >= D.R) return;
+    const int g = (int)(r / D.NB);
+    const int64_t bi = r % D.NB;
+    const int s = P.block_seq[bi];
     const int b0 = P.cu_blocks[s];
-    const int nb = P.cu_blocks[s + 1] - b0;
-    const int i0 = (gi - P.group_cu[s]) * RI;
-    const int i1 = min(i0 + RI, nb);
-    const int nrows = i1 - i0;
-    const int nqv = nrows * G;
-    const int tid = threadIdx.x;
-    const float inv_sqrt_d = 1.0f / sqrtf((float)HD);
-    float* scores = W.scores + (int64_t)g * D.tri_total + P.tri_off[s];
-
-    if (D.tau > 0.0) {
-        // query block means of this group's rows, rounded to fp32
-        for (int idx = tid; idx < kScoreQV * (HD / 4); idx += kScoreThreads) {
-            const int qv = idx / (HD / 4), e = (idx % (HD / 4)) * 4;
-            float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (qv < nqv) {
-                const int ri = qv / G, hl = qv % G;
-                const double* qp = W.qbar64 + ((int64_t)(b0 + i0 + ri) * D.Hq + g * G + hl) * HD + e;
-                f = make_float4((float)qp[0], (float)qp[1], (float)qp[2], (float)qp[3]);
-            }
-            *reinterpret_cast<float4*>(&S.q[qv][e]) = f;
+    const int i = (int)(bi - b0);
+    uint32_t* mask = P.kept_mask + r * D.mask_words;
+    int count = 0;
+    if (D.tau == 0.0) {
+        for (int w = lane; w < D.mask_words; w += 32) {
+            uint32_t bits = 0;
+            if (32 * w + 31 <= i) bits = 0xFFFFFFFFu;
+            else if (32 * w <= i) bits = (1u << (i - 32 * w + 1)) - 1u;
+            mask[w] = bits;
         }
-        const int tq = tid >> 3;   // 4 query vectors: 4*tq .. 4*tq+3
-        const int tk = tid & 7;    // 4 key blocks:   4*tk .. 4*tk+3
-        for (int jc = 0; jc < i1; jc += kScoreKC) {
-            __syncthreads();
-            for (int idx = tid; idx < kScoreKC * (HD / 4); idx += kScoreThreads) {
-                const int kv = idx / (HD / 4), e = (idx % (HD / 4)) * 4;
-                float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (jc + kv < nb) {
-                    const double* kp = W.kbar64 + ((int64_t)(b0 + jc + kv) * D.Hkv + g) * HD + e;
-                    f = make_float4((float)kp[0], (float)kp[1], (float)kp[2], (float)kp[3]);
-                }
-                *reinterpret_cast<float4*>(&S.k[kv][e]) = f;
-            }
-            __syncthreads();
-            float acc[4][4];
+        count = i + 1;
+    } else {
+        const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
+        const double C = 2.0 * (HD + 8) * (1.0 / 16777216.0) / sqrt((double)HD);
+        const double qn = W.qnorm[bi * D.Hkv + g];
+        const float* kn = W.knorm + (int64_t)b0 * D.Hkv + g;
+        // pass 1: largest lower bound of any score
+        double m_lo = -DBL_MAX;
+        for (int j = lane; j <= i; j += 32) m_lo = fmax(m_lo, (double)sc[j] - C * qn * kn[(int64_t)j * D.Hkv]);
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-#pragma unroll 4
-            for (int e = 0; e < HD; e += 4) {
-                float4 qa[4], kb[4];
-#pragma unroll
-                for (int a = 0; a < 4; ++a) qa[a] = *reinterpret_cast<const float4*>(&S.q[4 * tq + a][e]);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) kb[c] = *reinterpret_cast<const float4*>(&S.k[4 * tk + c][e]);
-#pragma unroll
-                for (int a = 0; a < 4; ++a)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        acc[a][c] = fmaf(qa[a].x, kb[c].x, acc[a][c]);
-                        acc[a][c] = fmaf(qa[a].y, kb[c].y, acc[a][c]);
-                        acc[a][c] = fmaf(qa[a].z, kb[c].z, acc[a][c]);
-                        acc[a][c] = fmaf(qa[a].w, kb[c].w, acc[a][c]);
-                    }
-            }
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) S.dots[4 * tq + a][4 * tk + c] = acc[a][c];
-            __syncthreads();
-            for (int idx = tid; idx < nrows * kScoreKC; idx += kScoreThreads) {
-                const int ri = idx / kScoreKC, jj = idx % kScoreKC;
-                const int i = i0 + ri, j = jc + jj;
-                if (j <= i) {
-                    float best = S.dots[ri * G][jj];
-                    for (int hl = 1; hl < G; ++hl) best = fmaxf(best, S.dots[ri * G + hl][jj]);
-                    scores[(int64_t)i * (i + 1) / 2 + j] = best * inv_sqrt_d;
-                }
+        for (int o = 16; o > 0; o >>= 1) m_lo = fmax(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o));
+        // pass 2: the row maximum in float64 over every candidate
+        double m = -DBL_MAX;
+        for (int jb = 0; jb <= i; jb += 32) {
+            const int j = jb + lane;
+            const bool cand = j <= i && (double)sc[j] + C * qn * kn[(int64_t)j * D.Hkv] >= m_lo;
+            uint32_t cb = __ballot_sync(0xffffffffu, cand);
+            while (cb) {
+                const int l = __ffs(cb) - 1;
+                cb &= cb - 1;
+                m = fmax(m, score64<HD>(D, W, bi, b0 + jb + l, g));
             }
         }
-        __syncthreads();
+        const double t = D.tau * m;
+        // pass 3: decisions (forced blocks 0 and i; uncertain ones in float64)
+        for (int w = 0; 32 * w <= i; ++w) {
+            const int j = 32 * w + lane;
+            bool keep = false, unsure = false;
+            if (j <= i) {
+                if (j == 0 || j == i) {
+                    keep = true;
+                } else {
+                    const double e = C * qn * kn[(int64_t)j * D.Hkv];
+                    const double x = (double)sc[j];
+                    if (x - e >= t) keep = true;
+                    else if (!(x + e < t)) unsure = true;
+                }
+            }
+            uint32_t ub = __ballot_sync(0xffffffffu, unsure);
+            while (ub) {
+                const int l = __ffs(ub) - 1;
+                ub &= ub - 1;
+                const double x64 = score64<HD>(D, W, bi, b0 + 32 * w + l, g);
+                if (lane == l) keep = x64 >= t;
+            }
+            const uint32_t bits = __ballot_sync(0xffffffffu, keep);
+            if (lane == 0) mask[w] = bits;
+            count += __popc(bits);
+        }
+        for (int w = i / 32 + 1 + lane; w < D.mask_words; w += 32) mask[w] = 0u;
     }
+    if (lane == 0) W.counts[r] = count;
+}
 
-    // ---- per-row threshold decision: one warp per row ----
-    const int warp = tid >> 5, lane = tid & 31;
-    const double C = 2.0 * (HD + 8) * (1.0 / 16777216.0) / sqrt((double)HD);
-    for (int ri = warp; ri < nrows; ri += kScoreThreads / 32) {
-        const int i = i0 + ri;
-        const int64_t bi = b0 + i;
-        const int64_t r = (int64_t)g * D.NB + bi;
-        uint32_t* mask = P.kept_mask + r * D.mask_words;
-        int count = 0;
-        if (D.tau == 0.0) {
-            for (int w = lane; w < D.mask_words; w += 32) {
-                uint32_t bits = 0;
-                if (32 * w + 31 <= i) bits = 0xFFFFFFFFu;
-                else if (32 * w <= i) bits = (1u << (i - 32 * w + 1)) - 1u;
-                mask[w] = bits;
-            }
-            count = i + 1;
-        } else {
-            const float* sc = scores + (int64_t)i * (i + 1) / 2;
-            const double qn = W.qnorm[bi * D.Hkv + g];
-            // pass 1: largest lower bound of any score
-            double m_lo = -DBL_MAX;
-            for (int j = lane; j <= i; j += 32) {
-                const double e = C * qn * W.knorm[(int64_t)(b0 + j) * D.Hkv + g];
-                m_lo = fmax(m_lo, (double)sc[j] - e);
-            }
+// ---------------------------------------------------------------------------
+// quant_means: e4m3 codes of the K / V block means for the FP8 correction
+// ---------------------------------------------------------------------------
+//
+// One CTA per (chunk of B blocks of one sequence, kv-head): the chunk is the
+// set of blocks one pseudo-key tile covers, so a pseudo tile needs a single
+// scale.  scale = absmax / 448 over the chunk's fp32 means (1 when all zero),
+// code = e4m3_rne_sat(mean / scale), both in fp32.
+
+__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+constexpr int kQuantMeansThreads = 1024;
+
+__global__ void __launch_bounds__(kQuantMeansThreads) k_quant_means(Dims D, PlanPtrs P) {
+    if (!*P.meta_valid) return;
+    const int s = blockIdx.y;
+    const int g = blockIdx.z;
+    const int b0 = P.cu_blocks[s];
+    if ((int64_t)blockIdx.x * D.B >= P.cu_blocks[s + 1] - b0) return;   // past the sequence
+    const int64_t b = b0 + (int64_t)blockIdx.x * D.B;                       // first block of the chunk
+    const int nblk = min((int64_t)D.B, (int64_t)P.cu_blocks[s + 1] - b);
+    const int d = D.d;
+    __shared__ float red[2][kQuantMeansThreads / 32];
+    float mk = 0.f, mv = 0.f;
+    for (int idx = 4 * threadIdx.x; idx < nblk * d; idx += 4 * blockDim.x) {
+        const int64_t off = ((b + idx / d) * D.Hkv + g) * d + idx % d;
+        const float4 k4 = *reinterpret_cast<const float4*>(P.kbar + off);
+        const float4 v4 = *reinterpret_cast<const float4*>(P.vbar + off);
+        mk = fmaxf(mk, fmaxf(fmaxf(fabsf(k4.x), fabsf(k4.y)), fmaxf(fabsf(k4.z), fabsf(k4.w))));
+        mv = fmaxf(mv, fmaxf(fmaxf(fabsf(v4.x), fabsf(v4.y)), fmaxf(fabsf(v4.z), fabsf(v4.w))));
+    }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m_lo = fmax(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o));
-            // pass 2: the row maximum in float64 over every candidate
-            double m = -DBL_MAX;
-            for (int jb = 0; jb <= i; jb += 32) {
-                const int j = jb + lane;
-                bool cand = false;
-                if (j <= i) {
-                    const double e = C * qn * W.knorm[(int64_t)(b0 + j) * D.Hkv + g];
-                    cand = (double)sc[j] + e >= m_lo;
-                }
-                uint32_t cb = __ballot_sync(0xffffffffu, cand);
-                while (cb) {
-                    const int l = __ffs(cb) - 1;
-                    cb &= cb - 1;
-                    m = fmax(m, score64<HD>(D, W, bi, b0 + jb + l, g));
-                }
-            }
-            const double t = D.tau * m;
-            // pass 3: decisions (forced blocks 0 and i; uncertain ones in float64)
-            for (int w = 0; 32 * w <= i; ++w) {
-                const int j = 32 * w + lane;
-                bool keep = false, unsure = false;
-                if (j <= i) {
-                    if (j == 0 || j == i) {
-                        keep = true;
-                    } else {
-                        const double e = C * qn * W.knorm[(int64_t)(b0 + j) * D.Hkv + g];
-                        const double x = (double)sc[j];
-                        if (x - e >= t) keep = true;
-                        else if (!(x + e < t)) unsure = true;
-                    }
-                }
-                uint32_t ub = __ballot_sync(0xffffffffu, unsure);
-                while (ub) {
-                    const int l = __ffs(ub) - 1;
-                    ub &= ub - 1;
-                    const double x64 = score64<HD>(D, W, bi, b0 + 32 * w + l, g);
-                    if (lane == l) keep = x64 >= t;
-                }
-                const uint32_t bits = __ballot_sync(0xffffffffu, keep);
-                if (lane == 0) mask[w] = bits;
-                count += __popc(bits);
-            }
-            for (int w = i / 32 + 1 + lane; w < D.mask_words; w += 32) mask[w] = 0u;
-        }
-        if (lane == 0) W.counts[r] = count;
+    for (int o = 16; o > 0; o >>= 1) {
+        mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, o));
+        mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, o));
+    }
+    if ((threadIdx.x & 31) == 0) {
+        red[0][threadIdx.x >> 5] = mk;
+        red[1][threadIdx.x >> 5] = mv;
+    }
+    __syncthreads();
+    mk = red[0][0];
+    mv = red[1][0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
+        mk = fmaxf(mk, red[0][w]);
+        mv = fmaxf(mv, red[1][w]);
+    }
+    const float sk = mk > 0.f ? __fdiv_rn(mk, 448.0f) : 1.0f;
+    const float sv = mv > 0.f ? __fdiv_rn(mv, 448.0f) : 1.0f;
+    if (threadIdx.x == 0) {
+        P.kbar_scale[b * D.Hkv + g] = sk;
+        P.vbar_scale[b * D.Hkv + g] = sv;
+    }
+    for (int idx = 4 * threadIdx.x; idx < nblk * d; idx += 4 * blockDim.x) {
+        const int64_t off = ((b + idx / d) * D.Hkv + g) * d + idx % d;
+        const float4 k4 = *reinterpret_cast<const float4*>(P.kbar + off);
+        const float4 v4 = *reinterpret_cast<const float4*>(P.vbar + off);
+        *reinterpret_cast<uint32_t*>(P.kbar8 + off) =
+            (uint32_t)e4m3x2(__fdiv_rn(k4.x, sk), __fdiv_rn(k4.y, sk)) |
+            ((uint32_t)e4m3x2(__fdiv_rn(k4.z, sk), __fdiv_rn(k4.w, sk)) << 16);
+        *reinterpret_cast<uint32_t*>(P.vbar8 + off) =
+            (uint32_t)e4m3x2(__fdiv_rn(v4.x, sv), __fdiv_rn(v4.y, sv)) |
+            ((uint32_t)e4m3x2(__fdiv_rn(v4.z, sv), __fdiv_rn(v4.w, sv)) << 16);
     }
 }
 
@@ -489,12 +580,16 @@ __global__ void k_compact(Dims D, PlanPtrs P) {
 
 template <int HD>
 int launch_score(const Dims& D, const PlanPtrs& P, const WsPtrs& W, cudaStream_t st) {
-    const size_t smem = sizeof(ScoreSmem<HD>);
-    if (cudaFuncSetAttribute(k_score<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return FP2_ERR_CUDA;
-    dim3 grid(D.n_groups_cap, D.Hkv);
-    k_score<HD><<<grid, kScoreThreads, smem, st>>>(D, P, W);
+    if (D.tau > 0.0) {
+        const size_t smem = sizeof(ScoreSmem<HD>);
+        if (cudaFuncSetAttribute(k_score<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
+            return FP2_ERR_CUDA;
+        const int max_chunks = (D.max_nb + kScoreKC - 1) / kScoreKC;
+        dim3 grid((unsigned)((int64_t)D.n_groups_cap * max_chunks), D.Hkv);
+        k_score<HD><<<grid, kScoreThreads, smem, st>>>(D, P, W, max_chunks);
+    }
+    k_threshold<HD><<<(unsigned)((D.R * 32 + 255) / 256), 256, 0, st>>>(D, P, W);
     return FP2_OK;
 }
 
@@ -516,6 +611,8 @@ int launch_plan(const Layout& L, const fp2_problem* p, const void* q, const void
     }
     int rc = D.d == 64 ? launch_score<64>(D, P, W, st) : launch_score<128>(D, P, W, st);
     if (rc != FP2_OK) return rc;
+    k_quant_means<<<dim3((unsigned)((D.max_nb + D.B - 1) / D.B), D.n_seqs, D.Hkv), kQuantMeansThreads, 0,
+                    st>>>(D, P);
     k_scan<<<1, kScanThreads, 0, st>>>(D, P, W);
     k_compact<<<(unsigned)((D.R * 32 + 255) / 256), 256, 0, st>>>(D, P);
     return cudaGetLastError() == cudaSuccess ? FP2_OK : FP2_ERR_CUDA;

@@ -133,9 +133,13 @@ typedef struct fp2_problem {
  *   kbar, vbar  float [num_blocks, Hkv, d] block means of K and V.
  *   kbar_bf16, vbar_bf16  the same means rounded to bfloat16 (operands of the
  *               correction's tensor-core products).
- *   kbar_e4m3, vbar_e4m3  uint8 [num_blocks, Hkv, d] e4m3 codes of the means,
- *   kbar_scale, vbar_scale float [num_blocks, Hkv] their per-(block, head)
- *               scales (absmax / 448); used by the FP8 path.
+ *   kbar_e4m3, vbar_e4m3  uint8 [num_blocks, Hkv, d] e4m3 codes of the fp32
+ *               means, with one scale per chunk of B consecutive blocks of a
+ *               sequence (blocks B*c .. B*c+B-1, the pseudo-key tile of the
+ *               FP8 correction) and kv-head: scale = absmax / 448 over the
+ *               chunk (1 when all zero), code = e4m3_rne_sat(mean / scale).
+ *   kbar_scale, vbar_scale float [num_blocks, Hkv]: the chunk scale, stored
+ *               at the chunk's first block (other entries unused).
  *   status      int32 [1] status word (FP2_STATUS_* bits), cleared by fp2_plan.
  *   (the rest is private to the library)
  */

@@ -229,3 +229,25 @@ def test_row_maximum_jump_inside_a_tile(pos):
     res = check_attention(wl, x, run, pl)
     assert res["finite"], res
     assert res["rel_l2"] <= REL_L2_BF16 and res["lse_max_abs"] <= LSE_ABS, res
+
+
+@pytest.mark.parametrize("name", ["ragged_d128", "two_pseudo_tiles", "paged_mix_small"])
+def test_mean_codes_for_the_fp8_correction(name):
+    # e4m3 codes of the block means with one scale per pseudo-tile chunk:
+    # bit-exact against the oracle (the quotient is taken in fp32 on both sides)
+    import torch
+    wl, x = _case(name)
+    run = GpuRun(wl, x).plan()
+    q, k, v = oracle_inputs(x, wl)
+    pl = oracle.plan(q, k, v, wl.seqlens, wl.B, wl.tau)
+    L = run.lay
+    NB, Hkv, d = int(L.num_blocks), wl.Hkv, wl.d
+    buf = run.plan_buf
+    for which, off_c, off_s in [("kbar", L.off_kbar_e4m3, L.off_kbar_scale),
+                                ("vbar", L.off_vbar_e4m3, L.off_vbar_scale)]:
+        codes = buf[off_c:off_c + NB * Hkv * d].view(torch.float8_e4m3fn).float().cpu().numpy()
+        scales = buf[off_s:off_s + NB * Hkv * 4].view(torch.float32).cpu().numpy().reshape(NB, Hkv)
+        ref_c, ref_s = oracle.quantize_means_e4m3(pl[which], wl.seqlens, wl.B)
+        starts = np.isfinite(ref_s[:, 0])
+        assert np.array_equal(scales[starts], ref_s[starts].astype(np.float32))
+        assert np.array_equal(codes.reshape(NB, Hkv, d).astype(np.float64), ref_c)
