@@ -262,7 +262,9 @@ int fp2_prefill(const fp2_problem* problem, const void* plan, size_t plan_bytes,
         if (q_scale || k_scale || v_scale) return FP2_ERR_INVALID_ARG;
     } else if (dtype == FP2_DTYPE_E4M3) {
         if (!q_scale || !k_scale || !v_scale) return FP2_ERR_INVALID_ARG;
-        return FP2_ERR_UNSUPPORTED;
+        if (!aligned(q_scale, 4) || !aligned(k_scale, 4) || !aligned(v_scale, 4))
+            return FP2_ERR_INVALID_ARG;
+        if (L.dims.d != 128) return FP2_ERR_UNSUPPORTED;
     } else {
         return FP2_ERR_INVALID_ARG;
     }

@@ -49,9 +49,10 @@ constexpr int kMmaWarp = 9;     // issues every MMA; owns the tensor memory
 // the 227 KiB of shared memory a CTA may use (at most 8).
 constexpr int kMaxSmem = 232448;
 constexpr int kMaxSlots = 8;
-template <int HD, int BLK>
+template <int HD, int BLK, bool F8>
 constexpr int ring_slots() {
-    const int avail = (kMaxSmem - 512 - 1024 - 2 * kTileM * HD * 2) / (BLK * HD * 2);
+    const int elt = F8 ? 1 : 2;
+    const int avail = (kMaxSmem - 512 - 1024 - 2 * kTileM * HD * elt) / (BLK * HD * elt);
     return avail < kMaxSlots ? avail : kMaxSlots;
 }
 
@@ -61,11 +62,19 @@ constexpr int pow2_ceil(int x) {
     return p;
 }
 
-template <int HD, int BLK>
+// F8: e4m3 Q/K/V (kind::f8f6f4 MMAs, K = 32 per instruction); otherwise bf16
+// (kind::f16, K = 16).  Operand rows are stored as 128-byte swizzle atoms.
+template <int HD, int BLK, bool F8>
 struct Cfg {
-    static constexpr int kSlots = ring_slots<HD, BLK>();
-    static constexpr int kQBytes = kTileM * HD * 2;      // one 128-row query tile (bf16)
-    static constexpr int kSlotBytes = BLK * HD * 2;      // one K or V tile (bf16)
+    static constexpr int kElt = F8 ? 1 : 2;              // bytes per element
+    static constexpr int kRowBytes = HD * kElt;          // one row of Q / K / V
+    static constexpr int kAtoms = kRowBytes / 128;       // 128-byte atoms per row
+    static constexpr int kAtomElems = 128 / kElt;        // elements per atom row
+    static constexpr int kKStep = F8 ? 32 : 16;          // K elements per MMA instruction
+    static_assert(kAtoms >= 1, "rows must span whole 128-byte atoms");
+    static constexpr int kSlots = ring_slots<HD, BLK, F8>();
+    static constexpr int kQBytes = kTileM * kRowBytes;   // one 128-row query tile
+    static constexpr int kSlotBytes = BLK * kRowBytes;   // one K or V tile
     static constexpr int kOffQ = 0;
     static constexpr int kOffSlot = 2 * kQBytes;
     static constexpr int kOffBar = kOffSlot + kSlots * kSlotBytes;
@@ -77,8 +86,17 @@ struct Cfg {
     static constexpr int kColO0 = 2 * BLK;
     static constexpr int kColO1 = 2 * BLK + HD;
     static constexpr int kTmemCols = pow2_ceil(2 * (BLK + HD));
-    static constexpr int kAtomQ = kTileM * 128;          // bytes between 64-column atoms of Q
-    static constexpr int kAtomKV = BLK * 128;            // bytes between 64-column atoms of K / V
+    static constexpr int kAtomQ = kTileM * 128;          // bytes between column atoms of Q
+    static constexpr int kAtomKV = BLK * 128;            // bytes between column atoms of K / V
+    // Each MMA covers kKStep elements = 32 bytes of a row, four per atom;
+    // P is packed 32 bits per TMEM column, so one K-step of P.V is 8 columns.
+    static constexpr uint32_t kIdescS =
+        F8 ? idesc_e4m3(kTileM, BLK, false) : idesc_bf16(kTileM, BLK, false);
+    static constexpr uint32_t kIdescO =
+        F8 ? idesc_e4m3(kTileM, HD, true) : idesc_bf16(kTileM, HD, true);
+    // P <= 2^headroom: bf16 P and fp32 sums allow 2^64; e4m3 P' = P s_V K_row
+    // must stay <= 448, which K_row = 448 / (2^8 max s_V) ensures for 2^8.
+    static constexpr float kHeadroom = F8 ? 8.0f : 64.0f;
 };
 
 struct Bars {
@@ -105,6 +123,14 @@ struct AttnParams {
     int32_t* status;
     uint16_t* o;
     float* lse;
+    // FP8 only: per-(block, head) scales of Q, K, V; per-chunk scales of the
+    // e4m3 block means; largest V scale per (sequence, kv-head)
+    const float* q_scale;
+    const float* k_scale;
+    const float* v_scale;
+    const float* kbar_scale;
+    const float* vbar_scale;
+    const float* vmax;
     uint32_t flags;
     int n_mtiles;   // 128-row query tiles per row = G * B / 128
     int n_pairs;    // work items per row = ceil(n_mtiles / 2)
@@ -234,14 +260,14 @@ __device__ __forceinline__ uint32_t col_bits(int kind, int tok, const TileWalk<B
 // producer (warp 8, one lane)
 // ---------------------------------------------------------------------------
 
-template <int HD, int BLK>
+template <int HD, int BLK, bool F8>
 __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUtensorMap* tm_q,
                          const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                          const CUtensorMap* tm_kbar, const CUtensorMap* tm_vbar) {
-    using C = Cfg<HD, BLK>;
+    using C = Cfg<HD, BLK, F8>;
     const Dims& D = P.D;
     uint32_t qcnt[2] = {0, 0}, qloaded[2] = {0, 0};
-    uint32_t ld = 0;                 // K/V loads issued (slot = ld % 3)
+    uint32_t ld = 0;                 // K/V loads issued (slot = ld % kSlots)
     constexpr int kSlots = C::kSlots;
     uint32_t issued[kMaxSlots] = {0, 0, 0, 0, 0, 0, 0, 0};
     const bool paged = D.page_size != 0;
@@ -260,9 +286,9 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
             for (int ht = 0; ht < kTileM / BLK; ++ht) {
                 const int hl = (kTileM * mt) / BLK + ht;
 #pragma unroll
-                for (int a = 0; a < HD / 64; ++a)
-                    tma_load_3d(qdst + a * C::kAtomQ + ht * BLK * 128, tm_q, &B.q_full[m], 64 * a,
-                                it.g * D.G + hl, it.tok0 + it.i * BLK);
+                for (int a = 0; a < C::kAtoms; ++a)
+                    tma_load_3d(qdst + a * C::kAtomQ + ht * BLK * 128, tm_q, &B.q_full[m],
+                                C::kAtomElems * a, it.g * D.G + hl, it.tok0 + it.i * BLK);
             }
         }
         TileWalk<BLK> walk;
@@ -281,13 +307,15 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
                 if (kind == kPseudo) {
                     const CUtensorMap* tm = kv == 0 ? tm_kbar : tm_vbar;
 #pragma unroll
-                    for (int a = 0; a < HD / 64; ++a)
-                        tma_load_3d(dst + a * C::kAtomKV, tm, bar, 64 * a, it.g, it.b0 + j * BLK);
+                    for (int a = 0; a < C::kAtoms; ++a)
+                        tma_load_3d(dst + a * C::kAtomKV, tm, bar, C::kAtomElems * a, it.g,
+                                    it.b0 + j * BLK);
                 } else if (!paged) {
                     const CUtensorMap* tm = kv == 0 ? tm_k : tm_v;
 #pragma unroll
-                    for (int a = 0; a < HD / 64; ++a)
-                        tma_load_3d(dst + a * C::kAtomKV, tm, bar, 64 * a, it.g, it.tok0 + j * BLK);
+                    for (int a = 0; a < C::kAtoms; ++a)
+                        tma_load_3d(dst + a * C::kAtomKV, tm, bar, C::kAtomElems * a, it.g,
+                                    it.tok0 + j * BLK);
                 } else {
                     const CUtensorMap* tm = kv == 0 ? tm_k : tm_v;
                     const int n_pages_s = (it.L + 63) / 64;
@@ -301,9 +329,9 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
                             else atomicOr(P.status, (int32_t)FP2_STATUS_BAD_PAGE);
                         }
 #pragma unroll
-                        for (int a = 0; a < HD / 64; ++a)
-                            tma_load_4d(dst + a * C::kAtomKV + pg * 64 * 128, tm, bar, 64 * a, it.g,
-                                        0, id);
+                        for (int a = 0; a < C::kAtoms; ++a)
+                            tma_load_4d(dst + a * C::kAtomKV + pg * 64 * 128, tm, bar,
+                                        C::kAtomElems * a, it.g, 0, id);
                     }
                 }
             }
@@ -330,25 +358,29 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) {
     return d + static_cast<uint64_t>(bytes >> 4);
 }
 
-template <int HD, int BLK>
+template <int HD, int BLK, bool F8>
 __device__ __forceinline__ void issue_s(uint32_t tmem_s, uint64_t q_desc, uint64_t k_desc) {
-    using C = Cfg<HD, BLK>;
-    constexpr uint32_t idesc = idesc_bf16(kTileM, BLK, false);
+    using C = Cfg<HD, BLK, F8>;
 #pragma unroll
-    for (int kk = 0; kk < HD / 16; ++kk) {
-        umma_f16(tmem_s, desc_add(q_desc, (kk / 4) * C::kAtomQ + (kk % 4) * 32),
-                 desc_add(k_desc, (kk / 4) * C::kAtomKV + (kk % 4) * 32), idesc, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < HD / C::kKStep; ++kk) {
+        const uint64_t a = desc_add(q_desc, (kk / 4) * C::kAtomQ + (kk % 4) * 32);
+        const uint64_t b = desc_add(k_desc, (kk / 4) * C::kAtomKV + (kk % 4) * 32);
+        if (F8) umma_f8(tmem_s, a, b, C::kIdescS, kk > 0 ? 1u : 0u);
+        else umma_f16(tmem_s, a, b, C::kIdescS, kk > 0 ? 1u : 0u);
     }
 }
 
-template <int HD, int BLK>
+template <int HD, int BLK, bool F8>
 __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint64_t v_desc,
                                          bool accumulate) {
-    constexpr uint32_t idesc = idesc_bf16(kTileM, HD, true);
+    using C = Cfg<HD, BLK, F8>;
 #pragma unroll
-    for (int kk = 0; kk < BLK / 16; ++kk)
-        umma_f16_ts(tmem_o, tmem_p + kk * 8, desc_add(v_desc, kk * 16 * 128), idesc,
-                    (accumulate || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < BLK / C::kKStep; ++kk) {
+        const uint64_t b = desc_add(v_desc, kk * C::kKStep * 128);
+        const uint32_t acc = (accumulate || kk > 0) ? 1u : 0u;
+        if (F8) umma_f8_ts(tmem_o, tmem_p + kk * 8, b, C::kIdescO, acc);
+        else umma_f16_ts(tmem_o, tmem_p + kk * 8, b, C::kIdescO, acc);
+    }
 }
 
 struct PrevTile {
@@ -360,9 +392,9 @@ struct PrevTile {
 // issuing thread ~50 cycles, about its 64-cycle execution time, so a single
 // thread issues every MMA in the order S0(n), P1(n-1).V, S1(n), P0(n).V
 // that keeps the two query tiles' chains interleaved.
-template <int HD, int BLK>
+template <int HD, int BLK, bool F8>
 __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
-    using C = Cfg<HD, BLK>;
+    using C = Cfg<HD, BLK, F8>;
     constexpr int kSlots = C::kSlots;
     const uint32_t tb = B.tmem_base;
     const uint32_t s_base = smem_u32(smem);
@@ -382,7 +414,7 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
         ++pcnt[1];
         if (pt.first && !mbar_wait(&B.o_free[1], (ocnt[1] & 1) ^ 1, &B.abort, P.status)) return false;
         tc_fence_after();
-        issue_pv<HD, BLK>(t_o[1], t_s[1], desc_add(v_desc0, pt.vslot * C::kSlotBytes), !pt.first);
+        issue_pv<HD, BLK, F8>(t_o[1], t_s[1], desc_add(v_desc0, pt.vslot * C::kSlotBytes), !pt.first);
         umma_commit(&B.kv_empty[pt.vslot]);
         if (pt.last) {
             umma_commit(&B.o_full[1]);
@@ -414,7 +446,7 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
             }
             if (!mbar_wait(&B.kv_full[ks], kuse & 1, &B.abort, P.status)) goto drain;
             tc_fence_after();
-            issue_s<HD, BLK>(t_s[0], q_desc[0], kd);
+            issue_s<HD, BLK, F8>(t_s[0], q_desc[0], kd);
             umma_commit(&B.s_full[0]);
             if (!it.has_m1) {
                 umma_commit(&B.kv_empty[ks]);
@@ -431,7 +463,7 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
                     ++qcnt[1];
                 }
                 tc_fence_after();
-                issue_s<HD, BLK>(t_s[1], q_desc[1], kd);
+                issue_s<HD, BLK, F8>(t_s[1], q_desc[1], kd);
                 umma_commit(&B.s_full[1]);
                 umma_commit(&B.kv_empty[ks]);
                 if (last) {
@@ -445,7 +477,7 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
             ++pcnt[0];
             if (first && !mbar_wait(&B.o_free[0], (ocnt[0] & 1) ^ 1, &B.abort, P.status)) goto drain;
             tc_fence_after();
-            issue_pv<HD, BLK>(t_o[0], t_s[0], vd, !first);
+            issue_pv<HD, BLK, F8>(t_o[0], t_s[0], vd, !first);
             if (!it.has_m1) umma_commit(&B.kv_empty[vs]);
             if (last) {
                 umma_commit(&B.o_full[0]);
@@ -468,36 +500,43 @@ __device__ __forceinline__ uint32_t chunk_bits(int kind, int tok, const TileWalk
     return MASKED ? col_bits(kind, tok, walk, j, c32) : 0xFFFFFFFFu;
 }
 
-// exp2 headroom of the running row maximum: P = 2^(x - m_ref) may reach
-// 2^kHeadroom before the reference is moved (bf16 P, fp32 row sums and fp32
-// O accumulators stay far from overflow).
-constexpr float kHeadroom = 64.0f;
-
-// 32 columns of P = 2^(s * scale + shift) as 16 packed bf16 pairs, written
-// into tensor memory over the first half of the 32 S columns just read
-// (P of keys 2c and 2c+1 in column c): the A operand of the P.V MMA.
-template <bool MASKED>
+// 32 columns of P = 2^(s * scale + shift), written into tensor memory over
+// the first part of the 32 S columns just read: the A operand of the P.V MMA.
+//   bf16: 16 packed pairs (keys 2c, 2c+1 in column c), columns [t_p, t_p+16).
+//   e4m3: P' = P * pfac packed four per column, columns [t_p, t_p+8).
+// The fp32 row sum accumulates the unscaled P.
+template <bool MASKED, bool F8>
 __device__ __forceinline__ void p32(const uint32_t (&r)[32], uint32_t vb, uint32_t t_p,
-                                    uint64_t scale2, uint64_t shift2, uint64_t& sum2) {
+                                    uint64_t scale2, uint64_t shift2, uint64_t& sum2, float pfac) {
+    float p[32];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int e = 0; e < 32; e += 2) {
+        float s0 = __uint_as_float(r[e]), s1 = __uint_as_float(r[e + 1]);
+        if (MASKED) {
+            s0 = ((vb >> e) & 1u) ? s0 : -INFINITY;
+            s1 = ((vb >> (e + 1)) & 1u) ? s1 : -INFINITY;
+        }
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(s0, s1), scale2, shift2), x0, x1);
+        p[e] = ex2_approx(x0);
+        p[e + 1] = ex2_approx(x1);
+        sum2 = f2_add(sum2, f2_pack(p[e], p[e + 1]));
+    }
+    if (F8) {
         uint32_t packed[8];
 #pragma unroll
-        for (int e2 = 0; e2 < 8; ++e2) {
-            const int e = 16 * h + 2 * e2;
-            float s0 = __uint_as_float(r[e]), s1 = __uint_as_float(r[e + 1]);
-            if (MASKED) {
-                s0 = ((vb >> e) & 1u) ? s0 : -INFINITY;
-                s1 = ((vb >> (e + 1)) & 1u) ? s1 : -INFINITY;
-            }
-            float x0, x1, p0, p1;
-            f2_unpack(f2_fma(f2_pack(s0, s1), scale2, shift2), x0, x1);
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-            sum2 = f2_add(sum2, f2_pack(p0, p1));
-            packed[e2] = pack_bf16x2(p0, p1);
+        for (int q = 0; q < 8; ++q)
+            packed[q] = pack_e4m3x4(p[4 * q] * pfac, p[4 * q + 1] * pfac, p[4 * q + 2] * pfac,
+                                    p[4 * q + 3] * pfac);
+        tmem_st8(t_p, packed);
+    } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t packed[8];
+#pragma unroll
+            for (int e2 = 0; e2 < 8; ++e2) packed[e2] = pack_bf16x2(p[16 * h + 2 * e2], p[16 * h + 2 * e2 + 1]);
+            tmem_st8(t_p + 8 * h, packed);
         }
-        tmem_st8(t_p + 8 * h, packed);
     }
 }
 
@@ -535,9 +574,9 @@ struct RowState {
 // written for it (cols [t_p0, t_p0 + n_pcols)) are scaled by 2^(m_ref - m_new).
 // Warp-collective (tensor memory accesses); lanes whose reference does not
 // move use the factor 1.
-template <int HD>
+template <int HD, bool F8>
 __device__ __forceinline__ void move_reference(RowState& st, float m_new, uint64_t& sum2, uint32_t t_p0,
-                                            int n_pcols) {
+                                               int n_pcols) {
     const float alpha = m_new > st.m_ref ? ex2_approx(st.m_ref - m_new) : 1.0f;
     if (m_new > st.m_ref) st.m_ref = m_new;
     st.l *= alpha;
@@ -560,9 +599,16 @@ __device__ __forceinline__ void move_reference(RowState& st, float m_new, uint64
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-            const float lo = __uint_as_float(r[e] << 16) * alpha;
-            const float hi = __uint_as_float(r[e] & 0xFFFF0000u) * alpha;
-            r[e] = pack_bf16x2(lo, hi);
+            if (F8) {
+                float a0, a1, a2, a3;
+                unpack_e4m3x2(static_cast<uint16_t>(r[e] & 0xFFFFu), a0, a1);
+                unpack_e4m3x2(static_cast<uint16_t>(r[e] >> 16), a2, a3);
+                r[e] = pack_e4m3x4(a0 * alpha, a1 * alpha, a2 * alpha, a3 * alpha);
+            } else {
+                const float lo = __uint_as_float(r[e] << 16) * alpha;
+                const float hi = __uint_as_float(r[e] & 0xFFFF0000u) * alpha;
+                r[e] = pack_bf16x2(lo, hi);
+            }
         }
         tmem_st16(t_p0 + c, r);
     }
@@ -570,17 +616,19 @@ __device__ __forceinline__ void move_reference(RowState& st, float m_new, uint64
 }
 
 // One pass over this thread's row of S: P = 2^(s * scale + bias - m_ref)
-// (zero where masked out) as bf16 pairs in place over S in tensor memory
-// (the P of chunk c goes to columns [16c, 16c+16) while the only loads in
-// flight cover [32(c+1), 32(c+3))).  Before a pair of 32-column chunks is
+// (zero where masked out) in place over S in tensor memory (the P of chunk c
+// goes to columns [16c, 16c+16) for bf16, [8c, 8c+8) for e4m3, while the only
+// loads in flight cover [32(c+1), 32(c+3))).  Before a pair of 32-column chunks is
 // written its maximum is checked against the reference; if it exceeds it by
 // more than the headroom the reference moves first.  Returns the fp32 row
 // sum of the tile.
-template <int BLK, int HD, bool MASKED>
+template <int BLK, int HD, bool MASKED, bool F8>
 __device__ __forceinline__ float tile_softmax(uint32_t t_s, int kind, int tok,
                                               const TileWalk<BLK>& walk, int j, float scale,
-                                              float bias, RowState& st) {
+                                              float bias, float pfac, RowState& st) {
     constexpr int NC = BLK / 32;
+    constexpr int kPColsPerChunk = F8 ? 8 : 16;   // TMEM columns of P per 32 keys
+    constexpr float kHeadroom = Cfg<HD, BLK, F8>::kHeadroom;
     const uint64_t scale2 = f2_pack(scale, scale);
     uint64_t shift2 = f2_pack(bias - st.m_ref, bias - st.m_ref);
     uint64_t sum2 = f2_pack(0.f, 0.f);
@@ -595,12 +643,12 @@ __device__ __forceinline__ float tile_softmax(uint32_t t_s, int kind, int tok,
         const float cm = fmaf(fmaxf(max32<MASKED>(ra, vba), max32<MASKED>(rb, vbb)), scale, bias);
         const bool need = cm > st.m_ref + kHeadroom;
         if (__any_sync(0xffffffffu, need)) {
-            move_reference<HD>(st, need ? cm : st.m_ref, sum2, t_s, 16 * c);
+            move_reference<HD, F8>(st, need ? cm : st.m_ref, sum2, t_s, kPColsPerChunk * c);
             shift2 = f2_pack(bias - st.m_ref, bias - st.m_ref);
         }
-        p32<MASKED>(ra, vba, t_s + 16 * c, scale2, shift2, sum2);
+        p32<MASKED, F8>(ra, vba, t_s + kPColsPerChunk * c, scale2, shift2, sum2, pfac);
         if (c + 2 < NC) tmem_ld32(t_s + 32 * (c + 2), ra);
-        p32<MASKED>(rb, vbb, t_s + 16 * (c + 1), scale2, shift2, sum2);
+        p32<MASKED, F8>(rb, vbb, t_s + kPColsPerChunk * (c + 1), scale2, shift2, sum2, pfac);
         if (c + 3 < NC) tmem_ld32(t_s + 32 * (c + 3), rb);
     }
     tmem_st_wait();
@@ -613,9 +661,9 @@ __device__ __forceinline__ float tile_softmax(uint32_t t_s, int kind, int tok,
 // softmax + correction + epilogue (warps 0-7)
 // ---------------------------------------------------------------------------
 
-template <int HD, int BLK>
+template <int HD, int BLK, bool F8>
 __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
-    using C = Cfg<HD, BLK>;
+    using C = Cfg<HD, BLK, F8>;
     const Dims& D = P.D;
     const int q4 = (threadIdx.x >> 5) & 3;        // TMEM lane quarter of this warp
     const int lane = threadIdx.x & 31;
@@ -638,6 +686,14 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
         const int pos = it.i * BLK + tok;
         const bool row_valid = pos < it.L;
         RowState st{-INFINITY, 0.f, t_o, false};
+        // e4m3: the logit scale folds in the Q scale of this row's block and
+        // head; P' = P s_V K_row with K_row = 448 / (2^8 max s_V) over the
+        // sequence and kv-head (so P' <= 448), undone in the epilogue.
+        float q_sc = 1.f, k_row = 1.f;
+        if (F8) {
+            q_sc = __ldg(P.q_scale + (int64_t)(it.b0 + it.i) * D.Hq + h);
+            k_row = 448.0f / (256.0f * __ldg(P.vmax + (int64_t)it.s * D.Hkv + it.g));
+        }
 
         TileWalk<BLK> walk;
         walk.init(P, it);
@@ -648,9 +704,18 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
             tc_fence_after();
             const bool masked = kind != kFull;
             const float bias = kind == kPseudo ? pseudo_bias : 0.f;
+            float tscale = scale, pfac = 1.f;
+            if (F8) {
+                // per-tile K and V scales: the block's, or a pseudo tile's chunk
+                const int64_t sb = (int64_t)it.b0 + (kind == kPseudo ? (int64_t)BLK * j : j);
+                const float* ks = kind == kPseudo ? P.kbar_scale : P.k_scale;
+                const float* vs = kind == kPseudo ? P.vbar_scale : P.v_scale;
+                tscale = scale * q_sc * __ldg(ks + sb * D.Hkv + it.g);
+                pfac = __ldg(vs + sb * D.Hkv + it.g) * k_row;
+            }
             const float rsum =
-                masked ? tile_softmax<BLK, HD, true>(t_s, kind, tok, walk, j, scale, bias, st)
-                       : tile_softmax<BLK, HD, false>(t_s, kind, tok, walk, j, scale, bias, st);
+                masked ? tile_softmax<BLK, HD, true, F8>(t_s, kind, tok, walk, j, tscale, bias, pfac, st)
+                       : tile_softmax<BLK, HD, false, F8>(t_s, kind, tok, walk, j, tscale, bias, pfac, st);
             st.o_valid = true;
             st.l += rsum;
             tc_fence_before();
@@ -663,7 +728,7 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
         if (!warp_wait(&B.o_full[m], ocnt & 1, B, P.status)) return;
         ++ocnt;
         tc_fence_after();
-        const float inv_l = 1.0f / st.l;
+        const float inv_l = 1.0f / (st.l * k_row);
         uint16_t* orow = P.o + ((int64_t)(it.tok0 + pos) * D.Hq + h) * HD;
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
@@ -689,12 +754,12 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
     }
 }
 
-template <int HD, int BLK>
+template <int HD, int BLK, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 k_attn(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap tm_q,
        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
        const __grid_constant__ CUtensorMap tm_kbar, const __grid_constant__ CUtensorMap tm_vbar) {
-    using C = Cfg<HD, BLK>;
+    using C = Cfg<HD, BLK, F8>;
     if (!*P.meta_valid) return;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -734,11 +799,11 @@ k_attn(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap
     tc_fence_after();
 
     if (warp < 8) {
-        softmax_wg<HD, BLK>(P, B, smem, warp >> 2);
+        softmax_wg<HD, BLK, F8>(P, B, smem, warp >> 2);
     } else if (warp == kProducerWarp) {
-        if (lane == 0) producer<HD, BLK>(P, B, smem, &tm_q, &tm_k, &tm_v, &tm_kbar, &tm_vbar);
+        if (lane == 0) producer<HD, BLK, F8>(P, B, smem, &tm_q, &tm_k, &tm_v, &tm_kbar, &tm_vbar);
     } else {
-        if (lane == 0) mma_issuer<HD, BLK>(P, B, smem);
+        if (lane == 0) mma_issuer<HD, BLK, F8>(P, B, smem);
     }
     __syncwarp();
     tc_fence_before();
@@ -772,53 +837,80 @@ EncodeTiledFn get_encode() {
     return fn;
 }
 
-// bf16 tensor map with 128-byte swizzle; dims innermost first, strides in
-// bytes for dims 1..rank-1.
+// Tensor map (bf16, or one-byte e4m3 codes) with 128-byte swizzle; dims
+// innermost first, strides in bytes for dims 1..rank-1.
 bool make_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
-              const cuuint64_t* strides, const cuuint32_t* box) {
+              const cuuint64_t* strides, const cuuint32_t* box, bool f8) {
     EncodeTiledFn enc = get_encode();
     if (!enc) return false;
     cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+    CUresult r = enc(map, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     rank, const_cast<void*>(base), dims,
                      strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-template <int HD, int BLK>
+// Largest V scale of every (sequence, kv-head): over the blocks' V scales and
+// the chunk scales of the e4m3 V block means (FP8 path).
+__global__ void __launch_bounds__(256) k_vmax(Dims D, PlanPtrs P, const float* __restrict__ v_scale) {
+    if (!*P.meta_valid) return;
+    const int s = blockIdx.x, g = blockIdx.y;
+    const int b0 = P.cu_blocks[s], b1 = P.cu_blocks[s + 1];
+    float mx = 0.f;
+    for (int b = b0 + threadIdx.x; b < b1; b += blockDim.x) {
+        mx = fmaxf(mx, v_scale[(int64_t)b * D.Hkv + g]);
+        if ((b - b0) % D.B == 0) mx = fmaxf(mx, P.vbar_scale[(int64_t)b * D.Hkv + g]);
+    }
+    __shared__ float red[8];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < 8; ++w) mx = fmaxf(mx, red[w]);
+        P.vmax[(int64_t)s * D.Hkv + g] = mx > 0.f ? mx : 1.0f;
+    }
+}
+
+template <int HD, int BLK, bool F8>
 int launch_attn_t(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, const void* q,
-                  const void* k, const void* v, void* o, float* lse, uint32_t flags,
-                  cudaStream_t st) {
-    using C = Cfg<HD, BLK>;
+                  const void* k, const void* v, const float* qs, const float* ks, const float* vs,
+                  void* o, float* lse, uint32_t flags, cudaStream_t st) {
+    using C = Cfg<HD, BLK, F8>;
     const Dims& D = L.dims;
+    const cuuint64_t eb = C::kElt;                         // bytes per element
+    const cuuint32_t ae = C::kAtomElems;                   // elements per 128-byte atom row
     CUtensorMap tq, tk, tv, tkb, tvb;
     {
         cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)D.Hq, (cuuint64_t)D.T};
-        cuuint64_t str[2] = {(cuuint64_t)HD * 2, (cuuint64_t)D.Hq * HD * 2};
-        cuuint32_t box[3] = {64, 1, (cuuint32_t)BLK};
-        if (!make_map(&tq, q, 3, dims, str, box)) return FP2_ERR_CUDA;
+        cuuint64_t str[2] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hq * HD * eb};
+        cuuint32_t box[3] = {ae, 1, (cuuint32_t)BLK};
+        if (!make_map(&tq, q, 3, dims, str, box, F8)) return FP2_ERR_CUDA;
     }
     if (D.page_size == 0) {
         cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)D.Hkv, (cuuint64_t)D.T};
-        cuuint64_t str[2] = {(cuuint64_t)HD * 2, (cuuint64_t)D.Hkv * HD * 2};
-        cuuint32_t box[3] = {64, 1, (cuuint32_t)BLK};
-        if (!make_map(&tk, k, 3, dims, str, box)) return FP2_ERR_CUDA;
-        if (!make_map(&tv, v, 3, dims, str, box)) return FP2_ERR_CUDA;
+        cuuint64_t str[2] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hkv * HD * eb};
+        cuuint32_t box[3] = {ae, 1, (cuuint32_t)BLK};
+        if (!make_map(&tk, k, 3, dims, str, box, F8)) return FP2_ERR_CUDA;
+        if (!make_map(&tv, v, 3, dims, str, box, F8)) return FP2_ERR_CUDA;
     } else {
         cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)D.Hkv, 64, (cuuint64_t)D.num_pages};
-        cuuint64_t str[3] = {(cuuint64_t)HD * 2, (cuuint64_t)D.Hkv * HD * 2,
-                             (cuuint64_t)64 * D.Hkv * HD * 2};
-        cuuint32_t box[4] = {64, 1, 64, 1};
-        if (!make_map(&tk, k, 4, dims, str, box)) return FP2_ERR_CUDA;
-        if (!make_map(&tv, v, 4, dims, str, box)) return FP2_ERR_CUDA;
+        cuuint64_t str[3] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hkv * HD * eb,
+                             (cuuint64_t)64 * D.Hkv * HD * eb};
+        cuuint32_t box[4] = {ae, 1, 64, 1};
+        if (!make_map(&tk, k, 4, dims, str, box, F8)) return FP2_ERR_CUDA;
+        if (!make_map(&tv, v, 4, dims, str, box, F8)) return FP2_ERR_CUDA;
     }
     {
         cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)D.Hkv, (cuuint64_t)D.NB};
-        cuuint64_t str[2] = {(cuuint64_t)HD * 2, (cuuint64_t)D.Hkv * HD * 2};
-        cuuint32_t box[3] = {64, 1, (cuuint32_t)BLK};
-        if (!make_map(&tkb, pp.kbar16, 3, dims, str, box)) return FP2_ERR_CUDA;
-        if (!make_map(&tvb, pp.vbar16, 3, dims, str, box)) return FP2_ERR_CUDA;
+        cuuint64_t str[2] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hkv * HD * eb};
+        cuuint32_t box[3] = {ae, 1, (cuuint32_t)BLK};
+        const void* kb = F8 ? static_cast<const void*>(pp.kbar8) : static_cast<const void*>(pp.kbar16);
+        const void* vb = F8 ? static_cast<const void*>(pp.vbar8) : static_cast<const void*>(pp.vbar16);
+        if (!make_map(&tkb, kb, 3, dims, str, box, F8)) return FP2_ERR_CUDA;
+        if (!make_map(&tvb, vb, 3, dims, str, box, F8)) return FP2_ERR_CUDA;
     }
     AttnParams P;
     P.D = D;
@@ -833,6 +925,12 @@ int launch_attn_t(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, con
     P.status = pp.status;
     P.o = static_cast<uint16_t*>(o);
     P.lse = lse;
+    P.q_scale = qs;
+    P.k_scale = ks;
+    P.v_scale = vs;
+    P.kbar_scale = pp.kbar_scale;
+    P.vbar_scale = pp.vbar_scale;
+    P.vmax = pp.vmax;
     P.flags = flags;
     P.n_mtiles = D.G * BLK / kTileM;
     P.n_pairs = (P.n_mtiles + 1) / 2;
@@ -840,10 +938,11 @@ int launch_attn_t(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, con
     const int sms = sm_count();
     if (sms <= 0) return FP2_ERR_CUDA;
     const int64_t grid = P.n_items < sms ? P.n_items : sms;
-    if (cudaFuncSetAttribute(k_attn<HD, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(k_attn<HD, BLK, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess)
         return FP2_ERR_CUDA;
-    k_attn<HD, BLK><<<(unsigned)grid, kThreads, C::kSmemBytes, st>>>(P, tq, tk, tv, tkb, tvb);
+    if (F8) k_vmax<<<dim3(D.n_seqs, D.Hkv), 256, 0, st>>>(D, pp, vs);
+    k_attn<HD, BLK, F8><<<(unsigned)grid, kThreads, C::kSmemBytes, st>>>(P, tq, tk, tv, tkb, tvb);
     return cudaGetLastError() == cudaSuccess ? FP2_OK : FP2_ERR_CUDA;
 }
 
@@ -852,15 +951,19 @@ int launch_attn_t(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, con
 int launch_prefill(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, const void* q,
                    const void* k, const void* v, const float* qs, const float* ks, const float* vs,
                    int dtype, void* o, float* lse, uint32_t flags, cudaStream_t st) {
-    (void)qs;
-    (void)ks;
-    (void)vs;
-    if (dtype != FP2_DTYPE_BF16) return FP2_ERR_UNSUPPORTED;
     const Dims& D = L.dims;
-    if (D.d == 128 && D.B == 128) return launch_attn_t<128, 128>(L, p, pp, q, k, v, o, lse, flags, st);
-    if (D.d == 128 && D.B == 64) return launch_attn_t<128, 64>(L, p, pp, q, k, v, o, lse, flags, st);
-    if (D.d == 64 && D.B == 128) return launch_attn_t<64, 128>(L, p, pp, q, k, v, o, lse, flags, st);
-    return launch_attn_t<64, 64>(L, p, pp, q, k, v, o, lse, flags, st);
+    if (dtype == FP2_DTYPE_E4M3) {
+        if (D.d != 128) return FP2_ERR_UNSUPPORTED;   // e4m3 rows must fill 128-byte atoms
+        if (D.B == 128) return launch_attn_t<128, 128, true>(L, p, pp, q, k, v, qs, ks, vs, o, lse, flags, st);
+        return launch_attn_t<128, 64, true>(L, p, pp, q, k, v, qs, ks, vs, o, lse, flags, st);
+    }
+    if (D.d == 128 && D.B == 128)
+        return launch_attn_t<128, 128, false>(L, p, pp, q, k, v, qs, ks, vs, o, lse, flags, st);
+    if (D.d == 128 && D.B == 64)
+        return launch_attn_t<128, 64, false>(L, p, pp, q, k, v, qs, ks, vs, o, lse, flags, st);
+    if (D.d == 64 && D.B == 128)
+        return launch_attn_t<64, 128, false>(L, p, pp, q, k, v, qs, ks, vs, o, lse, flags, st);
+    return launch_attn_t<64, 64, false>(L, p, pp, q, k, v, qs, ks, vs, o, lse, flags, st);
 }
 
 }  // namespace fp2

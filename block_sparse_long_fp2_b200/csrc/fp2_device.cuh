@@ -7,6 +7,7 @@
 #include <cstdint>
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "fp2_internal.h"
@@ -182,6 +183,29 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem], kind::f8f6f4 (e4m3 inputs, fp32 accumulate).
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem], kind::f8f6f4: A is read from tensor memory
+// (lane = row of A, each 32-bit column holds four consecutive e4m3 of a row).
+__device__ __forceinline__ void umma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // The mbarrier arrives once every tcgen05 operation this thread issued
 // before has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -288,6 +312,32 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
            | ((b_mn_major ? 1u : 0u) << 16)         // B major
            | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
+}
+
+// Instruction descriptor, kind::f8f6f4 with e4m3 A/B and fp32 D.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool b_mn_major) {
+    return (1u << 4)                                // D format: f32
+           | (0u << 7)                              // A format: e4m3
+           | (0u << 10)                             // B format: e4m3
+           | ((b_mn_major ? 1u : 0u) << 16)         // B major
+           | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
+}
+
+// Four floats -> four e4m3 codes (RNE, saturating), the first in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+    uint16_t lo, hi;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+    return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// Two e4m3 codes (low byte first) -> two floats (exact).
+__device__ __forceinline__ void unpack_e4m3x2(uint16_t v, float& lo, float& hi) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(v));
+    lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+    hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {

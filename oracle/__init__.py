@@ -40,4 +40,5 @@ from .fp2_oracle import (  # noqa: F401
     quantize_e4m3,
     dequantize_e4m3,
     quantize_means_e4m3,
+    dequantize_means_e4m3,
 )

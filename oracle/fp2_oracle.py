@@ -438,3 +438,18 @@ def quantize_means_e4m3(means, seqlens: Sequence[int], B: int):
                 codes[lo:hi, h, :] = e4m3_round(blk / sc)
     return codes, scales
 
+
+def dequantize_means_e4m3(codes, scales, seqlens: Sequence[int], B: int) -> np.ndarray:
+    """codes * the scale of the B-block chunk (of its sequence) each block
+    belongs to; inverse of quantize_means_e4m3 up to e4m3 rounding."""
+    codes = _as64(codes)
+    lay = block_layout(seqlens, B)
+    out = np.zeros_like(codes)
+    for s in range(len(lay["seqlens"])):
+        b0 = int(lay["cu_blocks"][s])
+        nb = int(lay["nb"][s])
+        for c0 in range(0, nb, B):
+            lo, hi = b0 + c0, b0 + min(c0 + B, nb)
+            out[lo:hi] = codes[lo:hi] * np.asarray(scales[lo], dtype=np.float64)[None, :, None]
+    return out
+

@@ -251,3 +251,58 @@ def test_mean_codes_for_the_fp8_correction(name):
         starts = np.isfinite(ref_s[:, 0])
         assert np.array_equal(scales[starts], ref_s[starts].astype(np.float32))
         assert np.array_equal(codes.reshape(NB, Hkv, d).astype(np.float64), ref_c)
+
+
+
+def _fp8_run(wl, x, run):
+    """Quantise q, k, v on the GPU and run the e4m3 prefill; returns the codes,
+    scales and outputs."""
+    import torch
+    NB = int(run.lay.num_blocks)
+    out = {}
+    for which, src, H in [(0, run.q, wl.Hq), (1, run.k, wl.Hkv), (2, run.v, wl.Hkv)]:
+        codes = torch.zeros(src.shape, dtype=torch.uint8, device="cuda")
+        scales = torch.zeros((NB, H), dtype=torch.float32, device="cuda")
+        fb.fp2_quantize_fp8(run.prob, run.plan_buf, src, which, codes, scales)
+        out[which] = (codes, scales)
+    o = torch.full((wl.T, wl.Hq, wl.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((wl.Hq, wl.T), float("nan"), dtype=torch.float32, device="cuda")
+    fb.fp2_prefill(run.prob, run.plan_buf, out[0][0], out[1][0], out[2][0], o, lse,
+                   q_scale=out[0][1], k_scale=out[1][1], v_scale=out[2][1],
+                   dtype=fb.FP2_DTYPE_E4M3)
+    return o.float().cpu().numpy(), lse.cpu().numpy()
+
+
+@pytest.mark.parametrize("name,gen", [("ragged_d128", "normal"), ("ragged_d128", "lowrank"),
+                                      ("B64_d128", "normal"), ("paged_mix_small", "normal")])
+def test_fp8_prefill(name, gen):
+    from fp2_harness import rel_l2, token_rows
+    seqlens, Hq, Hkv, d, B, tau, _, nn, page, pool = SMALL[name]
+    wl = synth.small_workload(seqlens, Hq, Hkv, d, B, tau, seed=700 + len(name), generator=gen,
+                              page_size=page, pool_pages=pool)
+    x = synth.generate(wl)
+    run = GpuRun(wl, x).plan()
+    O8, L8 = _fp8_run(wl, x, run)
+    assert run.status() == (fb.FP2_OK, 0)
+    q, k, v = oracle_inputs(x, wl)
+    pl = oracle.plan(q, k, v, wl.seqlens, wl.B, wl.tau)
+    # the oracle on the dequantised operands the FP8 path computes with
+    dq = [oracle.dequantize_e4m3(*oracle.quantize_e4m3(a, wl.seqlens, wl.B), wl.seqlens, wl.B)
+          for a in (q, k, v)]
+    pl_dq = dict(pl)
+    for key in ("kbar", "vbar"):
+        c, sc = oracle.quantize_means_e4m3(pl[key], wl.seqlens, wl.B)
+        pl_dq[key] = oracle.dequantize_means_e4m3(c, sc, wl.seqlens, wl.B)
+    rows = [(s, i) for s in range(len(wl.seqlens)) for i in range((wl.seqlens[s] + B - 1) // B)]
+    toks, O_dq, L_dq = oracle.attend_rows(dq[0], dq[1], dq[2], pl_dq, rows)
+    _, O_ref, L_ref = oracle.attend_rows(q, k, v, pl, rows)
+    assert np.isfinite(O8[toks]).all() and np.isfinite(L8[:, toks]).all()
+    e_dq = rel_l2(O8[toks], O_dq)
+    e_ref = rel_l2(O8[toks], O_ref)
+    l_dq = float(np.max(np.abs(L8[:, toks] - L_dq)))
+    print(f"fp8 {name}/{gen}: rel-L2 vs dequantised {e_dq:.3e}, vs plain {e_ref:.3e}, "
+          f"LSE vs dequantised {l_dq:.3e}")
+    assert l_dq <= LSE_ABS
+    assert e_dq <= 5e-2
+    if gen == "normal":
+        assert e_ref <= 5e-2

@@ -418,3 +418,6 @@ def test_quantize_means_chunks_follow_sequences():
             deq = codes[lo:hi, h] * scales[lo, h]
             big = np.abs(means[lo:hi, h]) > amax / 64
             assert np.all(np.abs(deq - means[lo:hi, h])[big] <= np.abs(means[lo:hi, h])[big] * 2 ** -4 + 1e-7)
+    deq_all = oracle.dequantize_means_e4m3(codes, scales, seqlens, 2)
+    assert np.array_equal(deq_all[2:4], codes[2:4] * scales[2][None, :, None])
+    assert np.array_equal(deq_all[7], codes[7] * scales[7][:, None])
