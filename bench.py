@@ -185,7 +185,67 @@ def run_ours(args, rank, world, local_rank):
     total_ms = t0.elapsed_time(t1)
     plan_ms = [e[0].elapsed_time(e[1]) for e in ev]
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    launches_per_step = (6 if wl.tau > 0 else 5) + 1
+    # plan: meta, pool, [norms, score], threshold, quant_means, scan, compact; prefill: attn
+    launches_per_step = (8 if wl.tau > 0 else 6) + 1
+
+    # FP8-e4m3 leg: plan (bf16) + direct online quantisation of Q, K, V + e4m3 prefill
+    fp8 = None
+    if not args.no_fp8 and wl.d == 128:
+        NB = int(lay.num_blocks)
+        q8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
+        k8 = torch.empty(k.shape, dtype=torch.uint8, device=dev)
+        v8 = torch.empty(v.shape, dtype=torch.uint8, device=dev)
+        qs = torch.empty((NB, wl.Hq), dtype=torch.float32, device=dev)
+        ks = torch.empty((NB, wl.Hkv), dtype=torch.float32, device=dev)
+        vs = torch.empty((NB, wl.Hkv), dtype=torch.float32, device=dev)
+
+        def step8(evs=None):
+            if evs is not None:
+                evs[0].record(stream)
+            fb.fp2_plan(prob, q, k, v, plan, ws, stream)
+            fb.fp2_quantize_fp8(prob, plan, q, 0, q8, qs, stream)
+            fb.fp2_quantize_fp8(prob, plan, k, 1, k8, ks, stream)
+            fb.fp2_quantize_fp8(prob, plan, v, 2, v8, vs, stream)
+            if evs is not None:
+                evs[1].record(stream)
+            fb.fp2_prefill(prob, plan, q8, k8, v8, o, lse, q_scale=qs, k_scale=ks, v_scale=vs,
+                           dtype=fb.FP2_DTYPE_E4M3, stream=stream)
+            if evs is not None:
+                evs[2].record(stream)
+
+        for _ in range(args.warmup):
+            step8()
+        torch.cuda.synchronize()
+        rc, st = fb.fp2_status_check(plan, stream)
+        if rc != 0:
+            raise RuntimeError(f"device status {st:#x} ({fb.strerror(rc)})")
+        ev8 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for s_ in range(args.steps):
+            step8(ev8[s_])
+        f1.record(stream)
+        torch.cuda.synchronize()
+        t8 = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t8, op=dist.ReduceOp.MAX)
+        ms8 = float(t8[0]) / args.steps
+        attn8 = statistics.mean(e[1].elapsed_time(e[2]) for e in ev8)
+        pre8 = statistics.mean(e[0].elapsed_time(e[1]) for e in ev8)
+        ach8 = nnz * kept_tile_flop(wl) / (attn8 * 1e-3) / 1e12
+        fp8 = {"ms_per_layer": round(ms8, 4), "ms_plan_and_quantize": round(pre8, 4),
+               "ms_attention": round(attn8, 4),
+               "value": round(world * dense_equiv_flop(wl) / (ms8 * 1e-3) / 1e12, 2),
+               "unit": UNIT, "dtype": "e4m3",
+               "roofline": {"bound": "tensor", "achieved": round(ach8, 1),
+                            "peak": round(2 * peaks()["bf16_sustained"], 1), "unit": "TFLOP/s",
+                            "frac": round(ach8 / (2 * peaks()["bf16_sustained"]), 4),
+                            "peak_kind": "e4m3 = 2 x measured bf16 sustained (nominal ratio)"},
+               "gpu_launches": (launches_per_step + 3 + 1) * args.steps}
 
     # end to end through the C ABI with host buffers (pinned), copies inside
     qh = torch.from_numpy(x["q"]).to(torch.bfloat16).pin_memory()
@@ -254,6 +314,7 @@ def run_ours(args, rank, world, local_rank):
                 "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
+        "fp8": fp8,
         "rows": R, "G": G,
     }
     return out, x
@@ -327,6 +388,7 @@ def main():
     ap.add_argument("--workload", default="qwen_128k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-e4m3 leg")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
