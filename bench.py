@@ -14,8 +14,13 @@ of the device time), inputs resident in HBM.  Each rank runs an independent
 layer (weak scaling, no collective on the data path); torch.distributed only
 provides the barrier and the max over ranks.
 
+The line also carries the FP8-e4m3 leg (plan + online quantisation + e4m3
+prefill on the same layer) and the dense baseline (the same kernels with
+tau = 0), each timed the same way.
+
 --impl reference runs the float64 CPU oracle on a bounded sample of the same
 workload (rank 0 only) and prints the same metric for it.
+--sweep prints one line per cell of the L x tau sweep (BF16 and FP8) instead.
 """
 
 from __future__ import annotations
@@ -188,6 +193,60 @@ def run_ours(args, rank, world, local_rank):
     # plan: meta, pool, [norms, score], threshold, quant_means, scan, compact; prefill: attn
     launches_per_step = (8 if wl.tau > 0 else 6) + 1
 
+    # dense baseline: the same kernels on the same inputs with tau = 0 (every
+    # causally visible block kept, no pseudo tiles)
+    dense = None
+    if not args.no_dense and wl.tau > 0:
+        prob0 = fb.Problem(wl.seqlens, cu, wl.Hq, wl.Hkv, wl.d, wl.B, 0.0,
+                           page_size=wl.page_size, page_table=pt,
+                           num_pages=int(x["k_pool"].shape[0]) if wl.page_size else 0)
+        lay0, plan0, ws0 = fb.allocate(prob0, dev)
+
+        def step0(evs=None):
+            if evs is not None:
+                evs[0].record(stream)
+            fb.fp2_plan(prob0, q, k, v, plan0, ws0, stream)
+            if evs is not None:
+                evs[1].record(stream)
+            fb.fp2_prefill(prob0, plan0, q, k, v, o, lse, stream=stream)
+            if evs is not None:
+                evs[2].record(stream)
+
+        for _ in range(args.warmup):
+            step0()
+        torch.cuda.synchronize()
+        rc, st = fb.fp2_status_check(plan0, stream)
+        if rc != 0:
+            raise RuntimeError(f"device status {st:#x} ({fb.strerror(rc)})")
+        nnz0 = int(fb.PlanView(plan0, lay0, wl.Hkv, wl.d).row_ptr[-1].item())
+        ev0 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        d0 = torch.cuda.Event(enable_timing=True)
+        d1 = torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for s_ in range(args.steps):
+            step0(ev0[s_])
+        d1.record(stream)
+        torch.cuda.synchronize()
+        t0d = torch.tensor([d0.elapsed_time(d1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t0d, op=dist.ReduceOp.MAX)
+        ms0 = float(t0d[0]) / args.steps
+        attn0 = statistics.mean(e[1].elapsed_time(e[2]) for e in ev0)
+        plan0_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev0)
+        ach0 = nnz0 * kept_tile_flop(wl) / (attn0 * 1e-3) / 1e12
+        dense = {"tau": 0.0, "ms_per_layer": round(ms0, 4), "ms_plan": round(plan0_ms, 4),
+                 "ms_attention": round(attn0, 4), "nnz": nnz0,
+                 "value": round(world * dense_equiv_flop(wl) / (ms0 * 1e-3) / 1e12, 2),
+                 "unit": UNIT,
+                 "roofline": {"bound": "tensor", "achieved": round(ach0, 1),
+                              "peak": peaks()["bf16_sustained"], "unit": "TFLOP/s",
+                              "frac": round(ach0 / peaks()["bf16_sustained"], 4)},
+                 "gpu_launches": 7 * args.steps}
+        del plan0, ws0
+
     # FP8-e4m3 leg: plan (bf16) + direct online quantisation of Q, K, V + e4m3 prefill
     fp8 = None
     if not args.no_fp8 and wl.d == 128:
@@ -315,6 +374,8 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "fp8": fp8,
+        "dense": dense,
+        "sparse_speedup_vs_dense": (round(dense["ms_per_layer"] / ms_step, 3) if dense else None),
         "rows": R, "G": G,
     }
     return out, x
@@ -380,6 +441,80 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+def run_sweep(args):
+    """Throughput of every cell of the dense-vs-sparse sweep (32 q / 8 kv heads,
+    d 128, block 128, L in 4K..128K, tau in {0, 0.05, 0.2}), BF16 and FP8-e4m3,
+    one JSON line per cell on stdout (not the benchmark line)."""
+    import torch
+    from block_sparse_long_fp2_b200 import binding as fb
+    from block_sparse_long_fp2_b200 import build as fbuild
+
+    fbuild.build()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+    names = sorted((n for n in synth.workloads() if n.startswith("sweep_")),
+                   key=lambda n: (synth.workloads()[n].T, synth.workloads()[n].tau))
+    for name in names:
+        wl = synth.workloads()[name]
+        x = synth.generate(wl)
+        q = torch.from_numpy(x["q"]).to(torch.bfloat16).to(dev)
+        k = torch.from_numpy(x["k"]).to(torch.bfloat16).to(dev)
+        v = torch.from_numpy(x["v"]).to(torch.bfloat16).to(dev)
+        cu = torch.from_numpy(x["cu_seqlens"]).to(dev)
+        prob = fb.Problem(wl.seqlens, cu, wl.Hq, wl.Hkv, wl.d, wl.B, wl.tau)
+        lay, plan, ws = fb.allocate(prob, dev)
+        o = torch.empty((wl.T, wl.Hq, wl.d), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((wl.Hq, wl.T), dtype=torch.float32, device=dev)
+        NB = int(lay.num_blocks)
+        q8, k8, v8 = (torch.empty(t.shape, dtype=torch.uint8, device=dev) for t in (q, k, v))
+        qs = torch.empty((NB, wl.Hq), dtype=torch.float32, device=dev)
+        ks = torch.empty((NB, wl.Hkv), dtype=torch.float32, device=dev)
+        vs = torch.empty((NB, wl.Hkv), dtype=torch.float32, device=dev)
+
+        def bf16_step(ev):
+            ev[0].record(stream)
+            fb.fp2_plan(prob, q, k, v, plan, ws, stream)
+            ev[1].record(stream)
+            fb.fp2_prefill(prob, plan, q, k, v, o, lse, stream=stream)
+            ev[2].record(stream)
+
+        def fp8_step(ev):
+            ev[0].record(stream)
+            fb.fp2_plan(prob, q, k, v, plan, ws, stream)
+            fb.fp2_quantize_fp8(prob, plan, q, 0, q8, qs, stream)
+            fb.fp2_quantize_fp8(prob, plan, k, 1, k8, ks, stream)
+            fb.fp2_quantize_fp8(prob, plan, v, 2, v8, vs, stream)
+            ev[1].record(stream)
+            fb.fp2_prefill(prob, plan, q8, k8, v8, o, lse, q_scale=qs, k_scale=ks, v_scale=vs,
+                           dtype=fb.FP2_DTYPE_E4M3, stream=stream)
+            ev[2].record(stream)
+
+        row = {"workload": name, "L": wl.seqlens[0], "tau": wl.tau}
+        for tag, fn in (("bf16", bf16_step), ("fp8", fp8_step)):
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                   for _ in range(args.warmup + args.steps)]
+            for e in evs:
+                fn(e)
+            torch.cuda.synchronize()
+            rc, st = fb.fp2_status_check(plan, stream)
+            if rc != 0:
+                raise RuntimeError(f"{name}: device status {st:#x}")
+            tim = evs[args.warmup:]
+            ms = statistics.median(e[0].elapsed_time(e[2]) for e in tim)
+            att = statistics.median(e[1].elapsed_time(e[2]) for e in tim)
+            nnz = int(fb.PlanView(plan, lay, wl.Hkv, wl.d).row_ptr[-1].item())
+            peak = pk["bf16_sustained"] * (2 if tag == "fp8" else 1)
+            row[tag] = {"ms_per_layer": round(ms, 4), "ms_attention": round(att, 4),
+                        "dense_equiv_tflops": round(dense_equiv_flop(wl) / (ms * 1e-3) / 1e12, 1),
+                        "tensor_frac": round(nnz * kept_tile_flop(wl) / (att * 1e-3) / 1e12 / peak,
+                                             4)}
+            row["density"] = round(nnz / float(lay.nnz_cap), 4)
+        print(json.dumps(row), flush=True)
+        del q, k, v, o, lse, plan, ws, q8, k8, v8
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -389,6 +524,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-e4m3 leg")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense tau = 0 leg")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one line per L x tau cell of the dense-vs-sparse sweep instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -396,6 +534,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.sweep:
+        run_sweep(args)
+        return
 
     if args.impl == "reference":
         out = run_reference(args, rank, world)

@@ -176,3 +176,84 @@ def check_attention(wl, x, run: GpuRun, pl, rows_si=None, correction=True):
     e_l = float(np.max(np.abs(LSE[:, toks] - L_ref)))
     return {"rel_l2": e_o, "lse_max_abs": e_l, "n_override": len(override),
             "finite": bool(np.isfinite(O[toks]).all() and np.isfinite(LSE[:, toks]).all())}
+
+
+REL_L2_FP8 = 5e-2
+
+
+def fp8_prefill(wl: synth.Workload, run: GpuRun):
+    """Quantises q, k, v on the GPU (fp2_quantize_fp8) and runs the e4m3
+    prefill on run's plan; returns (O, LSE) as float32 host arrays."""
+    import torch
+    NB = int(run.lay.num_blocks)
+    out = {}
+    for which, src, H in [(0, run.q, wl.Hq), (1, run.k, wl.Hkv), (2, run.v, wl.Hkv)]:
+        codes = torch.zeros(src.shape, dtype=torch.uint8, device="cuda")
+        scales = torch.zeros((NB, H), dtype=torch.float32, device="cuda")
+        fb.fp2_quantize_fp8(run.prob, run.plan_buf, src, which, codes, scales)
+        out[which] = (codes, scales)
+    o = torch.full((wl.T, wl.Hq, wl.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((wl.Hq, wl.T), float("nan"), dtype=torch.float32, device="cuda")
+    fb.fp2_prefill(run.prob, run.plan_buf, out[0][0], out[1][0], out[2][0], o, lse,
+                   q_scale=out[0][1], k_scale=out[1][1], v_scale=out[2][1],
+                   dtype=fb.FP2_DTYPE_E4M3)
+    res = (o.float().cpu().numpy(), lse.cpu().numpy())
+    del out, o, lse
+    return res
+
+
+def dequantised_operands(wl: synth.Workload, q, k, v, pl, rows_si):
+    """The operands the FP8 path computes with, from the oracle's own
+    quantiser: K and V whole, Q only on the query blocks `rows_si` (zeros
+    elsewhere), and a copy of the plan with the e4m3 block means of the
+    correction path.  Scales are per (block, head), so each block is
+    quantised on its own as a one-block sequence (same codes, less memory)."""
+    cu = np.concatenate([[0], np.cumsum(wl.seqlens)])
+
+    def dq_block(a, lo, hi, out):
+        c, sc = oracle.quantize_e4m3(np.asarray(a[lo:hi]), [hi - lo], wl.B)
+        out[lo:hi] = oracle.dequantize_e4m3(c, sc, [hi - lo], wl.B)
+
+    q_dq = np.zeros(np.shape(q))
+    k_dq = np.empty(np.shape(k))
+    v_dq = np.empty(np.shape(v))
+    for s, L in enumerate(wl.seqlens):
+        for i in range((L + wl.B - 1) // wl.B):
+            lo, hi = cu[s] + i * wl.B, cu[s] + min((i + 1) * wl.B, L)
+            dq_block(k, lo, hi, k_dq)
+            dq_block(v, lo, hi, v_dq)
+    for s, i in rows_si:
+        lo, hi = cu[s] + i * wl.B, cu[s] + min((i + 1) * wl.B, wl.seqlens[s])
+        dq_block(q, lo, hi, q_dq)
+    pl_dq = dict(pl)
+    for key in ("kbar", "vbar"):
+        c, sc = oracle.quantize_means_e4m3(pl[key], wl.seqlens, wl.B)
+        pl_dq[key] = oracle.dequantize_means_e4m3(c, sc, wl.seqlens, wl.B)
+    return q_dq, k_dq, v_dq, pl_dq
+
+
+def check_fp8(wl, x, run: GpuRun, pl, rows_si, O8, L8):
+    """FP8 O / LSE against the oracle on the dequantised operands (the FP8
+    path's own arithmetic: same codes, float64 math) and against the plain
+    bf16-input oracle (the accuracy cost of e4m3).  The GPU's block lists are
+    used where they differ inside the threshold band."""
+    q, k, v = oracle_inputs(x, wl)
+    gk = run.kept_lists()
+    nb = [(L + wl.B - 1) // wl.B for L in wl.seqlens]
+    cu_b = np.concatenate([[0], np.cumsum(nb)])
+    NB = int(cu_b[-1])
+    override = {}
+    for (s, i) in rows_si:
+        for g in range(wl.Hkv):
+            r = g * NB + int(cu_b[s]) + i
+            if list(pl["kept"][r]) != gk[r]:
+                override[(s, g, i)] = gk[r]
+    q_dq, k_dq, v_dq, pl_dq = dequantised_operands(wl, q, k, v, pl, rows_si)
+    toks, O_dq, L_dq = oracle.attend_rows(q_dq, k_dq, v_dq, pl_dq, rows_si, kept_override=override)
+    del q_dq, k_dq, v_dq
+    _, O_ref, L_ref = oracle.attend_rows(q, k, v, pl, rows_si, kept_override=override)
+    assert np.array_equal(toks, token_rows(wl, rows_si))
+    return {"rel_l2_dq": rel_l2(O8[toks], O_dq), "rel_l2_plain": rel_l2(O8[toks], O_ref),
+            "lse_dq": float(np.max(np.abs(L8[:, toks] - L_dq))),
+            "lse_plain": float(np.max(np.abs(L8[:, toks] - L_ref))),
+            "finite": bool(np.isfinite(O8[toks]).all() and np.isfinite(L8[:, toks]).all())}
