@@ -228,6 +228,13 @@ struct TileWalk {
         kind = kPseudo;
         return true;
     }
+    // Number of tiles of the walk (kept blocks + non-empty pseudo tiles), so a
+    // role that needs no column ids can count tiles without loading them.
+    __device__ __forceinline__ int count() const {
+        int n = n_kept + __popc(pt_bits);
+        for (int p = 32; p < n_pt; ++p) n += has_skip(p) ? 1 : 0;
+        return n;
+    }
     __device__ __forceinline__ bool is_last() const {
         if (t < n_kept) return false;
         int p = pt;
@@ -388,10 +395,28 @@ struct PrevTile {
     int vslot;
 };
 
+// Position in the K/V ring: slot and how many times it has been used before.
+struct RingPos {
+    int slot;
+    uint32_t use;
+};
+template <int kSlots>
+__device__ __forceinline__ RingPos ring_take(RingPos& next) {
+    const RingPos cur = next;
+    if (++next.slot == kSlots) {
+        next.slot = 0;
+        ++next.use;
+    }
+    return cur;
+}
+
 // The MMA issuer (one lane of warp kMmaWarp).  A tcgen05.mma costs its
 // issuing thread ~50 cycles, about its 64-cycle execution time, so a single
 // thread issues every MMA in the order S0(n), P1(n-1).V, S1(n), P0(n).V
-// that keeps the two query tiles' chains interleaved.
+// that keeps the two query tiles' chains interleaved.  The loop is rotated
+// so that S0(n+1) follows P0(n).V directly (the next tile's K is usually long
+// resident): the loop overhead and the wait for P1 fall on the other query
+// tile's chain, which is half a period behind.
 template <int HD, int BLK, bool F8>
 __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
     using C = Cfg<HD, BLK, F8>;
@@ -406,7 +431,7 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
     const uint32_t t_s[2] = {tb + C::kColS0, tb + C::kColS1};
     const uint32_t t_o[2] = {tb + C::kColO0, tb + C::kColO1};
     uint32_t qcnt[2] = {0, 0}, pcnt[2] = {0, 0}, ocnt[2] = {0, 0};
-    uint32_t ld = 0;
+    RingPos ring{0, 0};
     PrevTile prev{false, false, false, false, 0};
 
     auto pv1 = [&](const PrevTile& pt) -> bool {
@@ -422,36 +447,37 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
         }
         return true;
     };
+    // S0 = Q0 K^T of a tile whose K sits in ring slot k
+    auto s0 = [&](const RingPos& k, bool has_m1, bool last) -> bool {
+        if (!mbar_wait(&B.kv_full[k.slot], k.use & 1, &B.abort, P.status)) return false;
+        tc_fence_after();
+        issue_s<HD, BLK, F8>(t_s[0], q_desc[0], desc_add(k_desc0, k.slot * C::kSlotBytes));
+        umma_commit(&B.s_full[0]);
+        if (!has_m1) {
+            umma_commit(&B.kv_empty[k.slot]);
+            if (last) umma_commit(&B.q_empty[0]);
+        }
+        return true;
+    };
 
     for (int64_t w = blockIdx.x; w < P.n_items; w += gridDim.x) {
         const Item it = decode_item(P, w);
-        TileWalk<BLK> walk;
-        walk.init(P, it);
-        int kind, j, n = 0;
-        while (walk.next(kind, j)) {
+        // The issuer needs no column ids, only the tile count: its loop issues no
+        // global loads, which would otherwise hold up its barrier probes.
+        int n_tiles;
+        {
+            TileWalk<BLK> walk;
+            walk.init(P, it);
+            n_tiles = walk.count();
+        }
+        RingPos kp = ring_take<kSlots>(ring);
+        RingPos vp = ring_take<kSlots>(ring);
+        if (!mbar_wait(&B.q_full[0], qcnt[0] & 1, &B.abort, P.status)) goto drain;
+        ++qcnt[0];
+        if (!s0(kp, it.has_m1, n_tiles == 1)) goto drain;
+        for (int n = 0; n < n_tiles; ++n) {
             const bool first = n == 0;
-            const bool last = walk.is_last();
-            const int ks = ld % kSlots;
-            const uint32_t kuse = ld / kSlots;
-            ++ld;
-            const int vs = ld % kSlots;
-            const uint32_t vuse = ld / kSlots;
-            ++ld;
-            const uint64_t kd = desc_add(k_desc0, ks * C::kSlotBytes);
-            const uint64_t vd = desc_add(v_desc0, vs * C::kSlotBytes);
-            // S0 = Q0 K^T
-            if (first) {
-                if (!mbar_wait(&B.q_full[0], qcnt[0] & 1, &B.abort, P.status)) goto drain;
-                ++qcnt[0];
-            }
-            if (!mbar_wait(&B.kv_full[ks], kuse & 1, &B.abort, P.status)) goto drain;
-            tc_fence_after();
-            issue_s<HD, BLK, F8>(t_s[0], q_desc[0], kd);
-            umma_commit(&B.s_full[0]);
-            if (!it.has_m1) {
-                umma_commit(&B.kv_empty[ks]);
-                if (last) umma_commit(&B.q_empty[0]);
-            }
+            const bool last = n == n_tiles - 1;
             // P1.V of the previous tile
             if (prev.valid && prev.has_m1) {
                 if (!pv1(prev)) goto drain;
@@ -463,28 +489,33 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
                     ++qcnt[1];
                 }
                 tc_fence_after();
-                issue_s<HD, BLK, F8>(t_s[1], q_desc[1], kd);
+                issue_s<HD, BLK, F8>(t_s[1], q_desc[1], desc_add(k_desc0, kp.slot * C::kSlotBytes));
                 umma_commit(&B.s_full[1]);
-                umma_commit(&B.kv_empty[ks]);
+                umma_commit(&B.kv_empty[kp.slot]);
                 if (last) {
                     umma_commit(&B.q_empty[0]);
                     umma_commit(&B.q_empty[1]);
                 }
             }
             // P0.V of this tile
-            if (!mbar_wait(&B.kv_full[vs], vuse & 1, &B.abort, P.status)) goto drain;
+            if (!mbar_wait(&B.kv_full[vp.slot], vp.use & 1, &B.abort, P.status)) goto drain;
             if (!mbar_wait(&B.p_full[0], pcnt[0] & 1, &B.abort, P.status)) goto drain;
             ++pcnt[0];
             if (first && !mbar_wait(&B.o_free[0], (ocnt[0] & 1) ^ 1, &B.abort, P.status)) goto drain;
             tc_fence_after();
-            issue_pv<HD, BLK, F8>(t_o[0], t_s[0], vd, !first);
-            if (!it.has_m1) umma_commit(&B.kv_empty[vs]);
+            issue_pv<HD, BLK, F8>(t_o[0], t_s[0], desc_add(v_desc0, vp.slot * C::kSlotBytes), !first);
+            if (!it.has_m1) umma_commit(&B.kv_empty[vp.slot]);
             if (last) {
                 umma_commit(&B.o_full[0]);
                 ++ocnt[0];
             }
-            prev = PrevTile{true, it.has_m1, first, last, vs};
-            ++n;
+            prev = PrevTile{true, it.has_m1, first, last, vp.slot};
+            // S0 of the next tile right away
+            if (!last) {
+                kp = ring_take<kSlots>(ring);
+                vp = ring_take<kSlots>(ring);
+                if (!s0(kp, it.has_m1, n + 1 == n_tiles - 1)) goto drain;
+            }
         }
     }
     if (prev.valid && prev.has_m1) pv1(prev);
@@ -577,6 +608,7 @@ struct RowState {
 template <int HD, bool F8>
 __device__ __forceinline__ void move_reference(RowState& st, float m_new, uint64_t& sum2, uint32_t t_p0,
                                                int n_pcols) {
+    tmem_st_wait();   // the P columns read back below were stored by this thread
     const float alpha = m_new > st.m_ref ? ex2_approx(st.m_ref - m_new) : 1.0f;
     if (m_new > st.m_ref) st.m_ref = m_new;
     st.l *= alpha;
@@ -699,20 +731,21 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
         walk.init(P, it);
         int kind, j, n = 0;
         while (walk.next(kind, j)) {
-            if (!warp_wait(&B.s_full[m], scnt & 1, B, P.status)) return;
-            ++scnt;
-            tc_fence_after();
-            const bool masked = kind != kFull;
-            const float bias = kind == kPseudo ? pseudo_bias : 0.f;
             float tscale = scale, pfac = 1.f;
             if (F8) {
-                // per-tile K and V scales: the block's, or a pseudo tile's chunk
+                // per-tile K and V scales: the block's, or a pseudo tile's chunk;
+                // loaded before the S wait, which hides their latency
                 const int64_t sb = (int64_t)it.b0 + (kind == kPseudo ? (int64_t)BLK * j : j);
                 const float* ks = kind == kPseudo ? P.kbar_scale : P.k_scale;
                 const float* vs = kind == kPseudo ? P.vbar_scale : P.v_scale;
                 tscale = scale * q_sc * __ldg(ks + sb * D.Hkv + it.g);
                 pfac = __ldg(vs + sb * D.Hkv + it.g) * k_row;
             }
+            if (!warp_wait(&B.s_full[m], scnt & 1, B, P.status)) return;
+            ++scnt;
+            tc_fence_after();
+            const bool masked = kind != kFull;
+            const float bias = kind == kPseudo ? pseudo_bias : 0.f;
             const float rsum =
                 masked ? tile_softmax<BLK, HD, true, F8>(t_s, kind, tok, walk, j, tscale, bias, pfac, st)
                        : tile_softmax<BLK, HD, false, F8>(t_s, kind, tok, walk, j, tscale, bias, pfac, st);
