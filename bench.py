@@ -26,6 +26,7 @@ workload (rank 0 only) and prints the same metric for it.
 from __future__ import annotations
 
 import argparse
+import copy
 import json
 import os
 import statistics
@@ -56,6 +57,29 @@ def kept_tile_flop(wl) -> float:
     G heads x B tokens of the row = 4 * d * G * B^2."""
     G = wl.Hq // wl.Hkv
     return 4.0 * wl.d * G * wl.B * wl.B
+
+
+def rank_workload(name: str, rank: int):
+    """The workload a rank runs: the named layer with a rank-dependent seed,
+    so every rank processes an independent layer (weak scaling)."""
+    wl = copy.deepcopy(synth.workloads()[name])
+    wl.seed += 7919 * rank
+    return wl
+
+
+def max_over_ranks(values, world: int, device):
+    """Element-wise maximum of per-rank values (device times) over all ranks."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def whole_job_value(flop_per_rank: float, world: int, ms: float) -> float:
+    """Throughput of the whole job: the work of all ranks over the slowest rank's time."""
+    return world * flop_per_rank / (ms * 1e-3) / 1e12
 
 
 def peaks():
@@ -131,8 +155,7 @@ def run_ours(args, rank, world, local_rank):
     fbuild.build()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = synth.workloads()[args.workload]
-    wl.seed += 7919 * rank            # each rank: an independent layer
+    wl = rank_workload(args.workload, rank)
     x = synth.generate(wl)
     stream = torch.cuda.current_stream()
 
@@ -230,16 +253,13 @@ def run_ours(args, rank, world, local_rank):
             step0(ev0[s_])
         d1.record(stream)
         torch.cuda.synchronize()
-        t0d = torch.tensor([d0.elapsed_time(d1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t0d, op=dist.ReduceOp.MAX)
-        ms0 = float(t0d[0]) / args.steps
+        ms0 = max_over_ranks([d0.elapsed_time(d1)], world, dev)[0] / args.steps
         attn0 = statistics.mean(e[1].elapsed_time(e[2]) for e in ev0)
         plan0_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev0)
         ach0 = nnz0 * kept_tile_flop(wl) / (attn0 * 1e-3) / 1e12
         dense = {"tau": 0.0, "ms_per_layer": round(ms0, 4), "ms_plan": round(plan0_ms, 4),
                  "ms_attention": round(attn0, 4), "nnz": nnz0,
-                 "value": round(world * dense_equiv_flop(wl) / (ms0 * 1e-3) / 1e12, 2),
+                 "value": round(whole_job_value(dense_equiv_flop(wl), world, ms0), 2),
                  "unit": UNIT,
                  "roofline": {"bound": "tensor", "achieved": round(ach0, 1),
                               "peak": peaks()["bf16_sustained"], "unit": "TFLOP/s",
@@ -289,16 +309,13 @@ def run_ours(args, rank, world, local_rank):
             step8(ev8[s_])
         f1.record(stream)
         torch.cuda.synchronize()
-        t8 = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t8, op=dist.ReduceOp.MAX)
-        ms8 = float(t8[0]) / args.steps
+        ms8 = max_over_ranks([f0.elapsed_time(f1)], world, dev)[0] / args.steps
         attn8 = statistics.mean(e[1].elapsed_time(e[2]) for e in ev8)
         pre8 = statistics.mean(e[0].elapsed_time(e[1]) for e in ev8)
         ach8 = nnz * kept_tile_flop(wl) / (attn8 * 1e-3) / 1e12
         fp8 = {"ms_per_layer": round(ms8, 4), "ms_plan_and_quantize": round(pre8, 4),
                "ms_attention": round(attn8, 4),
-               "value": round(world * dense_equiv_flop(wl) / (ms8 * 1e-3) / 1e12, 2),
+               "value": round(whole_job_value(dense_equiv_flop(wl), world, ms8), 2),
                "unit": UNIT, "dtype": "e4m3",
                "roofline": {"bound": "tensor", "achieved": round(ach8, 1),
                             "peak": round(2 * peaks()["bf16_sustained"], 1), "unit": "TFLOP/s",
@@ -331,13 +348,10 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
     # max over ranks
-    vals = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = float(vals[0]), float(vals[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, dev)
     ms_step = total_ms / args.steps
     flop = dense_equiv_flop(wl)
-    value = world * flop / (ms_step * 1e-3) / 1e12
+    value = whole_job_value(flop, world, ms_step)
     pk = peaks()
     attn_avg = statistics.mean(attn_ms)
     plan_avg = statistics.mean(plan_ms)
@@ -368,7 +382,7 @@ def run_ours(args, rank, world, local_rank):
         "planning": {"achieved_gbs": round(plan_bytes / (plan_avg * 1e-3) / 1e9, 1),
                      "peak_gbs": pk["hbm_gbs"],
                      "frac": round(plan_bytes / (plan_avg * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
-        "e2e": {"value": round(world * flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+        "e2e": {"value": round(whole_job_value(flop, world, e2e_ms), 2), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(in_bytes),
                 "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4)},
         "gpu_launches": launches_per_step * args.steps,
@@ -552,7 +566,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     out, x = run_ours(args, rank, world, local_rank)
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         wl = synth.workloads()[args.workload]
         val, el, rows = oracle_sample(wl, x, 20.0)
         out["cpu_baseline"] = {
