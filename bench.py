@@ -21,6 +21,7 @@ tau = 0), each timed the same way.
 --impl reference runs the float64 CPU oracle on a bounded sample of the same
 workload (rank 0 only) and prints the same metric for it.
 --sweep prints one line per cell of the L x tau sweep (BF16 and FP8) instead.
+--correction-curve prints the mean-correction overhead and error vs tau at 64K.
 """
 
 from __future__ import annotations
@@ -455,6 +456,95 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+def run_correction_curve(args):
+    """Mean-correction overhead and accuracy at 64K (one 32 q / 8 kv-head, d 128,
+    B 128 layer; N(0,1) and low-rank generators): for each tau, attention time
+    with and without the correction (BF16 and FP8-e4m3) and the rel-L2 distance
+    of O to the dense (tau = 0) output of the same kernels, with and without it.
+    One JSON line per (generator, tau) on stdout (not the benchmark line)."""
+    import torch
+    from block_sparse_long_fp2_b200 import binding as fb
+    from block_sparse_long_fp2_b200 import build as fbuild
+
+    fbuild.build()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    L, taus = 65536, [0.05, 0.1, 0.2, 0.4]
+    for gen in ("normal", "lowrank"):
+        wl = synth.small_workload([L], 32, 8, 128, 128, 0.0, seed=2024, generator=gen)
+        x = synth.generate(wl)
+        q = torch.from_numpy(x["q"]).to(torch.bfloat16).to(dev)
+        k = torch.from_numpy(x["k"]).to(torch.bfloat16).to(dev)
+        v = torch.from_numpy(x["v"]).to(torch.bfloat16).to(dev)
+        cu = torch.from_numpy(x["cu_seqlens"]).to(dev)
+        o = torch.empty((wl.T, wl.Hq, wl.d), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((wl.Hq, wl.T), dtype=torch.float32, device=dev)
+
+        def plan_for(tau):
+            prob = fb.Problem(wl.seqlens, cu, wl.Hq, wl.Hkv, wl.d, wl.B, tau)
+            lay, plan, ws = fb.allocate(prob, dev)
+            fb.fp2_plan(prob, q, k, v, plan, ws, stream)
+            return prob, lay, plan
+
+        def quantised(prob, plan, NB):
+            out = []
+            for which, src, H in ((0, q, wl.Hq), (1, k, wl.Hkv), (2, v, wl.Hkv)):
+                c = torch.empty(src.shape, dtype=torch.uint8, device=dev)
+                sc = torch.empty((NB, H), dtype=torch.float32, device=dev)
+                fb.fp2_quantize_fp8(prob, plan, src, which, c, sc, stream)
+                out.append((c, sc))
+            return out
+
+        def timed(fn):
+            for _ in range(args.warmup):
+                fn()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / args.steps
+
+        prob0, lay0, plan0 = plan_for(0.0)
+        q80 = quantised(prob0, plan0, int(lay0.num_blocks))
+        fb.fp2_prefill(prob0, plan0, q, k, v, o, lse, stream=stream)
+        dense16 = o.float().clone()
+        fb.fp2_prefill(prob0, plan0, q80[0][0], q80[1][0], q80[2][0], o, lse, q_scale=q80[0][1],
+                       k_scale=q80[1][1], v_scale=q80[2][1], dtype=fb.FP2_DTYPE_E4M3, stream=stream)
+        dense8 = o.float().clone()
+        del plan0
+        for tau in taus:
+            prob, lay, plan = plan_for(tau)
+            q8 = quantised(prob, plan, int(lay.num_blocks))
+            nnz = int(fb.PlanView(plan, lay, wl.Hkv, wl.d).row_ptr[-1].item())
+            row = {"generator": gen, "L": L, "tau": tau, "density": round(nnz / float(lay.nnz_cap), 4)}
+            for tag, dense in (("bf16", dense16), ("fp8", dense8)):
+                for corr in (True, False):
+                    flags = 0 if corr else fb.FP2_NO_CORRECTION
+                    if tag == "bf16":
+                        def fn():
+                            fb.fp2_prefill(prob, plan, q, k, v, o, lse, flags=flags, stream=stream)
+                    else:
+                        def fn():
+                            fb.fp2_prefill(prob, plan, q8[0][0], q8[1][0], q8[2][0], o, lse,
+                                           q_scale=q8[0][1], k_scale=q8[1][1], v_scale=q8[2][1],
+                                           dtype=fb.FP2_DTYPE_E4M3, flags=flags, stream=stream)
+                    ms = timed(fn)
+                    rc, st = fb.fp2_status_check(plan, stream)
+                    if rc != 0:
+                        raise RuntimeError(f"device status {st:#x}")
+                    err = float((o.float() - dense).norm() / dense.norm())
+                    key = f"{tag}_{'corr' if corr else 'nocorr'}"
+                    row[key] = {"ms_attention": round(ms, 4), "rel_l2_to_dense": round(err, 5)}
+                row[f"{tag}_correction_overhead"] = round(
+                    row[f"{tag}_corr"]["ms_attention"] / row[f"{tag}_nocorr"]["ms_attention"] - 1.0, 4)
+            print(json.dumps(row), flush=True)
+            del plan, q8
+            torch.cuda.empty_cache()
+
+
 def run_sweep(args):
     """Throughput of every cell of the dense-vs-sparse sweep (32 q / 8 kv heads,
     d 128, block 128, L in 4K..128K, tau in {0, 0.05, 0.2}), BF16 and FP8-e4m3,
@@ -541,6 +631,8 @@ def main():
     ap.add_argument("--no-dense", action="store_true", help="skip the dense tau = 0 leg")
     ap.add_argument("--sweep", action="store_true",
                     help="one line per L x tau cell of the dense-vs-sparse sweep instead")
+    ap.add_argument("--correction-curve", action="store_true",
+                    help="mean-correction overhead and error vs tau at 64K instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -551,6 +643,9 @@ def main():
 
     if args.sweep:
         run_sweep(args)
+        return
+    if args.correction_curve:
+        run_correction_curve(args)
         return
 
     if args.impl == "reference":

@@ -281,6 +281,25 @@ def test_lse_rises_monotonically_as_tau_falls():
     assert np.max(np.abs(prev - Ld)) <= 1e-12
 
 
+def test_correction_lse_lies_between_uncorrected_and_dense():
+    # Jensen: a skipped block's tokens contribute sum_t e^{q.k_t} >= n e^{q.Kbar},
+    # so the pseudo-token (Figure 4) adds a lower bound of the skipped mass:
+    # LSE without correction <= LSE with correction <= dense LSE, row by row,
+    # for every tau; the first inequality is strict where a block is skipped.
+    wl = synth.small_workload([768, 320], 4, 2, 32, 32, 0.1, seed=37, generator="normal")
+    x = synth.generate(wl)
+    _, Ld = oracle.dense_attention(x["q"], x["k"], x["v"], wl.seqlens)
+    strict = False
+    for tau in [0.05, 0.2, 0.5, 1.0]:
+        pl = oracle.plan(x["q"], x["k"], x["v"], wl.seqlens, wl.B, tau)
+        _, L1 = oracle.attend(x["q"], x["k"], x["v"], pl, correction=True)
+        _, L0 = oracle.attend(x["q"], x["k"], x["v"], pl, correction=False)
+        assert np.all(L0 <= L1 + 1e-12)
+        assert np.all(L1 <= Ld + 1e-12)
+        strict |= bool(np.any(L1 > L0 + 1e-6))
+    assert strict
+
+
 def test_gqa_grouping_matches_replicated_heads():
     seqlens = [40]
     q, k, v = _rand_inputs(seqlens, 4, 2, 6, seed=12, scale=1.5)
