@@ -8,6 +8,8 @@
 #include <mutex>
 #include <vector>
 
+#include <cuda.h>
+
 #include "fp2_internal.h"
 
 namespace fp2 {
@@ -166,6 +168,44 @@ WsPtrs ws_ptrs(const Layout& L, void* ws) {
     w.scores = reinterpret_cast<float*>(b + L.ws_scores);
     w.counts = reinterpret_cast<int32_t*>(b + L.ws_counts);
     return w;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library).
+static EncodeTiledFn get_encode() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_tensor_map(void* map, const void* base, int rank, const uint64_t* dims,
+                     const uint64_t* strides, const uint32_t* box, MapType type) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    const cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
+    const CUtensorMapDataType dt = type == kMapF32  ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                   : type == kMapU8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const CUresult r = enc(static_cast<CUtensorMap*>(map), dt, static_cast<cuuint32_t>(rank),
+                           const_cast<void*>(base), reinterpret_cast<const cuuint64_t*>(dims),
+                           reinterpret_cast<const cuuint64_t*>(strides),
+                           reinterpret_cast<const cuuint32_t*>(box), elem_strides,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
 }
 
 int sm_count() {

@@ -851,40 +851,6 @@ k_attn(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap
 // host side: tensor maps and launch
 // ---------------------------------------------------------------------------
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// Tensor map (bf16, or one-byte e4m3 codes) with 128-byte swizzle; dims
-// innermost first, strides in bytes for dims 1..rank-1.
-bool make_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
-              const cuuint64_t* strides, const cuuint32_t* box, bool f8) {
-    EncodeTiledFn enc = get_encode();
-    if (!enc) return false;
-    cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
-    CUresult r = enc(map, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                     rank, const_cast<void*>(base), dims,
-                     strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 // Largest V scale of every (sequence, kv-head): over the blocks' V scales and
 // the chunk scales of the e4m3 V block means (FP8 path).
 __global__ void __launch_bounds__(256) k_vmax(Dims D, PlanPtrs P, const float* __restrict__ v_scale) {
@@ -920,21 +886,21 @@ int launch_attn_t(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, con
         cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)D.Hq, (cuuint64_t)D.T};
         cuuint64_t str[2] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hq * HD * eb};
         cuuint32_t box[3] = {ae, 1, (cuuint32_t)BLK};
-        if (!make_map(&tq, q, 3, dims, str, box, F8)) return FP2_ERR_CUDA;
+        if (!make_tensor_map(&tq, q, 3, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
     }
     if (D.page_size == 0) {
         cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)D.Hkv, (cuuint64_t)D.T};
         cuuint64_t str[2] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hkv * HD * eb};
         cuuint32_t box[3] = {ae, 1, (cuuint32_t)BLK};
-        if (!make_map(&tk, k, 3, dims, str, box, F8)) return FP2_ERR_CUDA;
-        if (!make_map(&tv, v, 3, dims, str, box, F8)) return FP2_ERR_CUDA;
+        if (!make_tensor_map(&tk, k, 3, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
+        if (!make_tensor_map(&tv, v, 3, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
     } else {
         cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)D.Hkv, 64, (cuuint64_t)D.num_pages};
         cuuint64_t str[3] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hkv * HD * eb,
                              (cuuint64_t)64 * D.Hkv * HD * eb};
         cuuint32_t box[4] = {ae, 1, 64, 1};
-        if (!make_map(&tk, k, 4, dims, str, box, F8)) return FP2_ERR_CUDA;
-        if (!make_map(&tv, v, 4, dims, str, box, F8)) return FP2_ERR_CUDA;
+        if (!make_tensor_map(&tk, k, 4, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
+        if (!make_tensor_map(&tv, v, 4, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
     }
     {
         cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)D.Hkv, (cuuint64_t)D.NB};
@@ -942,8 +908,8 @@ int launch_attn_t(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, con
         cuuint32_t box[3] = {ae, 1, (cuuint32_t)BLK};
         const void* kb = F8 ? static_cast<const void*>(pp.kbar8) : static_cast<const void*>(pp.kbar16);
         const void* vb = F8 ? static_cast<const void*>(pp.vbar8) : static_cast<const void*>(pp.vbar16);
-        if (!make_map(&tkb, kb, 3, dims, str, box, F8)) return FP2_ERR_CUDA;
-        if (!make_map(&tvb, vb, 3, dims, str, box, F8)) return FP2_ERR_CUDA;
+        if (!make_tensor_map(&tkb, kb, 3, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
+        if (!make_tensor_map(&tvb, vb, 3, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
     }
     AttnParams P;
     P.D = D;

@@ -314,6 +314,26 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
            | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
 }
 
+// D[tmem] (+)= A[smem] * B[smem], kind::tf32 (fp32 operands read as tf32, fp32 D).
+__device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Instruction descriptor, kind::tf32 with tf32 A/B (both K-major) and fp32 D.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
+    return (1u << 4)                                // D format: f32
+           | (2u << 7)                              // A format: tf32
+           | (2u << 10)                             // B format: tf32
+           | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
+}
+
 // Instruction descriptor, kind::f8f6f4 with e4m3 A/B and fp32 D.
 __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool b_mn_major) {
     return (1u << 4)                                // D format: f32

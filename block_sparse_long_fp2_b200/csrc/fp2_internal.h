@@ -93,4 +93,11 @@ int launch_prefill(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, co
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
+// A tiled TMA tensor map with 128-byte swizzle over `rank` dimensions
+// (innermost first; strides in bytes for dimensions 1..rank-1).  Element
+// types: bf16, uint8 (e4m3 codes) and fp32.  False when the driver rejects it.
+enum MapType { kMapBF16 = 0, kMapU8 = 1, kMapF32 = 2 };
+bool make_tensor_map(void* map, const void* base, int rank, const uint64_t* dims,
+                     const uint64_t* strides, const uint32_t* box, MapType type);
+
 }  // namespace fp2

@@ -355,6 +355,141 @@ k_score(Dims D, PlanPtrs P, WsPtrs W, int max_chunks) {
     }
 }
 
+// Tensor-core scores: one CTA per (sequence, kv-head, group of 128 / G query
+// blocks, chunk of 128 key blocks) inside the causal triangle.  The 128 query
+// vectors (G heads of each block of the group, the block means rounded to
+// fp32) and the 128 key block means are TMA-loaded as 128-byte-swizzled
+// K-major tiles and multiplied by tcgen05 MMAs of kind::tf32 (M = N = 128,
+// K = 8 per instruction) into tensor memory; four warps read the 128 x 128
+// dot products back, stage them in shared memory, and take the maximum over
+// each block's G heads.  TF32 keeps 10 of fp32's 23 mantissa bits, so a dot
+// product is within 2^-9 |Qbar| |Kbar| (plus fp32 accumulation) of the exact
+// one; the threshold kernel is given that bound with a factor 4 of margin and
+// re-scores in float64 every block it cannot decide.
+constexpr int kScoreTcKeys = 128;     // key blocks per CTA (MMA N)
+constexpr int kScoreTcThreads = 160;  // warps 0-3: epilogue (TMEM lanes); warp 4: TMA + MMA
+constexpr double kScoreTcRelErr = 1.0 / 128.0;   // 4 x (2^-10 + 2^-10 + accumulation)
+
+template <int HD>
+struct ScoreTcCfg {
+    static constexpr int kAtoms = HD * 4 / 128;          // 128-byte atoms per fp32 row
+    static constexpr int kAtomBytes = 128 * 128;         // one atom column of 128 rows
+    static constexpr int kTileBytes = kAtoms * kAtomBytes;
+    static constexpr int kDotsBytes = 128 * (kScoreTcKeys + 1) * 4;
+    static constexpr int kSmem = (2 * kTileBytes > kDotsBytes ? 2 * kTileBytes : kDotsBytes) + 1024;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(kScoreTcThreads)
+k_score_tc(Dims D, PlanPtrs P, WsPtrs W, int max_chunks, const __grid_constant__ CUtensorMap tm_q,
+           const __grid_constant__ CUtensorMap tm_k) {
+    using C = ScoreTcCfg<HD>;
+    if (!*P.meta_valid) return;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    __shared__ uint64_t bar_full, bar_done;
+    __shared__ uint32_t tmem_base;
+    __shared__ volatile int abort_flag;
+
+    const int gi = blockIdx.x / max_chunks;
+    const int jc = blockIdx.x % max_chunks;
+    const int g = blockIdx.y;
+    if (gi >= P.group_cu[D.n_seqs]) return;
+    const int s = P.group_seq[gi];
+    const int RI = D.rows_per_group;
+    const int G = D.G;
+    const int b0 = P.cu_blocks[s];
+    const int nb = P.cu_blocks[s + 1] - b0;
+    const int i0 = (gi - P.group_cu[s]) * RI;
+    const int i1 = min(i0 + RI, nb);
+    const int j0 = jc * kScoreTcKeys;
+    if (j0 > i1 - 1) return;                       // above the causal triangle
+    const int j1 = min(j0 + kScoreTcKeys, i1);
+    const int nrows = i1 - i0;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        mbar_init(&bar_full, 1);
+        mbar_init(&bar_done, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async_smem();
+    }
+    if (warp == 0) tmem_alloc(&tmem_base, kScoreTcKeys);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+    unsigned char* sa = smem;
+    unsigned char* sb = smem + C::kTileBytes;
+
+    if (warp == 4 && lane == 0) {
+        mbar_arrive_expect_tx(&bar_full, C::kAtoms * (G * RI * 128 + kScoreTcKeys * 128));
+#pragma unroll
+        for (int a = 0; a < C::kAtoms; ++a) {
+            tma_load_3d(sa + a * C::kAtomBytes, &tm_q, &bar_full, 32 * a, g * G, b0 + i0);
+            tma_load_3d(sb + a * C::kAtomBytes, &tm_k, &bar_full, 32 * a, g, b0 + j0);
+        }
+        if (mbar_wait(&bar_full, 0, &abort_flag, P.status)) {
+            tc_fence_after();
+            const uint64_t da = smem_desc_sw128(smem_u32(sa), 16, 1024);
+            const uint64_t db = smem_desc_sw128(smem_u32(sb), 16, 1024);
+            constexpr uint32_t idesc = idesc_tf32(128, kScoreTcKeys);
+#pragma unroll
+            for (int kk = 0; kk < HD / 8; ++kk) {
+                const uint32_t off = (kk / 4) * C::kAtomBytes + (kk % 4) * 32;
+                umma_tf32(tmem, da + (off >> 4), db + (off >> 4), idesc, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&bar_done);
+            // the CTA leaves only after its MMAs are done
+            mbar_wait_drain(&bar_done, 0, P.status);
+        }
+    }
+    float* dots = reinterpret_cast<float*>(smem);   // [128][kScoreTcKeys + 1], after the MMAs
+    bool ok = true;
+    if (warp < 4) {
+        ok = mbar_wait(&bar_done, 0, &abort_flag, P.status);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            tc_fence_after();
+            const int row = 32 * warp + lane;
+#pragma unroll 1
+            for (int c = 0; c < kScoreTcKeys / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32 * c, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    dots[row * (kScoreTcKeys + 1) + 32 * c + e] = __uint_as_float(r[e]);
+            }
+        } else {
+            abort_flag = 1;
+        }
+    }
+    __syncthreads();
+    if (!abort_flag) {
+        const float inv_sqrt_d = 1.0f / sqrtf((float)HD);
+        float* scores = W.scores + (int64_t)g * D.tri_total + P.tri_off[s];
+        for (int idx = tid; idx < nrows * kScoreTcKeys; idx += kScoreTcThreads) {
+            const int ri = idx / kScoreTcKeys, jj = idx % kScoreTcKeys;
+            const int i = i0 + ri, j = j0 + jj;
+            if (j <= i && j < j1) {
+                const float* col = dots + (ri * G) * (kScoreTcKeys + 1) + jj;
+                float best = col[0];
+                for (int hl = 1; hl < G; ++hl) best = fmaxf(best, col[hl * (kScoreTcKeys + 1)]);
+                scores[(int64_t)i * (i + 1) / 2 + j] = best * inv_sqrt_d;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kScoreTcKeys);
+    }
+}
+
 // float64 score of key block j for row (b_i, g): max over the group's heads
 // (warp-collective).
 template <int HD>
@@ -377,13 +512,15 @@ __device__ double score64(const Dims& D, const WsPtrs& W, int64_t b_i, int64_t b
 // threshold: one warp per row, decisions equal to the float64 ones
 // ---------------------------------------------------------------------------
 //
-// The float32 score of a block differs from the exact one by at most
-//   e_j = 2 (d + 8) 2^-24 max_h|Qbar_{i,h}| |Kbar_j| / sqrt(d)
-// (rounding of the means to fp32, the fp32 dot product, the scaling; with a
-// factor 2 of margin).  Every block whose score could be the row maximum and
-// every block whose score lies within e_j of tau * m is re-scored in float64.
+// The score of a block differs from the exact one by at most
+//   e_j = rel_err max_h|Qbar_{i,h}| |Kbar_j| / sqrt(d)
+// with rel_err = 2 (d + 8) 2^-24 for the fp32 scoring kernel (rounding of the
+// means to fp32, the fp32 dot product, the scaling; a factor 2 of margin) and
+// kScoreTcRelErr for the tf32 tensor-core one.  Every block whose score could
+// be the row maximum and every block whose score lies within e_j of tau * m is
+// re-scored in float64.
 template <int HD>
-__global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W) {
+__global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W, double rel_err) {
     if (!*P.meta_valid) return;
     const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
@@ -405,7 +542,7 @@ __global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W)
         count = i + 1;
     } else {
         const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
-        const double C = 2.0 * (HD + 8) * (1.0 / 16777216.0) / sqrt((double)HD);
+        const double C = rel_err / sqrt((double)HD);
         const double qn = W.qnorm[bi * D.Hkv + g];
         const float* kn = W.knorm + (int64_t)b0 * D.Hkv + g;
         // pass 1: largest lower bound of any score
@@ -578,18 +715,45 @@ __global__ void k_compact(Dims D, PlanPtrs P) {
     }
 }
 
+#ifndef FP2_SCORE_SIMT
+#define FP2_SCORE_SIMT 0
+#endif
+
 template <int HD>
 int launch_score(const Dims& D, const PlanPtrs& P, const WsPtrs& W, cudaStream_t st) {
+    double rel_err = 2.0 * (HD + 8) / 16777216.0;
     if (D.tau > 0.0) {
-        const size_t smem = sizeof(ScoreSmem<HD>);
-        if (cudaFuncSetAttribute(k_score<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess)
-            return FP2_ERR_CUDA;
-        const int max_chunks = (D.max_nb + kScoreKC - 1) / kScoreKC;
-        dim3 grid((unsigned)((int64_t)D.n_groups_cap * max_chunks), D.Hkv);
-        k_score<HD><<<grid, kScoreThreads, smem, st>>>(D, P, W, max_chunks);
+        if (FP2_SCORE_SIMT) {
+            const size_t smem = sizeof(ScoreSmem<HD>);
+            if (cudaFuncSetAttribute(k_score<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem) != cudaSuccess)
+                return FP2_ERR_CUDA;
+            const int max_chunks = (D.max_nb + kScoreKC - 1) / kScoreKC;
+            dim3 grid((unsigned)((int64_t)D.n_groups_cap * max_chunks), D.Hkv);
+            k_score<HD><<<grid, kScoreThreads, smem, st>>>(D, P, W, max_chunks);
+        } else {
+            // tensor maps over the fp32 query and key block means
+            CUtensorMap tq, tk;
+            const uint64_t qd[3] = {(uint64_t)HD, (uint64_t)D.Hq, (uint64_t)D.NB};
+            const uint64_t qs[2] = {(uint64_t)HD * 4, (uint64_t)D.Hq * HD * 4};
+            const uint32_t qb[3] = {32u, (uint32_t)D.G, (uint32_t)D.rows_per_group};
+            const uint64_t kd[3] = {(uint64_t)HD, (uint64_t)D.Hkv, (uint64_t)D.NB};
+            const uint64_t ks[2] = {(uint64_t)HD * 4, (uint64_t)D.Hkv * HD * 4};
+            const uint32_t kb[3] = {32u, 1u, (uint32_t)kScoreTcKeys};
+            if (!make_tensor_map(&tq, W.qbar32, 3, qd, qs, qb, kMapF32) ||
+                !make_tensor_map(&tk, P.kbar, 3, kd, ks, kb, kMapF32))
+                return FP2_ERR_CUDA;
+            const int smem = ScoreTcCfg<HD>::kSmem;
+            if (cudaFuncSetAttribute(k_score_tc<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     smem) != cudaSuccess)
+                return FP2_ERR_CUDA;
+            const int max_chunks = (D.max_nb + kScoreTcKeys - 1) / kScoreTcKeys;
+            dim3 grid((unsigned)((int64_t)D.n_groups_cap * max_chunks), D.Hkv);
+            k_score_tc<HD><<<grid, kScoreTcThreads, smem, st>>>(D, P, W, max_chunks, tq, tk);
+            rel_err = kScoreTcRelErr;
+        }
     }
-    k_threshold<HD><<<(unsigned)((D.R * 32 + 255) / 256), 256, 0, st>>>(D, P, W);
+    k_threshold<HD><<<(unsigned)((D.R * 32 + 255) / 256), 256, 0, st>>>(D, P, W, rel_err);
     return FP2_OK;
 }
 
