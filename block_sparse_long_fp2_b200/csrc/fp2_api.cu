@@ -55,7 +55,7 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     d.tau = p->tau;
     d.rows_per_group = kScoreQV / G;
 
-    int64_t T = 0, NB = 0, tri = 0, groups = 0;
+    int64_t T = 0, NB = 0, tri = 0, groups = 0, tiles = 0;
     int max_nb = 0, max_pages = 0;
     for (int s = 0; s < p->num_seqs; ++s) {
         const int64_t L = p->seqlens[s];
@@ -65,6 +65,8 @@ int compute_layout(const fp2_problem* p, Layout* out) {
         NB += nb;
         tri += nb * (nb + 1) / 2;
         groups += (nb + d.rows_per_group - 1) / d.rows_per_group;
+        for (int64_t i0 = 0; i0 < nb; i0 += d.rows_per_group)
+            tiles += (std::min<int64_t>(i0 + d.rows_per_group, nb) - 1) / kScoreKeys + 1;
         max_nb = std::max<int>(max_nb, (int)nb);
         max_pages = std::max<int>(max_pages, (int)((L + 63) / 64));
     }
@@ -82,6 +84,7 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     d.max_nb = max_nb;
     d.mask_words = (max_nb + 31) / 32;
     d.n_groups_cap = (int)groups;
+    d.score_tiles = tiles;
 
     Layout& L = *out;
     std::memset(&L, 0, sizeof(L));
@@ -116,12 +119,14 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     L.off_tri_off = c.take(sizeof(int64_t) * (n + 1));
     L.off_group_cu = c.take(sizeof(int32_t) * (n + 1));
     L.off_group_seq = c.take(sizeof(int32_t) * (size_t)std::max<int64_t>(1, groups));
+    L.off_tile_cu = c.take(sizeof(int32_t) * (size_t)(groups + 1));
     L.off_vmax = c.take(sizeof(float) * n * (size_t)d.Hkv);
     pub.plan_bytes = align_up(c.off, 256);
 
     Carver w;
     L.ws_qbar64 = w.take(sizeof(double) * (size_t)NB * d.Hq * d.d);
     L.ws_qbar32 = w.take(sizeof(float) * (size_t)NB * d.Hq * d.d);
+    L.ws_kbar_tf = w.take(sizeof(float) * mean_elems);
     L.ws_kbar64 = w.take(sizeof(double) * mean_elems);
     L.ws_qnorm = w.take(sizeof(float) * (size_t)NB * d.Hkv);
     L.ws_knorm = w.take(sizeof(float) * (size_t)NB * d.Hkv);
@@ -153,6 +158,7 @@ PlanPtrs plan_ptrs(const Layout& L, void* plan) {
     p.tri_off = reinterpret_cast<int64_t*>(b + L.off_tri_off);
     p.group_cu = reinterpret_cast<int32_t*>(b + L.off_group_cu);
     p.group_seq = reinterpret_cast<int32_t*>(b + L.off_group_seq);
+    p.tile_cu = reinterpret_cast<int32_t*>(b + L.off_tile_cu);
     p.vmax = reinterpret_cast<float*>(b + L.off_vmax);
     return p;
 }
@@ -162,6 +168,7 @@ WsPtrs ws_ptrs(const Layout& L, void* ws) {
     WsPtrs w;
     w.qbar64 = reinterpret_cast<double*>(b + L.ws_qbar64);
     w.qbar32 = reinterpret_cast<float*>(b + L.ws_qbar32);
+    w.kbar_tf = reinterpret_cast<float*>(b + L.ws_kbar_tf);
     w.kbar64 = reinterpret_cast<double*>(b + L.ws_kbar64);
     w.qnorm = reinterpret_cast<float*>(b + L.ws_qnorm);
     w.knorm = reinterpret_cast<float*>(b + L.ws_knorm);

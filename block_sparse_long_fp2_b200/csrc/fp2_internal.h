@@ -15,8 +15,10 @@ namespace fp2 {
 
 // Query rows of one PackGQA tile (M of one tcgen05 MMA).
 constexpr int kTileM = 128;
-// Query vectors scored together by one CTA of the scoring kernel.
+// Query vectors scored together by one CTA of the scoring kernel (MMA M).
 constexpr int kScoreQV = 128;
+// Key blocks scored together by one CTA of the scoring kernel (MMA N).
+constexpr int kScoreKeys = 128;
 
 // Derived sizes of one problem (host computed, passed to kernels by value).
 struct Dims {
@@ -28,6 +30,7 @@ struct Dims {
     int rows_per_group;   // query blocks per scoring CTA (kScoreQV / G)
     int n_groups_cap;     // upper bound of scoring row groups per kv-head
     int64_t T, NB, R, tri_total, nnz_cap;
+    int64_t score_tiles;  // (query group, 128-key-block chunk) tiles inside the causal triangles
     double tau;
 };
 
@@ -52,13 +55,15 @@ struct PlanPtrs {
     int64_t* tri_off;      // [n+1] prefix of nb (nb + 1) / 2
     int32_t* group_cu;     // [n+1] prefix of scoring CTAs per sequence
     int32_t* group_seq;    // [n_groups_cap]
+    int32_t* tile_cu;      // [n_groups_cap+1] prefix of scoring tiles per row group
     float* vmax;           // [n, Hkv]  largest V scale of each sequence and kv-head (FP8)
 };
 
 // Device pointers into fp2_plan's workspace.
 struct WsPtrs {
     double* qbar64;   // [NB, Hq, d]
-    float* qbar32;    // [NB, Hq, d]  the same means rounded to fp32
+    float* qbar32;    // [NB, Hq, d]  the same means rounded to tf32 (stored as fp32)
+    float* kbar_tf;   // [NB, Hkv, d] the key means rounded to tf32 (stored as fp32)
     double* kbar64;   // [NB, Hkv, d]
     float* qnorm;     // [NB, Hkv]  max over the group's heads of |Qbar|_2 (rounded up)
     float* knorm;     // [NB, Hkv]  |Kbar|_2 (rounded up)
@@ -71,8 +76,8 @@ struct Layout {
     Dims dims;
     fp2_plan_layout pub;
     size_t off_meta_valid, off_cu_blocks, off_block_seq, off_tri_off, off_group_cu, off_group_seq,
-        off_vmax;
-    size_t ws_qbar64, ws_qbar32, ws_kbar64, ws_qnorm, ws_knorm, ws_scores, ws_counts;
+        off_tile_cu, off_vmax;
+    size_t ws_qbar64, ws_qbar32, ws_kbar_tf, ws_kbar64, ws_qnorm, ws_knorm, ws_scores, ws_counts;
 };
 
 // Validates the problem on the host and computes sizes and offsets.

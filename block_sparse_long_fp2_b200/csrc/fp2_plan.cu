@@ -57,6 +57,17 @@ __global__ void k_meta(Dims D, const int32_t* __restrict__ cu_seqlens,
             P.cu_blocks[D.n_seqs] = (int32_t)nb_sum;
             P.tri_off[D.n_seqs] = tri;
             P.group_cu[D.n_seqs] = (int32_t)grp;
+            // scoring tiles per row group: the 128-key-block chunks its rows reach
+            int64_t tiles = 0;
+            for (int s = 0; s < D.n_seqs; ++s) {
+                const int nb = P.cu_blocks[s + 1] - P.cu_blocks[s];
+                for (int gi = P.group_cu[s], i0 = 0; gi < P.group_cu[s + 1]; ++gi, i0 += D.rows_per_group) {
+                    P.tile_cu[gi] = (int32_t)tiles;
+                    tiles += (min(i0 + D.rows_per_group, nb) - 1) / kScoreKeys + 1;
+                }
+            }
+            P.tile_cu[grp] = (int32_t)tiles;
+            valid = valid && tiles == D.score_tiles;
         }
         *P.status = valid ? 0 : (int32_t)FP2_STATUS_BAD_SEQLENS;
         *P.meta_valid = valid;
@@ -177,9 +188,12 @@ k_pool(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict
         double* dst = W.qbar64 + (b * D.Hq + head) * d + e0;
 #pragma unroll
         for (int e = 0; e < 8; e += 2) *reinterpret_cast<double2*>(dst + e) = make_double2(m[e], m[e + 1]);
+        // the scorer's operand: the means rounded to tf32
         float* d32 = W.qbar32 + (b * D.Hq + head) * d + e0;
-        *reinterpret_cast<float4*>(d32) = make_float4((float)m[0], (float)m[1], (float)m[2], (float)m[3]);
-        *reinterpret_cast<float4*>(d32 + 4) = make_float4((float)m[4], (float)m[5], (float)m[6], (float)m[7]);
+        *reinterpret_cast<float4*>(d32) = make_float4(round_tf32((float)m[0]), round_tf32((float)m[1]),
+                                                      round_tf32((float)m[2]), round_tf32((float)m[3]));
+        *reinterpret_cast<float4*>(d32 + 4) = make_float4(round_tf32((float)m[4]), round_tf32((float)m[5]),
+                                                          round_tf32((float)m[6]), round_tf32((float)m[7]));
     } else {
         const int64_t off = (b * D.Hkv + head) * d + e0;
         float* f32 = (which == 1 ? P.kbar : P.vbar) + off;
@@ -198,6 +212,11 @@ k_pool(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict
             double* dst = W.kbar64 + off;
 #pragma unroll
             for (int e = 0; e < 8; e += 2) *reinterpret_cast<double2*>(dst + e) = make_double2(m[e], m[e + 1]);
+            float* tf = W.kbar_tf + off;
+            *reinterpret_cast<float4*>(tf) = make_float4(round_tf32(f0.x), round_tf32(f0.y),
+                                                         round_tf32(f0.z), round_tf32(f0.w));
+            *reinterpret_cast<float4*>(tf + 4) = make_float4(round_tf32(f1.x), round_tf32(f1.y),
+                                                             round_tf32(f1.z), round_tf32(f1.w));
         }
     }
 }
@@ -246,142 +265,38 @@ __global__ void k_norms(Dims D, PlanPtrs P, WsPtrs W) {
 }
 
 // ---------------------------------------------------------------------------
-// score: float32 scores of every (row, visible key block), triangle-tiled
+// score: block scores of every (row, visible key block) on the tensor cores
 // ---------------------------------------------------------------------------
 
-constexpr int kScoreThreads = 256;
-constexpr int kScoreKC = 64;   // key blocks per tile
-
-template <int HD>
-struct ScoreSmem {
-    float q[kScoreQV][HD + 4];        // query block means of the tile's rows (padded rows)
-    union {
-        float k[kScoreKC][HD + 4];    // key block means of the tile's columns
-        float dots[kScoreQV][kScoreKC + 1];
-    };
-};
-
-// One CTA per (sequence, kv-head, group of rows_per_group query blocks,
-// chunk of kScoreKC key blocks) inside the causal triangle: 128 x 64 dot
-// products of length d from padded shared memory (4 query x 8 key register
-// tile per thread, conflict-free float4 loads), then the max over the
-// group's heads, written to the fp32 score scratch.
-template <int HD>
-__global__ void __launch_bounds__(kScoreThreads)
-k_score(Dims D, PlanPtrs P, WsPtrs W, int max_chunks) {
-    if (!*P.meta_valid) return;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    ScoreSmem<HD>& S = *reinterpret_cast<ScoreSmem<HD>*>(smem_raw);
-
-    const int gi = blockIdx.x / max_chunks;
-    const int jc = blockIdx.x % max_chunks;
-    const int g = blockIdx.y;
-    if (gi >= P.group_cu[D.n_seqs]) return;
-    const int s = P.group_seq[gi];
-    const int RI = D.rows_per_group;
-    const int G = D.G;
-    const int b0 = P.cu_blocks[s];
-    const int nb = P.cu_blocks[s + 1] - b0;
-    const int i0 = (gi - P.group_cu[s]) * RI;
-    const int i1 = min(i0 + RI, nb);
-    const int j0 = jc * kScoreKC;
-    if (j0 > i1 - 1) return;                       // above the causal triangle
-    const int j1 = min(j0 + kScoreKC, i1);
-    const int nrows = i1 - i0;
-    const int nqv = nrows * G;
-    const int tid = threadIdx.x;
-
-    for (int idx = tid; idx < kScoreQV * (HD / 4); idx += kScoreThreads) {
-        const int qv = idx / (HD / 4), e = (idx % (HD / 4)) * 4;
-        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (qv < nqv) {
-            const int ri = qv / G, hl = qv % G;
-            f = *reinterpret_cast<const float4*>(
-                W.qbar32 + ((int64_t)(b0 + i0 + ri) * D.Hq + g * G + hl) * HD + e);
-        }
-        *reinterpret_cast<float4*>(&S.q[qv][e]) = f;
-    }
-    for (int idx = tid; idx < kScoreKC * (HD / 4); idx += kScoreThreads) {
-        const int kv = idx / (HD / 4), e = (idx % (HD / 4)) * 4;
-        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (j0 + kv < j1)
-            f = *reinterpret_cast<const float4*>(P.kbar + ((int64_t)(b0 + j0 + kv) * D.Hkv + g) * HD + e);
-        *reinterpret_cast<float4*>(&S.k[kv][e]) = f;
-    }
-    __syncthreads();
-    // Thread (tq, tk) owns query vectors tq + 32a and key blocks tk + 8c: a warp
-    // reads 4 consecutive query rows and 8 consecutive key rows per load, which
-    // the 4-float row padding spreads over distinct banks.
-    const int tq = tid >> 3;   // 0..31
-    const int tk = tid & 7;    // 0..7
-    float acc[4][8];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
-#pragma unroll 2
-    for (int e = 0; e < HD; e += 4) {
-        float4 qa[4], kb[8];
-#pragma unroll
-        for (int a = 0; a < 4; ++a) qa[a] = *reinterpret_cast<const float4*>(&S.q[tq + 32 * a][e]);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) kb[c] = *reinterpret_cast<const float4*>(&S.k[tk + 8 * c][e]);
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                acc[a][c] = fmaf(qa[a].x, kb[c].x, acc[a][c]);
-                acc[a][c] = fmaf(qa[a].y, kb[c].y, acc[a][c]);
-                acc[a][c] = fmaf(qa[a].z, kb[c].z, acc[a][c]);
-                acc[a][c] = fmaf(qa[a].w, kb[c].w, acc[a][c]);
-            }
-    }
-    __syncthreads();                               // S.k is reused as S.dots
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) S.dots[tq + 32 * a][tk + 8 * c] = acc[a][c];
-    __syncthreads();
-    const float inv_sqrt_d = 1.0f / sqrtf((float)HD);
-    float* scores = W.scores + (int64_t)g * D.tri_total + P.tri_off[s];
-    for (int idx = tid; idx < nrows * kScoreKC; idx += kScoreThreads) {
-        const int ri = idx / kScoreKC, jj = idx % kScoreKC;
-        const int i = i0 + ri, j = j0 + jj;
-        if (j <= i && j < j1) {
-            float best = S.dots[ri * G][jj];
-            for (int hl = 1; hl < G; ++hl) best = fmaxf(best, S.dots[ri * G + hl][jj]);
-            scores[(int64_t)i * (i + 1) / 2 + j] = best * inv_sqrt_d;
-        }
-    }
-}
-
-// Tensor-core scores: one CTA per (sequence, kv-head, group of 128 / G query
-// blocks, chunk of 128 key blocks) inside the causal triangle.  The 128 query
-// vectors (G heads of each block of the group, the block means rounded to
-// fp32) and the 128 key block means are TMA-loaded as 128-byte-swizzled
-// K-major tiles and multiplied by tcgen05 MMAs of kind::tf32 (M = N = 128,
-// K = 8 per instruction) into tensor memory; four warps read the 128 x 128
-// dot products back, stage them in shared memory, and take the maximum over
-// each block's G heads.  TF32 keeps 10 of fp32's 23 mantissa bits, so a dot
-// product is within 2^-9 |Qbar| |Kbar| (plus fp32 accumulation) of the exact
-// one; the threshold kernel is given that bound with a factor 4 of margin and
-// re-scores in float64 every block it cannot decide.
-constexpr int kScoreTcKeys = 128;     // key blocks per CTA (MMA N)
+// Tensor-core scores.  A tile is (sequence, kv-head, group of 128 / G query
+// blocks, chunk of kScoreKeys key blocks) inside the causal triangle; the
+// tiles of all row groups are numbered through tile_cu and a persistent CTA
+// per SM walks them.  Per tile, the 128 query vectors (the G heads of each
+// block of the group) and the 128 key block means, both rounded to tf32, are
+// TMA-loaded as 128-byte-swizzled K-major tiles and multiplied by tcgen05 MMAs
+// of kind::tf32 (M = N = 128, K = 8 per instruction) into tensor memory; four
+// warps read the dot products back, stage them in shared memory, and take the
+// maximum over each block's G heads.  With both operands exact tf32 values
+// the products are exact and a dot product is within
+//   (2 * 2^-11 + d 2^-23) |Qbar| |Kbar|
+// of the one of the float64 means (tf32 rounding of both operands, fp32
+// accumulation); the threshold kernel is given 3 * 2^-10 (a factor of about
+// 2.8 of margin) and re-scores in float64 every block it cannot decide.
 constexpr int kScoreTcThreads = 160;  // warps 0-3: epilogue (TMEM lanes); warp 4: TMA + MMA
-constexpr double kScoreTcRelErr = 1.0 / 128.0;   // 4 x (2^-10 + 2^-10 + accumulation)
+constexpr double kScoreTcRelErr = 3.0 / 1024.0;
 
 template <int HD>
 struct ScoreTcCfg {
     static constexpr int kAtoms = HD * 4 / 128;          // 128-byte atoms per fp32 row
     static constexpr int kAtomBytes = 128 * 128;         // one atom column of 128 rows
     static constexpr int kTileBytes = kAtoms * kAtomBytes;
-    static constexpr int kDotsBytes = 128 * (kScoreTcKeys + 1) * 4;
+    static constexpr int kDotsBytes = 128 * (kScoreKeys + 1) * 4;
     static constexpr int kSmem = (2 * kTileBytes > kDotsBytes ? 2 * kTileBytes : kDotsBytes) + 1024;
 };
 
 template <int HD>
 __global__ void __launch_bounds__(kScoreTcThreads)
-k_score_tc(Dims D, PlanPtrs P, WsPtrs W, int max_chunks, const __grid_constant__ CUtensorMap tm_q,
+k_score_tc(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap tm_q,
            const __grid_constant__ CUtensorMap tm_k) {
     using C = ScoreTcCfg<HD>;
     if (!*P.meta_valid) return;
@@ -391,23 +306,10 @@ k_score_tc(Dims D, PlanPtrs P, WsPtrs W, int max_chunks, const __grid_constant__
     __shared__ uint64_t bar_full, bar_done;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
-
-    const int gi = blockIdx.x / max_chunks;
-    const int jc = blockIdx.x % max_chunks;
-    const int g = blockIdx.y;
-    if (gi >= P.group_cu[D.n_seqs]) return;
-    const int s = P.group_seq[gi];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int RI = D.rows_per_group;
     const int G = D.G;
-    const int b0 = P.cu_blocks[s];
-    const int nb = P.cu_blocks[s + 1] - b0;
-    const int i0 = (gi - P.group_cu[s]) * RI;
-    const int i1 = min(i0 + RI, nb);
-    const int j0 = jc * kScoreTcKeys;
-    if (j0 > i1 - 1) return;                       // above the causal triangle
-    const int j1 = min(j0 + kScoreTcKeys, i1);
-    const int nrows = i1 - i0;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_groups = P.group_cu[D.n_seqs];
 
     if (tid == 0) {
         mbar_init(&bar_full, 1);
@@ -416,77 +318,102 @@ k_score_tc(Dims D, PlanPtrs P, WsPtrs W, int max_chunks, const __grid_constant__
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async_smem();
     }
-    if (warp == 0) tmem_alloc(&tmem_base, kScoreTcKeys);
+    if (warp == 0) tmem_alloc(&tmem_base, kScoreKeys);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
     unsigned char* sa = smem;
     unsigned char* sb = smem + C::kTileBytes;
+    float* dots = reinterpret_cast<float*>(smem);   // [128][kScoreKeys + 1], after the MMAs
+    const float inv_sqrt_d = 1.0f / sqrtf((float)HD);
+    const int64_t n_items = D.score_tiles * D.Hkv;
+    uint32_t phase = 0;
 
-    if (warp == 4 && lane == 0) {
-        mbar_arrive_expect_tx(&bar_full, C::kAtoms * (G * RI * 128 + kScoreTcKeys * 128));
-#pragma unroll
-        for (int a = 0; a < C::kAtoms; ++a) {
-            tma_load_3d(sa + a * C::kAtomBytes, &tm_q, &bar_full, 32 * a, g * G, b0 + i0);
-            tma_load_3d(sb + a * C::kAtomBytes, &tm_k, &bar_full, 32 * a, g, b0 + j0);
+    for (int64_t w = blockIdx.x; w < n_items; w += gridDim.x, phase ^= 1u) {
+        const int g = (int)(w % D.Hkv);
+        const int tile = (int)(w / D.Hkv);
+        // row group of the tile: the last gi with tile_cu[gi] <= tile
+        int lo = 0, hi = n_groups - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (P.tile_cu[mid] <= tile) lo = mid;
+            else hi = mid - 1;
         }
-        if (mbar_wait(&bar_full, 0, &abort_flag, P.status)) {
-            tc_fence_after();
-            const uint64_t da = smem_desc_sw128(smem_u32(sa), 16, 1024);
-            const uint64_t db = smem_desc_sw128(smem_u32(sb), 16, 1024);
-            constexpr uint32_t idesc = idesc_tf32(128, kScoreTcKeys);
+        const int gi = lo;
+        const int jc = tile - P.tile_cu[gi];
+        const int s = P.group_seq[gi];
+        const int b0 = P.cu_blocks[s];
+        const int nb = P.cu_blocks[s + 1] - b0;
+        const int i0 = (gi - P.group_cu[s]) * RI;
+        const int i1 = min(i0 + RI, nb);
+        const int j0 = jc * kScoreKeys;
+        const int j1 = min(j0 + kScoreKeys, i1);
+        const int nrows = i1 - i0;
+
+        if (warp == 4 && lane == 0) {
+            mbar_arrive_expect_tx(&bar_full, C::kAtoms * (G * RI * 128 + kScoreKeys * 128));
 #pragma unroll
-            for (int kk = 0; kk < HD / 8; ++kk) {
-                const uint32_t off = (kk / 4) * C::kAtomBytes + (kk % 4) * 32;
-                umma_tf32(tmem, da + (off >> 4), db + (off >> 4), idesc, kk > 0 ? 1u : 0u);
+            for (int a = 0; a < C::kAtoms; ++a) {
+                tma_load_3d(sa + a * C::kAtomBytes, &tm_q, &bar_full, 32 * a, g * G, b0 + i0);
+                tma_load_3d(sb + a * C::kAtomBytes, &tm_k, &bar_full, 32 * a, g, b0 + j0);
             }
-            umma_commit(&bar_done);
-            // the CTA leaves only after its MMAs are done
-            mbar_wait_drain(&bar_done, 0, P.status);
+            if (mbar_wait(&bar_full, phase, &abort_flag, P.status)) {
+                tc_fence_after();
+                const uint64_t da = smem_desc_sw128(smem_u32(sa), 16, 1024);
+                const uint64_t db = smem_desc_sw128(smem_u32(sb), 16, 1024);
+                constexpr uint32_t idesc = idesc_tf32(128, kScoreKeys);
+#pragma unroll
+                for (int kk = 0; kk < HD / 8; ++kk) {
+                    const uint32_t off = (kk / 4) * C::kAtomBytes + (kk % 4) * 32;
+                    umma_tf32(tmem, da + (off >> 4), db + (off >> 4), idesc, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&bar_done);
+            } else {
+                // the copies may still land: wait for them before leaving
+                mbar_wait_drain(&bar_full, phase, P.status);
+            }
         }
-    }
-    float* dots = reinterpret_cast<float*>(smem);   // [128][kScoreTcKeys + 1], after the MMAs
-    bool ok = true;
-    if (warp < 4) {
-        ok = mbar_wait(&bar_done, 0, &abort_flag, P.status);
-        ok = __all_sync(0xffffffffu, ok);
-        if (ok) {
-            tc_fence_after();
-            const int row = 32 * warp + lane;
+        if (warp < 4) {
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_done, phase, &abort_flag, P.status));
+            if (ok) {
+                tc_fence_after();
+                const int row = 32 * warp + lane;
 #pragma unroll 1
-            for (int c = 0; c < kScoreTcKeys / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32 * c, r);
-                tmem_ld_wait();
+                for (int c = 0; c < kScoreKeys / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32 * c, r);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    dots[row * (kScoreTcKeys + 1) + 32 * c + e] = __uint_as_float(r[e]);
+                    for (int e = 0; e < 32; ++e)
+                        dots[row * (kScoreKeys + 1) + 32 * c + e] = __uint_as_float(r[e]);
+                }
+            } else {
+                abort_flag = 1;
             }
-        } else {
-            abort_flag = 1;
         }
-    }
-    __syncthreads();
-    if (!abort_flag) {
-        const float inv_sqrt_d = 1.0f / sqrtf((float)HD);
+        tc_fence_before();
+        __syncthreads();
+        if (abort_flag) break;
         float* scores = W.scores + (int64_t)g * D.tri_total + P.tri_off[s];
-        for (int idx = tid; idx < nrows * kScoreTcKeys; idx += kScoreTcThreads) {
-            const int ri = idx / kScoreTcKeys, jj = idx % kScoreTcKeys;
+        for (int idx = tid; idx < nrows * kScoreKeys; idx += kScoreTcThreads) {
+            const int ri = idx / kScoreKeys, jj = idx % kScoreKeys;
             const int i = i0 + ri, j = j0 + jj;
             if (j <= i && j < j1) {
-                const float* col = dots + (ri * G) * (kScoreTcKeys + 1) + jj;
+                const float* col = dots + (ri * G) * (kScoreKeys + 1) + jj;
                 float best = col[0];
-                for (int hl = 1; hl < G; ++hl) best = fmaxf(best, col[hl * (kScoreTcKeys + 1)]);
+                for (int hl = 1; hl < G; ++hl) best = fmaxf(best, col[hl * (kScoreKeys + 1)]);
                 scores[(int64_t)i * (i + 1) / 2 + j] = best * inv_sqrt_d;
             }
         }
+        __syncthreads();   // the staged dots are read before the next tile's copies land
+        tc_fence_after();
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kScoreTcKeys);
+        tmem_dealloc(tmem, kScoreKeys);
     }
 }
 
@@ -514,11 +441,9 @@ __device__ double score64(const Dims& D, const WsPtrs& W, int64_t b_i, int64_t b
 //
 // The score of a block differs from the exact one by at most
 //   e_j = rel_err max_h|Qbar_{i,h}| |Kbar_j| / sqrt(d)
-// with rel_err = 2 (d + 8) 2^-24 for the fp32 scoring kernel (rounding of the
-// means to fp32, the fp32 dot product, the scaling; a factor 2 of margin) and
-// kScoreTcRelErr for the tf32 tensor-core one.  Every block whose score could
-// be the row maximum and every block whose score lies within e_j of tau * m is
-// re-scored in float64.
+// with rel_err the scoring kernel's bound (kScoreTcRelErr).  Every block whose
+// score could be the row maximum and every block whose score lies within e_j of
+// tau * m is re-scored in float64.
 template <int HD>
 __global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W, double rel_err) {
     if (!*P.meta_valid) return;
@@ -715,45 +640,29 @@ __global__ void k_compact(Dims D, PlanPtrs P) {
     }
 }
 
-#ifndef FP2_SCORE_SIMT
-#define FP2_SCORE_SIMT 0
-#endif
-
 template <int HD>
 int launch_score(const Dims& D, const PlanPtrs& P, const WsPtrs& W, cudaStream_t st) {
-    double rel_err = 2.0 * (HD + 8) / 16777216.0;
     if (D.tau > 0.0) {
-        if (FP2_SCORE_SIMT) {
-            const size_t smem = sizeof(ScoreSmem<HD>);
-            if (cudaFuncSetAttribute(k_score<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)smem) != cudaSuccess)
-                return FP2_ERR_CUDA;
-            const int max_chunks = (D.max_nb + kScoreKC - 1) / kScoreKC;
-            dim3 grid((unsigned)((int64_t)D.n_groups_cap * max_chunks), D.Hkv);
-            k_score<HD><<<grid, kScoreThreads, smem, st>>>(D, P, W, max_chunks);
-        } else {
-            // tensor maps over the fp32 query and key block means
-            CUtensorMap tq, tk;
-            const uint64_t qd[3] = {(uint64_t)HD, (uint64_t)D.Hq, (uint64_t)D.NB};
-            const uint64_t qs[2] = {(uint64_t)HD * 4, (uint64_t)D.Hq * HD * 4};
-            const uint32_t qb[3] = {32u, (uint32_t)D.G, (uint32_t)D.rows_per_group};
-            const uint64_t kd[3] = {(uint64_t)HD, (uint64_t)D.Hkv, (uint64_t)D.NB};
-            const uint64_t ks[2] = {(uint64_t)HD * 4, (uint64_t)D.Hkv * HD * 4};
-            const uint32_t kb[3] = {32u, 1u, (uint32_t)kScoreTcKeys};
-            if (!make_tensor_map(&tq, W.qbar32, 3, qd, qs, qb, kMapF32) ||
-                !make_tensor_map(&tk, P.kbar, 3, kd, ks, kb, kMapF32))
-                return FP2_ERR_CUDA;
-            const int smem = ScoreTcCfg<HD>::kSmem;
-            if (cudaFuncSetAttribute(k_score_tc<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     smem) != cudaSuccess)
-                return FP2_ERR_CUDA;
-            const int max_chunks = (D.max_nb + kScoreTcKeys - 1) / kScoreTcKeys;
-            dim3 grid((unsigned)((int64_t)D.n_groups_cap * max_chunks), D.Hkv);
-            k_score_tc<HD><<<grid, kScoreTcThreads, smem, st>>>(D, P, W, max_chunks, tq, tk);
-            rel_err = kScoreTcRelErr;
-        }
+        // tensor maps over the tf32-rounded query and key block means
+        CUtensorMap tq, tk;
+        const uint64_t qd[3] = {(uint64_t)HD, (uint64_t)D.Hq, (uint64_t)D.NB};
+        const uint64_t qs[2] = {(uint64_t)HD * 4, (uint64_t)D.Hq * HD * 4};
+        const uint32_t qb[3] = {32u, (uint32_t)D.G, (uint32_t)D.rows_per_group};
+        const uint64_t kd[3] = {(uint64_t)HD, (uint64_t)D.Hkv, (uint64_t)D.NB};
+        const uint64_t ks[2] = {(uint64_t)HD * 4, (uint64_t)D.Hkv * HD * 4};
+        const uint32_t kb[3] = {32u, 1u, (uint32_t)kScoreKeys};
+        if (!make_tensor_map(&tq, W.qbar32, 3, qd, qs, qb, kMapF32) ||
+            !make_tensor_map(&tk, W.kbar_tf, 3, kd, ks, kb, kMapF32))
+            return FP2_ERR_CUDA;
+        const int smem = ScoreTcCfg<HD>::kSmem;
+        if (cudaFuncSetAttribute(k_score_tc<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem) != cudaSuccess)
+            return FP2_ERR_CUDA;
+        const int64_t items = D.score_tiles * D.Hkv;
+        const int grid = (int)std::min<int64_t>(items, std::max(1, sm_count()));
+        k_score_tc<HD><<<grid, kScoreTcThreads, smem, st>>>(D, P, W, tq, tk);
     }
-    k_threshold<HD><<<(unsigned)((D.R * 32 + 255) / 256), 256, 0, st>>>(D, P, W, rel_err);
+    k_threshold<HD><<<(unsigned)((D.R * 32 + 255) / 256), 256, 0, st>>>(D, P, W, kScoreTcRelErr);
     return FP2_OK;
 }
 
