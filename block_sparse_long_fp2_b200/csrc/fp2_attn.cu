@@ -534,11 +534,12 @@ __device__ __forceinline__ uint32_t chunk_bits(int kind, int tok, const TileWalk
 // 32 columns of P = 2^(s * scale + shift), written into tensor memory over
 // the first part of the 32 S columns just read: the A operand of the P.V MMA.
 //   bf16: 16 packed pairs (keys 2c, 2c+1 in column c), columns [t_p, t_p+16).
-//   e4m3: P' = P * pfac packed four per column, columns [t_p, t_p+8).
-// The fp32 row sum accumulates the unscaled P.
+//   e4m3: P' = P * pfac packed four per column, columns [t_p, t_p+8), pfac
+//   entering through the shift (as log2 pfac).
+// The fp32 row sum accumulates the P written (P' for e4m3).
 template <bool MASKED, bool F8>
 __device__ __forceinline__ void p32(const uint32_t (&r)[32], uint32_t vb, uint32_t t_p,
-                                    uint64_t scale2, uint64_t shift2, uint64_t& sum2, float pfac) {
+                                    uint64_t scale2, uint64_t shift2, uint64_t& sum2) {
     float p[32];
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
@@ -557,8 +558,7 @@ __device__ __forceinline__ void p32(const uint32_t (&r)[32], uint32_t vb, uint32
         uint32_t packed[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-            packed[q] = pack_e4m3x4(p[4 * q] * pfac, p[4 * q + 1] * pfac, p[4 * q + 2] * pfac,
-                                    p[4 * q + 3] * pfac);
+            packed[q] = pack_e4m3x4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
         tmem_st8(t_p, packed);
     } else {
 #pragma unroll
@@ -657,12 +657,13 @@ __device__ __forceinline__ void move_reference(RowState& st, float m_new, uint64
 template <int BLK, int HD, bool MASKED, bool F8>
 __device__ __forceinline__ float tile_softmax(uint32_t t_s, int kind, int tok,
                                               const TileWalk<BLK>& walk, int j, float scale,
-                                              float bias, float pfac, RowState& st) {
+                                              float bias, float lpf, float inv_pfac, RowState& st) {
     constexpr int NC = BLK / 32;
     constexpr int kPColsPerChunk = F8 ? 8 : 16;   // TMEM columns of P per 32 keys
     constexpr float kHeadroom = Cfg<HD, BLK, F8>::kHeadroom;
     const uint64_t scale2 = f2_pack(scale, scale);
-    uint64_t shift2 = f2_pack(bias - st.m_ref, bias - st.m_ref);
+    const float pbias = F8 ? bias + lpf : bias;   // shift of the P written
+    uint64_t shift2 = f2_pack(pbias - st.m_ref, pbias - st.m_ref);
     uint64_t sum2 = f2_pack(0.f, 0.f);
     uint32_t ra[32], rb[32];
     tmem_ld32(t_s, ra);
@@ -676,17 +677,17 @@ __device__ __forceinline__ float tile_softmax(uint32_t t_s, int kind, int tok,
         const bool need = cm > st.m_ref + kHeadroom;
         if (__any_sync(0xffffffffu, need)) {
             move_reference<HD, F8>(st, need ? cm : st.m_ref, sum2, t_s, kPColsPerChunk * c);
-            shift2 = f2_pack(bias - st.m_ref, bias - st.m_ref);
+            shift2 = f2_pack(pbias - st.m_ref, pbias - st.m_ref);
         }
-        p32<MASKED, F8>(ra, vba, t_s + kPColsPerChunk * c, scale2, shift2, sum2, pfac);
+        p32<MASKED, F8>(ra, vba, t_s + kPColsPerChunk * c, scale2, shift2, sum2);
         if (c + 2 < NC) tmem_ld32(t_s + 32 * (c + 2), ra);
-        p32<MASKED, F8>(rb, vbb, t_s + kPColsPerChunk * (c + 1), scale2, shift2, sum2, pfac);
+        p32<MASKED, F8>(rb, vbb, t_s + kPColsPerChunk * (c + 1), scale2, shift2, sum2);
         if (c + 3 < NC) tmem_ld32(t_s + 32 * (c + 3), rb);
     }
     tmem_st_wait();
     float a, b;
     f2_unpack(sum2, a, b);
-    return a + b;
+    return F8 ? (a + b) * inv_pfac : a + b;
 }
 
 // ---------------------------------------------------------------------------
@@ -731,7 +732,7 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
         walk.init(P, it);
         int kind, j, n = 0;
         while (walk.next(kind, j)) {
-            float tscale = scale, pfac = 1.f;
+            float tscale = scale, pfac = 1.f, lpf = 0.f, inv_pfac = 1.f;
             if (F8) {
                 // per-tile K and V scales: the block's, or a pseudo tile's chunk;
                 // loaded before the S wait, which hides their latency
@@ -746,9 +747,15 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
             tc_fence_after();
             const bool masked = kind != kFull;
             const float bias = kind == kPseudo ? pseudo_bias : 0.f;
+            if (F8) {
+                lpf = __log2f(pfac);
+                inv_pfac = __frcp_rn(pfac);
+            }
             const float rsum =
-                masked ? tile_softmax<BLK, HD, true, F8>(t_s, kind, tok, walk, j, tscale, bias, pfac, st)
-                       : tile_softmax<BLK, HD, false, F8>(t_s, kind, tok, walk, j, tscale, bias, pfac, st);
+                masked ? tile_softmax<BLK, HD, true, F8>(t_s, kind, tok, walk, j, tscale, bias, lpf,
+                                                         inv_pfac, st)
+                       : tile_softmax<BLK, HD, false, F8>(t_s, kind, tok, walk, j, tscale, bias, lpf,
+                                                          inv_pfac, st);
             st.o_valid = true;
             st.l += rsum;
             tc_fence_before();
