@@ -83,6 +83,24 @@ def whole_job_value(flop_per_rank: float, world: int, ms: float) -> float:
     return world * flop_per_rank / (ms * 1e-3) / 1e12
 
 
+def attn_traffic(workload: str, dtype: str):
+    """DRAM bytes per launch of the attention kernel on this workload, from the
+    committed single-pass ncu capture (profiles/k_attn_traffic.json), or None
+    when the kernel source changed since it was taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "k_attn_traffic.json")) as f:
+            rec = json.load(f)
+        src = os.path.join(ROOT, "block_sparse_long_fp2_b200", "csrc", "fp2_attn.cu")
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+        if rec.get("source_sha256") != digest or rec.get("workload") != workload:
+            return None
+        return rec.get(dtype)
+    except Exception:
+        return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -321,6 +339,7 @@ def run_ours(args, rank, world, local_rank):
                "roofline": {"bound": "tensor", "achieved": round(ach8, 1),
                             "peak": round(2 * peaks()["bf16_sustained"], 1), "unit": "TFLOP/s",
                             "frac": round(ach8 / (2 * peaks()["bf16_sustained"]), 4),
+                            "traffic": attn_traffic(wl.name, "fp8"),
                             "peak_kind": "e4m3 = 2 x measured bf16 sustained (nominal ratio)"},
                "gpu_launches": (launches_per_step + 3 + 1) * args.steps}
 
@@ -376,7 +395,9 @@ def run_ours(args, rank, world, local_rank):
         "dense_equiv_tflop": round(flop / 1e12, 3),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
                      "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
-                     "frac": round(achieved / pk["bf16_sustained"], 4), "traffic": None,
+                     "frac": round(achieved / pk["bf16_sustained"], 4),
+                     "traffic": attn_traffic(wl.name, "bf16"),
+                     "traffic_unit": "DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                      "kernel": "k_attn (sparse attention + correction)",
                      "peak_kind": f"bf16 sustained ({pk['source']})",
                      "frac_of_burst_peak": round(achieved / pk["bf16"], 4)},

@@ -151,8 +151,11 @@ __device__ __forceinline__ Item decode_item(const AttnParams& P, int64_t w) {
     Item it;
     const int64_t rank = w / P.n_pairs;
     it.mp = (int)(w % P.n_pairs);
-    it.b = P.D.NB - 1 - rank / P.D.Hkv;       // latest query blocks first (longest rows)
-    it.g = (int)(rank % P.D.Hkv);
+    // kv-head major, and within a kv-head the latest query blocks first (longest
+    // rows): the CTAs running at the same time read the K/V of one kv-head
+    // (64 MiB at 128K tokens, d = 128), which stays resident in L2
+    it.g = (int)(rank / P.D.NB);
+    it.b = P.D.NB - 1 - rank % P.D.NB;
     it.s = P.block_seq[it.b];
     it.b0 = P.cu_blocks[it.s];
     it.i = (int)(it.b - it.b0);
