@@ -36,7 +36,7 @@ FP2_NO_CORRECTION = 0x1
 FP2_DEBUG_DROP_Q_LOAD = 0x100
 
 EXPORTED = ["fp2_version", "fp2_strerror", "fp2_plan_sizes", "fp2_plan", "fp2_quantize_fp8",
-            "fp2_prefill", "fp2_status_check", "fp2_plan_static"]
+            "fp2_prefill", "fp2_status_check", "fp2_plan_static", "fp2_plan_kv8"]
 
 # Size of the library-held scratch of fp2_plan_static (FP2_STATIC_WORKSPACE_BYTES).
 FP2_STATIC_WORKSPACE_BYTES = 16 << 20
@@ -112,6 +112,10 @@ def lib():
         L.fp2_plan_static.argtypes = [ctypes.POINTER(fp2_problem), ctypes.c_void_p,
                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                       ctypes.c_size_t, ctypes.c_void_p]
+        L.fp2_plan_kv8.argtypes = [ctypes.POINTER(fp2_problem), ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                   ctypes.c_size_t, ctypes.c_void_p]
         L.fp2_quantize_fp8.argtypes = [ctypes.POINTER(fp2_problem), ctypes.c_void_p,
                                        ctypes.c_size_t, ctypes.c_void_p, ctypes.c_int32,
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
@@ -205,6 +209,15 @@ def fp2_plan_static(problem: Problem, q, k, v, plan, stream=None) -> None:
     workspace (for callers that cannot allocate device memory)."""
     _check(lib().fp2_plan_static(problem.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(plan),
                                  plan.numel(), _stream_ptr(stream)), "fp2_plan_static")
+
+
+def fp2_plan_kv8(problem: Problem, q, k_e4m3, v_e4m3, k_scale, v_scale, plan, workspace,
+                 stream=None) -> None:
+    """fp2_plan from an FP8 KV cache: e4m3 K/V codes with per-(block, kv-head)
+    scales, bf16 Q."""
+    _check(lib().fp2_plan_kv8(problem.ref, _ptr(q), _ptr(k_e4m3), _ptr(v_e4m3), _ptr(k_scale),
+                              _ptr(v_scale), _ptr(plan), plan.numel(), _ptr(workspace),
+                              workspace.numel(), _stream_ptr(stream)), "fp2_plan_kv8")
 
 
 def fp2_quantize_fp8(problem: Problem, plan, x, which: int, x_e4m3, scales, stream=None) -> None:

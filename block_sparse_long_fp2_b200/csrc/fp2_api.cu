@@ -280,6 +280,23 @@ int fp2_plan(const fp2_problem* problem, const void* q, const void* k, const voi
                        static_cast<cudaStream_t>(stream));
 }
 
+int fp2_plan_kv8(const fp2_problem* problem, const void* q, const void* k_e4m3, const void* v_e4m3,
+                 const float* k_scale, const float* v_scale, void* plan, size_t plan_bytes,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+    Layout L;
+    int rc = compute_layout(problem, &L);
+    if (rc != FP2_OK) return rc;
+    if (!q || !k_e4m3 || !v_e4m3 || !k_scale || !v_scale || !plan || !workspace)
+        return FP2_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_e4m3, 16) || !aligned(v_e4m3, 16) || !aligned(k_scale, 4) ||
+        !aligned(v_scale, 4) || !aligned(plan, 256) || !aligned(workspace, 256))
+        return FP2_ERR_INVALID_ARG;
+    if (plan_bytes < L.pub.plan_bytes || workspace_bytes < L.pub.workspace_bytes)
+        return FP2_ERR_CAPACITY;
+    return launch_plan(L, problem, q, k_e4m3, v_e4m3, plan_ptrs(L, plan), ws_ptrs(L, workspace),
+                       static_cast<cudaStream_t>(stream), k_scale, v_scale);
+}
+
 int fp2_quantize_fp8(const fp2_problem* problem, const void* plan, size_t plan_bytes, const void* x,
                      int32_t which, void* x_e4m3, float* scales, void* stream) {
     Layout L;

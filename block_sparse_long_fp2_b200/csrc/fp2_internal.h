@@ -86,8 +86,11 @@ PlanPtrs plan_ptrs(const Layout& L, void* plan);
 WsPtrs ws_ptrs(const Layout& L, void* ws);
 
 // Launchers (return FP2_OK or FP2_ERR_CUDA).
+// k_scale / v_scale non-null: k and v are e4m3 codes with per-(block, kv-head)
+// scales (planning from an FP8 KV cache); otherwise bf16.
 int launch_plan(const Layout& L, const fp2_problem* p, const void* q, const void* k,
-                const void* v, const PlanPtrs& pp, const WsPtrs& ws, cudaStream_t st);
+                const void* v, const PlanPtrs& pp, const WsPtrs& ws, cudaStream_t st,
+                const float* k_scale = nullptr, const float* v_scale = nullptr);
 int launch_quantize(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, const void* x,
                     int which, void* x8, float* scales, cudaStream_t st);
 int launch_prefill(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, const void* q,

@@ -114,10 +114,37 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
     return r;
 }
 
+// Eight e4m3 codes (8 bytes) added to eight float64 sums; e4m3 -> f16 -> f32
+// are exact conversions.
+__device__ __forceinline__ void accum8_e4m3(double (&acc)[8], uint2 x) {
+    const uint32_t w[2] = {x.x, x.y};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float lo, hi;
+            unpack_e4m3x2(static_cast<uint16_t>(w[e] >> (16 * h)), lo, hi);
+            acc[4 * e + 2 * h] += (double)lo;
+            acc[4 * e + 2 * h + 1] += (double)hi;
+        }
+    }
+}
+
+__device__ __forceinline__ uint2 ld_stream8(const uint2* p) {
+    uint2 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
+}
+
+// Block means of Q, K and V.  KV8: K and V are e4m3 codes with one fp32 scale
+// per (block, kv-head) (an FP8 KV cache); their means are the means of the
+// codes times the scale.
+template <bool KV8>
 __global__ void __launch_bounds__(kPoolThreads)
 k_pool(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ page_table,
-       const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
-       const uint16_t* __restrict__ v, PlanPtrs P, WsPtrs W) {
+       const uint16_t* __restrict__ q, const void* __restrict__ k,
+       const void* __restrict__ v, const float* __restrict__ k_scale,
+       const float* __restrict__ v_scale, PlanPtrs P, WsPtrs W) {
     if (!*P.meta_valid) return;
     const int vec = blockIdx.y * kPoolThreads + threadIdx.x;   // 8-element column chunk
     const int d = D.d;
@@ -141,8 +168,39 @@ k_pool(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.0;
 
-    if (which == 0 || D.page_size == 0) {
-        const uint16_t* base = which == 0 ? q : (which == 1 ? k : v);
+    if (KV8 && which != 0) {
+        // e4m3 K / V, contiguous [T, Hkv, d] or paged [P, 64, Hkv, d]
+        const uint8_t* base = static_cast<const uint8_t*>(which == 1 ? k : v);
+        const int64_t stride = (int64_t)D.Hkv * d / 8;   // uint2 per token
+        if (D.page_size == 0) {
+            const uint2* p = reinterpret_cast<const uint2*>(base + ((tok0 + t_begin) * D.Hkv + head) * d + e0);
+            int t = t_begin;
+            for (; t + kPoolUnroll <= t_end; t += kPoolUnroll) {
+                uint2 x[kPoolUnroll];
+#pragma unroll
+                for (int u = 0; u < kPoolUnroll; ++u) x[u] = ld_stream8(p + u * stride);
+#pragma unroll
+                for (int u = 0; u < kPoolUnroll; ++u) accum8_e4m3(acc, x[u]);
+                p += kPoolUnroll * stride;
+            }
+            for (; t < t_end; ++t) {
+                accum8_e4m3(acc, ld_stream8(p));
+                p += stride;
+            }
+        } else {
+            for (int t = t_begin; t < t_end; t += 64) {
+                const int id = page_table[(int64_t)s * D.pt_stride + t / 64];
+                const int n = min(64, t_end - t);
+                if (id < 0 || id >= D.num_pages) continue;   // recorded by k_meta; reads as zeros
+                const uint2* p = reinterpret_cast<const uint2*>(base + ((int64_t)id * 64 * D.Hkv + head) * d + e0);
+                for (int u = 0; u < n; ++u) accum8_e4m3(acc, ld_stream8(p + u * stride));
+            }
+        }
+        const double sc = (double)(which == 1 ? k_scale : v_scale)[b * D.Hkv + head];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] *= sc;
+    } else if (which == 0 || D.page_size == 0) {
+        const uint16_t* base = which == 0 ? q : static_cast<const uint16_t*>(which == 1 ? k : v);
         const int H = which == 0 ? D.Hq : D.Hkv;
         const uint4* p = reinterpret_cast<const uint4*>(base + ((tok0 + t_begin) * H + head) * d + e0);
         const int64_t stride = (int64_t)H * d / 8;   // uint4 per token
@@ -161,7 +219,7 @@ k_pool(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict
         }
     } else {
         // paged pool [num_pages, 64, Hkv, d]; blocks start on page boundaries (B % 64 == 0)
-        const uint16_t* pool = which == 1 ? k : v;
+        const uint16_t* pool = static_cast<const uint16_t*>(which == 1 ? k : v);
         const int64_t stride = (int64_t)D.Hkv * d / 8;
         for (int t = t_begin; t < t_end; t += 64) {
             const int id = page_table[(int64_t)s * D.pt_stride + t / 64];
@@ -669,15 +727,20 @@ int launch_score(const Dims& D, const PlanPtrs& P, const WsPtrs& W, cudaStream_t
 }  // namespace
 
 int launch_plan(const Layout& L, const fp2_problem* p, const void* q, const void* k, const void* v,
-                const PlanPtrs& P, const WsPtrs& W, cudaStream_t st) {
+                const PlanPtrs& P, const WsPtrs& W, cudaStream_t st, const float* k_scale,
+                const float* v_scale) {
     const Dims& D = L.dims;
     k_meta<<<1, 256, 0, st>>>(D, p->cu_seqlens, p->page_table, P);
     const int vecs = (D.Hq + 2 * D.Hkv) * D.d / 8;
     dim3 pool_grid((unsigned)D.NB, (vecs + kPoolThreads - 1) / kPoolThreads);
-    k_pool<<<pool_grid, kPoolThreads, 0, st>>>(D, p->cu_seqlens, p->page_table,
-                                               static_cast<const uint16_t*>(q),
-                                               static_cast<const uint16_t*>(k),
-                                               static_cast<const uint16_t*>(v), P, W);
+    if (k_scale)
+        k_pool<true><<<pool_grid, kPoolThreads, 0, st>>>(D, p->cu_seqlens, p->page_table,
+                                                         static_cast<const uint16_t*>(q), k, v,
+                                                         k_scale, v_scale, P, W);
+    else
+        k_pool<false><<<pool_grid, kPoolThreads, 0, st>>>(D, p->cu_seqlens, p->page_table,
+                                                          static_cast<const uint16_t*>(q), k, v,
+                                                          nullptr, nullptr, P, W);
     if (D.tau > 0.0) {
         const int64_t warps = D.NB * D.Hkv;
         k_norms<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(D, P, W);

@@ -188,13 +188,28 @@ int fp2_plan_sizes(const fp2_problem* problem, fp2_plan_layout* layout);
  * status word.  `workspace` (workspace_bytes >= layout.workspace_bytes,
  * device memory, 256-byte aligned) is scratch, free again once the enqueued
  * work completes.  Block lists are decided as if every score were computed in
- * float64: scores are computed in float32 and any block within the float32
- * error bound of the threshold (or of the row maximum) is re-scored in
- * float64.
+ * float64: scores are computed on the tensor cores (tf32 MMAs of the means
+ * rounded to tf32) and any block within that computation's error bound of the
+ * threshold (or of the row maximum) is re-scored in float64.
  */
 int fp2_plan(const fp2_problem* problem, const void* q, const void* k, const void* v,
              void* plan, size_t plan_bytes, void* workspace, size_t workspace_bytes,
              void* stream);
+
+/*
+ * Stage 1 from an FP8 KV cache: as fp2_plan, with K and V given as e4m3 codes
+ * (same layout as the bf16 tensors, one byte per element, contiguous or paged)
+ * and one fp32 scale per (block, kv-head) each, k_scale / v_scale [NB, Hkv]
+ * indexed by the global block (the layout fp2_quantize_fp8 writes); Q stays
+ * bf16.  The block means of K and V are the means of the dequantised values
+ * code * scale (computed as scale * mean of the codes, in float64), so the plan
+ * is the plan of the dequantised cache.  All pointers are device memory: q, k,
+ * v 16-byte aligned, scales 4-byte aligned; ownership, workspace and errors as
+ * for fp2_plan.
+ */
+int fp2_plan_kv8(const fp2_problem* problem, const void* q, const void* k_e4m3,
+                 const void* v_e4m3, const float* k_scale, const float* v_scale, void* plan,
+                 size_t plan_bytes, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Direct online FP8 quantisation (Table 1 footnote): for every (block, head)

@@ -129,6 +129,15 @@ def test_null_problem_and_buffers_rejected(lib):
     assert rc == fb.FP2_ERR_INVALID_ARG   # unknown flag
     rc = L.fp2_quantize_fp8(p.ref, 0x100000, lay.plan_bytes, 0x10000, 3, 0x10000, 0x10000, None)
     assert rc == fb.FP2_ERR_INVALID_ARG   # which out of range
+    rc = L.fp2_plan_kv8(p.ref, 0x10000, 0x10000, 0x10000, None, 0x10000, 0x100000, lay.plan_bytes,
+                        0x200000, lay.workspace_bytes, None)
+    assert rc == fb.FP2_ERR_INVALID_ARG   # missing K scales
+    rc = L.fp2_plan_kv8(p.ref, 0x10000, 0x10008, 0x10000, 0x10000, 0x10000, 0x100000,
+                        lay.plan_bytes, 0x200000, lay.workspace_bytes, None)
+    assert rc == fb.FP2_ERR_INVALID_ARG   # K codes not 16-byte aligned
+    rc = L.fp2_plan_kv8(p.ref, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 0x100000,
+                        lay.plan_bytes, 0x200000, lay.workspace_bytes - 256, None)
+    assert rc == fb.FP2_ERR_CAPACITY
 
 
 def test_no_cpu_fallback_in_product_path():

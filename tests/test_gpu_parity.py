@@ -306,3 +306,36 @@ def test_fp8_prefill(name, gen):
     assert e_dq <= 5e-2
     if gen == "normal":
         assert e_ref <= 5e-2
+
+
+@pytest.mark.parametrize("name", ["ragged_d128", "paged_mix_small", "B64_d128"])
+def test_plan_from_fp8_kv_cache(name):
+    # An FP8 KV cache: K and V quantised on the GPU (codes bit-exact with the
+    # oracle's quantiser, see test_quantize_fp8_matches_oracle_codes), then
+    # planned from the codes and scales; the oracle plans the dequantised cache.
+    import torch
+    from fp2_harness import dequantised_operands
+    wl, x = _case(name)
+    run = GpuRun(wl, x).plan()
+    NB = int(run.lay.num_blocks)
+    kv8 = []
+    for which, src in ((1, run.k), (2, run.v)):
+        codes = torch.zeros(src.shape, dtype=torch.uint8, device="cuda")
+        scales = torch.zeros((NB, wl.Hkv), dtype=torch.float32, device="cuda")
+        fb.fp2_quantize_fp8(run.prob, run.plan_buf, src, which, codes, scales)
+        kv8.append((codes, scales))
+    lay, plan8, ws8 = fb.allocate(run.prob)
+    fb.fp2_plan_kv8(run.prob, run.q, kv8[0][0], kv8[1][0], kv8[0][1], kv8[1][1], plan8, ws8)
+    rc, st = fb.fp2_status_check(plan8)
+    assert (rc, st) == (fb.FP2_OK, 0)
+    view = fb.PlanView(plan8, lay, wl.Hkv, wl.d)
+    q, k, v = oracle_inputs(x, wl)
+    _, k_dq, v_dq, _ = dequantised_operands(wl, q, k, v, oracle.plan(q, k, v, wl.seqlens, wl.B, 1.0), [])
+    pl = oracle.plan(q, k_dq, v_dq, wl.seqlens, wl.B, wl.tau)
+    rp = view.row_ptr.cpu().numpy()
+    ci = view.col_idx.cpu().numpy()
+    kept = {r: ci[rp[r]:rp[r + 1]].tolist() for r in range(len(rp) - 1)}
+    res = compare_plan(pl, kept)
+    assert res["outside_band"] == 0, res
+    assert np.allclose(view.kbar.cpu().numpy(), pl["kbar"], rtol=2e-7, atol=1e-7)
+    assert np.allclose(view.vbar.cpu().numpy(), pl["vbar"], rtol=2e-7, atol=1e-7)
