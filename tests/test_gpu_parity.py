@@ -41,6 +41,9 @@ SMALL = {
     "dense_tau0": ([1000, 300], 8, 2, 128, 128, 0.0, "lowrank", 0, 0, 0),
     "paged_mix_small": ([1500, 640, 97], 8, 2, 128, 128, 0.1, "lowrank", 0, 64, 60),
     "two_pseudo_tiles": ([9000], 2, 1, 64, 64, 0.2, "lowrank", 0, 0, 0),
+    # degenerate lengths: one token, two tokens, a block plus one, a partial block
+    "tiny_lengths": ([1, 2, 129, 3, 130], 8, 2, 128, 128, 0.5, "normal", 0, 0, 0),
+    "tiny_paged": ([1, 65, 64], 8, 2, 128, 128, 0.5, "normal", 0, 64, 8),
 }
 
 
