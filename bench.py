@@ -233,7 +233,8 @@ def run_ours(args, rank, world, local_rank):
     plan_ms = [e[0].elapsed_time(e[1]) for e in ev]
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
     # plan: meta, pool, [norms, score], threshold, quant_means, scan, compact; prefill: attn
-    launches_per_step = (8 if wl.tau > 0 else 6) + 1
+    # (+ the split merge when the schedule splits rows)
+    launches_per_step = (8 if wl.tau > 0 else 6) + 1 + (1 if lay.num_split_slots > 0 else 0)
 
     # dense baseline: the same kernels on the same inputs with tau = 0 (every
     # causally visible block kept, no pseudo tiles)
@@ -283,7 +284,7 @@ def run_ours(args, rank, world, local_rank):
                  "roofline": {"bound": "tensor", "achieved": round(ach0, 1),
                               "peak": peaks()["bf16_sustained"], "unit": "TFLOP/s",
                               "frac": round(ach0 / peaks()["bf16_sustained"], 4)},
-                 "gpu_launches": 7 * args.steps}
+                 "gpu_launches": (7 + (1 if lay.num_split_slots > 0 else 0)) * args.steps}
         del plan0, ws0
 
     # FP8-e4m3 leg: plan (bf16) + direct online quantisation of Q, K, V + e4m3 prefill

@@ -88,6 +88,8 @@ class fp2_plan_layout(ctypes.Structure):
         ("off_meta", ctypes.c_size_t),
         ("plan_bytes", ctypes.c_size_t),
         ("workspace_bytes", ctypes.c_size_t),
+        ("num_work_items", ctypes.c_int64),
+        ("num_split_slots", ctypes.c_int64),
     ]
 
 

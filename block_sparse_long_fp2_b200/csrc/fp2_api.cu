@@ -86,9 +86,45 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     d.n_groups_cap = (int)groups;
     d.score_tiles = tiles;
 
+    // attention schedule: split size from the layer's mean tiles per CTA,
+    // then the work items and the split rows' slots
+    SchedDims sd{};
+    sd.n_mtiles = G * d.B / kTileM;
+    sd.n_pairs = (sd.n_mtiles + 1) / 2;
+    int64_t units = 0;
+    for (int s = 0; s < p->num_seqs; ++s) {
+        const int64_t nb = (p->seqlens[s] + d.B - 1) / d.B;
+        for (int64_t i = 0; i < nb; ++i) units += row_tile_bound(i, d.B);
+    }
+    const int64_t share = (units * d.Hkv * sd.n_pairs + kSchedSMs - 1) / kSchedSMs;
+    const int64_t longest = row_tile_bound(max_nb - 1, d.B);
+    int64_t split = std::max<int64_t>({(int64_t)kMinSplitTiles, (share + 1) / 2,
+                                       (longest + kMaxSplits - 1) / kMaxSplits});
+    // no splits when no item outlasts a CTA's mean share, or when the longest
+    // row is too short to repay the merge
+    if (longest <= share || longest < kMinSplitRow) split = 0;
+    sd.split_c = (int)split;
+    int64_t items = 0, slots = 0;
+    for (int s = 0; s < p->num_seqs; ++s) {
+        const int64_t nb = (p->seqlens[s] + d.B - 1) / d.B;
+        for (int64_t i = 0; i < nb; ++i) {
+            const int S = row_splits(i, d.B, sd.split_c);
+            items += S;
+            if (S > 1) slots += S;
+        }
+    }
+    sd.n_items = items * d.Hkv * sd.n_pairs;
+    sd.split_slots = slots;
+    if (sd.n_items > ((int64_t)1 << 31) - 1 || slots * d.Hkv > ((int64_t)1 << 31) - 1 ||
+        row_splits(max_nb - 1, d.B, sd.split_c) > kMaxSplits || d.Hkv >= (1 << 16))
+        return FP2_ERR_UNSUPPORTED;
+    const int64_t head_kv_bytes = T * d.d * 4;   // bf16 K and V of one kv-head
+    sd.heads_per_chunk = (int)std::max<int64_t>(1, std::min<int64_t>(d.Hkv, kSchedL2Bytes / head_kv_bytes));
+
     Layout& L = *out;
     std::memset(&L, 0, sizeof(L));
     L.dims = d;
+    L.sched = sd;
     fp2_plan_layout& pub = L.pub;
     pub.num_tokens = T;
     pub.num_blocks = NB;
@@ -121,6 +157,13 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     L.off_group_seq = c.take(sizeof(int32_t) * (size_t)std::max<int64_t>(1, groups));
     L.off_tile_cu = c.take(sizeof(int32_t) * (size_t)(groups + 1));
     L.off_vmax = c.take(sizeof(float) * n * (size_t)d.Hkv);
+    L.off_sched = c.take(sizeof(int4) * (size_t)sd.n_items);
+    L.off_sched_cnt = c.take(sizeof(int32_t) * (size_t)max_nb);
+    L.off_sched_off = c.take(sizeof(int64_t) * (size_t)max_nb);
+    const size_t split_rows = (size_t)sd.split_slots * d.Hkv * d.G * d.B;
+    L.off_split_o = c.take(sizeof(float) * split_rows * d.d);
+    L.off_split_lse = c.take(sizeof(float) * split_rows);
+    L.off_slot_item = c.take(sizeof(int32_t) * (size_t)sd.split_slots * d.Hkv);
     pub.plan_bytes = align_up(c.off, 256);
 
     Carver w;
@@ -133,6 +176,8 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     L.ws_scores = w.take(sizeof(float) * (size_t)d.nnz_cap);
     L.ws_counts = w.take(sizeof(int32_t) * (size_t)d.R);
     pub.workspace_bytes = align_up(w.off, 256);
+    pub.num_work_items = sd.n_items;
+    pub.num_split_slots = sd.split_slots * d.Hkv;
     return FP2_OK;
 }
 
@@ -160,6 +205,12 @@ PlanPtrs plan_ptrs(const Layout& L, void* plan) {
     p.group_seq = reinterpret_cast<int32_t*>(b + L.off_group_seq);
     p.tile_cu = reinterpret_cast<int32_t*>(b + L.off_tile_cu);
     p.vmax = reinterpret_cast<float*>(b + L.off_vmax);
+    p.sched = reinterpret_cast<int4*>(b + L.off_sched);
+    p.sched_cnt = reinterpret_cast<int32_t*>(b + L.off_sched_cnt);
+    p.sched_off = reinterpret_cast<int64_t*>(b + L.off_sched_off);
+    p.split_o = reinterpret_cast<float*>(b + L.off_split_o);
+    p.split_lse = reinterpret_cast<float*>(b + L.off_split_lse);
+    p.slot_item = reinterpret_cast<int32_t*>(b + L.off_slot_item);
     return p;
 }
 

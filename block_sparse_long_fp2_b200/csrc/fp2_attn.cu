@@ -133,13 +133,20 @@ struct AttnParams {
     const float* vmax;
     uint32_t flags;
     int n_mtiles;   // 128-row query tiles per row = G * B / 128
-    int n_pairs;    // work items per row = ceil(n_mtiles / 2)
-    int64_t n_items;
+    // work schedule (built with the plan) and the scratch of split rows
+    const int4* sched;
+    float* split_o;
+    float* split_lse;
+    const int32_t* slot_item;
+    int64_t n_items;   // work items in the schedule
+    int64_t n_slots;   // n_items rounded up to whole passes of the grid
+    bool zigzag;       // odd passes run backwards
 };
 
-// One work item: row (s, g, i) and query tiles 2*mp, 2*mp+1.
+// One work item: split k of S of row (s, g, i), query tiles 2*mp, 2*mp+1.
 struct Item {
     int s, g, i, mp;
+    int k, S, slot;      // split, splits of the row, first split slot of the row
     int64_t b, r;
     int kbeg, kend;      // CSR range of the row
     int tok0, L;         // first token of the sequence, its length
@@ -147,15 +154,27 @@ struct Item {
     bool has_m1;
 };
 
+// The schedule lists the items longest row first (within a chunk of kv-heads
+// whose K/V share L2).  CTA c takes the c-th item of every pass over the grid;
+// with few passes (zigzag) it takes the c-th from the end on odd passes,
+// which evens out the rows' decreasing lengths across the CTAs (measured
+// 6-7 % faster at 8K-16K tokens per layer, 2 % slower at 128K, where the
+// passes are many and the lengths wrap around every kv-head).  Returns
+// n_items or more for a slot without an item.
+__device__ __forceinline__ int64_t sched_index(int64_t w, bool zigzag) {
+    const int64_t pass = w / gridDim.x;
+    return (zigzag && (pass & 1)) ? pass * gridDim.x + (gridDim.x - 1 - blockIdx.x) : w;
+}
+
 __device__ __forceinline__ Item decode_item(const AttnParams& P, int64_t w) {
     Item it;
-    const int64_t rank = w / P.n_pairs;
-    it.mp = (int)(w % P.n_pairs);
-    // kv-head major, and within a kv-head the latest query blocks first (longest
-    // rows): the CTAs running at the same time read the K/V of one kv-head
-    // (64 MiB at 128K tokens, d = 128), which stays resident in L2
-    it.g = (int)(rank / P.D.NB);
-    it.b = P.D.NB - 1 - rank % P.D.NB;
+    const int4 e = __ldg(P.sched + w);
+    it.b = e.x;
+    it.g = e.y & 0xFFFF;
+    it.mp = e.y >> 16;
+    it.k = e.z & 0xFFFF;
+    it.S = e.z >> 16;
+    it.slot = e.w;
     it.s = P.block_seq[it.b];
     it.b0 = P.cu_blocks[it.s];
     it.i = (int)(it.b - it.b0);
@@ -180,7 +199,7 @@ struct TileWalk {
     static constexpr int W = BLK / 32;
     const int32_t* cols;
     const uint32_t* mask;
-    int n_kept, t, i, pt, n_pt, mask_words;
+    int n_kept, t, i, pt, n_pt;
     int j_next;          // col_idx[t] (valid when t < n_kept)
     uint32_t pt_bits;    // bit p set: pseudo tile p (p < 32) holds a skipped block
 
@@ -190,22 +209,40 @@ struct TileWalk {
         t = 0;
         i = it.i;
         mask = P.kept_mask + it.r * P.D.mask_words;
-        mask_words = P.D.mask_words;
         pt = 0;
         n_pt = (P.flags & FP2_NO_CORRECTION) ? 0 : (it.i + BLK - 1) / BLK;
-        j_next = n_kept > 0 ? __ldg(cols) : 0;
         pt_bits = 0;
         const int n_small = n_pt < 32 ? n_pt : 32;
         for (int p = 0; p < n_small; ++p) pt_bits |= has_skip(p) ? (1u << p) : 0u;
+        if (it.S > 1) {
+            // count-balanced split: tiles [k n / S, (k + 1) n / S) of the n tiles
+            // of the row; the walk's ends are moved onto that range
+            const int n = count();
+            const int t0 = (int)((int64_t)it.k * n / it.S);
+            const int t1 = (int)((int64_t)(it.k + 1) * n / it.S);
+            if (t1 <= n_kept) {
+                n_kept = t1;
+                n_pt = 0;
+            } else {
+                int p = 0;
+                for (int r = t1 - n_kept; r > 0 && p < n_pt; ++p) r -= pt_nonempty(p) ? 1 : 0;
+                n_pt = p;
+            }
+            if (t0 <= n_kept) {
+                t = t0;
+            } else {
+                t = n_kept;
+                for (int r = t0 - n_kept; r > 0 && pt < n_pt; ++pt) r -= pt_nonempty(pt) ? 1 : 0;
+            }
+        }
+        j_next = t < n_kept ? __ldg(cols + t) : 0;
     }
     // skip bits of blocks BLK*pt + 32*w .. +31 (skipped = visible, j < i, not kept)
     __device__ __forceinline__ uint32_t skip_word(int p, int w) const {
         const int j0 = BLK * p + 32 * w;
         if (j0 >= i) return 0u;
         const uint32_t valid = (j0 + 32 <= i) ? 0xFFFFFFFFu : ((1u << (i - j0)) - 1u);
-        const int widx = j0 / 32;
-        const uint32_t kept = widx < mask_words ? __ldg(mask + widx) : 0xFFFFFFFFu;
-        return ~kept & valid;
+        return ~__ldg(mask + j0 / 32) & valid;
     }
     __device__ __forceinline__ bool has_skip(int p) const {
         uint32_t any = 0;
@@ -231,20 +268,24 @@ struct TileWalk {
         kind = kPseudo;
         return true;
     }
-    // Number of tiles of the walk (kept blocks + non-empty pseudo tiles), so a
-    // role that needs no column ids can count tiles without loading them.
+    // Tiles left in the walk (kept blocks + non-empty pseudo tiles), so a role
+    // that needs no column ids can count tiles without loading them.
     __device__ __forceinline__ int count() const {
-        int n = n_kept + __popc(pt_bits);
-        for (int p = 32; p < n_pt; ++p) n += has_skip(p) ? 1 : 0;
+        int n = n_kept - t;
+        const int hi = n_pt < 32 ? n_pt : 32;
+        if (pt < hi) {
+            const uint32_t below_hi = hi == 32 ? 0xFFFFFFFFu : ((1u << hi) - 1u);
+            n += __popc(pt_bits & below_hi & ~((1u << pt) - 1u));
+        }
+        for (int p = pt > 32 ? pt : 32; p < n_pt; ++p) n += has_skip(p) ? 1 : 0;
         return n;
     }
-    __device__ __forceinline__ bool is_last() const {
-        if (t < n_kept) return false;
-        int p = pt;
-        while (p < n_pt && !pt_nonempty(p)) ++p;
-        return p >= n_pt;
-    }
 };
+
+// Whether split k of S of a row with n tiles has any tile.
+__device__ __forceinline__ bool split_nonempty(int k, int S, int n) {
+    return (int64_t)(k + 1) * n / S > (int64_t)k * n / S;
+}
 
 // Uniform wait for a whole warp: every lane waits, then all agree.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars& B, int32_t* status) {
@@ -281,8 +322,13 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
     constexpr int kSlots = C::kSlots;
     uint32_t issued[kMaxSlots] = {0, 0, 0, 0, 0, 0, 0, 0};
     const bool paged = D.page_size != 0;
-    for (int64_t w = blockIdx.x; w < P.n_items; w += gridDim.x) {
-        const Item it = decode_item(P, w);
+    for (int64_t w = blockIdx.x; w < P.n_slots; w += gridDim.x) {
+        const int64_t o = sched_index(w, P.zigzag);
+        if (o >= P.n_items) continue;
+        const Item it = decode_item(P, o);
+        TileWalk<BLK> walk;
+        walk.init(P, it);
+        if (walk.count() == 0) continue;   // a split without tiles
         for (int m = 0; m < 2; ++m) {
             if (m == 1 && !it.has_m1) break;
             if (!mbar_wait(&B.q_empty[m], (qcnt[m] & 1) ^ 1, &B.abort, P.status)) goto drain;
@@ -301,8 +347,6 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
                                 C::kAtomElems * a, it.g * D.G + hl, it.tok0 + it.i * BLK);
             }
         }
-        TileWalk<BLK> walk;
-        walk.init(P, it);
         int kind, j;
         while (walk.next(kind, j)) {
             for (int kv = 0; kv < 2; ++kv) {
@@ -463,8 +507,10 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
         return true;
     };
 
-    for (int64_t w = blockIdx.x; w < P.n_items; w += gridDim.x) {
-        const Item it = decode_item(P, w);
+    for (int64_t w = blockIdx.x; w < P.n_slots; w += gridDim.x) {
+        const int64_t o = sched_index(w, P.zigzag);
+        if (o >= P.n_items) continue;
+        const Item it = decode_item(P, o);
         // The issuer needs no column ids, only the tile count: its loop issues no
         // global loads, which would otherwise hold up its barrier probes.
         int n_tiles;
@@ -473,6 +519,7 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
             walk.init(P, it);
             n_tiles = walk.count();
         }
+        if (n_tiles == 0) continue;
         RingPos kp = ring_take<kSlots>(ring);
         RingPos vp = ring_take<kSlots>(ring);
         if (!mbar_wait(&B.q_full[0], qcnt[0] & 1, &B.abort, P.status)) goto drain;
@@ -711,9 +758,15 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
     const float pseudo_bias = log2f((float)BLK);                   // ln n_j in log2 units
     uint32_t scnt = 0, ocnt = 0;
 
-    for (int64_t w = blockIdx.x; w < P.n_items; w += gridDim.x) {
-        const Item it = decode_item(P, w);
+    for (int64_t w = blockIdx.x; w < P.n_slots; w += gridDim.x) {
+        const int64_t o = sched_index(w, P.zigzag);
+        if (o >= P.n_items) continue;
+        const Item it = decode_item(P, o);
         if (m == 1 && !it.has_m1) continue;
+        TileWalk<BLK> walk;
+        walk.init(P, it);
+        if (walk.count() == 0) continue;   // a split without tiles
+        const int split_slot = it.S > 1 ? it.slot + it.k : -1;   // scratch slot of a split
         const int mt = 2 * it.mp + m;
         const int pr = kTileM * mt + prow;
         const int hl = pr / BLK;
@@ -731,8 +784,6 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
             k_row = 448.0f / (256.0f * __ldg(P.vmax + (int64_t)it.s * D.Hkv + it.g));
         }
 
-        TileWalk<BLK> walk;
-        walk.init(P, it);
         int kind, j, n = 0;
         while (walk.next(kind, j)) {
             float tscale = scale, pfac = 1.f, lpf = 0.f, inv_pfac = 1.f;
@@ -767,18 +818,29 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
             ++n;
         }
 
-        // epilogue: O / l as bf16, LSE = ln(l) + m_ref * ln 2
+        // epilogue: O / l as bf16, LSE = ln(l) + m_ref * ln 2; a split row
+        // writes its part's O / l in fp32 and log2(l) + m_ref to its slot
         if (!warp_wait(&B.o_full[m], ocnt & 1, B, P.status)) return;
         ++ocnt;
         tc_fence_after();
         const float inv_l = 1.0f / (st.l * k_row);
-        uint16_t* orow = P.o + ((int64_t)(it.tok0 + pos) * D.Hq + h) * HD;
+        const bool split = split_slot >= 0;
+        const int64_t srow = (int64_t)split_slot * (D.G * BLK) + pr;
+        const int64_t orow = (int64_t)(it.tok0 + pos) * D.Hq + h;
+        char* dst = split ? reinterpret_cast<char*>(P.split_o + srow * HD)
+                          : reinterpret_cast<char*>(P.o + orow * HD);
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
             uint32_t r[32];
             tmem_ld32(t_o + 32 * c, r);
             tmem_ld_wait();
-            if (row_valid) {
+            if (row_valid && split) {
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    reinterpret_cast<float4*>(dst)[(32 * c + e) / 4] =
+                        make_float4(__uint_as_float(r[e + 0]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
+                                    __uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
+            } else if (row_valid) {
 #pragma unroll
                 for (int e = 0; e < 32; e += 8) {
                     uint4 v;
@@ -786,11 +848,13 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
                     v.y = pack_bf16x2(__uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
                     v.z = pack_bf16x2(__uint_as_float(r[e + 4]) * inv_l, __uint_as_float(r[e + 5]) * inv_l);
                     v.w = pack_bf16x2(__uint_as_float(r[e + 6]) * inv_l, __uint_as_float(r[e + 7]) * inv_l);
-                    *reinterpret_cast<uint4*>(orow + 32 * c + e) = v;
+                    reinterpret_cast<uint4*>(dst)[(32 * c + e) / 8] = v;
                 }
             }
         }
-        if (row_valid) P.lse[(int64_t)h * D.T + it.tok0 + pos] = (st.m_ref + log2f(st.l)) * 0.6931471805599453f;
+        const float lse2 = st.m_ref + log2f(st.l);
+        if (row_valid && split) P.split_lse[srow] = lse2;
+        else if (row_valid) P.lse[(int64_t)h * D.T + it.tok0 + pos] = lse2 * 0.6931471805599453f;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.o_free[m]);
@@ -854,6 +918,91 @@ k_attn(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap
     if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(B.tmem_base, C::kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// merge of split rows
+// ---------------------------------------------------------------------------
+
+constexpr int kCombineThreads = 256;
+constexpr int kCombineRows = 32;   // query rows per CTA (4 per warp)
+
+// Grid (row split slot, query-tile pair x row chunk).  The CTAs of a split
+// row's first slot merge kCombineRows of its query rows each: a row's
+// non-empty splits k give lse = log2 sum_k 2^lse_k and
+// O = sum_k 2^(lse_k - lse) O_k (one split per lane for the weights, the
+// head dimension across the lanes for O); O goes out as bf16, LSE in
+// natural-log units.  The other slots' CTAs return at once.
+template <int HD, int BLK>
+__global__ void __launch_bounds__(kCombineThreads) k_combine(const __grid_constant__ AttnParams P) {
+    if (!*P.meta_valid) return;
+    const int slot = blockIdx.x;
+    const int64_t first = __ldg(P.slot_item + slot);
+    if (__ldg(P.sched + first).w != slot) return;
+    constexpr int kChunks = 2 * kTileM / kCombineRows;
+    const int mp = blockIdx.y / kChunks;
+    const Item it = decode_item(P, first + mp);
+    const Dims& D = P.D;
+    int n;   // tiles of the whole row, as the attention roles walked them
+    {
+        Item whole = it;
+        whole.S = 1;
+        TileWalk<BLK> walk;
+        walk.init(P, whole);
+        n = walk.count();
+    }
+    constexpr int E = HD / 32;   // elements per lane
+    const int lane = threadIdx.x & 31;
+    const int64_t gb = (int64_t)D.G * BLK;
+    const int r0 = (blockIdx.y % kChunks) * kCombineRows + (threadIdx.x >> 5) * (kCombineRows / 8);
+    for (int rr = r0; rr < r0 + kCombineRows / 8; ++rr) {
+        if (2 * it.mp + rr / kTileM >= P.n_mtiles) break;
+        const int pr = 2 * it.mp * kTileM + rr;
+        const int tok = pr % BLK;
+        const int h = it.g * D.G + pr / BLK;
+        const int pos = it.i * BLK + tok;
+        if (pos >= it.L) continue;
+        // lane k holds split k's log-sum-exp (-inf when the split had no tile)
+        const bool live = lane < it.S && split_nonempty(lane, it.S, n);
+        const float lk = live ? P.split_lse[(it.slot + lane) * gb + pr] : -INFINITY;
+        float mx = lk;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float wk = live ? exp2f(lk - mx) : 0.f;
+        float wsum = wk;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+        float acc[E];
+#pragma unroll
+        for (int x = 0; x < E; ++x) acc[x] = 0.f;
+        for (int k = 0; k < it.S; ++k) {
+            const float w = __shfl_sync(0xffffffffu, wk, k);
+            if (w == 0.f) continue;
+            const float* src = P.split_o + ((it.slot + k) * gb + pr) * HD + lane * E;
+            if constexpr (E == 4) {
+                const float4 v = *reinterpret_cast<const float4*>(src);
+                acc[0] += w * v.x;
+                acc[1] += w * v.y;
+                acc[2] += w * v.z;
+                acc[3] += w * v.w;
+            } else {
+                const float2 v = *reinterpret_cast<const float2*>(src);
+                acc[0] += w * v.x;
+                acc[1] += w * v.y;
+            }
+        }
+        const float inv = 1.0f / wsum;
+        uint16_t* orow = P.o + ((int64_t)(it.tok0 + pos) * D.Hq + h) * HD + lane * E;
+        if constexpr (E == 4) {
+            uint2 v;
+            v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+            v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+            *reinterpret_cast<uint2*>(orow) = v;
+        } else {
+            *reinterpret_cast<uint32_t*>(orow) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        }
+        if (lane == 0) P.lse[(int64_t)h * D.T + it.tok0 + pos] = (mx + log2f(wsum)) * 0.6931471805599453f;
     }
 }
 
@@ -941,17 +1090,26 @@ int launch_attn_t(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, con
     P.vbar_scale = pp.vbar_scale;
     P.vmax = pp.vmax;
     P.flags = flags;
-    P.n_mtiles = D.G * BLK / kTileM;
-    P.n_pairs = (P.n_mtiles + 1) / 2;
-    P.n_items = D.R * P.n_pairs;
+    const SchedDims& S = L.sched;
+    P.n_mtiles = S.n_mtiles;
+    P.n_items = S.n_items;
+    P.sched = pp.sched;
+    P.split_o = pp.split_o;
+    P.split_lse = pp.split_lse;
+    P.slot_item = pp.slot_item;
     const int sms = sm_count();
     if (sms <= 0) return FP2_ERR_CUDA;
-    const int64_t grid = P.n_items < sms ? P.n_items : sms;
+    const int64_t grid = S.n_items < sms ? S.n_items : sms;
+    P.n_slots = (S.n_items + grid - 1) / grid * grid;
+    P.zigzag = P.n_slots / grid <= kZigZagMaxPasses;
     if (cudaFuncSetAttribute(k_attn<HD, BLK, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess)
         return FP2_ERR_CUDA;
     if (F8) k_vmax<<<dim3(D.n_seqs, D.Hkv), 256, 0, st>>>(D, pp, vs);
     k_attn<HD, BLK, F8><<<(unsigned)grid, kThreads, C::kSmemBytes, st>>>(P, tq, tk, tv, tkb, tvb);
+    if (S.split_slots > 0)
+        k_combine<HD, BLK><<<dim3((unsigned)(S.split_slots * D.Hkv), S.n_pairs * (2 * kTileM / kCombineRows)),
+                             kCombineThreads, 0, st>>>(P);
     return cudaGetLastError() == cudaSuccess ? FP2_OK : FP2_ERR_CUDA;
 }
 

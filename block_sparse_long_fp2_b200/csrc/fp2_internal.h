@@ -20,6 +20,32 @@ constexpr int kScoreQV = 128;
 // Key blocks scored together by one CTA of the scoring kernel (MMA N).
 constexpr int kScoreKeys = 128;
 
+// Attention work schedule.  The rows of one chunk of kv-heads are taken
+// longest first; a chunk holds as many kv-heads as keep their bf16 K and V
+// within kSchedL2Bytes, so the CTAs that run together share K/V in L2.  When
+// the longest row's tile bound exceeds a CTA's mean share of the layer (taken
+// over kSchedSMs CTAs) and kMinSplitRow tiles, every row whose bound exceeds
+// half that share is cut into count-balanced splits of at least
+// kMinSplitTiles tiles (at most kMaxSplits), merged afterwards by their
+// log-sum-exp.  (The merge costs a launch of about 10 us; on a 16-row layer
+// with 17-tile rows, splitting measured slower than not.)
+constexpr int64_t kSchedL2Bytes = (int64_t)64 << 20;
+constexpr int kSchedSMs = 148;
+constexpr int kMinSplitTiles = 8;
+constexpr int kMinSplitRow = 32;
+constexpr int kMaxSplits = 32;   // splits of one row (the merge takes one per lane)
+// Passes over the grid up to which CTAs alternate their direction through the
+// schedule (fewer, longer items per CTA: evens out the decreasing lengths).
+constexpr int kZigZagMaxPasses = 16;
+
+// Upper bound of the tiles of row i (kept blocks 0..i plus pseudo tiles of
+// B block means each) and the number of splits it gets for split size c
+// (0: rows are never split).
+__host__ __device__ inline int64_t row_tile_bound(int64_t i, int B) { return i + 1 + (i + B - 1) / B; }
+__host__ __device__ inline int row_splits(int64_t i, int B, int c) {
+    return c ? (int)((row_tile_bound(i, B) + c - 1) / c) : 1;
+}
+
 // Derived sizes of one problem (host computed, passed to kernels by value).
 struct Dims {
     int n_seqs;
@@ -32,6 +58,17 @@ struct Dims {
     int64_t T, NB, R, tri_total, nnz_cap;
     int64_t score_tiles;  // (query group, 128-key-block chunk) tiles inside the causal triangles
     double tau;
+};
+
+// Sizes of the attention schedule (host computed; passed only to the kernels
+// that build or read the schedule).
+struct SchedDims {
+    int n_mtiles;           // 128-row query tiles per row, G * B / 128
+    int n_pairs;            // work items per row split, ceil(n_mtiles / 2)
+    int split_c;            // split size in tiles (0: no row is split)
+    int heads_per_chunk;    // kv-heads per schedule chunk
+    int64_t n_items;        // work items of the layer
+    int64_t split_slots;    // row splits of split rows, per kv-head
 };
 
 // Device pointers into the plan buffer.
@@ -57,6 +94,12 @@ struct PlanPtrs {
     int32_t* group_seq;    // [n_groups_cap]
     int32_t* tile_cu;      // [n_groups_cap+1] prefix of scoring tiles per row group
     float* vmax;           // [n, Hkv]  largest V scale of each sequence and kv-head (FP8)
+    int4* sched;           // [n_items]  {global block, g | pair << 16, split | splits << 16, slot}
+    int32_t* sched_cnt;    // [max_nb]   sequences longer than i blocks
+    int64_t* sched_off;    // [max_nb]   items of one kv-head's rows with a larger i
+    float* split_o;        // [Hkv * split_slots, G * B, d]  O of one split (normalised)
+    float* split_lse;      // [Hkv * split_slots, G * B]     its log2-sum-exp
+    int32_t* slot_item;    // [Hkv * split_slots]  schedule index of the slot's row (split 0, pair 0)
 };
 
 // Device pointers into fp2_plan's workspace.
@@ -74,9 +117,11 @@ struct WsPtrs {
 
 struct Layout {
     Dims dims;
+    SchedDims sched;
     fp2_plan_layout pub;
     size_t off_meta_valid, off_cu_blocks, off_block_seq, off_tri_off, off_group_cu, off_group_seq,
-        off_tile_cu, off_vmax;
+        off_tile_cu, off_vmax, off_sched, off_sched_cnt, off_sched_off, off_split_o, off_split_lse,
+        off_slot_item;
     size_t ws_qbar64, ws_qbar32, ws_kbar_tf, ws_kbar64, ws_qnorm, ws_knorm, ws_scores, ws_counts;
 };
 

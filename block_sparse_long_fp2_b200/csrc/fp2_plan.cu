@@ -3,7 +3,8 @@
 // scores under PackGQA, max-based thresholding and the CSR block index.
 //
 // Kernels, in launch order:
-//   meta     one CTA: checks cu_seqlens, derives block / scoring-group maps.
+//   meta     one CTA: checks cu_seqlens, derives block / scoring-group maps
+//            and the attention kernel's work schedule.
 //   pool     HBM-bound: streams Q, K, V once with 16-byte coalesced loads and
 //            accumulates each block's sum in float64 (exact for bf16 inputs),
 //            writing Qbar (fp64 workspace) and Kbar/Vbar (fp32, bf16, fp64).
@@ -29,10 +30,106 @@ namespace fp2 {
 namespace {
 
 // ---------------------------------------------------------------------------
-// meta: sequence -> block and scoring-group maps, device-side checks
+// meta: sequence -> block and scoring-group maps, device-side checks, and the
+// attention kernel's work schedule
 // ---------------------------------------------------------------------------
 
-__global__ void k_meta(Dims D, const int32_t* __restrict__ cu_seqlens,
+constexpr int kMetaThreads = 1024;
+
+// Exclusive prefix sum of v over the CTA (blockDim.x == kMetaThreads); every
+// thread gets the CTA's total in *total.
+__device__ int64_t block_excl_scan(int64_t v, int64_t* total) {
+    __shared__ int64_t warp_sum[kMetaThreads / 32];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int64_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sum[w] = x;
+    __syncthreads();
+    if (w == 0) {
+        int64_t t = warp_sum[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int64_t y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        warp_sum[lane] = t;
+    }
+    __syncthreads();
+    const int64_t before = (w ? warp_sum[w - 1] : 0) + x - v;
+    *total = warp_sum[kMetaThreads / 32 - 1];
+    __syncthreads();
+    return before;
+}
+
+// The attention kernel's work items in the order its CTAs take them: kv-head
+// chunks in order; inside a chunk the rows by block index i, largest first,
+// then kv-head, then sequence; inside a row its splits, then its query-tile
+// pairs.  Rows with the same i have the same number of items, so every
+// row's position follows from prefix sums over i.
+__device__ void build_schedule(const Dims& D, const SchedDims& S, const PlanPtrs& P) {
+    for (int i = threadIdx.x; i < D.max_nb; i += blockDim.x) {
+        int c = 0;
+        for (int s = 0; s < D.n_seqs; ++s) c += (P.cu_blocks[s + 1] - P.cu_blocks[s]) > i;
+        P.sched_cnt[i] = c;
+    }
+    __syncthreads();
+    // sched_off[i]: items of one kv-head's rows with a larger i (suffix sums,
+    // blockDim.x entries at a time from the largest i down)
+    int64_t per_head = 0, slots = 0;
+    for (int base = 0; base < D.max_nb; base += blockDim.x) {
+        const int i = D.max_nb - 1 - (base + (int)threadIdx.x);
+        int64_t v = 0, sv = 0;
+        if (i >= 0) {
+            const int ns = row_splits(i, D.B, S.split_c);
+            v = (int64_t)P.sched_cnt[i] * ns * S.n_pairs;
+            sv = ns > 1 ? (int64_t)P.sched_cnt[i] * ns : 0;
+        }
+        int64_t tot, stot;
+        const int64_t ex = block_excl_scan(v, &tot);
+        block_excl_scan(sv, &stot);
+        if (i >= 0) P.sched_off[i] = per_head + ex;
+        per_head += tot;
+        slots += stot;
+    }
+    if (per_head * D.Hkv != S.n_items || slots != S.split_slots) {
+        if (threadIdx.x == 0) {
+            *P.meta_valid = 0;
+            atomicOr(P.status, (int32_t)FP2_STATUS_BAD_SEQLENS);
+        }
+        return;
+    }
+    __syncthreads();
+    for (int64_t b = threadIdx.x; b < D.NB; b += blockDim.x) {
+        const int s = P.block_seq[b];
+        const int i = (int)(b - P.cu_blocks[s]);
+        int rank = 0;   // earlier sequences that also have a block i
+        for (int s2 = 0; s2 < s; ++s2) rank += (P.cu_blocks[s2 + 1] - P.cu_blocks[s2]) > i;
+        const int ns = row_splits(i, D.B, S.split_c);
+        const int64_t w = (int64_t)ns * S.n_pairs;
+        const int64_t cnt = P.sched_cnt[i], off = P.sched_off[i];
+        for (int g = 0; g < D.Hkv; ++g) {
+            const int g0 = g - g % S.heads_per_chunk;
+            const int nh = min(S.heads_per_chunk, D.Hkv - g0);
+            const int64_t in_chunk = off * nh + ((g - g0) * cnt + rank) * w;
+            const int64_t first = (int64_t)g0 * per_head + in_chunk;
+            // split rows come first in their chunk, so their items, counted in
+            // row splits, number the split slots
+            const int slot = ns > 1 ? (int)((int64_t)g0 * S.split_slots + in_chunk / S.n_pairs) : 0;
+            if (ns > 1)
+                for (int k = 0; k < ns; ++k) P.slot_item[slot + k] = (int32_t)first;
+            for (int k = 0; k < ns; ++k)
+                for (int mp = 0; mp < S.n_pairs; ++mp)
+                    P.sched[first + (int64_t)k * S.n_pairs + mp] =
+                        make_int4((int)b, g | (mp << 16), k | (ns << 16), slot);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kMetaThreads) k_meta(Dims D, SchedDims S, const int32_t* __restrict__ cu_seqlens,
                        const int32_t* __restrict__ page_table, PlanPtrs P) {
     __shared__ int s_valid;
     if (threadIdx.x == 0) {
@@ -88,6 +185,8 @@ __global__ void k_meta(Dims D, const int32_t* __restrict__ cu_seqlens,
             }
         }
     }
+    __syncthreads();
+    build_schedule(D, S, P);
 }
 
 // ---------------------------------------------------------------------------
@@ -730,7 +829,7 @@ int launch_plan(const Layout& L, const fp2_problem* p, const void* q, const void
                 const PlanPtrs& P, const WsPtrs& W, cudaStream_t st, const float* k_scale,
                 const float* v_scale) {
     const Dims& D = L.dims;
-    k_meta<<<1, 256, 0, st>>>(D, p->cu_seqlens, p->page_table, P);
+    k_meta<<<1, kMetaThreads, 0, st>>>(D, L.sched, p->cu_seqlens, p->page_table, P);
     const int vecs = (D.Hq + 2 * D.Hkv) * D.d / 8;
     dim3 pool_grid((unsigned)D.NB, (vecs + kPoolThreads - 1) / kPoolThreads);
     if (k_scale)

@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define FP2_VERSION 1
+#define FP2_VERSION 2
 
 /* ---- error codes -------------------------------------------------------- */
 #define FP2_OK 0
@@ -165,6 +165,8 @@ typedef struct fp2_plan_layout {
     size_t off_meta;
     size_t plan_bytes;        /* bytes the plan buffer must have      */
     size_t workspace_bytes;   /* bytes fp2_plan's scratch must have    */
+    int64_t num_work_items;   /* fp2_prefill's work items (rows x splits x query-tile pairs) */
+    int64_t num_split_slots;  /* row splits of the rows fp2_prefill splits (0: none)          */
 } fp2_plan_layout;
 
 /* Library version (FP2_VERSION of the build). */
@@ -233,8 +235,20 @@ int fp2_quantize_fp8(const fp2_problem* problem, const void* plan, size_t plan_b
  *   o    DEVICE bf16 [T, Hq, d]   attention output.
  *   lse  DEVICE float [Hq, T]     natural-log softmax denominator.
  *   flags  FP2_NO_CORRECTION and FP2_DEBUG_* bits.
- * Work is spread over one persistent CTA per SM; each CTA takes PackGQA
- * tiles (two 128-row query tiles of one kv-head) longest row first.
+ * Work is spread over one persistent CTA per SM.  A work item is two 128-row
+ * PackGQA query tiles of one row (kv-head g, query block i); fp2_plan lists
+ * the items longest row first within chunks of kv-heads whose K and V fit
+ * together in L2, and CTA c takes the c-th item of each pass over the grid
+ * (from the other end on odd passes, when there are at most 16 passes).  KV
+ * splitting (Table 7, "count-balanced CSR splits"): when the longest row's
+ * tile bound i + 1 + ceil(i / B) exceeds both 32 and the layer's mean tiles
+ * per CTA (over 148 CTAs), every row whose bound exceeds half that mean (and
+ * at least 8) is cut into
+ * splits of equal numbers of its tiles (kept blocks in CSR order, then pseudo
+ * tiles); each split writes its normalised fp32 O and log-sum-exp into the
+ * plan's private scratch, and a merge kernel combines them by log-sum-exp into
+ * o and lse.  Because fp2_prefill writes that scratch, two fp2_prefill calls
+ * on one plan must not overlap on the GPU (order them on one stream).
  */
 int fp2_prefill(const fp2_problem* problem, const void* plan, size_t plan_bytes,
                 const void* q, const void* k, const void* v,

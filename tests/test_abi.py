@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_strerror(lib):
-    assert fb.fp2_version() == 1
+    assert fb.fp2_version() == 2
     assert fb.strerror(0) == "ok"
     for code in [-1, -2, -3, -4, -5, -6]:
         assert fb.strerror(code) not in ("", "unknown error")

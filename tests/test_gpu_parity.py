@@ -44,6 +44,9 @@ SMALL = {
     # degenerate lengths: one token, two tokens, a block plus one, a partial block
     "tiny_lengths": ([1, 2, 129, 3, 130], 8, 2, 128, 128, 0.5, "normal", 0, 0, 0),
     "tiny_paged": ([1, 65, 64], 8, 2, 128, 128, 0.5, "normal", 0, 64, 8),
+    # one kv-head with long rows: the rows are cut into count-balanced splits
+    "split_long_rows": ([4096], 2, 1, 64, 64, 0.2, "lowrank", 0, 0, 0),
+    "split_d128_paged": ([3000, 700], 2, 1, 128, 64, 0.1, "normal", 0, 64, 70),
 }
 
 
@@ -105,6 +108,27 @@ def test_no_correction_flag_drops_the_surrogate():
     run2 = GpuRun(wl, x).plan().prefill()
     assert len(run2.kept_lists()[0]) >= 1
     assert float((run2.lse - run.lse).abs().max()) > 1e-2
+
+
+@pytest.mark.parametrize("flags", [0, fb.FP2_NO_CORRECTION])
+def test_split_rows_with_empty_splits_match_oracle(flags):
+    # One 4096-token sequence with 2/1 heads and B = 64 gives 64 rows of one
+    # query tile for 148 SMs, so the long rows are cut into count-balanced
+    # splits (row 63 into 9) merged by log-sum-exp.  At tau = 1 a row keeps 2
+    # or 3 blocks (plus one pseudo tile with the correction), so most of its
+    # splits have no tile at all.
+    wl = synth.small_workload([4096], 2, 1, 64, 64, 1.0, seed=98, generator="normal")
+    x = synth.generate(wl)
+    run = GpuRun(wl, x).plan()
+    assert run.lay.num_split_slots > 0 and run.lay.num_work_items > 64
+    run.prefill(flags=flags)
+    rc, st = run.status()
+    assert rc == fb.FP2_OK and st == 0
+    q, k, v = oracle_inputs(x, wl)
+    pl = oracle.plan(q, k, v, wl.seqlens, wl.B, wl.tau)
+    assert len(run.kept_lists()[63]) + 1 < 9   # fewer tiles than splits
+    res = check_attention(wl, x, run, pl, correction=flags == 0)
+    assert res["finite"] and res["rel_l2"] <= REL_L2_BF16 and res["lse_max_abs"] <= LSE_ABS, res
 
 
 def test_dense_tau0_equals_brute_force_dense():
@@ -277,7 +301,8 @@ def _fp8_run(wl, x, run):
 
 
 @pytest.mark.parametrize("name,gen", [("ragged_d128", "normal"), ("ragged_d128", "lowrank"),
-                                      ("B64_d128", "normal"), ("paged_mix_small", "normal")])
+                                      ("B64_d128", "normal"), ("paged_mix_small", "normal"),
+                                      ("split_d128_paged", "normal")])
 def test_fp8_prefill(name, gen):
     from fp2_harness import rel_l2, token_rows
     seqlens, Hq, Hkv, d, B, tau, _, nn, page, pool = SMALL[name]
