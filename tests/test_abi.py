@@ -61,6 +61,38 @@ def _problem(seqlens=(1000, 37), Hq=32, Hkv=8, d=128, B=128, tau=0.1, page_size=
     return p
 
 
+def _schedule_sizes(seqlens, Hq, Hkv, B):
+    # The documented split rule of fp2_prefill's work schedule, restated: the
+    # tile bound of row i is i + 1 + ceil(i / B); rows split only when the
+    # longest bound exceeds both 32 and the layer's mean tiles per CTA over 148
+    # CTAs, with split size max(8, ceil(mean / 2), ceil(longest / 32)).
+    G = Hq // Hkv
+    pairs = (G * B // 128 + 1) // 2
+    rows = [i for L in seqlens for i in range((L + B - 1) // B)]
+    bound = [i + 1 + (i + B - 1) // B for i in rows]
+    share = -(-sum(bound) * Hkv * pairs // 148)
+    longest = max(bound)
+    c = max(8, (share + 1) // 2, -(-longest // 32))
+    if longest <= share or longest < 32:
+        c = 0
+    splits = [-(-u // c) if c else 1 for u in bound]
+    return sum(splits) * Hkv * pairs, sum(x for x in splits if x > 1) * Hkv
+
+
+@pytest.mark.parametrize("shape", [((1024,), 4, 1, 64), ((4096,), 32, 8, 128), ((4096,), 2, 1, 64),
+                                   ((3000, 700), 2, 1, 64), ((131072,), 32, 8, 128),
+                                   ((4096, 9000, 16384, 30000, 65536, 1500), 32, 8, 128),
+                                   ((1, 2, 129, 3, 130), 8, 2, 128), ((9000,), 2, 1, 64)])
+def test_schedule_sizes_follow_the_split_rule(lib, shape):
+    seqlens, Hq, Hkv, B = shape
+    lay = fb.fp2_plan_sizes(_problem(seqlens, Hq, Hkv, 128 if B == 128 else 64, B))
+    items, slots = _schedule_sizes(seqlens, Hq, Hkv, B)
+    assert (lay.num_work_items, lay.num_split_slots) == (items, slots)
+    # every row has at least one item per query-tile pair
+    G = Hq // Hkv
+    assert lay.num_work_items >= lay.num_rows * ((G * B // 128 + 1) // 2)
+
+
 def test_plan_sizes_counts(lib):
     lay = fb.fp2_plan_sizes(_problem())
     nb = [8, 1]
