@@ -20,10 +20,13 @@ for Long-Context LLM Serving" (metallab.ai summary of arXiv 2608.19758):
 * Abstract -- "max-based dynamic thresholding" (Table 9 calls the threshold
   alpha; here it is tau).
 * Table 1 footnote / Table 7 -- FP8 via direct online quantisation.
+* Table 6 -- chunked prefill (a chunk of new queries over a KV cache holding
+  the earlier tokens): ``oracle.fp2_chunked``, under the reading stated in
+  its module docstring.
 
-Pinned by ``tests/test_oracle.py`` (see the module docstring of
-``oracle.fp2_oracle`` for which pin covers which function).  No function
-here is "parity unpinned".
+Pinned by ``tests/test_oracle.py`` and ``tests/test_oracle_chunked.py`` (see
+the module docstrings of ``oracle.fp2_oracle`` and ``oracle.fp2_chunked`` for
+which pin covers which function).  No function here is "parity unpinned".
 """
 
 from .fp2_oracle import (  # noqa: F401
@@ -41,4 +44,10 @@ from .fp2_oracle import (  # noqa: F401
     dequantize_e4m3,
     quantize_means_e4m3,
     dequantize_means_e4m3,
+)
+from .fp2_chunked import (  # noqa: F401
+    chunk_layout,
+    query_block_means,
+    plan_chunk,
+    attend_chunk,
 )
