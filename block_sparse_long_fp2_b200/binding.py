@@ -62,6 +62,8 @@ class fp2_problem(ctypes.Structure):
         ("num_pages", ctypes.c_int32),
         ("page_table", ctypes.c_void_p),
         ("page_table_stride", ctypes.c_int32),
+        ("q_seqlens", ctypes.POINTER(ctypes.c_int32)),
+        ("cu_q_seqlens", ctypes.c_void_p),
     ]
 
 
@@ -168,7 +170,8 @@ class Problem:
 
     def __init__(self, seqlens: Sequence[int], cu_seqlens, num_q_heads: int, num_kv_heads: int,
                  head_dim: int, block_size: int, tau: float, page_size: int = 0,
-                 page_table=None, num_pages: int = 0):
+                 page_table=None, num_pages: int = 0, q_seqlens: Optional[Sequence[int]] = None,
+                 cu_q_seqlens=None):
         self.seqlens_np = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
         self.cu_seqlens = cu_seqlens
         self.page_table = page_table
@@ -185,6 +188,13 @@ class Problem:
         self.c.num_pages = num_pages
         self.c.page_table = _ptr(page_table)
         self.c.page_table_stride = int(page_table.shape[1]) if page_table is not None else 0
+        # chunked prefill: new queries per sequence (host) and their prefix sums (device)
+        self.q_seqlens_np = None
+        self.cu_q_seqlens = cu_q_seqlens
+        if q_seqlens is not None:
+            self.q_seqlens_np = np.ascontiguousarray(np.asarray(q_seqlens, dtype=np.int32))
+            self.c.q_seqlens = self.q_seqlens_np.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+            self.c.cu_q_seqlens = _ptr(cu_q_seqlens)
 
     @property
     def ref(self):

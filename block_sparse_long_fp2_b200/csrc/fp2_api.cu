@@ -41,6 +41,14 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     if (G > kScoreQV) return FP2_ERR_UNSUPPORTED;
     if ((G * p->block_size) % kTileM != 0) return FP2_ERR_UNSUPPORTED;
     if (p->page_size != 0 && p->page_size != 64) return FP2_ERR_UNSUPPORTED;
+    const bool chunked = p->q_seqlens != nullptr;
+    if (chunked != (p->cu_q_seqlens != nullptr)) return FP2_ERR_INVALID_ARG;
+    int64_t Tq = 0;
+    if (chunked)
+        for (int s = 0; s < p->num_seqs; ++s) {
+            if (p->q_seqlens[s] < 1 || p->q_seqlens[s] > p->seqlens[s]) return FP2_ERR_INVALID_ARG;
+            Tq += p->q_seqlens[s];
+        }
 
     Dims d{};
     d.n_seqs = p->num_seqs;
@@ -91,10 +99,14 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     SchedDims sd{};
     sd.n_mtiles = G * d.B / kTileM;
     sd.n_pairs = (sd.n_mtiles + 1) / 2;
+    // rows of a chunked sequence start at the chunk's first query block
+    auto first_row = [&](int s) -> int64_t {
+        return chunked ? (int64_t)(p->seqlens[s] - p->q_seqlens[s]) / d.B : 0;
+    };
     int64_t units = 0;
     for (int s = 0; s < p->num_seqs; ++s) {
         const int64_t nb = (p->seqlens[s] + d.B - 1) / d.B;
-        for (int64_t i = 0; i < nb; ++i) units += row_tile_bound(i, d.B);
+        for (int64_t i = first_row(s); i < nb; ++i) units += row_tile_bound(i, d.B);
     }
     const int64_t share = (units * d.Hkv * sd.n_pairs + kSchedSMs - 1) / kSchedSMs;
     const int64_t longest = row_tile_bound(max_nb - 1, d.B);
@@ -107,7 +119,7 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     int64_t items = 0, slots = 0;
     for (int s = 0; s < p->num_seqs; ++s) {
         const int64_t nb = (p->seqlens[s] + d.B - 1) / d.B;
-        for (int64_t i = 0; i < nb; ++i) {
+        for (int64_t i = first_row(s); i < nb; ++i) {
             const int S = row_splits(i, d.B, sd.split_c);
             items += S;
             if (S > 1) slots += S;
@@ -125,6 +137,8 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     std::memset(&L, 0, sizeof(L));
     L.dims = d;
     L.sched = sd;
+    L.chunked = chunked;
+    L.Tq = chunked ? Tq : T;
     fp2_plan_layout& pub = L.pub;
     pub.num_tokens = T;
     pub.num_blocks = NB;
@@ -164,6 +178,7 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     L.off_split_o = c.take(sizeof(float) * split_rows * d.d);
     L.off_split_lse = c.take(sizeof(float) * split_rows);
     L.off_slot_item = c.take(sizeof(int32_t) * (size_t)sd.split_slots * d.Hkv);
+    L.off_q_off = c.take(sizeof(int32_t) * n);
     pub.plan_bytes = align_up(c.off, 256);
 
     Carver w;
@@ -211,6 +226,8 @@ PlanPtrs plan_ptrs(const Layout& L, void* plan) {
     p.split_o = reinterpret_cast<float*>(b + L.off_split_o);
     p.split_lse = reinterpret_cast<float*>(b + L.off_split_lse);
     p.slot_item = reinterpret_cast<int32_t*>(b + L.off_slot_item);
+    p.q_off = reinterpret_cast<int32_t*>(b + L.off_q_off);
+    p.cu_q = nullptr;
     return p;
 }
 
@@ -357,6 +374,7 @@ int fp2_quantize_fp8(const fp2_problem* problem, const void* plan, size_t plan_b
     if (!aligned(x, 16) || !aligned(x_e4m3, 16) || !aligned(scales, 4) || !aligned(plan, 256))
         return FP2_ERR_INVALID_ARG;
     if (plan_bytes < L.pub.plan_bytes) return FP2_ERR_CAPACITY;
+    if (L.chunked && which == 0) return FP2_ERR_UNSUPPORTED;   // e4m3 chunks: not built
     return launch_quantize(L, problem, plan_ptrs(L, const_cast<void*>(plan)), x, which, x_e4m3,
                            scales, static_cast<cudaStream_t>(stream));
 }
@@ -379,7 +397,7 @@ int fp2_prefill(const fp2_problem* problem, const void* plan, size_t plan_bytes,
         if (!q_scale || !k_scale || !v_scale) return FP2_ERR_INVALID_ARG;
         if (!aligned(q_scale, 4) || !aligned(k_scale, 4) || !aligned(v_scale, 4))
             return FP2_ERR_INVALID_ARG;
-        if (L.dims.d != 128) return FP2_ERR_UNSUPPORTED;
+        if (L.dims.d != 128 || L.chunked) return FP2_ERR_UNSUPPORTED;
     } else {
         return FP2_ERR_INVALID_ARG;
     }

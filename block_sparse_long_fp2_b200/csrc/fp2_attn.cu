@@ -138,6 +138,11 @@ struct AttnParams {
     float* split_o;
     float* split_lse;
     const int32_t* slot_item;
+    // queries: q, o and lse hold Tq tokens; sequence s's queries start at
+    // token cu_q[s] and position q_off[s] (a chunk; cu_seqlens and 0 otherwise)
+    const int32_t* cu_q;
+    const int32_t* q_off;
+    int64_t Tq;
     int64_t n_items;   // work items in the schedule
     int64_t n_slots;   // n_items rounded up to whole passes of the grid
     bool zigzag;       // odd passes run backwards
@@ -311,7 +316,7 @@ __device__ __forceinline__ uint32_t col_bits(int kind, int tok, const TileWalk<B
 // producer (warp 8, one lane)
 // ---------------------------------------------------------------------------
 
-template <int HD, int BLK, bool F8>
+template <int HD, int BLK, bool F8, bool CHUNK>
 __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUtensorMap* tm_q,
                          const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                          const CUtensorMap* tm_kbar, const CUtensorMap* tm_vbar) {
@@ -329,6 +334,10 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
         TileWalk<BLK> walk;
         walk.init(P, it);
         if (walk.count() == 0) continue;   // a split without tiles
+        // q token of position 0 of the sequence (for a chunk that starts inside
+        // the block, rows before the chunk read zeros or another sequence's
+        // queries: they are never written)
+        const int qtok = CHUNK ? P.cu_q[it.s] - P.q_off[it.s] : it.tok0;
         for (int m = 0; m < 2; ++m) {
             if (m == 1 && !it.has_m1) break;
             if (!mbar_wait(&B.q_empty[m], (qcnt[m] & 1) ^ 1, &B.abort, P.status)) goto drain;
@@ -344,7 +353,7 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
 #pragma unroll
                 for (int a = 0; a < C::kAtoms; ++a)
                     tma_load_3d(qdst + a * C::kAtomQ + ht * BLK * 128, tm_q, &B.q_full[m],
-                                C::kAtomElems * a, it.g * D.G + hl, it.tok0 + it.i * BLK);
+                                C::kAtomElems * a, it.g * D.G + hl, qtok + it.i * BLK);
             }
         }
         int kind, j;
@@ -744,7 +753,7 @@ __device__ __forceinline__ float tile_softmax(uint32_t t_s, int kind, int tok,
 // softmax + correction + epilogue (warps 0-7)
 // ---------------------------------------------------------------------------
 
-template <int HD, int BLK, bool F8>
+template <int HD, int BLK, bool F8, bool CHUNK>
 __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
     using C = Cfg<HD, BLK, F8>;
     const Dims& D = P.D;
@@ -773,7 +782,9 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
         const int tok = pr % BLK;
         const int h = it.g * D.G + hl;
         const int pos = it.i * BLK + tok;
-        const bool row_valid = pos < it.L;
+        const int qoff = CHUNK ? P.q_off[it.s] : 0;
+        const bool row_valid = pos < it.L && (!CHUNK || pos >= qoff);
+        const int64_t qtok = CHUNK ? (int64_t)P.cu_q[it.s] - qoff : it.tok0;   // q token of position 0
         RowState st{-INFINITY, 0.f, t_o, false};
         // e4m3: the logit scale folds in the Q scale of this row's block and
         // head; P' = P s_V K_row with K_row = 448 / (2^8 max s_V) over the
@@ -826,7 +837,7 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
         const float inv_l = 1.0f / (st.l * k_row);
         const bool split = split_slot >= 0;
         const int64_t srow = (int64_t)split_slot * (D.G * BLK) + pr;
-        const int64_t orow = (int64_t)(it.tok0 + pos) * D.Hq + h;
+        const int64_t orow = (qtok + pos) * D.Hq + h;
         char* dst = split ? reinterpret_cast<char*>(P.split_o + srow * HD)
                           : reinterpret_cast<char*>(P.o + orow * HD);
 #pragma unroll
@@ -854,14 +865,14 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
         }
         const float lse2 = st.m_ref + log2f(st.l);
         if (row_valid && split) P.split_lse[srow] = lse2;
-        else if (row_valid) P.lse[(int64_t)h * D.T + it.tok0 + pos] = lse2 * 0.6931471805599453f;
+        else if (row_valid) P.lse[(int64_t)h * (CHUNK ? P.Tq : D.T) + qtok + pos] = lse2 * 0.6931471805599453f;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.o_free[m]);
     }
 }
 
-template <int HD, int BLK, bool F8>
+template <int HD, int BLK, bool F8, bool CHUNK>
 __global__ void __launch_bounds__(kThreads, 1)
 k_attn(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap tm_q,
        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -906,9 +917,9 @@ k_attn(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap
     tc_fence_after();
 
     if (warp < 8) {
-        softmax_wg<HD, BLK, F8>(P, B, smem, warp >> 2);
+        softmax_wg<HD, BLK, F8, CHUNK>(P, B, smem, warp >> 2);
     } else if (warp == kProducerWarp) {
-        if (lane == 0) producer<HD, BLK, F8>(P, B, smem, &tm_q, &tm_k, &tm_v, &tm_kbar, &tm_vbar);
+        if (lane == 0) producer<HD, BLK, F8, CHUNK>(P, B, smem, &tm_q, &tm_k, &tm_v, &tm_kbar, &tm_vbar);
     } else {
         if (lane == 0) mma_issuer<HD, BLK, F8>(P, B, smem);
     }
@@ -962,7 +973,9 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(const __grid_consta
         const int tok = pr % BLK;
         const int h = it.g * D.G + pr / BLK;
         const int pos = it.i * BLK + tok;
-        if (pos >= it.L) continue;
+        const int qoff = P.q_off[it.s];
+        if (pos >= it.L || pos < qoff) continue;
+        const int64_t qtok = (int64_t)P.cu_q[it.s] - qoff;
         // lane k holds split k's log-sum-exp (-inf when the split had no tile)
         const bool live = lane < it.S && split_nonempty(lane, it.S, n);
         const float lk = live ? P.split_lse[(it.slot + lane) * gb + pr] : -INFINITY;
@@ -993,7 +1006,7 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(const __grid_consta
             }
         }
         const float inv = 1.0f / wsum;
-        uint16_t* orow = P.o + ((int64_t)(it.tok0 + pos) * D.Hq + h) * HD + lane * E;
+        uint16_t* orow = P.o + ((qtok + pos) * D.Hq + h) * HD + lane * E;
         if constexpr (E == 4) {
             uint2 v;
             v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
@@ -1002,7 +1015,7 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(const __grid_consta
         } else {
             *reinterpret_cast<uint32_t*>(orow) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
         }
-        if (lane == 0) P.lse[(int64_t)h * D.T + it.tok0 + pos] = (mx + log2f(wsum)) * 0.6931471805599453f;
+        if (lane == 0) P.lse[(int64_t)h * P.Tq + qtok + pos] = (mx + log2f(wsum)) * 0.6931471805599453f;
     }
 }
 
@@ -1042,7 +1055,7 @@ int launch_attn_t(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, con
     const cuuint32_t ae = C::kAtomElems;                   // elements per 128-byte atom row
     CUtensorMap tq, tk, tv, tkb, tvb;
     {
-        cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)D.Hq, (cuuint64_t)D.T};
+        cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)D.Hq, (cuuint64_t)L.Tq};
         cuuint64_t str[2] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hq * HD * eb};
         cuuint32_t box[3] = {ae, 1, (cuuint32_t)BLK};
         if (!make_tensor_map(&tq, q, 3, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
@@ -1097,16 +1110,22 @@ int launch_attn_t(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, con
     P.split_o = pp.split_o;
     P.split_lse = pp.split_lse;
     P.slot_item = pp.slot_item;
+    P.cu_q = L.chunked ? p->cu_q_seqlens : p->cu_seqlens;
+    P.q_off = pp.q_off;
+    P.Tq = L.Tq;
     const int sms = sm_count();
     if (sms <= 0) return FP2_ERR_CUDA;
     const int64_t grid = S.n_items < sms ? S.n_items : sms;
     P.n_slots = (S.n_items + grid - 1) / grid * grid;
     P.zigzag = P.n_slots / grid <= kZigZagMaxPasses;
-    if (cudaFuncSetAttribute(k_attn<HD, BLK, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
+    auto kernel = k_attn<HD, BLK, F8, false>;
+    if constexpr (!F8)
+        if (L.chunked) kernel = k_attn<HD, BLK, false, true>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+        cudaSuccess)
         return FP2_ERR_CUDA;
     if (F8) k_vmax<<<dim3(D.n_seqs, D.Hkv), 256, 0, st>>>(D, pp, vs);
-    k_attn<HD, BLK, F8><<<(unsigned)grid, kThreads, C::kSmemBytes, st>>>(P, tq, tk, tv, tkb, tvb);
+    kernel<<<(unsigned)grid, kThreads, C::kSmemBytes, st>>>(P, tq, tk, tv, tkb, tvb);
     if (S.split_slots > 0)
         k_combine<HD, BLK><<<dim3((unsigned)(S.split_slots * D.Hkv), S.n_pairs * (2 * kTileM / kCombineRows)),
                              kCombineThreads, 0, st>>>(P);

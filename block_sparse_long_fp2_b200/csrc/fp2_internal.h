@@ -100,6 +100,8 @@ struct PlanPtrs {
     float* split_o;        // [Hkv * split_slots, G * B, d]  O of one split (normalised)
     float* split_lse;      // [Hkv * split_slots, G * B]     its log2-sum-exp
     int32_t* slot_item;    // [Hkv * split_slots]  schedule index of the slot's row (split 0, pair 0)
+    int32_t* q_off;        // [n]  position of the first query (L - Q for a chunk, else 0)
+    const int32_t* cu_q;   // caller's cu_q_seqlens for a chunked problem, else null (set per call)
 };
 
 // Device pointers into fp2_plan's workspace.
@@ -118,10 +120,12 @@ struct WsPtrs {
 struct Layout {
     Dims dims;
     SchedDims sched;
+    bool chunked;   // q holds a chunk of each sequence (q_seqlens given)
+    int64_t Tq;     // query tokens (T unless chunked)
     fp2_plan_layout pub;
     size_t off_meta_valid, off_cu_blocks, off_block_seq, off_tri_off, off_group_cu, off_group_seq,
         off_tile_cu, off_vmax, off_sched, off_sched_cnt, off_sched_off, off_split_o, off_split_lse,
-        off_slot_item;
+        off_slot_item, off_q_off;
     size_t ws_qbar64, ws_qbar32, ws_kbar_tf, ws_kbar64, ws_qnorm, ws_knorm, ws_scores, ws_counts;
 };
 

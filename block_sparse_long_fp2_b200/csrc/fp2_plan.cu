@@ -65,6 +65,12 @@ __device__ int64_t block_excl_scan(int64_t v, int64_t* total) {
     return before;
 }
 
+// Whether sequence s has a row for query block i: i below its block count and
+// not below the first query block of its chunk.
+__device__ __forceinline__ bool has_row(const Dims& D, const PlanPtrs& P, int s, int i) {
+    return i < P.cu_blocks[s + 1] - P.cu_blocks[s] && i >= P.q_off[s] / D.B;
+}
+
 // The attention kernel's work items in the order its CTAs take them: kv-head
 // chunks in order; inside a chunk the rows by block index i, largest first,
 // then kv-head, then sequence; inside a row its splits, then its query-tile
@@ -73,7 +79,7 @@ __device__ int64_t block_excl_scan(int64_t v, int64_t* total) {
 __device__ void build_schedule(const Dims& D, const SchedDims& S, const PlanPtrs& P) {
     for (int i = threadIdx.x; i < D.max_nb; i += blockDim.x) {
         int c = 0;
-        for (int s = 0; s < D.n_seqs; ++s) c += (P.cu_blocks[s + 1] - P.cu_blocks[s]) > i;
+        for (int s = 0; s < D.n_seqs; ++s) c += has_row(D, P, s, i) ? 1 : 0;
         P.sched_cnt[i] = c;
     }
     __syncthreads();
@@ -106,8 +112,9 @@ __device__ void build_schedule(const Dims& D, const SchedDims& S, const PlanPtrs
     for (int64_t b = threadIdx.x; b < D.NB; b += blockDim.x) {
         const int s = P.block_seq[b];
         const int i = (int)(b - P.cu_blocks[s]);
-        int rank = 0;   // earlier sequences that also have a block i
-        for (int s2 = 0; s2 < s; ++s2) rank += (P.cu_blocks[s2 + 1] - P.cu_blocks[s2]) > i;
+        if (!has_row(D, P, s, i)) continue;   // query block below the chunk
+        int rank = 0;   // earlier sequences that also have a row i
+        for (int s2 = 0; s2 < s; ++s2) rank += has_row(D, P, s2, i) ? 1 : 0;
         const int ns = row_splits(i, D.B, S.split_c);
         const int64_t w = (int64_t)ns * S.n_pairs;
         const int64_t cnt = P.sched_cnt[i], off = P.sched_off[i];
@@ -129,15 +136,21 @@ __device__ void build_schedule(const Dims& D, const SchedDims& S, const PlanPtrs
     }
 }
 
-__global__ void __launch_bounds__(kMetaThreads) k_meta(Dims D, SchedDims S, const int32_t* __restrict__ cu_seqlens,
-                       const int32_t* __restrict__ page_table, PlanPtrs P) {
+// P.cu_q: prefix sums of a chunk's query counts (chunked prefill), or null;
+// Tq their total.
+__global__ void __launch_bounds__(kMetaThreads, 1) k_meta(Dims D, SchedDims S, const int32_t* __restrict__ cu_seqlens,
+                       const int32_t* __restrict__ page_table, int64_t Tq, PlanPtrs P) {
+    const int32_t* __restrict__ cu_q = P.cu_q;
     __shared__ int s_valid;
     if (threadIdx.x == 0) {
-        int valid = cu_seqlens[0] == 0;
+        int valid = cu_seqlens[0] == 0 && (!cu_q || cu_q[0] == 0);
         int64_t nb_sum = 0, tri = 0, grp = 0;
         for (int s = 0; s < D.n_seqs && valid; ++s) {
             const int64_t L = (int64_t)cu_seqlens[s + 1] - cu_seqlens[s];
             if (L < 1) { valid = 0; break; }
+            const int64_t Q = cu_q ? (int64_t)cu_q[s + 1] - cu_q[s] : L;
+            if (Q < 1 || Q > L) { valid = 0; break; }
+            P.q_off[s] = (int32_t)(L - Q);
             const int64_t nb = (L + D.B - 1) / D.B;
             if (nb > D.max_nb) { valid = 0; break; }
             if (D.page_size && (L + 63) / 64 > D.pt_stride) { valid = 0; break; }
@@ -150,7 +163,8 @@ __global__ void __launch_bounds__(kMetaThreads) k_meta(Dims D, SchedDims S, cons
             if (nb_sum > D.NB || grp > D.n_groups_cap) { valid = 0; break; }
         }
         if (valid) {
-            valid = (cu_seqlens[D.n_seqs] == D.T) && (nb_sum == D.NB) && (tri == D.tri_total);
+            valid = (cu_seqlens[D.n_seqs] == D.T) && (nb_sum == D.NB) && (tri == D.tri_total) &&
+                    (!cu_q || cu_q[D.n_seqs] == Tq);
             P.cu_blocks[D.n_seqs] = (int32_t)nb_sum;
             P.tri_off[D.n_seqs] = tri;
             P.group_cu[D.n_seqs] = (int32_t)grp;
@@ -237,8 +251,9 @@ __device__ __forceinline__ uint2 ld_stream8(const uint2* p) {
 
 // Block means of Q, K and V.  KV8: K and V are e4m3 codes with one fp32 scale
 // per (block, kv-head) (an FP8 KV cache); their means are the means of the
-// codes times the scale.
-template <bool KV8>
+// codes times the scale.  CHUNK: q holds a chunk of each sequence (positions
+// q_off .. L - 1), so a query block's mean covers only its chunk positions.
+template <bool KV8, bool CHUNK>
 __global__ void __launch_bounds__(kPoolThreads)
 k_pool(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ page_table,
        const uint16_t* __restrict__ q, const void* __restrict__ k,
@@ -253,15 +268,21 @@ k_pool(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict
     const int64_t b = blockIdx.x;
     const int s = P.block_seq[b];
     const int i = (int)(b - P.cu_blocks[s]);
-    const int64_t tok0 = cu_seqlens[s];
+    int64_t tok0 = cu_seqlens[s];
     const int L = cu_seqlens[s + 1] - cu_seqlens[s];
-    const int t_begin = i * D.B;
+    int t_begin = i * D.B;
     const int t_end = min(t_begin + D.B, L);
 
     int which, head, e0;
     if (col < qcols) { which = 0; head = col / d; e0 = col % d; }
     else if (col < qcols + kvcols) { which = 1; head = (col - qcols) / d; e0 = (col - qcols) % d; }
     else { which = 2; head = (col - qcols - kvcols) / d; e0 = (col - qcols - kvcols) % d; }
+    if (CHUNK && which == 0) {
+        // a chunk's queries: positions q_off .. L - 1 are q tokens cu_q[s] ..
+        const int off = P.q_off[s];
+        t_begin = max(t_begin, off);
+        tok0 = (int64_t)P.cu_q[s] - off;
+    }
 
     double acc[8];
 #pragma unroll
@@ -337,7 +358,8 @@ k_pool(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict
         }
     }
 
-    const double inv_n = 1.0 / (double)(t_end - t_begin);
+    // (a query block below a chunk has no query: its mean is left zero)
+    const double inv_n = (!CHUNK || t_end > t_begin) ? 1.0 / (double)(t_end - t_begin) : 0.0;
     double m[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) m[e] = acc[e] * inv_n;
@@ -601,7 +623,7 @@ __device__ double score64(const Dims& D, const WsPtrs& W, int64_t b_i, int64_t b
 // with rel_err the scoring kernel's bound (kScoreTcRelErr).  Every block whose
 // score could be the row maximum and every block whose score lies within e_j of
 // tau * m is re-scored in float64.
-template <int HD>
+template <int HD, bool CHUNK>
 __global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W, double rel_err) {
     if (!*P.meta_valid) return;
     const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -614,7 +636,10 @@ __global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W,
     const int i = (int)(bi - b0);
     uint32_t* mask = P.kept_mask + r * D.mask_words;
     int count = 0;
-    if (D.tau == 0.0) {
+    if (CHUNK && i < P.q_off[s] / D.B) {
+        // query block below a chunk: no row, nothing kept
+        for (int w = lane; w < D.mask_words; w += 32) mask[w] = 0u;
+    } else if (D.tau == 0.0) {
         for (int w = lane; w < D.mask_words; w += 32) {
             uint32_t bits = 0;
             if (32 * w + 31 <= i) bits = 0xFFFFFFFFu;
@@ -819,27 +844,38 @@ int launch_score(const Dims& D, const PlanPtrs& P, const WsPtrs& W, cudaStream_t
         const int grid = (int)std::min<int64_t>(items, std::max(1, sm_count()));
         k_score_tc<HD><<<grid, kScoreTcThreads, smem, st>>>(D, P, W, tq, tk);
     }
-    k_threshold<HD><<<(unsigned)((D.R * 32 + 255) / 256), 256, 0, st>>>(D, P, W, kScoreTcRelErr);
+    const unsigned grid = (unsigned)((D.R * 32 + 255) / 256);
+    if (P.cu_q)
+        k_threshold<HD, true><<<grid, 256, 0, st>>>(D, P, W, kScoreTcRelErr);
+    else
+        k_threshold<HD, false><<<grid, 256, 0, st>>>(D, P, W, kScoreTcRelErr);
     return FP2_OK;
 }
 
 }  // namespace
 
 int launch_plan(const Layout& L, const fp2_problem* p, const void* q, const void* k, const void* v,
-                const PlanPtrs& P, const WsPtrs& W, cudaStream_t st, const float* k_scale,
+                const PlanPtrs& P0, const WsPtrs& W, cudaStream_t st, const float* k_scale,
                 const float* v_scale) {
     const Dims& D = L.dims;
-    k_meta<<<1, kMetaThreads, 0, st>>>(D, L.sched, p->cu_seqlens, p->page_table, P);
+    PlanPtrs P = P0;
+    P.cu_q = L.chunked ? p->cu_q_seqlens : nullptr;
+    k_meta<<<1, kMetaThreads, 0, st>>>(D, L.sched, p->cu_seqlens, p->page_table, L.Tq, P);
     const int vecs = (D.Hq + 2 * D.Hkv) * D.d / 8;
     dim3 pool_grid((unsigned)D.NB, (vecs + kPoolThreads - 1) / kPoolThreads);
-    if (k_scale)
-        k_pool<true><<<pool_grid, kPoolThreads, 0, st>>>(D, p->cu_seqlens, p->page_table,
-                                                         static_cast<const uint16_t*>(q), k, v,
-                                                         k_scale, v_scale, P, W);
+    const uint16_t* q16 = static_cast<const uint16_t*>(q);
+    if (k_scale && L.chunked)
+        k_pool<true, true><<<pool_grid, kPoolThreads, 0, st>>>(D, p->cu_seqlens, p->page_table, q16, k,
+                                                               v, k_scale, v_scale, P, W);
+    else if (k_scale)
+        k_pool<true, false><<<pool_grid, kPoolThreads, 0, st>>>(D, p->cu_seqlens, p->page_table, q16,
+                                                                k, v, k_scale, v_scale, P, W);
+    else if (L.chunked)
+        k_pool<false, true><<<pool_grid, kPoolThreads, 0, st>>>(D, p->cu_seqlens, p->page_table, q16,
+                                                                k, v, nullptr, nullptr, P, W);
     else
-        k_pool<false><<<pool_grid, kPoolThreads, 0, st>>>(D, p->cu_seqlens, p->page_table,
-                                                          static_cast<const uint16_t*>(q), k, v,
-                                                          nullptr, nullptr, P, W);
+        k_pool<false, false><<<pool_grid, kPoolThreads, 0, st>>>(D, p->cu_seqlens, p->page_table, q16,
+                                                                 k, v, nullptr, nullptr, P, W);
     if (D.tau > 0.0) {
         const int64_t warps = D.NB * D.Hkv;
         k_norms<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(D, P, W);

@@ -103,6 +103,18 @@ extern "C" {
  *                describe the pool when page_size == 64; the stride must be
  *                >= ceil(max L_s / 64).  Page ids are checked on the device
  *                (FP2_STATUS_BAD_PAGE; such a page reads as zeros).
+ *   q_seqlens, cu_q_seqlens   chunked prefill (Table 6's serving mode); both
+ *                NULL for a full prefill.  q_seqlens HOST int32 [num_seqs]:
+ *                Q_s new queries of sequence s, 1 <= Q_s <= seqlens[s], at
+ *                positions seqlens[s] - Q_s .. seqlens[s] - 1; K and V hold all
+ *                seqlens[s] tokens (the earlier ones and the chunk's).
+ *                cu_q_seqlens DEVICE int32 [num_seqs + 1], their prefix sums
+ *                (checked on the device).  q, o and lse then have Tq = sum Q_s
+ *                tokens.  Blocks stay on the absolute position grid: query
+ *                block i holds the chunk's queries in [iB, (i+1)B) and its mean
+ *                covers only them; rows of query blocks below the chunk keep no
+ *                block.  BF16 only: fp2_quantize_fp8 of q and the e4m3
+ *                fp2_prefill return FP2_ERR_UNSUPPORTED for a chunked problem.
  */
 typedef struct fp2_problem {
     int32_t num_seqs;
@@ -117,6 +129,8 @@ typedef struct fp2_problem {
     int32_t num_pages;
     const int32_t* page_table;
     int32_t page_table_stride;
+    const int32_t* q_seqlens;
+    const int32_t* cu_q_seqlens;
 } fp2_problem;
 
 /*

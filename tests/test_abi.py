@@ -135,6 +135,40 @@ def test_plan_sizes_rejects(lib, kw, code):
     assert e.value.code == code
 
 
+def _chunk_problem(seqlens, q_seqlens, Hq=32, Hkv=8, B=128):
+    p = _problem(seqlens, Hq, Hkv, 128, B)
+    p.q_seqlens_np = np.ascontiguousarray(np.asarray(q_seqlens, dtype=np.int32))
+    p.c.q_seqlens = p.q_seqlens_np.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    p.c.cu_q_seqlens = 0x3000
+    return p
+
+
+@pytest.mark.parametrize("q_seqlens", [(0, 37), (1001, 37), (1000, 38)])
+def test_chunk_lengths_checked(lib, q_seqlens):
+    with pytest.raises(fb.Fp2Error) as e:
+        fb.fp2_plan_sizes(_chunk_problem((1000, 37), q_seqlens))
+    assert e.value.code == fb.FP2_ERR_INVALID_ARG
+
+
+def test_chunk_needs_both_lengths_and_offsets(lib):
+    p = _chunk_problem((1000, 37), (10, 37))
+    p.c.cu_q_seqlens = None
+    with pytest.raises(fb.Fp2Error) as e:
+        fb.fp2_plan_sizes(p)
+    assert e.value.code == fb.FP2_ERR_INVALID_ARG
+
+
+def test_chunk_schedule_counts_only_the_chunk_rows(lib):
+    # 131072 keys, the last 8192 queries: query blocks 960..1023 of 1024
+    full = fb.fp2_plan_sizes(_problem((131072,), 32, 8, 128, 128))
+    lay = fb.fp2_plan_sizes(_chunk_problem((131072,), (8192,)))
+    assert lay.num_rows == full.num_rows
+    assert lay.num_work_items == 8 * 2 * 64
+    # a chunk starting inside block 10 (position 1300) has rows 10..15
+    lay = fb.fp2_plan_sizes(_chunk_problem((2000,), (700,)))
+    assert lay.num_work_items == 8 * 2 * 6
+
+
 def test_paged_problem_accepted(lib):
     lay = fb.fp2_plan_sizes(_problem(page_size=64, page_table=16, num_pages=40))
     assert lay.num_blocks == 9
