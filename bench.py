@@ -641,6 +641,78 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+def chunk_dense_equiv_flop(wl, q_lens) -> float:
+    """Causal attention FLOP of the chunk's queries over all earlier keys:
+    4 * d * Hq * sum over query positions p of (p + 1)."""
+    tot = 0.0
+    for L, Q in zip(wl.seqlens, q_lens):
+        off = L - Q
+        tot += (L * (L + 1) - off * (off + 1)) / 2.0
+    return 4.0 * wl.d * wl.Hq * tot
+
+
+def run_chunked(args):
+    """Chunked prefill (Table 6's serving mode): the last C tokens of the 128K
+    layer as new queries over all 131072 keys, C in {8K, 16K}; plan + BF16
+    attention, one JSON line per chunk size on stdout (not the benchmark line)."""
+    import torch
+    from block_sparse_long_fp2_b200 import binding as fb
+    from block_sparse_long_fp2_b200 import build as fbuild
+
+    fbuild.build()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+    wl = synth.workloads()[args.workload]
+    x = synth.generate(wl)
+    k = torch.from_numpy(x["k"]).to(torch.bfloat16).to(dev)
+    v = torch.from_numpy(x["v"]).to(torch.bfloat16).to(dev)
+    cu = torch.from_numpy(x["cu_seqlens"]).to(dev)
+    for C in (8192, 16384):
+        q_lens = [min(C, L) for L in wl.seqlens]
+        parts, t0 = [], 0
+        for L, Q in zip(wl.seqlens, q_lens):
+            parts.append(x["q"][t0 + L - Q:t0 + L])
+            t0 += L
+        q = torch.from_numpy(np.concatenate(parts, axis=0)).to(torch.bfloat16).to(dev)
+        cu_q = torch.from_numpy(np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)).to(dev)
+        prob = fb.Problem(wl.seqlens, cu, wl.Hq, wl.Hkv, wl.d, wl.B, wl.tau, q_seqlens=q_lens,
+                          cu_q_seqlens=cu_q)
+        lay, plan, ws = fb.allocate(prob, dev)
+        Tq = sum(q_lens)
+        o = torch.empty((Tq, wl.Hq, wl.d), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((wl.Hq, Tq), dtype=torch.float32, device=dev)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+               for _ in range(args.warmup + args.steps)]
+        for e in evs:
+            e[0].record(stream)
+            fb.fp2_plan(prob, q, k, v, plan, ws, stream)
+            e[1].record(stream)
+            fb.fp2_prefill(prob, plan, q, k, v, o, lse, stream=stream)
+            e[2].record(stream)
+        torch.cuda.synchronize()
+        rc, st = fb.fp2_status_check(plan, stream)
+        if rc != 0:
+            raise RuntimeError(f"chunk {C}: device status {st:#x}")
+        tim = evs[args.warmup:]
+        ms = statistics.median(e[0].elapsed_time(e[2]) for e in tim)
+        plan_ms = statistics.median(e[0].elapsed_time(e[1]) for e in tim)
+        att = statistics.median(e[1].elapsed_time(e[2]) for e in tim)
+        nnz = int(fb.PlanView(plan, lay, wl.Hkv, wl.d).row_ptr[-1].item())
+        vis = sum((L + wl.B - 1) // wl.B * ((L + wl.B - 1) // wl.B + 1) // 2
+                  - ((L - Q) // wl.B) * ((L - Q) // wl.B + 1) // 2
+                  for L, Q in zip(wl.seqlens, q_lens)) * wl.Hkv
+        print(json.dumps({
+            "workload": f"{wl.name}_chunk{C // 1024}k", "kv_tokens": wl.T, "q_tokens": Tq,
+            "tau": wl.tau, "ms": round(ms, 4), "ms_plan": round(plan_ms, 4),
+            "ms_attention": round(att, 4), "density": round(nnz / vis, 4),
+            "dense_equiv_tflops": round(chunk_dense_equiv_flop(wl, q_lens) / (ms * 1e-3) / 1e12, 1),
+            "tensor_frac": round(nnz * kept_tile_flop(wl) / (att * 1e-3) / 1e12 / pk["bf16_sustained"], 4),
+        }), flush=True)
+        del q, o, lse, plan, ws
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -655,6 +727,8 @@ def main():
                     help="one line per L x tau cell of the dense-vs-sparse sweep instead")
     ap.add_argument("--correction-curve", action="store_true",
                     help="mean-correction overhead and error vs tau at 64K instead")
+    ap.add_argument("--chunked", action="store_true",
+                    help="chunked prefill of the last 8K / 16K tokens of the layer instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -665,6 +739,9 @@ def main():
 
     if args.sweep:
         run_sweep(args)
+        return
+    if args.chunked:
+        run_chunked(args)
         return
     if args.correction_curve:
         run_correction_curve(args)
