@@ -2,11 +2,16 @@
 // of arXiv 2608.19758): sparse attention over the selected key blocks with
 // the mean correction merged into the same online softmax.
 //
-// One persistent CTA per SM (320 threads) walks work items longest row
-// first.  A work item is one CSR row (sequence s, kv-head g, query block i)
-// restricted to two PackGQA query tiles of 128 rows each (the G heads x B
-// tokens of the row, packed head-major).  Both tiles share every K/V tile
-// the CTA streams, so K/V cross HBM once per kv-head (PackGQA).
+// One persistent CTA per SM (320 threads) takes work items from the schedule
+// the plan wrote (longest rows first within L2-sized chunks of kv-heads).  A
+// work item is one CSR row (sequence s, kv-head g, query block i), or one
+// count-balanced split of a long row's tiles (Table 7), restricted to two
+// PackGQA query tiles of 128 rows each (the G heads x B tokens of the row,
+// packed head-major).  Both tiles share every K/V tile the CTA streams, so
+// K/V cross HBM once per kv-head (PackGQA).  A split writes its normalised
+// O and log-sum-exp to scratch; k_combine merges a row's splits.  For
+// chunked prefill (CHUNK) the queries of sequence s are the positions from
+// its chunk offset on, read from and written to the chunk's own tokens.
 //
 // Roles (warp specialisation):
 //   warps 0-3   softmax warpgroup of query tile 0 (TMEM lanes 0-127)

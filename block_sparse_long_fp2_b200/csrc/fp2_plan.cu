@@ -3,19 +3,22 @@
 // scores under PackGQA, max-based thresholding and the CSR block index.
 //
 // Kernels, in launch order:
-//   meta     one CTA: checks cu_seqlens, derives block / scoring-group maps
-//            and the attention kernel's work schedule.
+//   meta     one CTA: checks cu_seqlens (and a chunk's cu_q_seqlens),
+//            derives block / scoring-group maps, the chunk offsets and the
+//            attention kernel's work schedule.
 //   pool     HBM-bound: streams Q, K, V once with 16-byte coalesced loads and
 //            accumulates each block's sum in float64 (exact for bf16 inputs),
 //            writing Qbar (fp64 workspace) and Kbar/Vbar (fp32, bf16, fp64).
 //   norms    |Qbar|, |Kbar| per block and kv-head (for the score error bound).
-//   score    one CTA per tile of the causal triangle (128 query vectors of a
-//            group of query blocks x 64 key blocks, one kv-head): float32
-//            block scores, max over the group's heads, to a scratch array.
+//   score    persistent, one CTA per SM over the tiles of the causal
+//            triangles (128 query vectors of a group of query blocks x 128 key
+//            blocks, one kv-head): tf32 tcgen05 MMAs of the means rounded to
+//            tf32 (exact products, fp32 sums), max over the group's heads, to
+//            a scratch array.
 //   threshold  one warp per row: the threshold decision.  A block whose
-//            float32 score lies within the float32 rounding bound of the
-//            threshold, and every candidate for the row maximum, is re-scored
-//            in float64, so the kept set is the one float64 scores give.
+//            score lies within the scores' error bound of the threshold, and
+//            every candidate for the row maximum, is re-scored in float64, so
+//            the kept set is the one float64 scores give.
 //   scan     row_ptr = exclusive prefix sum of kept counts.
 //   quant_means  e4m3 codes of Kbar / Vbar with one scale per pseudo-tile
 //            chunk (used by the FP8 correction).
