@@ -74,3 +74,16 @@ def test_two_gloo_ranks_independent_layers_and_max_time():
     assert val0 == val1 == pytest.approx(2 * flop / 11e-3 / 1e12)
     # reference arm: rank 0 reports, rank 1 does no work
     assert ref0 == ("reference", 2, "oracle") and ref1 is None
+
+
+def test_chunk_flop_counts():
+    # a chunk that is the whole sequence counts the full causal layer; the
+    # last C queries count the causal pairs of positions L - C .. L - 1
+    import bench  # noqa: E402
+    from block_sparse_long_fp2_b200 import synth
+    wl = synth.workloads()["qwen_128k"]
+    L = wl.seqlens[0]
+    assert bench.chunk_dense_equiv_flop(wl, [L]) == bench.dense_equiv_flop(wl)
+    C = 8192
+    pairs = sum(p + 1 for p in range(L - C, L))
+    assert bench.chunk_dense_equiv_flop(wl, [C]) == 4.0 * wl.d * wl.Hq * pairs
