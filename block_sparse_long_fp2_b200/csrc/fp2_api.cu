@@ -354,6 +354,7 @@ int fp2_plan_kv8(const fp2_problem* problem, const void* q, const void* k_e4m3, 
     Layout L;
     int rc = compute_layout(problem, &L);
     if (rc != FP2_OK) return rc;
+    if (L.chunked) return FP2_ERR_UNSUPPORTED;   // chunks over an FP8 cache: not built
     if (!q || !k_e4m3 || !v_e4m3 || !k_scale || !v_scale || !plan || !workspace)
         return FP2_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k_e4m3, 16) || !aligned(v_e4m3, 16) || !aligned(k_scale, 4) ||

@@ -867,10 +867,7 @@ int launch_plan(const Layout& L, const fp2_problem* p, const void* q, const void
     const int vecs = (D.Hq + 2 * D.Hkv) * D.d / 8;
     dim3 pool_grid((unsigned)D.NB, (vecs + kPoolThreads - 1) / kPoolThreads);
     const uint16_t* q16 = static_cast<const uint16_t*>(q);
-    if (k_scale && L.chunked)
-        k_pool<true, true><<<pool_grid, kPoolThreads, 0, st>>>(D, p->cu_seqlens, p->page_table, q16, k,
-                                                               v, k_scale, v_scale, P, W);
-    else if (k_scale)
+    if (k_scale)   // (an FP8 KV cache is never chunked: the entry point rejects it)
         k_pool<true, false><<<pool_grid, kPoolThreads, 0, st>>>(D, p->cu_seqlens, p->page_table, q16,
                                                                 k, v, k_scale, v_scale, P, W);
     else if (L.chunked)

@@ -113,8 +113,9 @@ extern "C" {
  *                tokens.  Blocks stay on the absolute position grid: query
  *                block i holds the chunk's queries in [iB, (i+1)B) and its mean
  *                covers only them; rows of query blocks below the chunk keep no
- *                block.  BF16 only: fp2_quantize_fp8 of q and the e4m3
- *                fp2_prefill return FP2_ERR_UNSUPPORTED for a chunked problem.
+ *                block.  BF16 only: fp2_quantize_fp8 of q, the e4m3
+ *                fp2_prefill and fp2_plan_kv8 return FP2_ERR_UNSUPPORTED for a
+ *                chunked problem.
  */
 typedef struct fp2_problem {
     int32_t num_seqs;

@@ -158,6 +158,15 @@ def test_chunk_needs_both_lengths_and_offsets(lib):
     assert e.value.code == fb.FP2_ERR_INVALID_ARG
 
 
+def test_chunked_planning_from_an_fp8_cache_is_rejected(lib):
+    # rejected on the host before anything is enqueued
+    p = _chunk_problem((1000, 37), (10, 37))
+    lay = fb.fp2_plan_sizes(p)
+    rc = lib.fp2_plan_kv8(p.ref, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 0x100000,
+                          lay.plan_bytes, 0x200000, lay.workspace_bytes, None)
+    assert rc == fb.FP2_ERR_UNSUPPORTED
+
+
 def test_chunk_schedule_counts_only_the_chunk_rows(lib):
     # 131072 keys, the last 8192 queries: query blocks 960..1023 of 1024
     full = fb.fp2_plan_sizes(_problem((131072,), 32, 8, 128, 128))
