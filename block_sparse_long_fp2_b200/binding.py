@@ -39,7 +39,7 @@ EXPORTED = ["fp2_version", "fp2_strerror", "fp2_plan_sizes", "fp2_plan", "fp2_qu
             "fp2_prefill", "fp2_status_check", "fp2_plan_static", "fp2_plan_kv8"]
 
 # Size of the library-held scratch of fp2_plan_static (FP2_STATIC_WORKSPACE_BYTES).
-FP2_STATIC_WORKSPACE_BYTES = 16 << 20
+FP2_STATIC_WORKSPACE_BYTES = 32 << 20
 
 
 class Fp2Error(RuntimeError):

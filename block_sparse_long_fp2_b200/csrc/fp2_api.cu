@@ -108,7 +108,10 @@ int compute_layout(const fp2_problem* p, Layout* out) {
         const int64_t nb = (p->seqlens[s] + d.B - 1) / d.B;
         for (int64_t i = first_row(s); i < nb; ++i) units += row_tile_bound(i, d.B);
     }
-    const int64_t share = (units * d.Hkv * sd.n_pairs + kSchedSMs - 1) / kSchedSMs;
+    // one attention CTA per SM of the current device (the attention kernel's grid)
+    int64_t ctas = sm_count();
+    if (ctas <= 0) ctas = kDefaultSchedSMs;
+    const int64_t share = (units * d.Hkv * sd.n_pairs + ctas - 1) / ctas;
     const int64_t longest = row_tile_bound(max_nb - 1, d.B);
     int64_t split = std::max<int64_t>({(int64_t)kMinSplitTiles, (share + 1) / 2,
                                        (longest + kMaxSplits - 1) / kMaxSplits});
@@ -287,7 +290,10 @@ int sm_count() {
     static std::mutex mu;
     static std::vector<int> cache;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();   // no device visible: leave no sticky error behind
+        return 0;
+    }
     std::lock_guard<std::mutex> lock(mu);
     if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
     if (cache[dev] == 0) {

@@ -24,13 +24,14 @@ constexpr int kScoreKeys = 128;
 // longest first; a chunk holds as many kv-heads as keep their bf16 K and V
 // within kSchedL2Bytes, so the CTAs that run together share K/V in L2.  When
 // the longest row's tile bound exceeds a CTA's mean share of the layer (taken
-// over kSchedSMs CTAs) and kMinSplitRow tiles, every row whose bound exceeds
+// over one CTA per SM of the current device, kDefaultSchedSMs when no device
+// is visible) and kMinSplitRow tiles, every row whose bound exceeds
 // half that share is cut into count-balanced splits of at least
 // kMinSplitTiles tiles (at most kMaxSplits), merged afterwards by their
 // log-sum-exp.  (The merge costs a launch of about 10 us; on a 16-row layer
 // with 17-tile rows, splitting measured slower than not.)
 constexpr int64_t kSchedL2Bytes = (int64_t)64 << 20;
-constexpr int kSchedSMs = 148;
+constexpr int kDefaultSchedSMs = 148;   // a B200
 constexpr int kMinSplitTiles = 8;
 constexpr int kMinSplitRow = 32;
 constexpr int kMaxSplits = 32;   // splits of one row (the merge takes one per lane)

@@ -10,9 +10,6 @@
 // the library's device image (kStaticWorkspaceBytes below).  The array is
 // created when the library is loaded onto a device and is held by every
 // device that loads the library until the process exits.
-#include <mutex>
-#include <vector>
-
 #include "fp2_internal.h"
 
 namespace fp2 {
@@ -26,22 +23,14 @@ constexpr size_t kStaticWorkspaceBytes = FP2_STATIC_WORKSPACE_BYTES;
 // cudaGetSymbolAddress below and only that address is handed to kernels.
 static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
 
-std::mutex g_mu;
-std::vector<void*> g_addr;   // per device: device address of g_static_workspace
-
-// Device address of the array on the current device, looked up once per
-// device (with that device current).  nullptr on failure.
+// Device address of the array in the current device's context, or nullptr.
+// It is looked up on every call rather than cached: after cudaDeviceReset or
+// a re-created primary context the array lives at a new address, and a cached
+// one would point into freed memory.  The lookup is a host-side table read.
 void* static_workspace_address() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if ((int)g_addr.size() <= dev) g_addr.resize(dev + 1, nullptr);
-    if (!g_addr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess) return nullptr;
-        g_addr[dev] = p;
-    }
-    return g_addr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess) return nullptr;
+    return p;
 }
 
 }  // namespace

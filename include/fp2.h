@@ -191,8 +191,10 @@ int fp2_version(void);
 const char* fp2_strerror(int code);
 
 /*
- * Host-only and pure: validates *problem (device pointers are not
- * dereferenced) and fills *layout.  nnz_cap is the dense count
+ * Host-only: validates *problem (device pointers are not dereferenced) and
+ * fills *layout.  The work schedule's split rule (fp2_prefill) depends on the
+ * current device's SM count, read here (148 when no device is visible), so
+ * call it with the device current that will run the plan.  nnz_cap is the dense count
  * Hkv * sum_s nb_s (nb_s + 1) / 2, so the CSR can never overflow.
  */
 int fp2_plan_sizes(const fp2_problem* problem, fp2_plan_layout* layout);
@@ -257,7 +259,7 @@ int fp2_quantize_fp8(const fp2_problem* problem, const void* plan, size_t plan_b
  * (from the other end on odd passes, when there are at most 16 passes).  KV
  * splitting (Table 7, "count-balanced CSR splits"): when the longest row's
  * tile bound i + 1 + ceil(i / B) exceeds both 32 and the layer's mean tiles
- * per CTA (over 148 CTAs), every row whose bound exceeds half that mean (and
+ * per CTA (one CTA per SM of the current device; 148 when no device is visible), every row whose bound exceeds half that mean (and
  * at least 8) is cut into
  * splits of equal numbers of its tiles (kept blocks in CSR order, then pseudo
  * tiles); each split writes its normalised fp32 O and log-sum-exp into the
@@ -278,20 +280,23 @@ int fp2_prefill(const fp2_problem* problem, const void* plan, size_t plan_bytes,
  * runtime and has no allocator of its own).  The paper has no counterpart:
  * this is an interface convenience of this library.
  *
- * The scratch lives in one fixed array of FP2_STATIC_WORKSPACE_BYTES inside
- * the library's device image, which every device that loads the library
- * holds until the process exits.  Problems whose layout.workspace_bytes
- * exceed it are rejected with FP2_ERR_CAPACITY (16 MiB covers, e.g., one
- * 32K-token layer with 32 query / 8 kv heads of dim 128).  The call
- * allocates and frees nothing.  Its first call on a device looks up the
- * array's device address (cudaGetSymbolAddress) with that device current;
- * make that first call before any stream capture.  Every call shares the
- * one array and leaves the last call's scratch in it (no entry needs to
- * start at zero), so calls whose work overlaps on the GPU -- on two streams,
- * or from two threads -- race; order them on one stream.  Arguments,
- * outputs and errors are otherwise those of fp2_plan.
+ * The scratch lives in one fixed array of FP2_STATIC_WORKSPACE_BYTES (32 MiB)
+ * inside the library's device image, which every device that loads the
+ * library holds until the process exits.  Problems whose
+ * layout.workspace_bytes exceed it are rejected with FP2_ERR_CAPACITY; it
+ * covers, e.g., one 32K-token layer with 32 query / 8 kv heads of dim 128 and
+ * block 128 (about 16.8 MB of scratch), not a 64K-token one of that shape.
+ * The call allocates and frees nothing.  Every call looks up the array's
+ * device address in the current device's context (cudaGetSymbolAddress, with
+ * the device the caller made current), so a reset or re-created context is
+ * followed; the first lookup on a device loads the library's device code
+ * there, so make the first call on each device before any stream capture.
+ * Every call shares the one array and leaves the last call's scratch in it
+ * (no entry needs to start at zero), so calls whose work overlaps on the GPU
+ * -- on two streams, or from two threads -- race; order them on one stream.
+ * Arguments, outputs and errors are otherwise those of fp2_plan.
  */
-#define FP2_STATIC_WORKSPACE_BYTES ((size_t)16 << 20)
+#define FP2_STATIC_WORKSPACE_BYTES ((size_t)32 << 20)
 int fp2_plan_static(const fp2_problem* problem, const void* q, const void* k, const void* v,
                     void* plan, size_t plan_bytes, void* stream);
 

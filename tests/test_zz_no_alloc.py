@@ -33,6 +33,23 @@ def test_rejects_problems_beyond_the_fixed_scratch():
     assert rc == fb.FP2_ERR_CAPACITY
 
 
+def test_documented_shape_fits_the_fixed_scratch():
+    _lib()
+    # the header names one 32K-token layer (32 q / 8 kv heads, d 128, B 128)
+    # as fitting the fixed array, and a 64K-token one as not
+    for L, fits in ((32768, True), (65536, False)):
+        p = fb.Problem([L], 0x1000, 32, 8, 128, 128, 0.1)
+        assert (fb.fp2_plan_sizes(p).workspace_bytes <= fb.FP2_STATIC_WORKSPACE_BYTES) == fits, L
+
+
+def test_binding_constant_matches_the_header():
+    import os
+    import re
+    hdr = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "fp2.h")
+    m = re.search(r"#define FP2_STATIC_WORKSPACE_BYTES \(\(size_t\)(\d+) << (\d+)\)", open(hdr).read())
+    assert m and int(m.group(1)) << int(m.group(2)) == fb.FP2_STATIC_WORKSPACE_BYTES
+
+
 @pytest.mark.gpu
 @pytest.mark.parametrize("case", ["ragged_d128", "pr1_ref_1k", "paged"])
 def test_static_plan_equals_workspace_plan_twice(case):
