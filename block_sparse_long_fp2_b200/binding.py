@@ -92,6 +92,7 @@ class fp2_plan_layout(ctypes.Structure):
         ("workspace_bytes", ctypes.c_size_t),
         ("num_work_items", ctypes.c_int64),
         ("num_split_slots", ctypes.c_int64),
+        ("off_kbar_e4m3_lo", ctypes.c_size_t),
     ]
 
 

@@ -165,6 +165,7 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     pub.off_vbar_bf16 = c.take(sizeof(uint16_t) * mean_elems);
     pub.off_kbar_e4m3 = c.take(mean_elems);
     pub.off_vbar_e4m3 = c.take(mean_elems);
+    pub.off_kbar_e4m3_lo = c.take(mean_elems);
     pub.off_kbar_scale = c.take(sizeof(float) * (size_t)NB * d.Hkv);
     pub.off_vbar_scale = c.take(sizeof(float) * (size_t)NB * d.Hkv);
     L.off_cu_blocks = c.take(sizeof(int32_t) * (n + 1));
@@ -211,6 +212,7 @@ PlanPtrs plan_ptrs(const Layout& L, void* plan) {
     p.kbar16 = reinterpret_cast<uint16_t*>(b + u.off_kbar_bf16);
     p.vbar16 = reinterpret_cast<uint16_t*>(b + u.off_vbar_bf16);
     p.kbar8 = reinterpret_cast<uint8_t*>(b + u.off_kbar_e4m3);
+    p.kbar8lo = reinterpret_cast<uint8_t*>(b + u.off_kbar_e4m3_lo);
     p.vbar8 = reinterpret_cast<uint8_t*>(b + u.off_vbar_e4m3);
     p.kbar_scale = reinterpret_cast<float*>(b + u.off_kbar_scale);
     p.vbar_scale = reinterpret_cast<float*>(b + u.off_vbar_scale);

@@ -18,8 +18,9 @@
 //   warps 4-7   softmax warpgroup of query tile 1
 //   warp 8      TMA producer: Q tiles, then per kept block its K and V tiles
 //               (through the page table when paged), then per pseudo tile
-//               up to B bf16 block means Kbar/Vbar; a ring of K-or-V slots
-//               (as many as shared memory holds, 5 at d = B = 128).
+//               up to B block means Kbar/Vbar (bf16; e4m3 with the key means
+//               in two terms, hi and lo, in two ring slots); a ring of K-or-V
+//               slots (as many as shared memory holds, 5 at d = B = 128).
 //   warp 9      allocates tensor memory and issues every tcgen05 MMA:
 //               S_m = Q_m K^T into TMEM, O_m += P_m V with P_m read from TMEM
 //               (P overwrites its own S columns).  Issue order for K/V tile n:
@@ -33,7 +34,9 @@
 // pseudo-key with key Kbar_j, value Vbar_j and logit bias ln n_j = ln B.
 // Up to B skipped blocks form one pseudo tile, run through exactly the same
 // MMA + softmax path as a real K/V tile, with the columns of kept blocks
-// (and of blocks j >= i) masked out.
+// (and of blocks j >= i) masked out.  In e4m3 the pseudo logits are
+// Q (Kbar_hi + Kbar_lo)^T, two MMAs into the same accumulator, so the key
+// means enter with about 2^-8 relative error rather than e4m3's 2^-4.
 //
 // Every wait is bounded (about a second); a timeout records
 // FP2_STATUS_TIMEOUT, all roles stop, in-flight copies and MMAs are drained
@@ -324,7 +327,8 @@ __device__ __forceinline__ uint32_t col_bits(int kind, int tok, const TileWalk<B
 template <int HD, int BLK, bool F8, bool CHUNK>
 __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUtensorMap* tm_q,
                          const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                         const CUtensorMap* tm_kbar, const CUtensorMap* tm_vbar) {
+                         const CUtensorMap* tm_kbar, const CUtensorMap* tm_vbar,
+                         const CUtensorMap* tm_kbar_lo) {
     using C = Cfg<HD, BLK, F8>;
     const Dims& D = P.D;
     uint32_t qcnt[2] = {0, 0}, qloaded[2] = {0, 0};
@@ -332,6 +336,10 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
     constexpr int kSlots = C::kSlots;
     uint32_t issued[kMaxSlots] = {0, 0, 0, 0, 0, 0, 0, 0};
     const bool paged = D.page_size != 0;
+    // K/V tiles (and block means) are re-read by every row of the kv-head:
+    // keep them in L2 over the query tiles, which each item reads once
+    const uint64_t pol_kv = l2_policy_evict_last();
+    const uint64_t pol_q = l2_policy_evict_first();
     for (int64_t w = blockIdx.x; w < P.n_slots; w += gridDim.x) {
         const int64_t o = sched_index(w, P.zigzag);
         if (o >= P.n_items) continue;
@@ -357,13 +365,17 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
                 const int hl = (kTileM * mt) / BLK + ht;
 #pragma unroll
                 for (int a = 0; a < C::kAtoms; ++a)
-                    tma_load_3d(qdst + a * C::kAtomQ + ht * BLK * 128, tm_q, &B.q_full[m],
-                                C::kAtomElems * a, it.g * D.G + hl, qtok + it.i * BLK);
+                    tma_load_3d_hint(qdst + a * C::kAtomQ + ht * BLK * 128, tm_q, &B.q_full[m],
+                                     C::kAtomElems * a, it.g * D.G + hl, qtok + it.i * BLK, pol_q);
             }
         }
         int kind, j;
         while (walk.next(kind, j)) {
-            for (int kv = 0; kv < 2; ++kv) {
+            // ring entries of the tile: K and V; an e4m3 pseudo tile's keys
+            // take two (the two e4m3 terms of the key means)
+            const int n_ent = (F8 && kind == kPseudo) ? 3 : 2;
+            for (int e = 0; e < n_ent; ++e) {
+                const int kv = e == n_ent - 1 ? 1 : 0;
                 const int slot = ld % kSlots;
                 const uint32_t use = ld / kSlots;
                 if (!mbar_wait(&B.kv_empty[slot], (use & 1) ^ 1, &B.abort, P.status)) goto drain;
@@ -373,17 +385,17 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
                 mbar_arrive_expect_tx(bar, C::kSlotBytes);
                 uint8_t* dst = smem + C::kOffSlot + slot * C::kSlotBytes;
                 if (kind == kPseudo) {
-                    const CUtensorMap* tm = kv == 0 ? tm_kbar : tm_vbar;
+                    const CUtensorMap* tm = kv == 1 ? tm_vbar : (e == 0 ? tm_kbar : tm_kbar_lo);
 #pragma unroll
                     for (int a = 0; a < C::kAtoms; ++a)
-                        tma_load_3d(dst + a * C::kAtomKV, tm, bar, C::kAtomElems * a, it.g,
-                                    it.b0 + j * BLK);
+                        tma_load_3d_hint(dst + a * C::kAtomKV, tm, bar, C::kAtomElems * a, it.g,
+                                         it.b0 + j * BLK, pol_kv);
                 } else if (!paged) {
                     const CUtensorMap* tm = kv == 0 ? tm_k : tm_v;
 #pragma unroll
                     for (int a = 0; a < C::kAtoms; ++a)
-                        tma_load_3d(dst + a * C::kAtomKV, tm, bar, C::kAtomElems * a, it.g,
-                                    it.tok0 + j * BLK);
+                        tma_load_3d_hint(dst + a * C::kAtomKV, tm, bar, C::kAtomElems * a, it.g,
+                                         it.tok0 + j * BLK, pol_kv);
                 } else {
                     const CUtensorMap* tm = kv == 0 ? tm_k : tm_v;
                     const int n_pages_s = (it.L + 63) / 64;
@@ -398,8 +410,8 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
                         }
 #pragma unroll
                         for (int a = 0; a < C::kAtoms; ++a)
-                            tma_load_4d(dst + a * C::kAtomKV + pg * 64 * 128, tm, bar,
-                                        C::kAtomElems * a, it.g, 0, id);
+                            tma_load_4d_hint(dst + a * C::kAtomKV + pg * 64 * 128, tm, bar,
+                                             C::kAtomElems * a, it.g, 0, id, pol_kv);
                     }
                 }
             }
@@ -426,15 +438,18 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) {
     return d + static_cast<uint64_t>(bytes >> 4);
 }
 
+// S = Q K^T (accumulate: S += Q K^T, for the second term of e4m3 key means).
 template <int HD, int BLK, bool F8>
-__device__ __forceinline__ void issue_s(uint32_t tmem_s, uint64_t q_desc, uint64_t k_desc) {
+__device__ __forceinline__ void issue_s(uint32_t tmem_s, uint64_t q_desc, uint64_t k_desc,
+                                        bool accumulate = false) {
     using C = Cfg<HD, BLK, F8>;
 #pragma unroll
     for (int kk = 0; kk < HD / C::kKStep; ++kk) {
         const uint64_t a = desc_add(q_desc, (kk / 4) * C::kAtomQ + (kk % 4) * 32);
         const uint64_t b = desc_add(k_desc, (kk / 4) * C::kAtomKV + (kk % 4) * 32);
-        if (F8) umma_f8(tmem_s, a, b, C::kIdescS, kk > 0 ? 1u : 0u);
-        else umma_f16(tmem_s, a, b, C::kIdescS, kk > 0 ? 1u : 0u);
+        const uint32_t acc = (accumulate || kk > 0) ? 1u : 0u;
+        if (F8) umma_f8(tmem_s, a, b, C::kIdescS, acc);
+        else umma_f16(tmem_s, a, b, C::kIdescS, acc);
     }
 }
 
@@ -508,14 +523,33 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
         }
         return true;
     };
-    // S0 = Q0 K^T of a tile whose K sits in ring slot k
-    auto s0 = [&](const RingPos& k, bool has_m1, bool last) -> bool {
-        if (!mbar_wait(&B.kv_full[k.slot], k.use & 1, &B.abort, P.status)) return false;
+    // The K ring entries of one tile: its K tile, and for an e4m3 pseudo tile
+    // the second term of the key means in the next entry (lo).
+    struct KPos {
+        RingPos k, lo;
+        bool two;
+    };
+    auto kdesc = [&](const RingPos& r) { return desc_add(k_desc0, r.slot * C::kSlotBytes); };
+    // S_m = Q_m K^T of the tile's K entries (waits for them to land)
+    auto issue_sm = [&](int m, const KPos& kk) -> bool {
+        if (!mbar_wait(&B.kv_full[kk.k.slot], kk.k.use & 1, &B.abort, P.status)) return false;
+        if (kk.two && !mbar_wait(&B.kv_full[kk.lo.slot], kk.lo.use & 1, &B.abort, P.status))
+            return false;
         tc_fence_after();
-        issue_s<HD, BLK, F8>(t_s[0], q_desc[0], desc_add(k_desc0, k.slot * C::kSlotBytes));
+        issue_s<HD, BLK, F8>(t_s[m], q_desc[m], kdesc(kk.k));
+        if (kk.two) issue_s<HD, BLK, F8>(t_s[m], q_desc[m], kdesc(kk.lo), true);
+        return true;
+    };
+    auto release_k = [&](const KPos& kk) {
+        umma_commit(&B.kv_empty[kk.k.slot]);
+        if (kk.two) umma_commit(&B.kv_empty[kk.lo.slot]);
+    };
+    // S0 = Q0 K^T
+    auto s0 = [&](const KPos& kk, bool has_m1, bool last) -> bool {
+        if (!issue_sm(0, kk)) return false;
         umma_commit(&B.s_full[0]);
         if (!has_m1) {
-            umma_commit(&B.kv_empty[k.slot]);
+            release_k(kk);
             if (last) umma_commit(&B.q_empty[0]);
         }
         return true;
@@ -525,17 +559,26 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
         const int64_t o = sched_index(w, P.zigzag);
         if (o >= P.n_items) continue;
         const Item it = decode_item(P, o);
-        // The issuer needs no column ids, only the tile count: its loop issues no
-        // global loads, which would otherwise hold up its barrier probes.
-        int n_tiles;
+        // The issuer needs no column ids, only the tile count (and, for e4m3,
+        // where the pseudo tiles start): its loop issues no global loads,
+        // which would otherwise hold up its barrier probes.
+        int n_tiles, n_real;
         {
             TileWalk<BLK> walk;
             walk.init(P, it);
             n_tiles = walk.count();
+            n_real = walk.n_kept - walk.t;   // tiles before the pseudo tiles
         }
         if (n_tiles == 0) continue;
-        RingPos kp = ring_take<kSlots>(ring);
-        RingPos vp = ring_take<kSlots>(ring);
+        auto take_tile = [&](int n, KPos& kk, RingPos& v) {
+            kk.k = ring_take<kSlots>(ring);
+            kk.two = F8 && n >= n_real;
+            if (kk.two) kk.lo = ring_take<kSlots>(ring);
+            v = ring_take<kSlots>(ring);
+        };
+        KPos kp;
+        RingPos vp;
+        take_tile(0, kp, vp);
         if (!mbar_wait(&B.q_full[0], qcnt[0] & 1, &B.abort, P.status)) goto drain;
         ++qcnt[0];
         if (!s0(kp, it.has_m1, n_tiles == 1)) goto drain;
@@ -552,10 +595,9 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
                     if (!mbar_wait(&B.q_full[1], qcnt[1] & 1, &B.abort, P.status)) goto drain;
                     ++qcnt[1];
                 }
-                tc_fence_after();
-                issue_s<HD, BLK, F8>(t_s[1], q_desc[1], desc_add(k_desc0, kp.slot * C::kSlotBytes));
+                if (!issue_sm(1, kp)) goto drain;
                 umma_commit(&B.s_full[1]);
-                umma_commit(&B.kv_empty[kp.slot]);
+                release_k(kp);
                 if (last) {
                     umma_commit(&B.q_empty[0]);
                     umma_commit(&B.q_empty[1]);
@@ -576,8 +618,7 @@ __device__ void mma_issuer(const AttnParams& P, Bars& B, uint8_t* smem) {
             prev = PrevTile{true, it.has_m1, first, last, vp.slot};
             // S0 of the next tile right away
             if (!last) {
-                kp = ring_take<kSlots>(ring);
-                vp = ring_take<kSlots>(ring);
+                take_tile(n + 1, kp, vp);
                 if (!s0(kp, it.has_m1, n + 1 == n_tiles - 1)) goto drain;
             }
         }
@@ -864,7 +905,7 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
                     v.y = pack_bf16x2(__uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
                     v.z = pack_bf16x2(__uint_as_float(r[e + 4]) * inv_l, __uint_as_float(r[e + 5]) * inv_l);
                     v.w = pack_bf16x2(__uint_as_float(r[e + 6]) * inv_l, __uint_as_float(r[e + 7]) * inv_l);
-                    reinterpret_cast<uint4*>(dst)[(32 * c + e) / 8] = v;
+                    st_stream_v4(reinterpret_cast<uint4*>(dst) + (32 * c + e) / 8, v);
                 }
             }
         }
@@ -881,7 +922,8 @@ template <int HD, int BLK, bool F8, bool CHUNK>
 __global__ void __launch_bounds__(kThreads, 1)
 k_attn(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap tm_q,
        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-       const __grid_constant__ CUtensorMap tm_kbar, const __grid_constant__ CUtensorMap tm_vbar) {
+       const __grid_constant__ CUtensorMap tm_kbar, const __grid_constant__ CUtensorMap tm_vbar,
+       const __grid_constant__ CUtensorMap tm_kbar_lo) {
     using C = Cfg<HD, BLK, F8>;
     if (!*P.meta_valid) return;
     extern __shared__ uint8_t smem_raw[];
@@ -915,6 +957,7 @@ k_attn(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
         tma_prefetch_desc(&tm_kbar);
+        if (F8) tma_prefetch_desc(&tm_kbar_lo);
         tma_prefetch_desc(&tm_vbar);
     }
     tc_fence_before();
@@ -924,7 +967,8 @@ k_attn(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap
     if (warp < 8) {
         softmax_wg<HD, BLK, F8, CHUNK>(P, B, smem, warp >> 2);
     } else if (warp == kProducerWarp) {
-        if (lane == 0) producer<HD, BLK, F8, CHUNK>(P, B, smem, &tm_q, &tm_k, &tm_v, &tm_kbar, &tm_vbar);
+        if (lane == 0) producer<HD, BLK, F8, CHUNK>(P, B, smem, &tm_q, &tm_k, &tm_v, &tm_kbar, &tm_vbar,
+                                                    &tm_kbar_lo);
     } else {
         if (lane == 0) mma_issuer<HD, BLK, F8>(P, B, smem);
     }
@@ -1058,7 +1102,7 @@ int launch_attn_t(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, con
     const Dims& D = L.dims;
     const cuuint64_t eb = C::kElt;                         // bytes per element
     const cuuint32_t ae = C::kAtomElems;                   // elements per 128-byte atom row
-    CUtensorMap tq, tk, tv, tkb, tvb;
+    CUtensorMap tq, tk, tv, tkb, tvb, tkb_lo;
     {
         cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)D.Hq, (cuuint64_t)L.Tq};
         cuuint64_t str[2] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hq * HD * eb};
@@ -1087,6 +1131,9 @@ int launch_attn_t(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, con
         const void* vb = F8 ? static_cast<const void*>(pp.vbar8) : static_cast<const void*>(pp.vbar16);
         if (!make_tensor_map(&tkb, kb, 3, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
         if (!make_tensor_map(&tvb, vb, 3, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
+        // the second e4m3 term of the key means (e4m3 only; unused for bf16)
+        const void* kl = F8 ? static_cast<const void*>(pp.kbar8lo) : kb;
+        if (!make_tensor_map(&tkb_lo, kl, 3, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
     }
     AttnParams P;
     P.D = D;
@@ -1130,7 +1177,7 @@ int launch_attn_t(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, con
         cudaSuccess)
         return FP2_ERR_CUDA;
     if (F8) k_vmax<<<dim3(D.n_seqs, D.Hkv), 256, 0, st>>>(D, pp, vs);
-    kernel<<<(unsigned)grid, kThreads, C::kSmemBytes, st>>>(P, tq, tk, tv, tkb, tvb);
+    kernel<<<(unsigned)grid, kThreads, C::kSmemBytes, st>>>(P, tq, tk, tv, tkb, tvb, tkb_lo);
     if (S.split_slots > 0)
         k_combine<HD, BLK><<<dim3((unsigned)(S.split_slots * D.Hkv), S.n_pairs * (2 * kTileM / kCombineRows)),
                              kCombineThreads, 0, st>>>(P);

@@ -82,6 +82,7 @@ struct PlanPtrs {
     uint16_t* kbar16;
     uint16_t* vbar16;
     uint8_t* kbar8;
+    uint8_t* kbar8lo;   // e4m3 residual of kbar / chunk scale - kbar8
     uint8_t* vbar8;
     float* kbar_scale;
     float* vbar_scale;

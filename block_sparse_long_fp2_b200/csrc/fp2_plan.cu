@@ -710,7 +710,10 @@ __global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W,
 // One CTA per (chunk of B blocks of one sequence, kv-head): the chunk is the
 // set of blocks one pseudo-key tile covers, so a pseudo tile needs a single
 // scale.  scale = absmax / 448 over the chunk's fp32 means (1 when all zero),
-// code = e4m3_rne_sat(mean / scale), both in fp32.
+// code = e4m3_rne_sat(mean / scale), both in fp32.  The key means get a second
+// e4m3 term, lo = e4m3_rne_sat(mean / scale - code), so that the pseudo-key
+// logits (one MMA over both terms) carry about 2^-8 relative error instead of
+// the 2^-4 of one e4m3 rounding.
 
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
     uint16_t r;
@@ -764,9 +767,18 @@ __global__ void __launch_bounds__(kQuantMeansThreads) k_quant_means(Dims D, Plan
         const int64_t off = ((b + idx / d) * D.Hkv + g) * d + idx % d;
         const float4 k4 = *reinterpret_cast<const float4*>(P.kbar + off);
         const float4 v4 = *reinterpret_cast<const float4*>(P.vbar + off);
-        *reinterpret_cast<uint32_t*>(P.kbar8 + off) =
-            (uint32_t)e4m3x2(__fdiv_rn(k4.x, sk), __fdiv_rn(k4.y, sk)) |
-            ((uint32_t)e4m3x2(__fdiv_rn(k4.z, sk), __fdiv_rn(k4.w, sk)) << 16);
+        const float kq[4] = {__fdiv_rn(k4.x, sk), __fdiv_rn(k4.y, sk), __fdiv_rn(k4.z, sk),
+                             __fdiv_rn(k4.w, sk)};
+        const uint16_t h01 = e4m3x2(kq[0], kq[1]), h23 = e4m3x2(kq[2], kq[3]);
+        *reinterpret_cast<uint32_t*>(P.kbar8 + off) = (uint32_t)h01 | ((uint32_t)h23 << 16);
+        // second term: the residual of the quotient (exact in fp32, since the
+        // e4m3 value is within a factor 2 of it), rounded to e4m3 on its own
+        float hv[4];
+        unpack_e4m3x2(h01, hv[0], hv[1]);
+        unpack_e4m3x2(h23, hv[2], hv[3]);
+        *reinterpret_cast<uint32_t*>(P.kbar8lo + off) =
+            (uint32_t)e4m3x2(kq[0] - hv[0], kq[1] - hv[1]) |
+            ((uint32_t)e4m3x2(kq[2] - hv[2], kq[3] - hv[3]) << 16);
         *reinterpret_cast<uint32_t*>(P.vbar8 + off) =
             (uint32_t)e4m3x2(__fdiv_rn(v4.x, sv), __fdiv_rn(v4.y, sv)) |
             ((uint32_t)e4m3x2(__fdiv_rn(v4.z, sv), __fdiv_rn(v4.w, sv)) << 16);

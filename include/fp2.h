@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define FP2_VERSION 2
+#define FP2_VERSION 3
 
 /* ---- error codes -------------------------------------------------------- */
 #define FP2_OK 0
@@ -155,6 +155,11 @@ typedef struct fp2_problem {
  *               chunk (1 when all zero), code = e4m3_rne_sat(mean / scale).
  *   kbar_scale, vbar_scale float [num_blocks, Hkv]: the chunk scale, stored
  *               at the chunk's first block (other entries unused).
+ *   kbar_e4m3_lo  uint8 [num_blocks, Hkv, d] e4m3 codes of the residual
+ *               mean / scale - kbar_e4m3 (same chunk scale), so that
+ *               kbar ~ scale * (kbar_e4m3 + kbar_e4m3_lo) to about 2^-8
+ *               relative: the FP8 correction's pseudo-key logits use both
+ *               terms (one e4m3 term alone, 2^-4, moves the LSE by ~2e-3).
  *   status      int32 [1] status word (FP2_STATUS_* bits), cleared by fp2_plan.
  *   (the rest is private to the library)
  */
@@ -182,6 +187,7 @@ typedef struct fp2_plan_layout {
     size_t workspace_bytes;   /* bytes fp2_plan's scratch must have    */
     int64_t num_work_items;   /* fp2_prefill's work items (rows x splits x query-tile pairs) */
     int64_t num_split_slots;  /* row splits of the rows fp2_prefill splits (0: none)          */
+    size_t off_kbar_e4m3_lo;
 } fp2_plan_layout;
 
 /* Library version (FP2_VERSION of the build). */

@@ -42,8 +42,6 @@ from .fp2_oracle import (  # noqa: F401
     e4m3_round,
     quantize_e4m3,
     dequantize_e4m3,
-    quantize_means_e4m3,
-    dequantize_means_e4m3,
 )
 from .fp2_chunked import (  # noqa: F401
     chunk_layout,

@@ -407,49 +407,3 @@ def dequantize_e4m3(codes, scales, seqlens: Sequence[int], B: int) -> np.ndarray
             lo, hi = t0 + i * B, t0 + min((i + 1) * B, int(L))
             out[lo:hi] = codes[lo:hi] * scales[b0 + i][None, :, None]
     return out
-
-
-def quantize_means_e4m3(means, seqlens: Sequence[int], B: int):
-    """e4m3 codes of block means for the FP8 correction path.
-
-    means [NB, H, d] (float64 block means).  They are stored as float32, and
-    every chunk of B consecutive blocks of a sequence (the blocks one
-    pseudo-key tile covers) shares one scale per head: scale = absmax / 448
-    over the chunk (1 when all zero), code = e4m3_round(mean / scale), the
-    scale and the quotient rounded to float32 as the kernel computes them.
-    Returns (codes [NB, H, d] float64, scales [NB, H] float64 with the chunk's
-    scale at its first block and NaN elsewhere).
-    """
-    m32 = np.asarray(means, dtype=np.float32)
-    lay = block_layout(seqlens, B)
-    NB, H, d = m32.shape
-    codes = np.zeros((NB, H, d))
-    scales = np.full((NB, H), np.nan)
-    for s in range(len(lay["seqlens"])):
-        b0 = int(lay["cu_blocks"][s])
-        nb = int(lay["nb"][s])
-        for c0 in range(0, nb, B):
-            lo, hi = b0 + c0, b0 + min(c0 + B, nb)
-            for h in range(H):
-                blk = m32[lo:hi, h, :]
-                amax = np.float32(np.abs(blk).max())
-                sc = amax / np.float32(E4M3_MAX) if amax > 0 else np.float32(1.0)
-                scales[lo, h] = sc
-                codes[lo:hi, h, :] = e4m3_round(blk / sc)
-    return codes, scales
-
-
-def dequantize_means_e4m3(codes, scales, seqlens: Sequence[int], B: int) -> np.ndarray:
-    """codes * the scale of the B-block chunk (of its sequence) each block
-    belongs to; inverse of quantize_means_e4m3 up to e4m3 rounding."""
-    codes = _as64(codes)
-    lay = block_layout(seqlens, B)
-    out = np.zeros_like(codes)
-    for s in range(len(lay["seqlens"])):
-        b0 = int(lay["cu_blocks"][s])
-        nb = int(lay["nb"][s])
-        for c0 in range(0, nb, B):
-            lo, hi = b0 + c0, b0 + min(c0 + B, nb)
-            out[lo:hi] = codes[lo:hi] * np.asarray(scales[lo], dtype=np.float64)[None, :, None]
-    return out
-

@@ -151,6 +151,34 @@ def csr_rows(wl: synth.Workload, rows_si: Sequence[tuple]) -> List[int]:
     return [g * NB + int(cu_b[s]) + i for g in range(wl.Hkv) for (s, i) in rows_si]
 
 
+def attend_rows_mt(q, k, v, pl, rows_si, correction=True, kept_override=None, workers=None):
+    """oracle.attend_rows over the query blocks rows_si, one call per block,
+    the calls spread over the host's cores by threads (NumPy releases the GIL
+    inside its matrix products and element-wise loops; BLAS is held to one
+    thread per call so the threads do not oversubscribe).  The oracle is
+    unchanged: every (s, i) block is computed on its own, so splitting the
+    list does not change any value.  Returns what attend_rows returns for the
+    whole list, in its order."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    from threadpoolctl import threadpool_limits
+    rows_si = list(rows_si)
+    if not rows_si:
+        return oracle.attend_rows(q, k, v, pl, rows_si, correction, kept_override)
+    workers = workers or len(os.sched_getaffinity(0))
+    order = sorted(range(len(rows_si)), key=lambda n: -rows_si[n][1])   # longest rows first
+
+    def one(n):
+        return n, oracle.attend_rows(q, k, v, pl, [rows_si[n]], correction=correction,
+                                     kept_override=kept_override)
+
+    with threadpool_limits(1), ThreadPoolExecutor(max_workers=workers) as ex:
+        res = dict(ex.map(one, order))
+    parts = [res[n] for n in range(len(rows_si))]
+    return (np.concatenate([p[0] for p in parts]), np.concatenate([p[1] for p in parts], axis=0),
+            np.concatenate([p[2] for p in parts], axis=1))
+
+
 def check_attention(wl, x, run: GpuRun, pl, rows_si=None, correction=True):
     """O / LSE of the GPU against the oracle on the given query blocks, with
     the oracle using the GPU's block lists where the two differ inside the
@@ -168,8 +196,8 @@ def check_attention(wl, x, run: GpuRun, pl, rows_si=None, correction=True):
             r = g * NB + int(cu_b[s]) + i
             if list(pl["kept"][r]) != gk[r]:
                 override[(s, g, i)] = gk[r]
-    toks, O_ref, L_ref = oracle.attend_rows(q, k, v, pl, rows_si, correction=correction,
-                                            kept_override=override)
+    toks, O_ref, L_ref = attend_rows_mt(q, k, v, pl, rows_si, correction=correction,
+                                        kept_override=override)
     O, LSE = run.outputs()
     assert np.array_equal(toks, token_rows(wl, rows_si))
     e_o = rel_l2(O[toks], O_ref)
@@ -202,11 +230,14 @@ def fp8_prefill(wl: synth.Workload, run: GpuRun):
     return res
 
 
-def dequantised_operands(wl: synth.Workload, q, k, v, pl, rows_si):
-    """The operands the FP8 path computes with, from the oracle's own
-    quantiser: K and V whole, Q only on the query blocks `rows_si` (zeros
-    elsewhere), and a copy of the plan with the e4m3 block means of the
-    correction path.  Scales are per (block, head), so each block is
+def dequantised_operands(wl: synth.Workload, q, k, v, rows_si):
+    """The FP8 path's inputs as its definition gives them: Q, K and V after
+    direct online quantisation (per (block, head) scale = absmax / 448,
+    e4m3 round-to-nearest-even, saturating) and dequantisation, from the
+    oracle's quantiser -- K and V whole, Q only on the query blocks rows_si
+    (zeros elsewhere).  The block means stay the plan's float64 means: how
+    the kernel carries them into its e4m3 products is its own business and
+    part of its error.  Scales are per (block, head), so each block is
     quantised on its own as a one-block sequence (same codes, less memory)."""
     cu = np.concatenate([[0], np.cumsum(wl.seqlens)])
 
@@ -225,18 +256,24 @@ def dequantised_operands(wl: synth.Workload, q, k, v, pl, rows_si):
     for s, i in rows_si:
         lo, hi = cu[s] + i * wl.B, cu[s] + min((i + 1) * wl.B, wl.seqlens[s])
         dq_block(q, lo, hi, q_dq)
-    pl_dq = dict(pl)
-    for key in ("kbar", "vbar"):
-        c, sc = oracle.quantize_means_e4m3(pl[key], wl.seqlens, wl.B)
-        pl_dq[key] = oracle.dequantize_means_e4m3(c, sc, wl.seqlens, wl.B)
-    return q_dq, k_dq, v_dq, pl_dq
+    return q_dq, k_dq, v_dq
+
+
+# Regression guard for the distance of the FP8 output to the plain oracle
+# (bf16 inputs, no quantisation).  e4m3 rounding of Q, K and V alone moves O
+# by 4e-2 (N(0,1) inputs) to 7e-2 (low-rank generator) rel-L2 in the float64
+# oracle itself (tests/test_oracle.py), and e4m3 P in the P.V product adds
+# about 3e-2; the stated 5e-2 is checked against the oracle on the
+# quantised inputs (REL_L2_FP8 above).
+REL_L2_FP8_PLAIN_GUARD = 0.15
 
 
 def check_fp8(wl, x, run: GpuRun, pl, rows_si, O8, L8):
-    """FP8 O / LSE against the oracle on the dequantised operands (the FP8
-    path's own arithmetic: same codes, float64 math) and against the plain
-    bf16-input oracle (the accuracy cost of e4m3).  The GPU's block lists are
-    used where they differ inside the threshold band."""
+    """FP8 O / LSE against the oracle on the quantised inputs (Q, K, V through
+    the direct online quantisation, then float64 arithmetic with the plan's
+    float64 block means) and against the plain bf16-input oracle (the
+    accuracy cost of e4m3).  The GPU's block lists are used where they differ
+    inside the threshold band."""
     q, k, v = oracle_inputs(x, wl)
     gk = run.kept_lists()
     nb = [(L + wl.B - 1) // wl.B for L in wl.seqlens]
@@ -248,12 +285,21 @@ def check_fp8(wl, x, run: GpuRun, pl, rows_si, O8, L8):
             r = g * NB + int(cu_b[s]) + i
             if list(pl["kept"][r]) != gk[r]:
                 override[(s, g, i)] = gk[r]
-    q_dq, k_dq, v_dq, pl_dq = dequantised_operands(wl, q, k, v, pl, rows_si)
-    toks, O_dq, L_dq = oracle.attend_rows(q_dq, k_dq, v_dq, pl_dq, rows_si, kept_override=override)
+    q_dq, k_dq, v_dq = dequantised_operands(wl, q, k, v, rows_si)
+    toks, O_dq, L_dq = attend_rows_mt(q_dq, k_dq, v_dq, pl, rows_si, kept_override=override)
     del q_dq, k_dq, v_dq
-    _, O_ref, L_ref = oracle.attend_rows(q, k, v, pl, rows_si, kept_override=override)
+    _, O_ref, L_ref = attend_rows_mt(q, k, v, pl, rows_si, kept_override=override)
     assert np.array_equal(toks, token_rows(wl, rows_si))
     return {"rel_l2_dq": rel_l2(O8[toks], O_dq), "rel_l2_plain": rel_l2(O8[toks], O_ref),
             "lse_dq": float(np.max(np.abs(L8[:, toks] - L_dq))),
             "lse_plain": float(np.max(np.abs(L8[:, toks] - L_ref))),
             "finite": bool(np.isfinite(O8[toks]).all() and np.isfinite(L8[:, toks]).all())}
+
+
+def assert_fp8(res):
+    """The FP8 tolerances: O rel-L2 <= 5e-2 and LSE <= 1e-3 against the oracle
+    on the quantised inputs; the distance to the plain oracle under its guard."""
+    assert res["finite"], res
+    assert res["rel_l2_dq"] <= REL_L2_FP8, res
+    assert res["lse_dq"] <= LSE_ABS, res
+    assert res["rel_l2_plain"] <= REL_L2_FP8_PLAIN_GUARD, res

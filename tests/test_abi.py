@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_strerror(lib):
-    assert fb.fp2_version() == 2
+    assert fb.fp2_version() == 3
     assert fb.strerror(0) == "ok"
     for code in [-1, -2, -3, -4, -5, -6]:
         assert fb.strerror(code) not in ("", "unknown error")
@@ -101,7 +101,7 @@ def test_plan_sizes_counts(lib):
     assert lay.mask_words == 1 and lay.max_blocks_per_seq == 8
     offs = [lay.off_status, lay.off_row_ptr, lay.off_col_idx, lay.off_kept_mask, lay.off_kbar,
             lay.off_vbar, lay.off_kbar_bf16, lay.off_vbar_bf16, lay.off_kbar_e4m3,
-            lay.off_vbar_e4m3, lay.off_kbar_scale, lay.off_vbar_scale]
+            lay.off_vbar_e4m3, lay.off_kbar_scale, lay.off_vbar_scale, lay.off_kbar_e4m3_lo]
     assert lay.off_status == 0
     assert all(o % 256 == 0 for o in offs)
     assert len(set(offs)) == len(offs) and max(offs) < lay.plan_bytes

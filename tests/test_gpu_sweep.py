@@ -3,11 +3,11 @@
 0.05, 0.2}, BF16 and FP8-e4m3, low-rank generator, and the FP8-e4m3 run of the
 128K needles layer.
 
-Each cell is checked on a seeded sample of query blocks (always the first and
-the last): block lists on 16 blocks per sequence across every kv-head, O / LSE
-on three of them across every query head and token.  FP8 is checked against
-the oracle on the dequantised operands (the path's own arithmetic) and its
-distance to the plain oracle is recorded.
+Each cell is checked on a seeded sample of 16 query blocks (always the first
+and the last) across every kv-head and query head: block lists, and O / LSE.
+FP8 is checked against the oracle on the quantised inputs (direct online
+quantisation of Q, K, V; float64 block means) and its distance to the plain
+oracle is held under a regression guard.
 """
 
 import numpy as np
@@ -17,7 +17,7 @@ import oracle
 from block_sparse_long_fp2_b200 import binding as fb
 from block_sparse_long_fp2_b200 import synth
 
-from fp2_harness import (LSE_ABS, REL_L2_BF16, REL_L2_FP8, GpuRun, check_attention, check_fp8,
+from fp2_harness import (LSE_ABS, REL_L2_BF16, GpuRun, assert_fp8, check_attention, check_fp8,
                          compare_plan, csr_rows, fp8_prefill, oracle_inputs, sample_rows)
 
 pytestmark = pytest.mark.gpu
@@ -47,7 +47,7 @@ def _cell(name, fp8=True):
     pl = oracle.plan(q, k, v, wl.seqlens, wl.B, wl.tau, rows=rows_plan)
     res = compare_plan(pl, run.kept_lists(), rows=csr_rows(wl, rows_plan))
     assert res["outside_band"] == 0, res
-    rows_o = [rows_plan[0], rows_plan[len(rows_plan) // 2], rows_plan[-1]]
+    rows_o = rows_plan
     att = check_attention(wl, x, run, pl, rows_si=rows_o)
     out = {"plan": res, "bf16": att}
     if fp8:
@@ -65,15 +65,4 @@ def test_sweep_cell(name):
     res = _cell(name)
     bf = res["bf16"]
     assert bf["finite"] and bf["rel_l2"] <= REL_L2_BF16 and bf["lse_max_abs"] <= LSE_ABS, bf
-    f8 = res["fp8"]
-    assert f8["finite"], f8
-    assert f8["lse_dq"] <= LSE_ABS, f8
-    assert f8["rel_l2_dq"] <= REL_L2_FP8, f8
-
-
-def test_fp8_on_the_128k_needles_layer():
-    res = _cell("qwen_128k")
-    f8 = res["fp8"]
-    assert f8["finite"], f8
-    assert f8["lse_dq"] <= LSE_ABS, f8
-    assert f8["rel_l2_dq"] <= REL_L2_FP8, f8
+    assert_fp8(res["fp8"])

@@ -418,30 +418,6 @@ def test_quantize_roundtrip_error_bound_and_scales():
     assert np.all(cz == 0) and sz[0, 0] == 1.0
 
 
-def test_quantize_means_chunks_follow_sequences():
-    # 2 sequences with 5 and 3 blocks, B = 2 -> chunks {0,1},{2,3},{4} | {5,6},{7}
-    seqlens = [10, 6]
-    NB, H, d = 8, 2, 4
-    rng = np.random.default_rng(1)
-    means = rng.standard_normal((NB, H, d))
-    means[4] = 0.0                                  # an all-zero chunk
-    codes, scales = oracle.quantize_means_e4m3(means, seqlens, 2)
-    starts = [0, 2, 4, 5, 7]
-    assert np.all(np.isfinite(scales[starts])) and np.all(np.isnan(np.delete(scales, starts, 0)))
-    assert np.all(scales[4] == 1.0) and np.all(codes[4] == 0.0)
-    for lo, hi in [(0, 2), (2, 4), (5, 7), (7, 8)]:
-        for h in range(H):
-            amax = np.abs(means[lo:hi, h].astype(np.float32)).max()
-            assert scales[lo, h] == np.float32(amax) / np.float32(448)
-            assert np.abs(codes[lo:hi, h]).max() == 448.0          # the absmax maps to 448
-            deq = codes[lo:hi, h] * scales[lo, h]
-            big = np.abs(means[lo:hi, h]) > amax / 64
-            assert np.all(np.abs(deq - means[lo:hi, h])[big] <= np.abs(means[lo:hi, h])[big] * 2 ** -4 + 1e-7)
-    deq_all = oracle.dequantize_means_e4m3(codes, scales, seqlens, 2)
-    assert np.array_equal(deq_all[2:4], codes[2:4] * scales[2][None, :, None])
-    assert np.array_equal(deq_all[7], codes[7] * scales[7][:, None])
-
-
 def test_e4m3_operand_rounding_alone_moves_o_by_percents():
     # The FP8 path's own definition: Q, K, V rounded to e4m3 with one absmax
     # scale per (block, head), then exact attention.  The rounding alone moves
