@@ -22,6 +22,7 @@ tau = 0), each timed the same way.
 workload (rank 0 only) and prints the same metric for it.
 --sweep prints one line per cell of the L x tau sweep (BF16 and FP8) instead.
 --correction-curve prints the mean-correction overhead and error vs tau at 64K.
+--density prints attention time against density on the 128K topics layers.
 """
 
 from __future__ import annotations
@@ -644,6 +645,91 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+def pseudo_tiles(kept_mask: np.ndarray, wl) -> int:
+    """Pseudo tiles the attention kernel runs: per row (s, g, i), the groups of
+    B consecutive blocks below i holding at least one skipped block."""
+    B = wl.B
+    n, r = 0, 0
+    for _g in range(wl.Hkv):
+        for L in wl.seqlens:
+            nb = (L + B - 1) // B
+            for i in range(nb):
+                words = kept_mask[r]
+                bits = np.unpackbits(words.view(np.uint8), bitorder="little")[:i]
+                skipped = np.flatnonzero(bits == 0)
+                n += len(np.unique(skipped // B))
+                r += 1
+    return n
+
+
+def run_density(args):
+    """Attention time against density on the 128K layer shape with block-level
+    topics (about 5, 10 and 20 % of the blocks kept; the pages' real prompts
+    keep 4.6-9.4 % at 64K-128K, Table 3), BF16: ms, executed-block tensor
+    fraction, and the time the dense (tau = 0) run of the same inputs predicts
+    when time is proportional to the tiles executed (kept blocks + pseudo
+    tiles of the correction) -- Figure 5's "tracks the theoretical bound".
+    One JSON line per density on stdout (not the benchmark line)."""
+    import torch
+    from block_sparse_long_fp2_b200 import binding as fb
+    from block_sparse_long_fp2_b200 import build as fbuild
+
+    fbuild.build()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+    names = [n for n in synth.workloads() if n.startswith("topics_128k_")]
+    for name in names:
+        wl = synth.workloads()[name]
+        x = synth.generate(wl)
+        q = torch.from_numpy(x["q"]).to(torch.bfloat16).to(dev)
+        k = torch.from_numpy(x["k"]).to(torch.bfloat16).to(dev)
+        v = torch.from_numpy(x["v"]).to(torch.bfloat16).to(dev)
+        del x
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(wl.seqlens)]).astype(np.int32), device=dev)
+        o = torch.empty((wl.T, wl.Hq, wl.d), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((wl.Hq, wl.T), dtype=torch.float32, device=dev)
+        row = {"workload": name, "L": wl.seqlens[0], "tau": wl.tau}
+        for tag, tau in (("sparse", wl.tau), ("dense", 0.0)):
+            prob = fb.Problem(wl.seqlens, cu, wl.Hq, wl.Hkv, wl.d, wl.B, tau)
+            lay, plan, ws = fb.allocate(prob, dev)
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                   for _ in range(args.warmup + args.steps)]
+            for e in evs:
+                e[0].record(stream)
+                fb.fp2_plan(prob, q, k, v, plan, ws, stream)
+                e[1].record(stream)
+                fb.fp2_prefill(prob, plan, q, k, v, o, lse, stream=stream)
+                e[2].record(stream)
+            torch.cuda.synchronize()
+            rc, st = fb.fp2_status_check(plan, stream)
+            if rc != 0:
+                raise RuntimeError(f"{name}: device status {st:#x}")
+            tim = evs[args.warmup:]
+            view = fb.PlanView(plan, lay, wl.Hkv, wl.d)
+            nnz = int(view.row_ptr[-1].item())
+            att = statistics.median(e[1].elapsed_time(e[2]) for e in tim)
+            ent = {"ms_per_layer": round(statistics.median(e[0].elapsed_time(e[2]) for e in tim), 4),
+                   "ms_plan": round(statistics.median(e[0].elapsed_time(e[1]) for e in tim), 4),
+                   "ms_attention": round(att, 4), "nnz": nnz,
+                   "density": round(nnz / float(lay.nnz_cap), 4),
+                   "tensor_frac": round(nnz * kept_tile_flop(wl) / (att * 1e-3) / 1e12
+                                        / pk["bf16_sustained"], 4)}
+            if tag == "sparse":
+                ent["pseudo_tiles"] = pseudo_tiles(view.kept_mask.cpu().numpy(), wl)
+            row[tag] = ent
+            del plan, ws
+        sp, dn = row["sparse"], row["dense"]
+        per_tile = dn["ms_attention"] / dn["nnz"]
+        pred = per_tile * (sp["nnz"] + sp["pseudo_tiles"])
+        row["predicted_ms_attention"] = round(pred, 4)
+        row["actual_over_predicted"] = round(sp["ms_attention"] / pred, 4)
+        row["speedup_vs_dense"] = round(dn["ms_per_layer"] / sp["ms_per_layer"], 3)
+        print(json.dumps(row), flush=True)
+        del q, k, v, o, lse
+        torch.cuda.empty_cache()
+
+
 def chunk_dense_equiv_flop(wl, q_lens) -> float:
     """Causal attention FLOP of the chunk's queries over all earlier keys:
     4 * d * Hq * sum over query positions p of (p + 1)."""
@@ -730,6 +816,8 @@ def main():
                     help="one line per L x tau cell of the dense-vs-sparse sweep instead")
     ap.add_argument("--correction-curve", action="store_true",
                     help="mean-correction overhead and error vs tau at 64K instead")
+    ap.add_argument("--density", action="store_true",
+                    help="attention time against density on the 128K topics layers")
     ap.add_argument("--chunked", action="store_true",
                     help="chunked prefill of the last 8K / 16K tokens of the layer instead")
     args = ap.parse_args()
@@ -748,6 +836,9 @@ def main():
         return
     if args.correction_curve:
         run_correction_curve(args)
+        return
+    if args.density:
+        run_density(args)
         return
 
     if args.impl == "reference":

@@ -336,10 +336,6 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
     constexpr int kSlots = C::kSlots;
     uint32_t issued[kMaxSlots] = {0, 0, 0, 0, 0, 0, 0, 0};
     const bool paged = D.page_size != 0;
-    // K/V tiles (and block means) are re-read by every row of the kv-head:
-    // keep them in L2 over the query tiles, which each item reads once
-    const uint64_t pol_kv = l2_policy_evict_last();
-    const uint64_t pol_q = l2_policy_evict_first();
     for (int64_t w = blockIdx.x; w < P.n_slots; w += gridDim.x) {
         const int64_t o = sched_index(w, P.zigzag);
         if (o >= P.n_items) continue;
@@ -365,8 +361,8 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
                 const int hl = (kTileM * mt) / BLK + ht;
 #pragma unroll
                 for (int a = 0; a < C::kAtoms; ++a)
-                    tma_load_3d_hint(qdst + a * C::kAtomQ + ht * BLK * 128, tm_q, &B.q_full[m],
-                                     C::kAtomElems * a, it.g * D.G + hl, qtok + it.i * BLK, pol_q);
+                    tma_load_3d(qdst + a * C::kAtomQ + ht * BLK * 128, tm_q, &B.q_full[m],
+                                C::kAtomElems * a, it.g * D.G + hl, qtok + it.i * BLK);
             }
         }
         int kind, j;
@@ -388,14 +384,14 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
                     const CUtensorMap* tm = kv == 1 ? tm_vbar : (e == 0 ? tm_kbar : tm_kbar_lo);
 #pragma unroll
                     for (int a = 0; a < C::kAtoms; ++a)
-                        tma_load_3d_hint(dst + a * C::kAtomKV, tm, bar, C::kAtomElems * a, it.g,
-                                         it.b0 + j * BLK, pol_kv);
+                        tma_load_3d(dst + a * C::kAtomKV, tm, bar, C::kAtomElems * a, it.g,
+                                    it.b0 + j * BLK);
                 } else if (!paged) {
                     const CUtensorMap* tm = kv == 0 ? tm_k : tm_v;
 #pragma unroll
                     for (int a = 0; a < C::kAtoms; ++a)
-                        tma_load_3d_hint(dst + a * C::kAtomKV, tm, bar, C::kAtomElems * a, it.g,
-                                         it.tok0 + j * BLK, pol_kv);
+                        tma_load_3d(dst + a * C::kAtomKV, tm, bar, C::kAtomElems * a, it.g,
+                                    it.tok0 + j * BLK);
                 } else {
                     const CUtensorMap* tm = kv == 0 ? tm_k : tm_v;
                     const int n_pages_s = (it.L + 63) / 64;
@@ -410,8 +406,8 @@ __device__ void producer(const AttnParams& P, Bars& B, uint8_t* smem, const CUte
                         }
 #pragma unroll
                         for (int a = 0; a < C::kAtoms; ++a)
-                            tma_load_4d_hint(dst + a * C::kAtomKV + pg * 64 * 128, tm, bar,
-                                             C::kAtomElems * a, it.g, 0, id, pol_kv);
+                            tma_load_4d(dst + a * C::kAtomKV + pg * 64 * 128, tm, bar,
+                                        C::kAtomElems * a, it.g, 0, id);
                     }
                 }
             }
@@ -905,7 +901,7 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
                     v.y = pack_bf16x2(__uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
                     v.z = pack_bf16x2(__uint_as_float(r[e + 4]) * inv_l, __uint_as_float(r[e + 5]) * inv_l);
                     v.w = pack_bf16x2(__uint_as_float(r[e + 6]) * inv_l, __uint_as_float(r[e + 7]) * inv_l);
-                    st_stream_v4(reinterpret_cast<uint4*>(dst) + (32 * c + e) / 8, v);
+                    reinterpret_cast<uint4*>(dst)[(32 * c + e) / 8] = v;
                 }
             }
         }

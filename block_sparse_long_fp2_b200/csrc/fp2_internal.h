@@ -72,6 +72,18 @@ struct SchedDims {
     int64_t split_slots;    // row splits of split rows, per kv-head
 };
 
+// Block and token offsets of up to kMapSeqs sequences, computed on the host
+// from the problem's host arrays and passed to the pooling kernel by value,
+// so that it needs no device-side map and can run before k_meta.
+constexpr int kMapSeqs = 64;
+struct SeqMap {
+    int32_t n;
+    int32_t cu_blocks[kMapSeqs + 1];
+    int32_t cu_tok[kMapSeqs + 1];
+    int32_t cu_q[kMapSeqs + 1];   // query tokens (chunked prefill), else cu_tok
+    int32_t q_off[kMapSeqs];      // position of the first query (L - Q, else 0)
+};
+
 // Device pointers into the plan buffer.
 struct PlanPtrs {
     int32_t* row_ptr;

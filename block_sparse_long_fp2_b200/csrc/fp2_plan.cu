@@ -24,6 +24,7 @@
 //            chunk (used by the FP8 correction).
 //   compact  col_idx from the kept-block bit masks, ascending per row.
 #include <cfloat>
+#include <cstring>
 #include <cmath>
 
 #include "fp2_device.cuh"
@@ -139,6 +140,9 @@ __device__ void build_schedule(const Dims& D, const SchedDims& S, const PlanPtrs
     }
 }
 
+__device__ void meta_maps(const Dims& D, const SchedDims& S, const int32_t* __restrict__ cu_seqlens,
+                          const int32_t* __restrict__ page_table, const PlanPtrs& P);
+
 // P.cu_q: prefix sums of a chunk's query counts (chunked prefill), or null;
 // Tq their total.
 __global__ void __launch_bounds__(kMetaThreads, 1) k_meta(Dims D, SchedDims S, const int32_t* __restrict__ cu_seqlens,
@@ -188,7 +192,16 @@ __global__ void __launch_bounds__(kMetaThreads, 1) k_meta(Dims D, SchedDims S, c
         s_valid = valid;
     }
     __syncthreads();
-    if (!s_valid) return;
+    if (s_valid) meta_maps(D, S, cu_seqlens, page_table, P);
+    // k_meta may run beside the pooling kernel launched before it (which
+    // needs none of its outputs); it completes only after that kernel, so
+    // the kernels after it see both
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Block -> sequence and scoring-group maps, page-id checks, the schedule.
+__device__ void meta_maps(const Dims& D, const SchedDims& S, const int32_t* __restrict__ cu_seqlens,
+                          const int32_t* __restrict__ page_table, const PlanPtrs& P) {
     for (int s = 0; s < D.n_seqs; ++s) {
         const int b0 = P.cu_blocks[s], b1 = P.cu_blocks[s + 1];
         for (int b = b0 + threadIdx.x; b < b1; b += blockDim.x) P.block_seq[b] = s;
@@ -252,46 +265,116 @@ __device__ __forceinline__ uint2 ld_stream8(const uint2* p) {
     return r;
 }
 
+__device__ __forceinline__ double warp_sum_d(double x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+__device__ __forceinline__ float round_up_f(double x) {
+    // a float not below x (x >= 0)
+    float f = (float)x;
+    if ((double)f < x) f = nextafterf(f, FLT_MAX);
+    return f * (1.0f + 1.0f / 1048576.0f);
+}
+
+// Sequence of global block b, its block index i, and its token offsets.
+// BYVAL: from the host-computed map passed by value (the pool then needs no
+// device-side map and can run before k_meta); otherwise from k_meta's maps.
+struct BlockLoc {
+    int s, i;
+    int64_t tok0;   // first K/V token of the sequence
+    int64_t qtok0;  // q token of position 0 of the sequence (chunked: cu_q - q_off)
+    int L, q_off;
+};
+
+template <bool BYVAL>
+__device__ __forceinline__ BlockLoc locate_block(const Dims& D, const SeqMap& M, const PlanPtrs& P,
+                                                 const int32_t* __restrict__ cu_seqlens, int64_t b) {
+    BlockLoc r;
+    if (BYVAL) {
+        int lo = 0, hi = M.n - 1;   // the last s with cu_blocks[s] <= b
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (M.cu_blocks[mid] <= b) lo = mid;
+            else hi = mid - 1;
+        }
+        r.s = lo;
+        r.i = (int)(b - M.cu_blocks[lo]);
+        r.tok0 = M.cu_tok[lo];
+        r.L = M.cu_tok[lo + 1] - M.cu_tok[lo];
+        r.q_off = M.q_off[lo];
+        r.qtok0 = (int64_t)M.cu_q[lo] - r.q_off;
+    } else {
+        r.s = P.block_seq[b];
+        r.i = (int)(b - P.cu_blocks[r.s]);
+        r.tok0 = cu_seqlens[r.s];
+        r.L = cu_seqlens[r.s + 1] - cu_seqlens[r.s];
+        r.q_off = P.cu_q ? P.q_off[r.s] : 0;
+        r.qtok0 = P.cu_q ? (int64_t)P.cu_q[r.s] - r.q_off : r.tok0;
+    }
+    return r;
+}
+
 // Block means of Q, K and V.  KV8: K and V are e4m3 codes with one fp32 scale
 // per (block, kv-head) (an FP8 KV cache); their means are the means of the
 // codes times the scale.  CHUNK: q holds a chunk of each sequence (positions
 // q_off .. L - 1), so a query block's mean covers only its chunk positions.
-template <bool KV8, bool CHUNK>
+// BYVAL: block -> sequence from the map passed by value (see locate_block);
+// the kernel then reads only token rows inside [0, T) (or [0, Tq) of q), so a
+// cu_seqlens that disagrees with the host sizes (k_meta flags it) cannot make
+// it read out of bounds.  NORMS: also writes |Kbar| per (block, kv-head) and
+// the largest |Qbar| over each kv-head's G query heads (both rounded up), the
+// threshold's error-bound inputs; needs the G heads of a group inside one CTA.
+template <bool KV8, bool CHUNK, bool BYVAL, bool NORMS>
 __global__ void __launch_bounds__(kPoolThreads)
-k_pool(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ page_table,
-       const uint16_t* __restrict__ q, const void* __restrict__ k,
-       const void* __restrict__ v, const float* __restrict__ k_scale,
+k_pool(Dims D, SeqMap M, int64_t Tq, const int32_t* __restrict__ cu_seqlens,
+       const int32_t* __restrict__ page_table, const uint16_t* __restrict__ q,
+       const void* __restrict__ k, const void* __restrict__ v, const float* __restrict__ k_scale,
        const float* __restrict__ v_scale, PlanPtrs P, WsPtrs W) {
-    if (!*P.meta_valid) return;
+    // the next kernel (k_meta) may start while the pool runs: it reads none
+    // of the pool's outputs and waits for the pool before it completes
+    if (BYVAL) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (!BYVAL && !*P.meta_valid) return;
     const int vec = blockIdx.y * kPoolThreads + threadIdx.x;   // 8-element column chunk
     const int d = D.d;
     const int qcols = D.Hq * d, kvcols = D.Hkv * d;
     const int col = vec * 8;
-    if (col >= qcols + 2 * kvcols) return;
+    const bool active = col < qcols + 2 * kvcols;
     const int64_t b = blockIdx.x;
-    const int s = P.block_seq[b];
-    const int i = (int)(b - P.cu_blocks[s]);
-    int64_t tok0 = cu_seqlens[s];
-    const int L = cu_seqlens[s + 1] - cu_seqlens[s];
-    int t_begin = i * D.B;
-    const int t_end = min(t_begin + D.B, L);
+    const BlockLoc loc = locate_block<BYVAL>(D, M, P, cu_seqlens, b);
+    const int s = loc.s;
+    int64_t tok0 = loc.tok0;
+    const int L = loc.L;
+    int t_begin = loc.i * D.B;
+    int t_end = min(t_begin + D.B, L);
 
-    int which, head, e0;
+    int which = 0, head = 0, e0 = 0;
     if (col < qcols) { which = 0; head = col / d; e0 = col % d; }
     else if (col < qcols + kvcols) { which = 1; head = (col - qcols) / d; e0 = (col - qcols) % d; }
     else { which = 2; head = (col - qcols - kvcols) / d; e0 = (col - qcols - kvcols) % d; }
-    if (CHUNK && which == 0) {
-        // a chunk's queries: positions q_off .. L - 1 are q tokens cu_q[s] ..
-        const int off = P.q_off[s];
-        t_begin = max(t_begin, off);
-        tok0 = (int64_t)P.cu_q[s] - off;
+    int64_t tok_lim = D.T;   // rows of the tensor read
+    if (which == 0) {
+        tok_lim = Tq;
+        if (CHUNK) {
+            // a chunk's queries: positions q_off .. L - 1 are q tokens cu_q[s] ..
+            t_begin = max(t_begin, loc.q_off);
+            tok0 = loc.qtok0;
+        }
+    }
+    if (BYVAL) {
+        // keep every row read inside the tensor, whatever cu_seqlens holds
+        if ((int64_t)t_begin < -tok0) t_begin = (int)(-tok0);
+        if ((int64_t)t_end > tok_lim - tok0) t_end = (int)(tok_lim - tok0);
     }
 
     double acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.0;
 
-    if (KV8 && which != 0) {
+    if (!active) {
+        // no column: only takes part in the CTA's barrier below
+    } else if (KV8 && which != 0) {
         // e4m3 K / V, contiguous [T, Hkv, d] or paged [P, 64, Hkv, d]
         const uint8_t* base = static_cast<const uint8_t*>(which == 1 ? k : v);
         const int64_t stride = (int64_t)D.Hkv * d / 8;   // uint2 per token
@@ -362,11 +445,11 @@ k_pool(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict
     }
 
     // (a query block below a chunk has no query: its mean is left zero)
-    const double inv_n = (!CHUNK || t_end > t_begin) ? 1.0 / (double)(t_end - t_begin) : 0.0;
+    const double inv_n = t_end > t_begin ? 1.0 / (double)(t_end - t_begin) : 0.0;
     double m[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) m[e] = acc[e] * inv_n;
-    if (which == 0) {
+    if (active && which == 0) {
         double* dst = W.qbar64 + (b * D.Hq + head) * d + e0;
 #pragma unroll
         for (int e = 0; e < 8; e += 2) *reinterpret_cast<double2*>(dst + e) = make_double2(m[e], m[e + 1]);
@@ -376,7 +459,7 @@ k_pool(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict
                                                       round_tf32((float)m[2]), round_tf32((float)m[3]));
         *reinterpret_cast<float4*>(d32 + 4) = make_float4(round_tf32((float)m[4]), round_tf32((float)m[5]),
                                                           round_tf32((float)m[6]), round_tf32((float)m[7]));
-    } else {
+    } else if (active) {
         const int64_t off = (b * D.Hkv + head) * d + e0;
         float* f32 = (which == 1 ? P.kbar : P.vbar) + off;
         uint16_t* h16 = (which == 1 ? P.kbar16 : P.vbar16) + off;
@@ -401,24 +484,33 @@ k_pool(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict
                                                              round_tf32(f1.z), round_tf32(f1.w));
         }
     }
+    if (NORMS) {
+        // |mean|^2 of this thread's head: the d / 8 threads of a head are
+        // consecutive lanes of one warp (d / 8 in {8, 16})
+        double sq = 0.0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sq = fma(m[e], m[e], sq);
+        const int tph = d / 8;
+        for (int o = tph / 2; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        const bool lead = active && (vec % tph) == 0;
+        if (lead && which == 1) W.knorm[b * D.Hkv + head] = round_up_f(sqrt(sq));
+        // the largest over the G query heads of a kv-head: the group's heads
+        // lie in this CTA (G d divides the CTA's 1024 columns)
+        __shared__ double head_sq[kPoolThreads];
+        const int hl = threadIdx.x / tph;   // head slot within the CTA
+        if (lead) head_sq[hl] = sq;
+        __syncthreads();
+        if (lead && which == 0 && head % D.G == 0) {
+            double mx = 0.0;
+            for (int u = 0; u < D.G; ++u) mx = fmax(mx, head_sq[hl + u]);
+            W.qnorm[b * D.Hkv + head / D.G] = round_up_f(sqrt(mx));
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
 // norms: one warp per (block, kv-head)
 // ---------------------------------------------------------------------------
-
-__device__ __forceinline__ double warp_sum_d(double x) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    return x;
-}
-
-__device__ __forceinline__ float round_up_f(double x) {
-    // a float not below x (x >= 0)
-    float f = (float)x;
-    if ((double)f < x) f = nextafterf(f, FLT_MAX);
-    return f * (1.0f + 1.0f / 1048576.0f);
-}
 
 __global__ void k_norms(Dims D, PlanPtrs P, WsPtrs W) {
     if (!*P.meta_valid) return;
@@ -481,7 +573,12 @@ __global__ void __launch_bounds__(kScoreTcThreads)
 k_score_tc(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap tm_q,
            const __grid_constant__ CUtensorMap tm_k) {
     using C = ScoreTcCfg<HD>;
-    if (!*P.meta_valid) return;
+    // runs beside k_quant_means (launched before it as its programmatic
+    // dependent) and completes only after it
+    if (!*P.meta_valid) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        return;
+    }
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -597,6 +694,224 @@ k_score_tc(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap tm_
         tc_fence_after();
         tmem_dealloc(tmem, kScoreKeys);
     }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Pipelined tensor-core scores (G a power of two, at most 32).  A persistent CTA per SM takes
+// work items (row group of 128 / G query blocks, kv-head), the row groups of
+// a sequence from the last (longest rows) down, kv-heads inner, one item per
+// CTA per pass over the grid (odd passes from the other end).  Roles:
+//   warp 4  TMA: the item's 128 query vectors (tf32 values in fp32) once,
+//           then its 128-key-block chunks into a 2-slot ring;
+//   warp 5  MMA: per chunk 16 (d = 128) tcgen05 kind::tf32 MMAs
+//           (M = N = 128, K = 8) into one of two 128-column TMEM accumulators;
+//   warps 0-3  epilogue: each thread reads its query vector's 128 dot
+//           products from TMEM, the G heads of a block (G adjacent lanes)
+//           take their maximum by shuffles, and the block's first lane
+//           stores the scores j <= i of that chunk.
+// The loads of chunk c + 1 and its MMAs overlap the epilogue of chunk c.
+// Products and error bound as for k_score_tc.
+constexpr int kScorePThreads = 192;
+
+template <int HD>
+struct ScorePCfg {
+    static constexpr int kAtoms = HD * 4 / 128;          // 128-byte atoms per fp32 row
+    static constexpr int kAtomBytes = 128 * 128;         // one atom column of 128 rows
+    static constexpr int kTileBytes = kAtoms * kAtomBytes;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kTileBytes;             // two K slots
+    static constexpr int kSmem = 3 * kTileBytes + 1024;
+};
+
+struct ScoreItem {
+    int g, s, b0, nb, i0, i1, n_chunks;
+};
+
+__device__ __forceinline__ ScoreItem score_item(const Dims& D, const PlanPtrs& P, int64_t w,
+                                                int n_groups) {
+    const int64_t n_items = (int64_t)n_groups * D.Hkv;
+    const int64_t pass = w / gridDim.x;
+    const int64_t o = (pass & 1) ? pass * gridDim.x + (gridDim.x - 1 - blockIdx.x) : w;
+    ScoreItem it;
+    it.n_chunks = 0;
+    if (o >= n_items) return it;
+    const int gi = n_groups - 1 - (int)(o / D.Hkv);
+    it.g = (int)(o % D.Hkv);
+    it.s = P.group_seq[gi];
+    it.b0 = P.cu_blocks[it.s];
+    it.nb = P.cu_blocks[it.s + 1] - it.b0;
+    it.i0 = (gi - P.group_cu[it.s]) * D.rows_per_group;
+    it.i1 = min(it.i0 + D.rows_per_group, it.nb);
+    it.n_chunks = (it.i1 - 1) / kScoreKeys + 1;
+    return it;
+}
+
+template <int HD>
+__global__ void __launch_bounds__(kScorePThreads, 1)
+k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap tm_q,
+             const __grid_constant__ CUtensorMap tm_k) {
+    using C = ScorePCfg<HD>;
+    // runs beside k_quant_means (launched before it as its programmatic
+    // dependent) and completes only after it
+    if (!*P.meta_valid) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        return;
+    }
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    __shared__ uint64_t q_full, q_empty, k_full[2], k_empty[2], acc_full[2], acc_empty[2], drain;
+    __shared__ uint32_t tmem_base;
+    __shared__ volatile int abort_flag;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_groups = P.group_cu[D.n_seqs];
+    const int64_t n_items = (int64_t)n_groups * D.Hkv;
+    const int64_t n_slots = (n_items + gridDim.x - 1) / gridDim.x * gridDim.x;
+
+    if (tid == 0) {
+        mbar_init(&q_full, 1);
+        mbar_init(&q_empty, 1);
+        mbar_init(&drain, 1);
+        for (int u = 0; u < 2; ++u) {
+            mbar_init(&k_full[u], 1);
+            mbar_init(&k_empty[u], 1);
+            mbar_init(&acc_full[u], 1);
+            mbar_init(&acc_empty[u], 4);
+        }
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async_smem();
+    }
+    if (warp == 5) tmem_alloc(&tmem_base, 2 * kScoreKeys);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+
+    if (warp == 4) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            uint32_t qn = 0, kn = 0;   // Q loads, K chunk loads issued
+            uint32_t kuse[2] = {0, 0};  // loads issued into each K slot
+            for (int64_t w = blockIdx.x; w < n_slots; w += gridDim.x) {
+                const ScoreItem it = score_item(D, P, w, n_groups);
+                if (it.n_chunks == 0) continue;
+                if (!mbar_wait(&q_empty, (qn & 1) ^ 1, &abort_flag, P.status)) break;
+                ++qn;
+                mbar_arrive_expect_tx(&q_full, C::kAtoms * kScoreQV * 128);
+#pragma unroll
+                for (int a = 0; a < C::kAtoms; ++a)
+                    tma_load_3d(smem + C::kOffQ + a * C::kAtomBytes, &tm_q, &q_full, 32 * a, it.g * D.G,
+                                it.b0 + it.i0);
+                bool ok = true;
+                for (int c = 0; c < it.n_chunks && ok; ++c, ++kn) {
+                    const int slot = kn & 1;
+                    if (!mbar_wait(&k_empty[slot], ((kn >> 1) & 1) ^ 1, &abort_flag, P.status)) {
+                        ok = false;
+                        break;
+                    }
+                    ++kuse[slot];
+                    mbar_arrive_expect_tx(&k_full[slot], C::kAtoms * kScoreKeys * 128);
+#pragma unroll
+                    for (int a = 0; a < C::kAtoms; ++a)
+                        tma_load_3d(smem + C::kOffK + slot * C::kTileBytes + a * C::kAtomBytes, &tm_k,
+                                    &k_full[slot], 32 * a, it.g, it.b0 + kScoreKeys * c);
+                }
+                if (!ok) break;
+            }
+            // let the copies in flight land before the CTA may exit
+            if (qn) mbar_wait_drain(&q_full, (qn - 1) & 1, P.status);
+            for (int u = 0; u < 2; ++u)
+                if (kuse[u]) mbar_wait_drain(&k_full[u], (kuse[u] - 1) & 1, P.status);
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {
+            const uint64_t dq = smem_desc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
+            constexpr uint32_t idesc = idesc_tf32(128, kScoreKeys);
+            uint32_t qn = 0, kn = 0, an = 0;
+            for (int64_t w = blockIdx.x; w < n_slots; w += gridDim.x) {
+                const ScoreItem it = score_item(D, P, w, n_groups);
+                if (it.n_chunks == 0) continue;
+                if (!mbar_wait(&q_full, qn & 1, &abort_flag, P.status)) break;
+                ++qn;
+                bool ok = true;
+                for (int c = 0; c < it.n_chunks; ++c, ++kn, ++an) {
+                    const int slot = kn & 1, buf = an & 1;
+                    if (!mbar_wait(&k_full[slot], (kn >> 1) & 1, &abort_flag, P.status) ||
+                        !mbar_wait(&acc_empty[buf], ((an >> 1) & 1) ^ 1, &abort_flag, P.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t dk = smem_desc_sw128(smem_u32(smem + C::kOffK + slot * C::kTileBytes), 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < HD / 8; ++kk) {
+                        const uint32_t off = (kk / 4) * C::kAtomBytes + (kk % 4) * 32;
+                        umma_tf32(tmem + buf * kScoreKeys, dq + (off >> 4), dk + (off >> 4), idesc,
+                                  kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&k_empty[slot]);
+                    umma_commit(&acc_full[buf]);
+                }
+                if (!ok) break;
+                umma_commit(&q_empty);
+            }
+            // every MMA issued above completes before the CTA may exit
+            umma_commit(&drain);
+            mbar_wait_drain(&drain, 0, P.status);
+        }
+    } else {
+        // epilogue warps 0-3: thread = query vector (block ri, head hl) of the item
+        const float inv_sqrt_d = 1.0f / sqrtf((float)HD);
+        const int G = D.G;
+        const int row = 32 * warp + lane;
+        const int ri = row / G, hl = row % G;
+        uint32_t an = 0;
+        for (int64_t w = blockIdx.x; w < n_slots; w += gridDim.x) {
+            const ScoreItem it = score_item(D, P, w, n_groups);
+            if (it.n_chunks == 0) continue;
+            const int i = it.i0 + ri;
+            const bool row_ok = i < it.i1 && hl == 0;
+            float* sc_row = W.scores + (int64_t)it.g * D.tri_total + P.tri_off[it.s] + (int64_t)i * (i + 1) / 2;
+            bool ok = true;
+            for (int c = 0; c < it.n_chunks; ++c, ++an) {
+                const int buf = an & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (an >> 1) & 1, &abort_flag, P.status))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll 1
+                for (int cc = 0; cc < kScoreKeys / 32; ++cc) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + buf * kScoreKeys + 32 * cc, r);
+                    tmem_ld_wait();
+                    const int jb = kScoreKeys * c + 32 * cc;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        float v = __uint_as_float(r[e]);
+                        for (int o = 1; o < G; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                        if (row_ok && jb + e <= i) sc_row[jb + e] = v * inv_sqrt_d;
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            }
+            if (!ok) {
+                abort_flag = 1;
+                break;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 2 * kScoreKeys);
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // float64 score of key block j for row (b_i, g): max over the group's heads
@@ -626,8 +941,66 @@ __device__ double score64(const Dims& D, const WsPtrs& W, int64_t b_i, int64_t b
 // with rel_err the scoring kernel's bound (kScoreTcRelErr).  Every block whose
 // score could be the row maximum and every block whose score lies within e_j of
 // tau * m is re-scored in float64.
+// Rows of up to 32 * kThrRegs blocks load their scores in one pass.
+constexpr int kThrRegs = 32;
+
+// The decision of one row (warp-collective), given the largest lower bound
+// m_lo of its scores: the row maximum in float64 over every block whose upper
+// bound reaches m_lo, then keep / drop per block, re-scoring in float64 every
+// block within its bound Cq * |Kbar_j| of the threshold.  Writes the mask
+// words 0 .. i / 32 and zeroes the rest; adds the kept count to `count`.
+template <int HD>
+__device__ __forceinline__ void thr_decide(const Dims& D, const WsPtrs& W, const float* sc,
+                                           const float* kn, double Cq, double m_lo, int i,
+                                           int64_t bi, int b0, int g, int lane, uint32_t* mask,
+                                           int& count) {
+    double m = -DBL_MAX;
+#pragma unroll 1
+    for (int jb = 0; jb <= i; jb += 32) {
+        const int j = jb + lane;
+        const bool cand = j <= i && (double)__ldg(sc + j) + Cq * __ldg(kn + (int64_t)j * D.Hkv) >= m_lo;
+        uint32_t cb = __ballot_sync(0xffffffffu, cand);
+        while (cb) {
+            const int l = __ffs(cb) - 1;
+            cb &= cb - 1;
+            m = fmax(m, score64<HD>(D, W, bi, b0 + jb + l, g));
+        }
+    }
+    const double t = D.tau * m;
+#pragma unroll 1
+    for (int w = 0; 32 * w <= i; ++w) {
+        const int j = 32 * w + lane;
+        bool keep = false, unsure = false;
+        if (j <= i) {
+            if (j == 0 || j == i) {
+                keep = true;
+            } else {
+                const double e = Cq * __ldg(kn + (int64_t)j * D.Hkv);
+                const double x = (double)__ldg(sc + j);
+                if (x - e >= t) keep = true;
+                else if (!(x + e < t)) unsure = true;
+            }
+        }
+        uint32_t ub = __ballot_sync(0xffffffffu, unsure);
+        while (ub) {
+            const int l = __ffs(ub) - 1;
+            ub &= ub - 1;
+            const double x64 = score64<HD>(D, W, bi, b0 + 32 * w + l, g);
+            if (lane == l) keep = x64 >= t;
+        }
+        const uint32_t bits = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) mask[w] = bits;
+        count += __popc(bits);
+    }
+    for (int w = i / 32 + 1 + lane; w < D.mask_words; w += 32) mask[w] = 0u;
+}
+
 template <int HD, bool CHUNK>
 __global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W, double rel_err) {
+    // launched as a programmatic dependent: everything before it is complete
+    // once the wait returns
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (!*P.meta_valid) return;
     const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
@@ -650,55 +1023,43 @@ __global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W,
             mask[w] = bits;
         }
         count = i + 1;
+    } else if (i < 32 * kThrRegs) {
+        // one pass of loads with every load of the row in flight at once (the
+        // row's scores and key norms, 32 per lane, in registers), then the two
+        // decision passes over the same lines from L1
+        const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
+        const double C = rel_err / sqrt((double)HD);
+        const double qn = W.qnorm[bi * D.Hkv + g];
+        const float* kn = W.knorm + (int64_t)b0 * D.Hkv + g;
+        float x[kThrRegs], kv[kThrRegs];
+#pragma unroll
+        for (int u = 0; u < kThrRegs; ++u) {
+            const int j = 32 * u + lane;
+            const bool in = j <= i;
+            x[u] = in ? __ldg(sc + j) : 0.f;
+            kv[u] = in ? __ldg(kn + (int64_t)j * D.Hkv) : 0.f;
+        }
+        // largest lower bound of any score
+        double m_lo = -DBL_MAX;
+#pragma unroll
+        for (int u = 0; u < kThrRegs; ++u)
+            if (32 * u + lane <= i) m_lo = fmax(m_lo, (double)x[u] - C * qn * kv[u]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m_lo = fmax(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o));
+        thr_decide<HD>(D, W, sc, kn, C * qn, m_lo, i, bi, b0, g, lane, mask, count);
     } else {
         const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
         const double C = rel_err / sqrt((double)HD);
         const double qn = W.qnorm[bi * D.Hkv + g];
         const float* kn = W.knorm + (int64_t)b0 * D.Hkv + g;
-        // pass 1: largest lower bound of any score
+        // largest lower bound of any score
         double m_lo = -DBL_MAX;
-        for (int j = lane; j <= i; j += 32) m_lo = fmax(m_lo, (double)sc[j] - C * qn * kn[(int64_t)j * D.Hkv]);
+#pragma unroll 8
+        for (int j = lane; j <= i; j += 32)
+            m_lo = fmax(m_lo, (double)__ldg(sc + j) - C * qn * __ldg(kn + (int64_t)j * D.Hkv));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m_lo = fmax(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o));
-        // pass 2: the row maximum in float64 over every candidate
-        double m = -DBL_MAX;
-        for (int jb = 0; jb <= i; jb += 32) {
-            const int j = jb + lane;
-            const bool cand = j <= i && (double)sc[j] + C * qn * kn[(int64_t)j * D.Hkv] >= m_lo;
-            uint32_t cb = __ballot_sync(0xffffffffu, cand);
-            while (cb) {
-                const int l = __ffs(cb) - 1;
-                cb &= cb - 1;
-                m = fmax(m, score64<HD>(D, W, bi, b0 + jb + l, g));
-            }
-        }
-        const double t = D.tau * m;
-        // pass 3: decisions (forced blocks 0 and i; uncertain ones in float64)
-        for (int w = 0; 32 * w <= i; ++w) {
-            const int j = 32 * w + lane;
-            bool keep = false, unsure = false;
-            if (j <= i) {
-                if (j == 0 || j == i) {
-                    keep = true;
-                } else {
-                    const double e = C * qn * kn[(int64_t)j * D.Hkv];
-                    const double x = (double)sc[j];
-                    if (x - e >= t) keep = true;
-                    else if (!(x + e < t)) unsure = true;
-                }
-            }
-            uint32_t ub = __ballot_sync(0xffffffffu, unsure);
-            while (ub) {
-                const int l = __ffs(ub) - 1;
-                ub &= ub - 1;
-                const double x64 = score64<HD>(D, W, bi, b0 + 32 * w + l, g);
-                if (lane == l) keep = x64 >= t;
-            }
-            const uint32_t bits = __ballot_sync(0xffffffffu, keep);
-            if (lane == 0) mask[w] = bits;
-            count += __popc(bits);
-        }
-        for (int w = i / 32 + 1 + lane; w < D.mask_words; w += 32) mask[w] = 0u;
+        thr_decide<HD>(D, W, sc, kn, C * qn, m_lo, i, bi, b0, g, lane, mask, count);
     }
     if (lane == 0) W.counts[r] = count;
 }
@@ -724,6 +1085,9 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
 constexpr int kQuantMeansThreads = 1024;
 
 __global__ void __launch_bounds__(kQuantMeansThreads) k_quant_means(Dims D, PlanPtrs P) {
+    // the scorer, launched next, may run beside this kernel (it needs nothing
+    // from it) and waits for it before it completes
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (!*P.meta_valid) return;
     const int s = blockIdx.y;
     const int g = blockIdx.z;
@@ -792,28 +1156,24 @@ __global__ void __launch_bounds__(kQuantMeansThreads) k_quant_means(Dims D, Plan
 constexpr int kScanThreads = 1024;
 
 __global__ void __launch_bounds__(kScanThreads) k_scan(Dims D, PlanPtrs P, WsPtrs W) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // (a programmatic dependent)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (!*P.meta_valid) return;
-    __shared__ int64_t part[kScanThreads];
+    static_assert(kScanThreads == kMetaThreads, "block_excl_scan is sized for kMetaThreads");
     const int64_t R = D.R;
     const int64_t per = (R + kScanThreads - 1) / kScanThreads;
     const int64_t lo = R < (int64_t)threadIdx.x * per ? R : (int64_t)threadIdx.x * per;
     const int64_t hi = R < lo + per ? R : lo + per;
     int64_t sum = 0;
+#pragma unroll 4
     for (int64_t r = lo; r < hi; ++r) sum += W.counts[r];
-    part[threadIdx.x] = sum;
-    __syncthreads();
-    for (int o = 1; o < kScanThreads; o <<= 1) {
-        int64_t add = threadIdx.x >= o ? part[threadIdx.x - o] : 0;
-        __syncthreads();
-        part[threadIdx.x] += add;
-        __syncthreads();
-    }
-    int64_t run = part[threadIdx.x] - sum;
+    int64_t total;
+    int64_t run = block_excl_scan(sum, &total);
     for (int64_t r = lo; r < hi; ++r) {
         P.row_ptr[r] = (int32_t)run;
         run += W.counts[r];
     }
-    if (threadIdx.x == kScanThreads - 1) P.row_ptr[R] = (int32_t)part[kScanThreads - 1];
+    if (threadIdx.x == 0) P.row_ptr[R] = (int32_t)total;
 }
 
 // ---------------------------------------------------------------------------
@@ -821,6 +1181,7 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(Dims D, PlanPtrs P, WsPtr
 // ---------------------------------------------------------------------------
 
 __global__ void k_compact(Dims D, PlanPtrs P) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // (a programmatic dependent)
     if (!*P.meta_valid) return;
     const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
@@ -837,6 +1198,27 @@ __global__ void k_compact(Dims D, PlanPtrs P) {
     }
 }
 
+// Launch with programmatic stream serialization: the kernel may begin before
+// the one before it in the stream completes; what it may read before its
+// griddepcontrol.wait is stated at each kernel.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+               Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? FP2_OK : FP2_ERR_CUDA;
+}
+
+// Scores (tau > 0; launched right after k_quant_means, beside which it runs)
+// and the threshold.
 template <int HD>
 int launch_score(const Dims& D, const PlanPtrs& P, const WsPtrs& W, cudaStream_t st) {
     if (D.tau > 0.0) {
@@ -851,20 +1233,59 @@ int launch_score(const Dims& D, const PlanPtrs& P, const WsPtrs& W, cudaStream_t
         if (!make_tensor_map(&tq, W.qbar32, 3, qd, qs, qb, kMapF32) ||
             !make_tensor_map(&tk, W.kbar_tf, 3, kd, ks, kb, kMapF32))
             return FP2_ERR_CUDA;
-        const int smem = ScoreTcCfg<HD>::kSmem;
-        if (cudaFuncSetAttribute(k_score_tc<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smem) != cudaSuccess)
-            return FP2_ERR_CUDA;
-        const int64_t items = D.score_tiles * D.Hkv;
-        const int grid = (int)std::min<int64_t>(items, std::max(1, sm_count()));
-        k_score_tc<HD><<<grid, kScoreTcThreads, smem, st>>>(D, P, W, tq, tk);
+        int rc;
+        if (D.G <= 32 && (D.G & (D.G - 1)) == 0) {
+            // the G heads of a block are G aligned, adjacent lanes of one warp
+            const int smem = ScorePCfg<HD>::kSmem;
+            if (cudaFuncSetAttribute(k_score_pipe<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     smem) != cudaSuccess)
+                return FP2_ERR_CUDA;
+            const int64_t items = (int64_t)D.n_groups_cap * D.Hkv;
+            const int grid = (int)std::min<int64_t>(items, std::max(1, sm_count()));
+            rc = launch_pdl(k_score_pipe<HD>, dim3(grid), dim3(kScorePThreads), smem, st, D, P, W, tq, tk);
+        } else {
+            const int smem = ScoreTcCfg<HD>::kSmem;
+            if (cudaFuncSetAttribute(k_score_tc<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     smem) != cudaSuccess)
+                return FP2_ERR_CUDA;
+            const int64_t items = D.score_tiles * D.Hkv;
+            const int grid = (int)std::min<int64_t>(items, std::max(1, sm_count()));
+            rc = launch_pdl(k_score_tc<HD>, dim3(grid), dim3(kScoreTcThreads), smem, st, D, P, W, tq, tk);
+        }
+        if (rc != FP2_OK) return rc;
     }
-    const unsigned grid = (unsigned)((D.R * 32 + 255) / 256);
-    if (P.cu_q)
-        k_threshold<HD, true><<<grid, 256, 0, st>>>(D, P, W, kScoreTcRelErr);
-    else
-        k_threshold<HD, false><<<grid, 256, 0, st>>>(D, P, W, kScoreTcRelErr);
-    return FP2_OK;
+    const dim3 grid((unsigned)((D.R * 32 + 255) / 256));
+    if (P.cu_q) return launch_pdl(k_threshold<HD, true>, grid, dim3(256), 0, st, D, P, W, kScoreTcRelErr);
+    return launch_pdl(k_threshold<HD, false>, grid, dim3(256), 0, st, D, P, W, kScoreTcRelErr);
+}
+
+}  // namespace
+
+namespace {
+
+template <bool KV8, bool CHUNK, bool BYVAL, bool NORMS>
+void launch_pool(const Layout& L, const fp2_problem* p, const SeqMap& M, const void* q,
+                 const void* k, const void* v, const float* k_scale, const float* v_scale,
+                 const PlanPtrs& P, const WsPtrs& W, cudaStream_t st) {
+    const Dims& D = L.dims;
+    const int vecs = (D.Hq + 2 * D.Hkv) * D.d / 8;
+    dim3 grid((unsigned)D.NB, (vecs + kPoolThreads - 1) / kPoolThreads);
+    k_pool<KV8, CHUNK, BYVAL, NORMS><<<grid, kPoolThreads, 0, st>>>(
+        D, M, L.Tq, p->cu_seqlens, p->page_table, static_cast<const uint16_t*>(q), k, v, k_scale,
+        v_scale, P, W);
+}
+
+template <bool KV8, bool CHUNK>
+void launch_pool_kv(const Layout& L, const fp2_problem* p, const SeqMap& M, bool byval, bool norms,
+                    const void* q, const void* k, const void* v, const float* ks, const float* vs,
+                    const PlanPtrs& P, const WsPtrs& W, cudaStream_t st) {
+    if (byval) {
+        if (norms) launch_pool<KV8, CHUNK, true, true>(L, p, M, q, k, v, ks, vs, P, W, st);
+        else launch_pool<KV8, CHUNK, true, false>(L, p, M, q, k, v, ks, vs, P, W, st);
+    } else {
+        if (norms) launch_pool<KV8, CHUNK, false, true>(L, p, M, q, k, v, ks, vs, P, W, st);
+        else launch_pool<KV8, CHUNK, false, false>(L, p, M, q, k, v, ks, vs, P, W, st);
+    }
 }
 
 }  // namespace
@@ -875,29 +1296,70 @@ int launch_plan(const Layout& L, const fp2_problem* p, const void* q, const void
     const Dims& D = L.dims;
     PlanPtrs P = P0;
     P.cu_q = L.chunked ? p->cu_q_seqlens : nullptr;
-    k_meta<<<1, kMetaThreads, 0, st>>>(D, L.sched, p->cu_seqlens, p->page_table, L.Tq, P);
-    const int vecs = (D.Hq + 2 * D.Hkv) * D.d / 8;
-    dim3 pool_grid((unsigned)D.NB, (vecs + kPoolThreads - 1) / kPoolThreads);
-    const uint16_t* q16 = static_cast<const uint16_t*>(q);
-    if (k_scale)   // (an FP8 KV cache is never chunked: the entry point rejects it)
-        k_pool<true, false><<<pool_grid, kPoolThreads, 0, st>>>(D, p->cu_seqlens, p->page_table, q16,
-                                                                k, v, k_scale, v_scale, P, W);
-    else if (L.chunked)
-        k_pool<false, true><<<pool_grid, kPoolThreads, 0, st>>>(D, p->cu_seqlens, p->page_table, q16,
-                                                                k, v, nullptr, nullptr, P, W);
-    else
-        k_pool<false, false><<<pool_grid, kPoolThreads, 0, st>>>(D, p->cu_seqlens, p->page_table, q16,
-                                                                 k, v, nullptr, nullptr, P, W);
-    if (D.tau > 0.0) {
+    // The pooling kernel runs first when the sequences fit the by-value map:
+    // it then needs nothing from k_meta, which is launched after it as a
+    // programmatic dependent (it may start once every pooling CTA has begun,
+    // overlapping the pool's last wave) and waits for it before completing.
+    const bool byval = D.n_seqs <= kMapSeqs;
+    SeqMap M;
+    std::memset(&M, 0, sizeof(M));
+    if (byval) {
+        M.n = D.n_seqs;
+        for (int s = 0; s < D.n_seqs; ++s) {
+            const int Ls = p->seqlens[s];
+            const int Qs = L.chunked ? p->q_seqlens[s] : Ls;
+            M.cu_blocks[s + 1] = M.cu_blocks[s] + (Ls + D.B - 1) / D.B;
+            M.cu_tok[s + 1] = M.cu_tok[s] + Ls;
+            M.cu_q[s + 1] = M.cu_q[s] + Qs;
+            M.q_off[s] = Ls - Qs;
+        }
+    }
+    // the threshold's error-bound norms come out of the pooling kernel when
+    // the G query heads of a kv-head fall into one pooling CTA (1024 columns)
+    const bool norms_in_pool = D.tau > 0.0 && (kPoolThreads * 8) % (D.G * D.d) == 0;
+    auto meta = [&]() -> int {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(1);
+        cfg.blockDim = dim3(kMetaThreads);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = byval ? 1 : 0;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, k_meta, D, L.sched, p->cu_seqlens, p->page_table, L.Tq, P) ==
+                       cudaSuccess
+                   ? FP2_OK
+                   : FP2_ERR_CUDA;
+    };
+    auto pool = [&]() {
+        if (k_scale)   // (an FP8 KV cache is never chunked: the entry point rejects it)
+            launch_pool_kv<true, false>(L, p, M, byval, norms_in_pool, q, k, v, k_scale, v_scale, P, W, st);
+        else if (L.chunked)
+            launch_pool_kv<false, true>(L, p, M, byval, norms_in_pool, q, k, v, nullptr, nullptr, P, W, st);
+        else
+            launch_pool_kv<false, false>(L, p, M, byval, norms_in_pool, q, k, v, nullptr, nullptr, P, W, st);
+    };
+    if (byval) {
+        pool();
+        if (meta() != FP2_OK) return FP2_ERR_CUDA;
+    } else {
+        if (meta() != FP2_OK) return FP2_ERR_CUDA;
+        pool();
+    }
+    if (D.tau > 0.0 && !norms_in_pool) {
         const int64_t warps = D.NB * D.Hkv;
         k_norms<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(D, P, W);
     }
-    int rc = D.d == 64 ? launch_score<64>(D, P, W, st) : launch_score<128>(D, P, W, st);
-    if (rc != FP2_OK) return rc;
+    // e4m3 block means (needs the pool's K/V means only); the scorer runs beside it
     k_quant_means<<<dim3((unsigned)((D.max_nb + D.B - 1) / D.B), D.n_seqs, D.Hkv), kQuantMeansThreads, 0,
                     st>>>(D, P);
-    k_scan<<<1, kScanThreads, 0, st>>>(D, P, W);
-    k_compact<<<(unsigned)((D.R * 32 + 255) / 256), 256, 0, st>>>(D, P);
+    int rc = D.d == 64 ? launch_score<64>(D, P, W, st) : launch_score<128>(D, P, W, st);
+    if (rc != FP2_OK) return rc;
+    if (launch_pdl(k_scan, dim3(1), dim3(kScanThreads), 0, st, D, P, W) != FP2_OK ||
+        launch_pdl(k_compact, dim3((unsigned)((D.R * 32 + 255) / 256)), dim3(256), 0, st, D, P) != FP2_OK)
+        return FP2_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? FP2_OK : FP2_ERR_CUDA;
 }
 

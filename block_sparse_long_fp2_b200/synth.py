@@ -24,6 +24,15 @@ Every head draws from its own generator spawned from the workload seed.
   shared part about 2).  The keys of the first 4 tokens of every sequence
   are scaled by 8 (attention sinks).  V ~ N(0, 1).
 * ``lowrank+needles`` -- ``lowrank`` plus needles at uniform positions.
+* ``topics``   -- block-level structure that the block means carry (the
+  retrieval structure that makes the pages' real prompts 5-9 % dense): per
+  kv-head, ``n_topics`` orthonormal directions w_t; every key block j draws
+  a topic t_j and every query block i a topic t'_i (uniform, per kv-head);
+  K = N(0, 1) + 3 w_{t_j} on the tokens of block j, Q = N(0, 1) + 3 w_{t'_i}
+  on the tokens of block i (all G query heads of the kv-head), V ~ N(0, 1).
+  A block's score is about 9 / sqrt(d) when the topics match and near zero
+  otherwise, so a threshold between them keeps about 1 / n_topics of the
+  blocks (plus the forced sink and diagonal blocks).
 
 A paged layout places every sequence's 64-token pages at a seeded random
 permutation of a larger pool.  Whole pages that no sequence uses are filled
@@ -88,6 +97,7 @@ class Workload:
     pool_pages: int = 0         # pages in the pool when paged
     dtype: str = "bf16"
     seed: int = 0
+    n_topics: int = 0           # "topics" generator: topics per kv-head
 
     @property
     def T(self) -> int:
@@ -105,6 +115,12 @@ def workloads() -> Dict[str, Workload]:
         "paged_mix": Workload("paged_mix", [4096, 9000, 16384, 30000, 65536, 1500], 32, 8, 128, 128,
                               0.1, "lowrank", 0, page_size=64, pool_pages=2048, seed=1003),
     }
+    # low-density layers: the 128K shape with block-level topics, about 5, 10
+    # and 20 % of the blocks kept (Table 3's 64K-128K densities are 4.6-9.4 %)
+    for pct, nt in ((5, 20), (10, 10), (20, 5)):
+        name = f"topics_128k_{pct}pct"
+        w[name] = Workload(name, [131072], 32, 8, 128, 128, 0.5, "topics", 0, seed=1100 + pct,
+                           n_topics=nt)
     for li, L in enumerate([4096, 8192, 16384, 32768, 65536, 131072]):
         for ti, tau in enumerate([0.0, 0.05, 0.2]):
             name = f"sweep_{L // 1024}k_tau{tau:g}"
@@ -132,6 +148,19 @@ def _fill_head(seed_seq, out: np.ndarray, h: int, W: Optional[np.ndarray]) -> No
     z = _normal(rng, (T, W.shape[0]))
     out[:, h, :] = _normal(rng, (T, d))
     out[:, h, :] += z @ W
+
+
+def _fill_head_topic(seed_seq, out: np.ndarray, h: int, dirs: np.ndarray, tok_topic: np.ndarray,
+                     amp: float) -> None:
+    """out[:, h, :] = N(0, 1) + amp * dirs[tok_topic[t]] (the topic direction of
+    the block each token t belongs to), from the head's own generator."""
+    rng = np.random.Generator(np.random.PCG64(seed_seq))
+    T, _, d = out.shape
+    out[:, h, :] = _normal(rng, (T, d))
+    chunk = 1 << 16
+    for lo in range(0, T, chunk):
+        hi = min(T, lo + chunk)
+        out[lo:hi, h, :] += amp * dirs[tok_topic[lo:hi]]
 
 
 def _fill_heads(children, out: np.ndarray, Ws) -> None:
@@ -188,6 +217,27 @@ def generate(wl: Workload) -> Dict[str, object]:
         for L in wl.seqlens:
             k[t0:t0 + min(4, L)] *= 8.0
             t0 += L
+    elif wl.generator == "topics":
+        nt = wl.n_topics
+        assert 1 <= nt <= d
+        # per kv-head orthonormal topic directions; per (kv-head, block) topics
+        dirs = [np.linalg.qr(rng.standard_normal((d, nt)))[0].T.astype(np.float32)
+                for _ in range(Hkv)]
+        nbs = [(L + wl.B - 1) // wl.B for L in wl.seqlens]
+        NB = int(sum(nbs))
+        ktop = rng.integers(0, nt, size=(Hkv, NB))
+        qtop = rng.integers(0, nt, size=(Hkv, NB))
+        tok_block = np.concatenate([b0 + np.arange(L) // wl.B for b0, L in
+                                    zip(np.concatenate([[0], np.cumsum(nbs)[:-1]]), wl.seqlens)])
+        import concurrent.futures
+        import os
+        with concurrent.futures.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
+            jobs = [ex.submit(_fill_head_topic, kids[h], q, h, dirs[h // G], qtop[h // G][tok_block], 3.0)
+                    for h in range(Hq)]
+            jobs += [ex.submit(_fill_head_topic, kids[Hq + g], k, g, dirs[g], ktop[g][tok_block], 3.0)
+                     for g in range(Hkv)]
+            for j in jobs:
+                j.result()
     elif wl.generator == "needles" or wl.generator == "normal":
         _fill_heads(kids[:Hq], q, [None] * Hq)
         _fill_heads(kids[Hq:Hq + Hkv], k, [None] * Hkv)
@@ -243,10 +293,10 @@ def make_paged(rng, k: np.ndarray, v: np.ndarray, seqlens: Sequence[int], page: 
 
 
 def small_workload(seqlens, Hq, Hkv, d, B, tau, seed, generator="lowrank", n_needles=0,
-                   page_size=0, pool_pages=0) -> Workload:
+                   page_size=0, pool_pages=0, n_topics=0) -> Workload:
     """A test-sized workload with the same generators."""
     return Workload(f"small_{seed}", list(seqlens), Hq, Hkv, d, B, tau, generator, n_needles,
-                    page_size=page_size, pool_pages=pool_pages, seed=seed)
+                    page_size=page_size, pool_pages=pool_pages, seed=seed, n_topics=n_topics)
 
 
 def sample_qblocks(nb: int, count: int, seed: int) -> List[int]:
