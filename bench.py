@@ -8,11 +8,12 @@ attention with mean correction).  The default workload is the 128K-token
 Qwen3-4B-shaped layer (32 query / 8 kv heads, head dim 128, block 128,
 tau 0.05, low-rank + needle generator).
 
-Prints one JSON line.  `value` is dense-equivalent TFLOP/s of the whole job
-(sum over ranks of 2*d*Hq*sum L(L+1) per step, divided by the max over ranks
-of the device time), inputs resident in HBM.  Each rank runs an independent
-layer (weak scaling, no collective on the data path); torch.distributed only
-provides the barrier and the max over ranks.
+Prints one JSON line.  `value` is dense-equivalent TFLOP/s of the whole layer
+(2*d*Hq*sum L(L+1) per step, divided by the max over ranks of the device
+time), inputs resident in HBM.  On N GPUs the layer is split by kv-head: rank
+r runs its contiguous share of the kv-heads (and their query heads) in place
+in the full-layer tensors (strong scaling, no collective on the data path);
+torch.distributed only provides the barrier and the max over ranks.
 
 The line also carries the FP8-e4m3 leg (plan + online quantisation + e4m3
 prefill on the same layer) and the dense baseline (the same kernels with
@@ -28,7 +29,6 @@ workload (rank 0 only) and prints the same metric for it.
 from __future__ import annotations
 
 import argparse
-import copy
 import json
 import os
 import statistics
@@ -61,12 +61,22 @@ def kept_tile_flop(wl) -> float:
     return 4.0 * wl.d * G * wl.B * wl.B
 
 
-def rank_workload(name: str, rank: int):
-    """The workload a rank runs: the named layer with a rank-dependent seed,
-    so every rank processes an independent layer (weak scaling)."""
-    wl = copy.deepcopy(synth.workloads()[name])
-    wl.seed += 7919 * rank
-    return wl
+def plan_launches(wl, tau=None) -> int:
+    """Kernels fp2_plan launches: pool, meta, e4m3 means, threshold, scan and
+    compact; with tau > 0 the scorer, and the separate norms kernel when the G
+    query heads of a kv-head do not fall into one pooling CTA (1024 columns)."""
+    tau = wl.tau if tau is None else tau
+    G = wl.Hq // wl.Hkv
+    return 6 + (1 if tau > 0 else 0) + (1 if tau > 0 and 1024 % (G * wl.d) != 0 else 0)
+
+
+def rank_slice(wl, world: int, rank: int):
+    """The kv-heads a rank runs: the layer split over the ranks by kv-head
+    (each kv-head with its G query heads is planned and attended on its own,
+    so the ranks exchange nothing on the data path).  Returns (first kv-head,
+    kv-heads)."""
+    from block_sparse_long_fp2_b200.binding import kv_head_slice
+    return kv_head_slice(wl.Hkv, world, rank)
 
 
 def max_over_ranks(values, world: int, device):
@@ -79,9 +89,10 @@ def max_over_ranks(values, world: int, device):
     return [float(v) for v in t.cpu()]
 
 
-def whole_job_value(flop_per_rank: float, world: int, ms: float) -> float:
-    """Throughput of the whole job: the work of all ranks over the slowest rank's time."""
-    return world * flop_per_rank / (ms * 1e-3) / 1e12
+def whole_job_value(flop: float, ms: float) -> float:
+    """Throughput of the whole job: the layer's work (all ranks' slices
+    together) over the slowest rank's time."""
+    return flop / (ms * 1e-3) / 1e12
 
 
 def attn_traffic(workload: str, dtype: str):
@@ -175,8 +186,11 @@ def run_ours(args, rank, world, local_rank):
     fbuild.build()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = rank_workload(args.workload, rank)
+    wl = synth.workloads()[args.workload]
     x = synth.generate(wl)
+    h0, hn = rank_slice(wl, world, rank)   # this rank's kv-heads of the layer
+    G = wl.Hq // wl.Hkv
+    slice_kw = {"kv_head_begin": h0, "num_kv_heads_total": wl.Hkv}
     stream = torch.cuda.current_stream()
 
     def dev_bf16(a):
@@ -190,13 +204,14 @@ def run_ours(args, rank, world, local_rank):
         k, v = dev_bf16(x["k"]), dev_bf16(x["v"])
         pt = None
     cu = torch.from_numpy(x["cu_seqlens"]).to(dev)
-    prob = fb.Problem(wl.seqlens, cu, wl.Hq, wl.Hkv, wl.d, wl.B, wl.tau,
+    prob = fb.Problem(wl.seqlens, cu, G * hn, hn, wl.d, wl.B, wl.tau,
                       page_size=wl.page_size, page_table=pt,
-                      num_pages=int(x["k_pool"].shape[0]) if wl.page_size else 0)
+                      num_pages=int(x["k_pool"].shape[0]) if wl.page_size else 0, **slice_kw)
     lay, plan, ws = fb.allocate(prob, dev)
     o = torch.empty((wl.T, wl.Hq, wl.d), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((wl.Hq, wl.T), dtype=torch.float32, device=dev)
-    in_bytes = (q.numel() + k.numel() + v.numel()) * 2
+    in_bytes = (q.numel() + k.numel() + v.numel()) * 2          # the layer's Q, K, V
+    slice_bytes = in_bytes * hn // wl.Hkv                          # this rank's heads of them
 
     def step():
         fb.fp2_plan(prob, q, k, v, plan, ws, stream)
@@ -208,7 +223,7 @@ def run_ours(args, rank, world, local_rank):
     rc, st = fb.fp2_status_check(plan, stream)
     if rc != 0:
         raise RuntimeError(f"device status {st:#x} ({fb.strerror(rc)})")
-    nnz = int(fb.PlanView(plan, lay, wl.Hkv, wl.d).row_ptr[-1].item())
+    nnz = int(fb.PlanView(plan, lay, hn, wl.d).row_ptr[-1].item())
 
     # timed region: K steps, per-stage events on the launching stream
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
@@ -235,15 +250,15 @@ def run_ours(args, rank, world, local_rank):
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
     # plan: meta, pool, [norms, score], threshold, quant_means, scan, compact; prefill: attn
     # (+ the split merge when the schedule splits rows)
-    launches_per_step = (8 if wl.tau > 0 else 6) + 1 + (1 if lay.num_split_slots > 0 else 0)
+    launches_per_step = plan_launches(wl) + 1 + (1 if lay.num_split_slots > 0 else 0)
 
     # dense baseline: the same kernels on the same inputs with tau = 0 (every
     # causally visible block kept, no pseudo tiles)
     dense = None
     if not args.no_dense and wl.tau > 0:
-        prob0 = fb.Problem(wl.seqlens, cu, wl.Hq, wl.Hkv, wl.d, wl.B, 0.0,
+        prob0 = fb.Problem(wl.seqlens, cu, G * hn, hn, wl.d, wl.B, 0.0,
                            page_size=wl.page_size, page_table=pt,
-                           num_pages=int(x["k_pool"].shape[0]) if wl.page_size else 0)
+                           num_pages=int(x["k_pool"].shape[0]) if wl.page_size else 0, **slice_kw)
         lay0, plan0, ws0 = fb.allocate(prob0, dev)
 
         def step0(evs=None):
@@ -262,7 +277,7 @@ def run_ours(args, rank, world, local_rank):
         rc, st = fb.fp2_status_check(plan0, stream)
         if rc != 0:
             raise RuntimeError(f"device status {st:#x} ({fb.strerror(rc)})")
-        nnz0 = int(fb.PlanView(plan0, lay0, wl.Hkv, wl.d).row_ptr[-1].item())
+        nnz0 = int(fb.PlanView(plan0, lay0, hn, wl.d).row_ptr[-1].item())
         ev0 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
         if world > 1:
             dist.barrier()
@@ -280,12 +295,13 @@ def run_ours(args, rank, world, local_rank):
         ach0 = nnz0 * kept_tile_flop(wl) / (attn0 * 1e-3) / 1e12
         dense = {"tau": 0.0, "ms_per_layer": round(ms0, 4), "ms_plan": round(plan0_ms, 4),
                  "ms_attention": round(attn0, 4), "nnz": nnz0,
-                 "value": round(whole_job_value(dense_equiv_flop(wl), world, ms0), 2),
+                 "value": round(whole_job_value(dense_equiv_flop(wl), ms0), 2),
                  "unit": UNIT,
                  "roofline": {"bound": "tensor", "achieved": round(ach0, 1),
                               "peak": peaks()["bf16_sustained"], "unit": "TFLOP/s",
                               "frac": round(ach0 / peaks()["bf16_sustained"], 4)},
-                 "gpu_launches": (7 + (1 if lay.num_split_slots > 0 else 0)) * args.steps}
+                 "gpu_launches": (plan_launches(wl, 0.0) + 1
+                                  + (1 if lay0.num_split_slots > 0 else 0)) * args.steps}
         del plan0, ws0
 
     # FP8-e4m3 leg: plan (bf16) + direct online quantisation of Q, K, V + e4m3 prefill
@@ -295,17 +311,15 @@ def run_ours(args, rank, world, local_rank):
         q8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
         k8 = torch.empty(k.shape, dtype=torch.uint8, device=dev)
         v8 = torch.empty(v.shape, dtype=torch.uint8, device=dev)
-        qs = torch.empty((NB, wl.Hq), dtype=torch.float32, device=dev)
-        ks = torch.empty((NB, wl.Hkv), dtype=torch.float32, device=dev)
-        vs = torch.empty((NB, wl.Hkv), dtype=torch.float32, device=dev)
+        qs = torch.empty((NB, G * hn), dtype=torch.float32, device=dev)
+        ks = torch.empty((NB, hn), dtype=torch.float32, device=dev)
+        vs = torch.empty((NB, hn), dtype=torch.float32, device=dev)
 
         def step8(evs=None):
             if evs is not None:
                 evs[0].record(stream)
             fb.fp2_plan(prob, q, k, v, plan, ws, stream)
-            fb.fp2_quantize_fp8(prob, plan, q, 0, q8, qs, stream)
-            fb.fp2_quantize_fp8(prob, plan, k, 1, k8, ks, stream)
-            fb.fp2_quantize_fp8(prob, plan, v, 2, v8, vs, stream)
+            fb.fp2_quantize_fp8_qkv(prob, plan, q, k, v, q8, k8, v8, qs, ks, vs, stream)
             if evs is not None:
                 evs[1].record(stream)
             fb.fp2_prefill(prob, plan, q8, k8, v8, o, lse, q_scale=qs, k_scale=ks, v_scale=vs,
@@ -336,14 +350,14 @@ def run_ours(args, rank, world, local_rank):
         ach8 = nnz * kept_tile_flop(wl) / (attn8 * 1e-3) / 1e12
         fp8 = {"ms_per_layer": round(ms8, 4), "ms_plan_and_quantize": round(pre8, 4),
                "ms_attention": round(attn8, 4),
-               "value": round(whole_job_value(dense_equiv_flop(wl), world, ms8), 2),
+               "value": round(whole_job_value(dense_equiv_flop(wl), ms8), 2),
                "unit": UNIT, "dtype": "e4m3",
                "roofline": {"bound": "tensor", "achieved": round(ach8, 1),
                             "peak": round(2 * peaks()["bf16_sustained"], 1), "unit": "TFLOP/s",
                             "frac": round(ach8 / (2 * peaks()["bf16_sustained"]), 4),
                             "traffic": attn_traffic(wl.name, "fp8"),
                             "peak_kind": "e4m3 = 2 x measured bf16 sustained (nominal ratio)"},
-               "gpu_launches": (launches_per_step + 3 + 1) * args.steps}
+               "gpu_launches": (launches_per_step + 1 + 1) * args.steps}
 
     # end to end through the C ABI with host buffers (pinned), copies inside
     qh = torch.from_numpy(x["q"]).to(torch.bfloat16).pin_memory()
@@ -373,24 +387,24 @@ def run_ours(args, rank, world, local_rank):
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, dev)
     ms_step = total_ms / args.steps
     flop = dense_equiv_flop(wl)
-    value = whole_job_value(flop, world, ms_step)
+    value = whole_job_value(flop, ms_step)
     pk = peaks()
     attn_avg = statistics.mean(attn_ms)
     plan_avg = statistics.mean(plan_ms)
     executed = nnz * kept_tile_flop(wl)
     achieved = executed / (attn_avg * 1e-3) / 1e12
-    G = wl.Hq // wl.Hkv
     R = int(lay.num_rows)
     density = nnz / float(lay.nnz_cap)
-    plan_bytes = in_bytes + int(lay.num_blocks) * wl.Hkv * wl.d * (4 + 4 + 2 + 2)
+    plan_bytes = slice_bytes + int(lay.num_blocks) * hn * wl.d * (4 + 4 + 2 + 2)
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded low-rank + needles generator; no model weights)",
         "config": {"workload": wl.name, "seqlens": wl.seqlens, "Hq": wl.Hq, "Hkv": wl.Hkv,
                    "head_dim": wl.d, "block": wl.B, "tau": wl.tau, "paged": bool(wl.page_size),
-                   "parallelism": f"independent layer per GPU x{world}",
+                   "parallelism": f"kv-head split of one layer x{world}",
+                   "kv_heads_per_rank": [list(rank_slice(wl, world, r_)) for r_ in range(world)],
                    "l2": "inputs (%.2f GB) larger than L2 (126 MB), no flush" % (in_bytes / 1e9)},
         "ms_per_layer": round(ms_step, 4), "ms_plan": round(plan_avg, 4),
         "ms_attention": round(attn_avg, 4), "density": round(density, 5), "nnz": nnz,
@@ -406,7 +420,7 @@ def run_ours(args, rank, world, local_rank):
         "planning": {"achieved_gbs": round(plan_bytes / (plan_avg * 1e-3) / 1e9, 1),
                      "peak_gbs": pk["hbm_gbs"],
                      "frac": round(plan_bytes / (plan_avg * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
-        "e2e": {"value": round(whole_job_value(flop, world, e2e_ms), 2), "unit": UNIT,
+        "e2e": {"value": round(whole_job_value(flop, e2e_ms), 2), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps,
                 "how": "torch copy_ of pinned host Q/K/V into the device tensors, fp2_plan + "
                        "fp2_prefill through the C ABI, copy_ of O and LSE back, per step",
@@ -472,7 +486,7 @@ def run_reference(args, rank, world):
               f"query blocks (all kv-heads) of the {wl.seqlens[0]}-token layer, float64 NumPy")
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name, "seqlens": wl.seqlens, "Hq": wl.Hq, "Hkv": wl.Hkv,
                        "head_dim": wl.d, "block": wl.B, "tau": wl.tau},
@@ -612,9 +626,7 @@ def run_sweep(args):
         def fp8_step(ev):
             ev[0].record(stream)
             fb.fp2_plan(prob, q, k, v, plan, ws, stream)
-            fb.fp2_quantize_fp8(prob, plan, q, 0, q8, qs, stream)
-            fb.fp2_quantize_fp8(prob, plan, k, 1, k8, ks, stream)
-            fb.fp2_quantize_fp8(prob, plan, v, 2, v8, vs, stream)
+            fb.fp2_quantize_fp8_qkv(prob, plan, q, k, v, q8, k8, v8, qs, ks, vs, stream)
             ev[1].record(stream)
             fb.fp2_prefill(prob, plan, q8, k8, v8, o, lse, q_scale=qs, k_scale=ks, v_scale=vs,
                            dtype=fb.FP2_DTYPE_E4M3, stream=stream)

@@ -36,7 +36,8 @@ FP2_NO_CORRECTION = 0x1
 FP2_DEBUG_DROP_Q_LOAD = 0x100
 
 EXPORTED = ["fp2_version", "fp2_strerror", "fp2_plan_sizes", "fp2_plan", "fp2_quantize_fp8",
-            "fp2_prefill", "fp2_status_check", "fp2_plan_static", "fp2_plan_kv8"]
+            "fp2_quantize_fp8_qkv", "fp2_prefill", "fp2_status_check", "fp2_plan_static",
+            "fp2_plan_kv8"]
 
 # Size of the library-held scratch of fp2_plan_static (FP2_STATIC_WORKSPACE_BYTES).
 FP2_STATIC_WORKSPACE_BYTES = 32 << 20
@@ -64,6 +65,10 @@ class fp2_problem(ctypes.Structure):
         ("page_table_stride", ctypes.c_int32),
         ("q_seqlens", ctypes.POINTER(ctypes.c_int32)),
         ("cu_q_seqlens", ctypes.c_void_p),
+        ("kv_head_begin", ctypes.c_int32),
+        ("num_kv_heads_total", ctypes.c_int32),
+        ("prev_kbar", ctypes.c_void_p),
+        ("prev_vbar", ctypes.c_void_p),
     ]
 
 
@@ -124,6 +129,8 @@ def lib():
         L.fp2_quantize_fp8.argtypes = [ctypes.POINTER(fp2_problem), ctypes.c_void_p,
                                        ctypes.c_size_t, ctypes.c_void_p, ctypes.c_int32,
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+        L.fp2_quantize_fp8_qkv.argtypes = [ctypes.POINTER(fp2_problem), ctypes.c_void_p,
+                                           ctypes.c_size_t] + [ctypes.c_void_p] * 10
         L.fp2_prefill.argtypes = [ctypes.POINTER(fp2_problem), ctypes.c_void_p, ctypes.c_size_t,
                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -172,7 +179,8 @@ class Problem:
     def __init__(self, seqlens: Sequence[int], cu_seqlens, num_q_heads: int, num_kv_heads: int,
                  head_dim: int, block_size: int, tau: float, page_size: int = 0,
                  page_table=None, num_pages: int = 0, q_seqlens: Optional[Sequence[int]] = None,
-                 cu_q_seqlens=None):
+                 cu_q_seqlens=None, kv_head_begin: int = 0, num_kv_heads_total: int = 0,
+                 prev_kbar=None, prev_vbar=None):
         self.seqlens_np = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
         self.cu_seqlens = cu_seqlens
         self.page_table = page_table
@@ -196,6 +204,13 @@ class Problem:
             self.q_seqlens_np = np.ascontiguousarray(np.asarray(q_seqlens, dtype=np.int32))
             self.c.q_seqlens = self.q_seqlens_np.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
             self.c.cu_q_seqlens = _ptr(cu_q_seqlens)
+        # a slice of the layer's kv-heads, run in place in full-layer tensors
+        self.c.kv_head_begin = int(kv_head_begin)
+        self.c.num_kv_heads_total = int(num_kv_heads_total)
+        # chunked prefill: block means already held for blocks before the chunk
+        self.prev = (prev_kbar, prev_vbar)
+        self.c.prev_kbar = _ptr(prev_kbar)
+        self.c.prev_vbar = _ptr(prev_vbar)
 
     @property
     def ref(self):
@@ -239,6 +254,14 @@ def fp2_quantize_fp8(problem: Problem, plan, x, which: int, x_e4m3, scales, stre
            "fp2_quantize_fp8")
 
 
+def fp2_quantize_fp8_qkv(problem: Problem, plan, q, k, v, q8, k8, v8, qs, ks, vs,
+                         stream=None) -> None:
+    """fp2_quantize_fp8 of q, k and v in one launch."""
+    _check(lib().fp2_quantize_fp8_qkv(problem.ref, _ptr(plan), plan.numel(), _ptr(q), _ptr(k),
+                                      _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(qs), _ptr(ks),
+                                      _ptr(vs), _stream_ptr(stream)), "fp2_quantize_fp8_qkv")
+
+
 def fp2_prefill(problem: Problem, plan, q, k, v, o, lse, q_scale=None, k_scale=None,
                 v_scale=None, dtype: int = FP2_DTYPE_BF16, flags: int = 0, stream=None) -> None:
     _check(lib().fp2_prefill(problem.ref, _ptr(plan), plan.numel(), _ptr(q), _ptr(k), _ptr(v),
@@ -280,6 +303,17 @@ class PlanView:
         self.kbar_bf16 = view(L.off_kbar_bf16, n_mean, torch.bfloat16, mean_shape)
         self.vbar_bf16 = view(L.off_vbar_bf16, n_mean, torch.bfloat16, mean_shape)
         self.status = view(L.off_status, 1, torch.int32, (1,))
+
+
+def kv_head_slice(num_kv_heads: int, world: int, rank: int) -> tuple:
+    """(first kv-head, kv-heads) of rank's share of a layer split over world
+    ranks by kv-head: contiguous, as equal as the counts allow, earlier ranks
+    taking the remainder."""
+    if not 1 <= world <= num_kv_heads or not 0 <= rank < world:
+        raise ValueError(f"cannot split {num_kv_heads} kv-heads over {world} ranks")
+    base, extra = divmod(num_kv_heads, world)
+    begin = rank * base + min(rank, extra)
+    return begin, base + (1 if rank < extra else 0)
 
 
 def allocate(problem: Problem, device="cuda"):

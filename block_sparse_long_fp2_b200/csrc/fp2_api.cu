@@ -4,6 +4,7 @@
 // device memory or synchronises, except fp2_status_check (which
 // synchronises the stream and reads the 4-byte status word).
 #include <algorithm>
+#include <type_traits>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -43,6 +44,10 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     if (p->page_size != 0 && p->page_size != 64) return FP2_ERR_UNSUPPORTED;
     const bool chunked = p->q_seqlens != nullptr;
     if (chunked != (p->cu_q_seqlens != nullptr)) return FP2_ERR_INVALID_ARG;
+    if ((p->prev_kbar != nullptr) != (p->prev_vbar != nullptr)) return FP2_ERR_INVALID_ARG;
+    if (p->prev_kbar && (!chunked || (reinterpret_cast<uintptr_t>(p->prev_kbar) |
+                                      reinterpret_cast<uintptr_t>(p->prev_vbar)) % 16 != 0))
+        return FP2_ERR_INVALID_ARG;
     int64_t Tq = 0;
     if (chunked)
         for (int s = 0; s < p->num_seqs; ++s) {
@@ -50,10 +55,19 @@ int compute_layout(const fp2_problem* p, Layout* out) {
             Tq += p->q_seqlens[s];
         }
 
+    // a slice of a layer's heads, in place
+    const int hkv_total = p->num_kv_heads_total ? p->num_kv_heads_total : p->num_kv_heads;
+    if (p->kv_head_begin < 0 || p->num_kv_heads_total < 0 ||
+        (int64_t)p->kv_head_begin + p->num_kv_heads > hkv_total)
+        return FP2_ERR_INVALID_ARG;
+
     Dims d{};
     d.n_seqs = p->num_seqs;
     d.Hq = p->num_q_heads;
     d.Hkv = p->num_kv_heads;
+    d.Hkv_str = hkv_total;
+    d.Hq_str = G * hkv_total;
+    d.head0 = p->kv_head_begin;
     d.G = G;
     d.d = p->head_dim;
     d.B = p->block_size;
@@ -314,6 +328,15 @@ namespace {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// The first element of a head slice: `heads` heads of `elt`-byte elements
+// past the tensor's start (the tensors keep all heads of each token).
+template <typename T>
+T* head_offset(T* p, int64_t heads, int d, int elt) {
+    if (!p) return p;
+    using B = typename std::conditional<std::is_const<T>::value, const char, char>::type;
+    return reinterpret_cast<T*>(reinterpret_cast<B*>(p) + heads * d * elt);
+}
+
 }  // namespace
 
 extern "C" {
@@ -352,8 +375,10 @@ int fp2_plan(const fp2_problem* problem, const void* q, const void* k, const voi
     if (!aligned(plan, 256) || !aligned(workspace, 256)) return FP2_ERR_INVALID_ARG;
     if (plan_bytes < L.pub.plan_bytes || workspace_bytes < L.pub.workspace_bytes)
         return FP2_ERR_CAPACITY;
-    return launch_plan(L, problem, q, k, v, plan_ptrs(L, plan), ws_ptrs(L, workspace),
-                       static_cast<cudaStream_t>(stream));
+    const Dims& D = L.dims;
+    return launch_plan(L, problem, head_offset(q, (int64_t)D.G * D.head0, D.d, 2),
+                       head_offset(k, D.head0, D.d, 2), head_offset(v, D.head0, D.d, 2),
+                       plan_ptrs(L, plan), ws_ptrs(L, workspace), static_cast<cudaStream_t>(stream));
 }
 
 int fp2_plan_kv8(const fp2_problem* problem, const void* q, const void* k_e4m3, const void* v_e4m3,
@@ -370,8 +395,11 @@ int fp2_plan_kv8(const fp2_problem* problem, const void* q, const void* k_e4m3, 
         return FP2_ERR_INVALID_ARG;
     if (plan_bytes < L.pub.plan_bytes || workspace_bytes < L.pub.workspace_bytes)
         return FP2_ERR_CAPACITY;
-    return launch_plan(L, problem, q, k_e4m3, v_e4m3, plan_ptrs(L, plan), ws_ptrs(L, workspace),
-                       static_cast<cudaStream_t>(stream), k_scale, v_scale);
+    const Dims& D = L.dims;
+    return launch_plan(L, problem, head_offset(q, (int64_t)D.G * D.head0, D.d, 2),
+                       head_offset(k_e4m3, D.head0, D.d, 1), head_offset(v_e4m3, D.head0, D.d, 1),
+                       plan_ptrs(L, plan), ws_ptrs(L, workspace), static_cast<cudaStream_t>(stream),
+                       k_scale, v_scale);
 }
 
 int fp2_quantize_fp8(const fp2_problem* problem, const void* plan, size_t plan_bytes, const void* x,
@@ -383,9 +411,41 @@ int fp2_quantize_fp8(const fp2_problem* problem, const void* plan, size_t plan_b
     if (!aligned(x, 16) || !aligned(x_e4m3, 16) || !aligned(scales, 4) || !aligned(plan, 256))
         return FP2_ERR_INVALID_ARG;
     if (plan_bytes < L.pub.plan_bytes) return FP2_ERR_CAPACITY;
-    if (L.chunked && which == 0) return FP2_ERR_UNSUPPORTED;   // e4m3 chunks: not built
-    return launch_quantize(L, problem, plan_ptrs(L, const_cast<void*>(plan)), x, which, x_e4m3,
-                           scales, static_cast<cudaStream_t>(stream));
+    const Dims& D = L.dims;
+    const int64_t h0 = which == 0 ? (int64_t)D.G * D.head0 : D.head0;
+    const void* xs[1] = {head_offset(x, h0, D.d, 2)};
+    void* x8s[1] = {head_offset(x_e4m3, h0, D.d, 1)};
+    float* ss[1] = {scales};
+    return launch_quantize(L, problem, plan_ptrs(L, const_cast<void*>(plan)), xs, x8s, ss, which, 1,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int fp2_quantize_fp8_qkv(const fp2_problem* problem, const void* plan, size_t plan_bytes,
+                         const void* q, const void* k, const void* v, void* q_e4m3, void* k_e4m3,
+                         void* v_e4m3, float* q_scales, float* k_scales, float* v_scales,
+                         void* stream) {
+    Layout L;
+    int rc = compute_layout(problem, &L);
+    if (rc != FP2_OK) return rc;
+    const void* xs[3] = {q, k, v};
+    void* x8s[3] = {q_e4m3, k_e4m3, v_e4m3};
+    float* ss[3] = {q_scales, k_scales, v_scales};
+    if (!plan || !aligned(plan, 256)) return FP2_ERR_INVALID_ARG;
+    for (int w = 0; w < 3; ++w)
+        if (!xs[w] || !x8s[w] || !ss[w] || !aligned(xs[w], 16) || !aligned(x8s[w], 16) ||
+            !aligned(ss[w], 4))
+            return FP2_ERR_INVALID_ARG;
+    if (plan_bytes < L.pub.plan_bytes) return FP2_ERR_CAPACITY;
+    const Dims& D = L.dims;
+    const int64_t hq0 = (int64_t)D.G * D.head0;
+    xs[0] = head_offset(q, hq0, D.d, 2);
+    xs[1] = head_offset(k, D.head0, D.d, 2);
+    xs[2] = head_offset(v, D.head0, D.d, 2);
+    x8s[0] = head_offset(q_e4m3, hq0, D.d, 1);
+    x8s[1] = head_offset(k_e4m3, D.head0, D.d, 1);
+    x8s[2] = head_offset(v_e4m3, D.head0, D.d, 1);
+    return launch_quantize(L, problem, plan_ptrs(L, const_cast<void*>(plan)), xs, x8s, ss, 0, 3,
+                           static_cast<cudaStream_t>(stream));
 }
 
 int fp2_prefill(const fp2_problem* problem, const void* plan, size_t plan_bytes, const void* q,
@@ -406,14 +466,20 @@ int fp2_prefill(const fp2_problem* problem, const void* plan, size_t plan_bytes,
         if (!q_scale || !k_scale || !v_scale) return FP2_ERR_INVALID_ARG;
         if (!aligned(q_scale, 4) || !aligned(k_scale, 4) || !aligned(v_scale, 4))
             return FP2_ERR_INVALID_ARG;
-        if (L.dims.d != 128 || L.chunked) return FP2_ERR_UNSUPPORTED;
+        if (L.dims.d != 128) return FP2_ERR_UNSUPPORTED;
     } else {
         return FP2_ERR_INVALID_ARG;
     }
     const uint32_t known = FP2_NO_CORRECTION | FP2_DEBUG_DROP_Q_LOAD;
     if (flags & ~known) return FP2_ERR_INVALID_ARG;
-    return launch_prefill(L, problem, plan_ptrs(L, const_cast<void*>(plan)), q, k, v, q_scale,
-                          k_scale, v_scale, dtype, o, lse, flags,
+    const Dims& D = L.dims;
+    const int elt = dtype == FP2_DTYPE_E4M3 ? 1 : 2;
+    const int64_t hq0 = (int64_t)D.G * D.head0;
+    // lse is [G * num_kv_heads_total, Tq]: the slice's rows are contiguous
+    return launch_prefill(L, problem, plan_ptrs(L, const_cast<void*>(plan)),
+                          head_offset(q, hq0, D.d, elt), head_offset(k, D.head0, D.d, elt),
+                          head_offset(v, D.head0, D.d, elt), q_scale, k_scale, v_scale, dtype,
+                          head_offset(o, hq0, D.d, 2), lse + hq0 * L.Tq, flags,
                           static_cast<cudaStream_t>(stream));
 }
 

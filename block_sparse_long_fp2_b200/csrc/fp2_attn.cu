@@ -638,9 +638,22 @@ __device__ __forceinline__ uint32_t chunk_bits(int kind, int tok, const TileWalk
 //   e4m3: P' = P * pfac packed four per column, columns [t_p, t_p+8), pfac
 //   entering through the shift (as log2 pfac).
 // The fp32 row sum accumulates the P written (P' for e4m3).
+// Exponentials computed on the FMA pipe (exp2_fma2) instead of MUFU ex2: the
+// pairs p of a 32-column chunk with p % 8 < kEmuPairs / 2, i.e. kEmuPairs of
+// the 16 pairs (both units then share the softmax's exponentials).
+#ifndef FP2_EXP2_FMA_PAIRS_BF16
+#define FP2_EXP2_FMA_PAIRS_BF16 0
+#endif
+#ifndef FP2_EXP2_FMA_PAIRS_E4M3
+#define FP2_EXP2_FMA_PAIRS_E4M3 0
+#endif
+template <bool F8>
+constexpr int emu_pairs() { return F8 ? FP2_EXP2_FMA_PAIRS_E4M3 : FP2_EXP2_FMA_PAIRS_BF16; }
+
 template <bool MASKED, bool F8>
 __device__ __forceinline__ void p32(const uint32_t (&r)[32], uint32_t vb, uint32_t t_p,
                                     uint64_t scale2, uint64_t shift2, uint64_t& sum2) {
+    constexpr int kEmu = emu_pairs<F8>();
     float p[32];
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
@@ -649,10 +662,15 @@ __device__ __forceinline__ void p32(const uint32_t (&r)[32], uint32_t vb, uint32
             s0 = ((vb >> e) & 1u) ? s0 : -INFINITY;
             s1 = ((vb >> (e + 1)) & 1u) ? s1 : -INFINITY;
         }
-        float x0, x1;
-        f2_unpack(f2_fma(f2_pack(s0, s1), scale2, shift2), x0, x1);
-        p[e] = ex2_approx(x0);
-        p[e + 1] = ex2_approx(x1);
+        const uint64_t x2 = f2_fma(f2_pack(s0, s1), scale2, shift2);
+        if ((e / 2) % 8 < kEmu / 2) {
+            f2_unpack(exp2_fma2(x2), p[e], p[e + 1]);
+        } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p[e] = ex2_approx(x0);
+            p[e + 1] = ex2_approx(x1);
+        }
         sum2 = f2_add(sum2, f2_pack(p[e], p[e + 1]));
     }
     if (F8) {
@@ -879,7 +897,7 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
         const float inv_l = 1.0f / (st.l * k_row);
         const bool split = split_slot >= 0;
         const int64_t srow = (int64_t)split_slot * (D.G * BLK) + pr;
-        const int64_t orow = (qtok + pos) * D.Hq + h;
+        const int64_t orow = (qtok + pos) * D.Hq_str + h;
         char* dst = split ? reinterpret_cast<char*>(P.split_o + srow * HD)
                           : reinterpret_cast<char*>(P.o + orow * HD);
 #pragma unroll
@@ -1051,7 +1069,7 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(const __grid_consta
             }
         }
         const float inv = 1.0f / wsum;
-        uint16_t* orow = P.o + ((qtok + pos) * D.Hq + h) * HD + lane * E;
+        uint16_t* orow = P.o + ((qtok + pos) * D.Hq_str + h) * HD + lane * E;
         if constexpr (E == 4) {
             uint2 v;
             v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
@@ -1101,20 +1119,20 @@ int launch_attn_t(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, con
     CUtensorMap tq, tk, tv, tkb, tvb, tkb_lo;
     {
         cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)D.Hq, (cuuint64_t)L.Tq};
-        cuuint64_t str[2] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hq * HD * eb};
+        cuuint64_t str[2] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hq_str * HD * eb};
         cuuint32_t box[3] = {ae, 1, (cuuint32_t)BLK};
         if (!make_tensor_map(&tq, q, 3, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
     }
     if (D.page_size == 0) {
         cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)D.Hkv, (cuuint64_t)D.T};
-        cuuint64_t str[2] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hkv * HD * eb};
+        cuuint64_t str[2] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hkv_str * HD * eb};
         cuuint32_t box[3] = {ae, 1, (cuuint32_t)BLK};
         if (!make_tensor_map(&tk, k, 3, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
         if (!make_tensor_map(&tv, v, 3, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
     } else {
         cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)D.Hkv, 64, (cuuint64_t)D.num_pages};
-        cuuint64_t str[3] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hkv * HD * eb,
-                             (cuuint64_t)64 * D.Hkv * HD * eb};
+        cuuint64_t str[3] = {(cuuint64_t)HD * eb, (cuuint64_t)D.Hkv_str * HD * eb,
+                             (cuuint64_t)64 * D.Hkv_str * HD * eb};
         cuuint32_t box[4] = {ae, 1, 64, 1};
         if (!make_tensor_map(&tk, k, 4, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
         if (!make_tensor_map(&tv, v, 4, dims, str, box, F8 ? kMapU8 : kMapBF16)) return FP2_ERR_CUDA;
@@ -1166,9 +1184,7 @@ int launch_attn_t(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, con
     const int64_t grid = S.n_items < sms ? S.n_items : sms;
     P.n_slots = (S.n_items + grid - 1) / grid * grid;
     P.zigzag = P.n_slots / grid <= kZigZagMaxPasses;
-    auto kernel = k_attn<HD, BLK, F8, false>;
-    if constexpr (!F8)
-        if (L.chunked) kernel = k_attn<HD, BLK, false, true>;
+    auto kernel = L.chunked ? k_attn<HD, BLK, F8, true> : k_attn<HD, BLK, F8, false>;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
         return FP2_ERR_CUDA;

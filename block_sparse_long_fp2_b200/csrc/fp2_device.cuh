@@ -392,6 +392,40 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// 2^x of two floats on the FMA pipe (the MUFU ex2 unit is the softmax's
+// scarcest resource): x = j + f with j = round(x) (through the 1.5 * 2^23
+// shift, exact for |x| < 2^22) and f in [-1/2, 1/2]; 2^f by a cubic whose
+// coefficients were fitted by the Remez exchange for minimax relative error
+// on [-1/2, 1/2] (7.5e-5, below bf16's 2^-9 and e4m3's 2^-4 rounding of P);
+// 2^j enters by adding j to the exponent field.  Inputs are clamped to
+// >= -125, so -inf (a masked logit) gives about 2^-125 instead of 0; inputs
+// above 64 do not occur (the softmax keeps P <= 2^64).
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x2) {
+    constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
+    float a, b;
+    f2_unpack(x2, a, b);
+    const uint64_t xc = f2_pack(fmaxf(a, -125.0f), fmaxf(b, -125.0f));
+    const uint64_t t = f2_add(xc, f2_pack(kShift, kShift));
+    const uint64_t f = f2_sub(xc, f2_sub(t, f2_pack(kShift, kShift)));
+    uint64_t p = f2_fma(f, f2_pack(0.0551716685295105f, 0.0551716685295105f),
+                        f2_pack(0.2426111251115799f, 0.2426111251115799f));
+    p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+    p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+    float p0, p1, t0, t1;
+    f2_unpack(p, p0, p1);
+    f2_unpack(t, t0, t1);
+    // the low bits of t hold j (two's complement); j << 23 moves it into the exponent
+    const uint32_t y0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
+    const uint32_t y1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
+    return f2_pack(__uint_as_float(y0), __uint_as_float(y1));
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));

@@ -51,6 +51,8 @@ __host__ __device__ inline int row_splits(int64_t i, int B, int c) {
 struct Dims {
     int n_seqs;
     int Hq, Hkv, G, d, B;
+    int Hq_str, Hkv_str;  // heads per token of the q / o and k / v tensors (>= Hq, Hkv for a slice)
+    int head0;            // first kv-head of the slice in those tensors
     int page_size, num_pages, pt_stride;
     int mask_words;       // 32-bit words per kept-mask row
     int max_nb;           // largest nb_s
@@ -154,8 +156,10 @@ WsPtrs ws_ptrs(const Layout& L, void* ws);
 int launch_plan(const Layout& L, const fp2_problem* p, const void* q, const void* k,
                 const void* v, const PlanPtrs& pp, const WsPtrs& ws, cudaStream_t st,
                 const float* k_scale = nullptr, const float* v_scale = nullptr);
-int launch_quantize(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, const void* x,
-                    int which, void* x8, float* scales, cudaStream_t st);
+// Quantises count tensors (which = first .. first + count - 1: 0 q, 1 k, 2 v)
+// in one launch.
+int launch_quantize(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, const void* const* x,
+                    void* const* x8, float* const* scales, int first, int count, cudaStream_t st);
 int launch_prefill(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, const void* q,
                    const void* k, const void* v, const float* qs, const float* ks,
                    const float* vs, int dtype, void* o, float* lse, uint32_t flags,

@@ -331,7 +331,8 @@ __global__ void __launch_bounds__(kPoolThreads)
 k_pool(Dims D, SeqMap M, int64_t Tq, const int32_t* __restrict__ cu_seqlens,
        const int32_t* __restrict__ page_table, const uint16_t* __restrict__ q,
        const void* __restrict__ k, const void* __restrict__ v, const float* __restrict__ k_scale,
-       const float* __restrict__ v_scale, PlanPtrs P, WsPtrs W) {
+       const float* __restrict__ v_scale, const float* __restrict__ prev_kbar,
+       const float* __restrict__ prev_vbar, PlanPtrs P, WsPtrs W) {
     // the next kernel (k_meta) may start while the pool runs: it reads none
     // of the pool's outputs and waits for the pool before it completes
     if (BYVAL) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -371,15 +372,26 @@ k_pool(Dims D, SeqMap M, int64_t Tq, const int32_t* __restrict__ cu_seqlens,
     double acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+    // chunked prefill with the caller's means of the blocks wholly before the
+    // chunk: those K / V means are copied, not pooled from K and V again
+    const float* prev = which == 1 ? prev_kbar : prev_vbar;
+    const bool reuse = CHUNK && which != 0 && prev && (loc.i + 1) * D.B <= loc.q_off;
 
     if (!active) {
         // no column: only takes part in the CTA's barrier below
+    } else if (reuse) {
+        const float* src = prev + (b * D.Hkv + head) * d + e0;
+        const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+        const float4 c = __ldg(reinterpret_cast<const float4*>(src + 4));
+        const float f[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = (double)f[e];   // the means themselves
     } else if (KV8 && which != 0) {
         // e4m3 K / V, contiguous [T, Hkv, d] or paged [P, 64, Hkv, d]
         const uint8_t* base = static_cast<const uint8_t*>(which == 1 ? k : v);
-        const int64_t stride = (int64_t)D.Hkv * d / 8;   // uint2 per token
+        const int64_t stride = (int64_t)D.Hkv_str * d / 8;   // uint2 per token
         if (D.page_size == 0) {
-            const uint2* p = reinterpret_cast<const uint2*>(base + ((tok0 + t_begin) * D.Hkv + head) * d + e0);
+            const uint2* p = reinterpret_cast<const uint2*>(base + ((tok0 + t_begin) * D.Hkv_str + head) * d + e0);
             int t = t_begin;
             for (; t + kPoolUnroll <= t_end; t += kPoolUnroll) {
                 uint2 x[kPoolUnroll];
@@ -398,7 +410,7 @@ k_pool(Dims D, SeqMap M, int64_t Tq, const int32_t* __restrict__ cu_seqlens,
                 const int id = page_table[(int64_t)s * D.pt_stride + t / 64];
                 const int n = min(64, t_end - t);
                 if (id < 0 || id >= D.num_pages) continue;   // recorded by k_meta; reads as zeros
-                const uint2* p = reinterpret_cast<const uint2*>(base + ((int64_t)id * 64 * D.Hkv + head) * d + e0);
+                const uint2* p = reinterpret_cast<const uint2*>(base + ((int64_t)id * 64 * D.Hkv_str + head) * d + e0);
                 for (int u = 0; u < n; ++u) accum8_e4m3(acc, ld_stream8(p + u * stride));
             }
         }
@@ -407,7 +419,7 @@ k_pool(Dims D, SeqMap M, int64_t Tq, const int32_t* __restrict__ cu_seqlens,
         for (int e = 0; e < 8; ++e) acc[e] *= sc;
     } else if (which == 0 || D.page_size == 0) {
         const uint16_t* base = which == 0 ? q : static_cast<const uint16_t*>(which == 1 ? k : v);
-        const int H = which == 0 ? D.Hq : D.Hkv;
+        const int H = which == 0 ? D.Hq_str : D.Hkv_str;   // heads per token of the tensor
         const uint4* p = reinterpret_cast<const uint4*>(base + ((tok0 + t_begin) * H + head) * d + e0);
         const int64_t stride = (int64_t)H * d / 8;   // uint4 per token
         int t = t_begin;
@@ -426,12 +438,12 @@ k_pool(Dims D, SeqMap M, int64_t Tq, const int32_t* __restrict__ cu_seqlens,
     } else {
         // paged pool [num_pages, 64, Hkv, d]; blocks start on page boundaries (B % 64 == 0)
         const uint16_t* pool = static_cast<const uint16_t*>(which == 1 ? k : v);
-        const int64_t stride = (int64_t)D.Hkv * d / 8;
+        const int64_t stride = (int64_t)D.Hkv_str * d / 8;
         for (int t = t_begin; t < t_end; t += 64) {
             const int id = page_table[(int64_t)s * D.pt_stride + t / 64];
             const int n = min(64, t_end - t);
             if (id < 0 || id >= D.num_pages) continue;   // recorded by k_meta; reads as zeros
-            const uint4* p = reinterpret_cast<const uint4*>(pool + ((int64_t)id * 64 * D.Hkv + head) * d + e0);
+            const uint4* p = reinterpret_cast<const uint4*>(pool + ((int64_t)id * 64 * D.Hkv_str + head) * d + e0);
             int u0 = 0;
             for (; u0 + kPoolUnroll <= n; u0 += kPoolUnroll) {
                 uint4 x[kPoolUnroll];
@@ -445,7 +457,7 @@ k_pool(Dims D, SeqMap M, int64_t Tq, const int32_t* __restrict__ cu_seqlens,
     }
 
     // (a query block below a chunk has no query: its mean is left zero)
-    const double inv_n = t_end > t_begin ? 1.0 / (double)(t_end - t_begin) : 0.0;
+    const double inv_n = reuse ? 1.0 : t_end > t_begin ? 1.0 / (double)(t_end - t_begin) : 0.0;
     double m[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) m[e] = acc[e] * inv_n;
@@ -1272,7 +1284,7 @@ void launch_pool(const Layout& L, const fp2_problem* p, const SeqMap& M, const v
     dim3 grid((unsigned)D.NB, (vecs + kPoolThreads - 1) / kPoolThreads);
     k_pool<KV8, CHUNK, BYVAL, NORMS><<<grid, kPoolThreads, 0, st>>>(
         D, M, L.Tq, p->cu_seqlens, p->page_table, static_cast<const uint16_t*>(q), k, v, k_scale,
-        v_scale, P, W);
+        v_scale, CHUNK ? p->prev_kbar : nullptr, CHUNK ? p->prev_vbar : nullptr, P, W);
 }
 
 template <bool KV8, bool CHUNK>

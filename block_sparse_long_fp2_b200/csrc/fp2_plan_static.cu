@@ -55,6 +55,10 @@ extern "C" int fp2_plan_static(const fp2_problem* problem, const void* q, const 
     if (!ws) return FP2_ERR_CUDA;
     // No part of the workspace has to start at zero: every kernel writes the
     // scratch entries it reads later in the same call.
-    return launch_plan(L, problem, q, k, v, plan_ptrs(L, plan), ws_ptrs(L, ws),
+    const Dims& D = L.dims;
+    const char* qb = static_cast<const char*>(q) + (int64_t)D.G * D.head0 * D.d * 2;
+    const char* kb = static_cast<const char*>(k) + (int64_t)D.head0 * D.d * 2;
+    const char* vb = static_cast<const char*>(v) + (int64_t)D.head0 * D.d * 2;
+    return launch_plan(L, problem, qb, kb, vb, plan_ptrs(L, plan), ws_ptrs(L, ws),
                        static_cast<cudaStream_t>(stream));
 }

@@ -3,7 +3,8 @@
 // per (block, head) finds the absmax of the block's bf16 values, sets
 // scale = absmax / 448 (1 for an all-zero block) and writes
 // e4m3 = round-to-nearest-even-saturating(x / scale), with scale and quotient
-// in fp32.  Memory bound: the block is read twice (the second pass mostly
+// in fp32.  For a chunked problem a query block covers the chunk's positions
+// in it (a block below the chunk gets scale 1 and no codes).  Memory bound: the block is read twice (the second pass mostly
 // from L2) and written once at a quarter of the size.
 #include "fp2_device.cuh"
 
@@ -26,30 +27,58 @@ struct Addr {
     const int32_t* cu_seqlens;
     const int32_t* page_table;
     bool paged;
-    int H;
+    int H;      // heads per token of the tensor (all of a layer's heads for a slice)
+    int pos0;   // position of the sequence's first row (a chunk's first query)
     __device__ __forceinline__ int64_t operator()(int s, int t, int h, int e) const {
-        if (!paged) return ((int64_t)(cu_seqlens[s] + t) * H + h) * D->d + e;
+        if (!paged) return ((int64_t)(cu_seqlens[s] + t - pos0) * H + h) * D->d + e;
         const int id = page_table[(int64_t)s * D->pt_stride + t / 64];
         if (id < 0 || id >= D->num_pages) return -1;
         return (((int64_t)id * 64 + t % 64) * H + h) * D->d + e;
     }
 };
 
+// The tensors of one launch: q, k and v with their codes and scales (a
+// single-tensor launch fills only `which`).
+struct QuantArgs {
+    const uint16_t* x[3];
+    uint8_t* x8[3];
+    float* scales[3];
+};
+
+// One CTA per (block, head): blockIdx.y runs over the heads of the tensors
+// the launch quantises, q's Hq heads first, then k's and v's Hkv heads.
 __global__ void __launch_bounds__(kQuantThreads)
 k_quant(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ page_table,
-        PlanPtrs P, const uint16_t* __restrict__ x, uint8_t* __restrict__ x8,
-        float* __restrict__ scales, int which) {
+        PlanPtrs P, QuantArgs A, int first) {
     if (!*P.meta_valid) return;
     const int64_t b = blockIdx.x;
-    const int h = blockIdx.y;
+    int which = first, h = blockIdx.y;
+    while (h >= (which == 0 ? D.Hq : D.Hkv)) {
+        h -= which == 0 ? D.Hq : D.Hkv;
+        ++which;
+    }
+    const uint16_t* __restrict__ x = A.x[which];
+    uint8_t* __restrict__ x8 = A.x8[which];
+    float* __restrict__ scales = A.scales[which];
     const int H = which == 0 ? D.Hq : D.Hkv;
     const int s = P.block_seq[b];
     const int i = (int)(b - P.cu_blocks[s]);
     const int L = cu_seqlens[s + 1] - cu_seqlens[s];
-    const int t0 = i * D.B, t1 = min(t0 + D.B, L);
-    Addr addr{&D, cu_seqlens, page_table, which != 0 && D.page_size != 0, H};
+    int t0 = i * D.B;
+    const int t1 = min(t0 + D.B, L);
+    // q of a chunked problem holds positions q_off .. L - 1 of each sequence:
+    // a query block's scale covers its chunk positions (none below the chunk)
+    const int32_t* base = cu_seqlens;
+    int pos0 = 0;
+    if (which == 0 && P.cu_q) {
+        t0 = max(t0, P.q_off[s]);
+        base = P.cu_q;
+        pos0 = P.q_off[s];
+    }
+    Addr addr{&D, base, page_table, which != 0 && D.page_size != 0,
+              which == 0 ? D.Hq_str : D.Hkv_str, pos0};
     const int vpt = D.d / 8;                       // 16-byte vectors per token
-    const int nvec = (t1 - t0) * vpt;
+    const int nvec = t1 > t0 ? (t1 - t0) * vpt : 0;
 
     float amax = 0.f;
     for (int idx = threadIdx.x; idx < nvec; idx += kQuantThreads) {
@@ -95,13 +124,21 @@ k_quant(Dims D, const int32_t* __restrict__ cu_seqlens, const int32_t* __restric
 
 }  // namespace
 
-int launch_quantize(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, const void* x,
-                    int which, void* x8, float* scales, cudaStream_t st) {
+int launch_quantize(const Layout& L, const fp2_problem* p, const PlanPtrs& pp, const void* const* x,
+                    void* const* x8, float* const* scales, int first, int count, cudaStream_t st) {
     const Dims& D = L.dims;
-    dim3 grid((unsigned)D.NB, which == 0 ? D.Hq : D.Hkv);
-    k_quant<<<grid, kQuantThreads, 0, st>>>(D, p->cu_seqlens, p->page_table, pp,
-                                            static_cast<const uint16_t*>(x),
-                                            static_cast<uint8_t*>(x8), scales, which);
+    PlanPtrs P = pp;
+    P.cu_q = L.chunked ? p->cu_q_seqlens : nullptr;
+    QuantArgs A{};
+    int heads = 0;
+    for (int w = first; w < first + count; ++w) {
+        A.x[w] = static_cast<const uint16_t*>(x[w - first]);
+        A.x8[w] = static_cast<uint8_t*>(x8[w - first]);
+        A.scales[w] = scales[w - first];
+        heads += w == 0 ? D.Hq : D.Hkv;
+    }
+    dim3 grid((unsigned)D.NB, (unsigned)heads);
+    k_quant<<<grid, kQuantThreads, 0, st>>>(D, p->cu_seqlens, p->page_table, P, A, first);
     return cudaGetLastError() == cudaSuccess ? FP2_OK : FP2_ERR_CUDA;
 }
 

@@ -113,9 +113,37 @@ extern "C" {
  *                tokens.  Blocks stay on the absolute position grid: query
  *                block i holds the chunk's queries in [iB, (i+1)B) and its mean
  *                covers only them; rows of query blocks below the chunk keep no
- *                block.  BF16 only: fp2_quantize_fp8 of q, the e4m3
- *                fp2_prefill and fp2_plan_kv8 return FP2_ERR_UNSUPPORTED for a
- *                chunked problem.
+ *                block.  The e4m3 path takes a chunk too: fp2_quantize_fp8
+ *                of q gives a query block the scale of its chunk positions.
+ *                fp2_plan_kv8 returns FP2_ERR_UNSUPPORTED for a chunked
+ *                problem.
+ *   kv_head_begin, num_kv_heads_total   a slice of a layer's heads, run in
+ *                place (the kv-head split of one layer across GPUs: each
+ *                kv-head and its G query heads are planned and attended on
+ *                their own).  num_kv_heads_total = 0 (or num_kv_heads, with
+ *                kv_head_begin = 0): the tensors hold exactly the problem's
+ *                heads.  Otherwise q, o are [T(q), G * num_kv_heads_total, d],
+ *                k, v are [T, num_kv_heads_total, d] (or the paged pool
+ *                [num_pages, 64, num_kv_heads_total, d]) and lse is
+ *                [G * num_kv_heads_total, T(q)]; the call reads and writes only
+ *                kv-heads kv_head_begin .. kv_head_begin + num_kv_heads - 1 and
+ *                their query heads G * kv_head_begin .. (every other head of o,
+ *                lse and of fp2_quantize_fp8's output is left untouched), with
+ *                0 <= kv_head_begin and kv_head_begin + num_kv_heads <=
+ *                num_kv_heads_total.  The plan and every per-(block, head)
+ *                scale array (fp2_quantize_fp8, fp2_prefill, fp2_plan_kv8)
+ *                cover the slice's heads only, numbered from 0.
+ *   prev_kbar, prev_vbar   chunked prefill only (NULL otherwise, and both or
+ *                neither): DEVICE float [num_blocks, num_kv_heads, d], 16-byte
+ *                aligned, the K and V block means the caller already holds for
+ *                the blocks that lie wholly before each sequence's chunk
+ *                (blocks j with (j + 1) * block_size <= seqlens[s] - q_seqlens[s]),
+ *                numbered like the plan's kbar / vbar of this problem (e.g. an
+ *                earlier chunk's plan of a single sequence).  fp2_plan copies
+ *                those blocks' means instead of reading their K and V again,
+ *                so planning a chunk reads only the chunk's tokens; other
+ *                entries are not read.  The float64 re-scoring of such blocks
+ *                then uses these fp32 means.
  */
 typedef struct fp2_problem {
     int32_t num_seqs;
@@ -132,6 +160,10 @@ typedef struct fp2_problem {
     int32_t page_table_stride;
     const int32_t* q_seqlens;
     const int32_t* cu_q_seqlens;
+    int32_t kv_head_begin;
+    int32_t num_kv_heads_total;
+    const float* prev_kbar;
+    const float* prev_vbar;
 } fp2_problem;
 
 /*
@@ -248,6 +280,17 @@ int fp2_plan_kv8(const fp2_problem* problem, const void* q, const void* k_e4m3,
  */
 int fp2_quantize_fp8(const fp2_problem* problem, const void* plan, size_t plan_bytes,
                      const void* x, int32_t which, void* x_e4m3, float* scales, void* stream);
+
+/*
+ * fp2_quantize_fp8 of q, k and v in one launch (which = 0, 1, 2 in turn):
+ * the same codes and scales as three fp2_quantize_fp8 calls, with one launch
+ * instead of three (the launches dominate on short layers).  Arguments as for
+ * fp2_quantize_fp8, one tensor, code tensor and scale array per input.
+ */
+int fp2_quantize_fp8_qkv(const fp2_problem* problem, const void* plan, size_t plan_bytes,
+                         const void* q, const void* k, const void* v, void* q_e4m3,
+                         void* k_e4m3, void* v_e4m3, float* q_scales, float* k_scales,
+                         float* v_scales, void* stream);
 
 /*
  * Stage 2, sparse attention with mean correction (Figure 3 / Figure 4).

@@ -210,7 +210,7 @@ REL_L2_FP8 = 5e-2
 
 
 def fp8_prefill(wl: synth.Workload, run: GpuRun):
-    """Quantises q, k, v on the GPU (fp2_quantize_fp8) and runs the e4m3
+    """Quantises q, k, v on the GPU (fp2_quantize_fp8_qkv) and runs the e4m3
     prefill on run's plan; returns (O, LSE) as float32 host arrays."""
     import torch
     NB = int(run.lay.num_blocks)
@@ -218,8 +218,9 @@ def fp8_prefill(wl: synth.Workload, run: GpuRun):
     for which, src, H in [(0, run.q, wl.Hq), (1, run.k, wl.Hkv), (2, run.v, wl.Hkv)]:
         codes = torch.zeros(src.shape, dtype=torch.uint8, device="cuda")
         scales = torch.zeros((NB, H), dtype=torch.float32, device="cuda")
-        fb.fp2_quantize_fp8(run.prob, run.plan_buf, src, which, codes, scales)
         out[which] = (codes, scales)
+    fb.fp2_quantize_fp8_qkv(run.prob, run.plan_buf, run.q, run.k, run.v, out[0][0], out[1][0],
+                            out[2][0], out[0][1], out[1][1], out[2][1])
     o = torch.full((wl.T, wl.Hq, wl.d), float("nan"), dtype=torch.bfloat16, device="cuda")
     lse = torch.full((wl.Hq, wl.T), float("nan"), dtype=torch.float32, device="cuda")
     fb.fp2_prefill(run.prob, run.plan_buf, out[0][0], out[1][0], out[2][0], o, lse,

@@ -222,3 +222,21 @@ def test_no_cpu_fallback_in_product_path():
         if f.endswith(".py"):
             src = open(os.path.join(pkg, f)).read()
             assert "import oracle" not in src and "from oracle" not in src, f
+
+
+def test_head_slice_arguments_and_sizes():
+    # a slice of the layer's kv-heads: its plan is sized for its own heads, and
+    # a slice that does not fit in the tensors' heads is rejected on the host
+    lib = fb.lib()
+    full = fb.Problem([1000, 300], 0x1000, 32, 8, 128, 128, 0.1)
+    half = fb.Problem([1000, 300], 0x1000, 16, 4, 128, 128, 0.1, kv_head_begin=4,
+                      num_kv_heads_total=8)
+    compact = fb.Problem([1000, 300], 0x1000, 16, 4, 128, 128, 0.1)
+    lf, lh, lc = fb.fp2_plan_sizes(full), fb.fp2_plan_sizes(half), fb.fp2_plan_sizes(compact)
+    assert lh.num_rows * 2 == lf.num_rows and lh.nnz_cap * 2 == lf.nnz_cap
+    assert (lh.plan_bytes, lh.workspace_bytes) == (lc.plan_bytes, lc.workspace_bytes)
+    lay = fb.fp2_plan_layout()
+    for begin, total in ((5, 8), (-1, 8), (0, 3), (0, -2)):
+        bad = fb.Problem([1000, 300], 0x1000, 16, 4, 128, 128, 0.1, kv_head_begin=begin,
+                         num_kv_heads_total=total)
+        assert lib.fp2_plan_sizes(bad.ref, ctypes.byref(lay)) == fb.FP2_ERR_INVALID_ARG, (begin, total)

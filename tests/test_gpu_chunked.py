@@ -176,11 +176,118 @@ def test_whole_sequence_chunk_equals_the_full_prefill_bitwise():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-def test_chunked_fp8_is_rejected():
-    run = ChunkRun("mid_block")
+def _dq_chunk_q(run):
+    """The chunk's queries after direct online quantisation per (query block,
+    head) over the chunk positions in the block (the first block may be
+    partial), by the oracle's quantiser: codes, scales per global block and
+    the dequantised values."""
+    B = run.B
+    nbs = [(L + B - 1) // B for L in run.kv]
+    cu_b = np.concatenate([[0], np.cumsum(nbs)])
+    q = np.asarray(run.q64)
+    codes = np.zeros_like(q)
+    deq = np.zeros_like(q)
+    scales = np.ones((int(cu_b[-1]), q.shape[1]))
+    t0 = 0
+    for s, (L, Q) in enumerate(zip(run.kv, run.ql)):
+        off = L - Q
+        for i in range(off // B, nbs[s]):
+            lo, hi = max(i * B, off) - off + t0, min((i + 1) * B, L) - off + t0
+            c, sc = oracle.quantize_e4m3(q[lo:hi], [hi - lo], hi - lo)
+            codes[lo:hi] = c
+            scales[cu_b[s] + i] = sc[0]
+            deq[lo:hi] = oracle.dequantize_e4m3(c, sc, [hi - lo], hi - lo)
+        t0 += Q
+    return codes, scales, deq
+
+
+def _dq_full(a, lens, B):
+    """K or V after direct online quantisation per (block, head)."""
+    c, sc = oracle.quantize_e4m3(a, lens, B)
+    return oracle.dequantize_e4m3(c, sc, lens, B)
+
+
+@pytest.mark.parametrize("name", ["mid_block", "varlen_B64", "paged"])
+def test_chunked_fp8_matches_oracle(name):
+    # the e4m3 path on a chunk: Q quantised per query block over its chunk
+    # positions (codes and scales bit-exact with the oracle's quantiser), K / V
+    # per block; O / LSE against the chunked oracle on the quantised inputs
+    # (float64 block means of the plan)
     import torch
-    codes = torch.zeros(run.q.shape, dtype=torch.uint8, device="cuda")
-    scales = torch.zeros((int(run.lay.num_blocks), run.Hq), dtype=torch.float32, device="cuda")
-    with pytest.raises(fb.Fp2Error) as e:
-        fb.fp2_quantize_fp8(run.prob, run.plan_buf, run.q, 0, codes, scales)
-    assert e.value.code == fb.FP2_ERR_UNSUPPORTED
+    from fp2_harness import REL_L2_FP8
+    run = ChunkRun(name).run()
+    NB = int(run.lay.num_blocks)
+    out = {}
+    for which, src, H in ((0, run.q, run.Hq), (1, run.k, run.Hkv), (2, run.v, run.Hkv)):
+        codes = torch.zeros(src.shape, dtype=torch.uint8, device="cuda")
+        scales = torch.ones((NB, H), dtype=torch.float32, device="cuda")
+        fb.fp2_quantize_fp8(run.prob, run.plan_buf, src, which, codes, scales)
+        out[which] = (codes, scales)
+    qc, qs, q_dq = _dq_chunk_q(run)
+    got_c = out[0][0].view(torch.float8_e4m3fn).float().cpu().numpy()
+    assert np.array_equal(got_c.astype(np.float64), qc)
+    assert np.array_equal(out[0][1].cpu().numpy(), qs.astype(np.float32))
+    o = torch.full((run.Tq, run.Hq, run.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((run.Hq, run.Tq), float("nan"), dtype=torch.float32, device="cuda")
+    fb.fp2_prefill(run.prob, run.plan_buf, out[0][0], out[1][0], out[2][0], o, lse,
+                   q_scale=out[0][1], k_scale=out[1][1], v_scale=out[2][1],
+                   dtype=fb.FP2_DTYPE_E4M3)
+    assert fb.fp2_status_check(run.plan_buf) == (fb.FP2_OK, 0)
+    pl = ch.plan_chunk(run.q64, run.k64, run.v64, run.ql, run.kv, run.B, run.tau)
+    active, _ = _rows(run, pl)
+    gk = run.kept_lists()
+    for rg, ro in active:
+        if gk[rg] != list(pl["kept"][ro]):
+            pl["kept"][ro] = np.asarray(gk[rg], dtype=np.int64)
+    O_dq, L_dq = ch.attend_chunk(q_dq, _dq_full(run.k64, run.kv, run.B),
+                                 _dq_full(run.v64, run.kv, run.B), pl)
+    O = o.float().cpu().numpy()
+    L = lse.cpu().numpy()
+    assert np.isfinite(O).all() and np.isfinite(L).all()
+    e = rel_l2(O, O_dq)
+    l_err = float(np.max(np.abs(L - L_dq)))
+    print(f"fp8 chunk {name}: rel-L2 {e:.3e}, LSE {l_err:.3e}")
+    assert e <= REL_L2_FP8 and l_err <= LSE_ABS
+
+
+@pytest.mark.parametrize("name", ["mid_block", "varlen_B64", "paged"])
+def test_chunk_with_held_block_means(name):
+    # a serving caller keeps the K / V block means of earlier blocks: passing
+    # them (prev_kbar / prev_vbar) for the blocks wholly before each chunk must
+    # give the same plan and outputs as pooling those blocks again; entries of
+    # the other blocks are poisoned with NaN and must not be read
+    import torch
+    run = ChunkRun(name).run()
+    full = fb.Problem(run.kv, run.cu, run.Hq, run.Hkv, run.d, run.B, run.tau,
+                      **({} if not run.wl.page_size else
+                         dict(page_size=64, page_table=run.pt, num_pages=int(run.x["k_pool"].shape[0]))))
+    lay_f, plan_f, ws_f = fb.allocate(full)
+    full_q = to_bf16_device(np.asarray(run.x["q"]))
+    fb.fp2_plan(full, full_q, run.k, run.v, plan_f, ws_f)
+    assert fb.fp2_status_check(plan_f) == (fb.FP2_OK, 0)
+    vf = fb.PlanView(plan_f, lay_f, run.Hkv, run.d)
+    kb, vb = vf.kbar.clone(), vf.vbar.clone()
+    # poison every block that is not wholly before its sequence's chunk
+    b0 = 0
+    for L, Q in zip(run.kv, run.ql):
+        nb = (L + run.B - 1) // run.B
+        keep = (L - Q) // run.B
+        kb[b0 + keep:b0 + nb] = float("nan")
+        vb[b0 + keep:b0 + nb] = float("nan")
+        b0 += nb
+    extra = {} if not run.wl.page_size else dict(page_size=64, page_table=run.pt,
+                                                 num_pages=int(run.x["k_pool"].shape[0]))
+    prob = fb.Problem(run.kv, run.cu, run.Hq, run.Hkv, run.d, run.B, run.tau, q_seqlens=run.ql,
+                      cu_q_seqlens=run.cu_q, prev_kbar=kb, prev_vbar=vb, **extra)
+    lay, plan, ws = fb.allocate(prob)
+    fb.fp2_plan(prob, run.q, run.k, run.v, plan, ws)
+    o = torch.zeros_like(run.o)
+    lse = torch.zeros_like(run.lse)
+    fb.fp2_prefill(prob, plan, run.q, run.k, run.v, o, lse)
+    assert fb.fp2_status_check(plan) == (fb.FP2_OK, 0)
+    view = fb.PlanView(plan, lay, run.Hkv, run.d)
+    assert torch.equal(view.kbar, run.view.kbar) and torch.equal(view.vbar, run.view.vbar)
+    n = int(run.view.row_ptr[-1])
+    assert torch.equal(view.row_ptr, run.view.row_ptr)
+    assert torch.equal(view.col_idx[:n], run.view.col_idx[:n])
+    assert torch.equal(o, run.o) and torch.equal(lse, run.lse)

@@ -213,6 +213,17 @@ def test_quantize_fp8_matches_oracle_codes():
         ref, ref_s = oracle.quantize_e4m3(x[name], wl.seqlens, wl.B)
         assert np.array_equal(scales.cpu().numpy().astype(np.float64), ref_s)
         assert np.array_equal(got, ref)
+    # the one-launch form gives the same codes and scales
+    outs = [(torch.zeros(t.shape, dtype=torch.uint8, device="cuda"),
+             torch.zeros((NB, t.shape[1]), dtype=torch.float32, device="cuda"))
+            for t in (run.q, run.k, run.v)]
+    fb.fp2_quantize_fp8_qkv(run.prob, run.plan_buf, run.q, run.k, run.v, outs[0][0], outs[1][0],
+                            outs[2][0], outs[0][1], outs[1][1], outs[2][1])
+    for which, name in ((0, "q"), (1, "k"), (2, "v")):
+        ref, ref_s = oracle.quantize_e4m3(x[name], wl.seqlens, wl.B)
+        got = outs[which][0].view(torch.float8_e4m3fn).to(torch.float64).cpu().numpy()
+        assert np.array_equal(got, ref)
+        assert np.array_equal(outs[which][1].cpu().numpy().astype(np.float64), ref_s)
 
 
 def test_bounded_wait_times_out_and_context_survives():
