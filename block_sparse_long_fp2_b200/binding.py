@@ -16,6 +16,7 @@ import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libfp2.so")
+DEBUG_LIB_PATH = os.path.join(_PKG, "libfp2_debug.so")
 
 FP2_OK = 0
 FP2_ERR_INVALID_ARG = -1
@@ -28,6 +29,7 @@ FP2_ERR_DEVICE_CHECK = -6
 FP2_STATUS_BAD_SEQLENS = 0x1
 FP2_STATUS_BAD_PAGE = 0x2
 FP2_STATUS_TIMEOUT = 0x4
+FP2_STATUS_BOUNDS = 0x8
 
 FP2_DTYPE_BF16 = 0
 FP2_DTYPE_E4M3 = 1
@@ -102,11 +104,22 @@ class fp2_plan_layout(ctypes.Structure):
 
 
 _lib = None
+_loaded = {}
+
+
+def use_debug_library(on: bool) -> None:
+    """Route every call through libfp2_debug.so (the FP2_DEBUG build, whose
+    index checks record FP2_STATUS_BOUNDS) instead of libfp2.so, or back."""
+    global LIB_PATH, _lib
+    LIB_PATH = DEBUG_LIB_PATH if on else os.path.join(_PKG, "libfp2.so")
+    _lib = None
 
 
 def lib():
     """The loaded libfp2 (raises if it has not been built)."""
     global _lib
+    if _lib is None and LIB_PATH in _loaded:
+        _lib = _loaded[LIB_PATH]
     if _lib is None:
         if not os.path.exists(LIB_PATH):
             raise RuntimeError(f"libfp2 is not built ({LIB_PATH} missing); run "
@@ -141,6 +154,7 @@ def lib():
         for name in EXPORTED:
             getattr(L, name).restype = ctypes.c_int if name != "fp2_strerror" else ctypes.c_char_p
         _lib = L
+        _loaded[LIB_PATH] = L
     return _lib
 
 

@@ -3,8 +3,10 @@
     python -m block_sparse_long_fp2_b200.build [--verbose]
 
 Objects go to ``block_sparse_long_fp2_b200/_build/``; the shared library to
-``block_sparse_long_fp2_b200/libfp2.so``.  Rebuilds only when a source or
-header is newer than the library.
+``block_sparse_long_fp2_b200/libfp2.so``, and the debug build (the same
+sources with FP2_DEBUG: index checks that record FP2_STATUS_BOUNDS) to
+``libfp2_debug.so``.  Rebuilds only when a source or header is newer than the
+library.
 """
 
 from __future__ import annotations
@@ -20,6 +22,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libfp2.so")
+# The debug build: the same sources with FP2_DEBUG, whose index checks record
+# FP2_STATUS_BOUNDS in the plan's status word instead of accessing out of range.
+DEBUG_LIB = os.path.join(PKG, "libfp2_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O3",
@@ -44,22 +49,20 @@ def _deps():
     return files
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(f) > t for f in _deps())
 
 
-def build(verbose: bool = False, force: bool = False) -> str:
-    if not force and not needs_build():
-        return LIB
+def _build_one(lib: str, defines, objdir: str, verbose: bool) -> None:
     nvcc = _nvcc()
-    os.makedirs(BUILD, exist_ok=True)
-    extra = ["-Xptxas", "-v"] if verbose else []
+    os.makedirs(objdir, exist_ok=True)
+    extra = (["-Xptxas", "-v"] if verbose else []) + [f"-D{d}" for d in defines]
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
         cmd = [nvcc] + ARCH + NVCC_FLAGS + extra + ["-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -72,12 +75,20 @@ def build(verbose: bool = False, force: bool = False) -> str:
         for _, log in results:
             sys.stderr.write(log)
     objs = [o for o, _ in results]
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nvcc] + ARCH + ["-shared", "-o", tmp] + objs
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(verbose: bool = False, force: bool = False, debug: bool = True) -> str:
+    """Builds libfp2.so and (debug=True) libfp2_debug.so when a source is newer."""
+    if force or needs_build(LIB):
+        _build_one(LIB, [], BUILD, verbose)
+    if debug and (force or needs_build(DEBUG_LIB)):
+        _build_one(DEBUG_LIB, ["FP2_DEBUG"], os.path.join(BUILD, "debug"), verbose)
     return LIB
 
 

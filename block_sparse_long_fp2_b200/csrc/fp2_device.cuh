@@ -14,6 +14,20 @@
 
 namespace fp2 {
 
+// Index checks of the debug build (compiled with FP2_DEBUG: libfp2_debug.so):
+// a failed check records FP2_STATUS_BOUNDS in the status word and returns
+// false, and the caller clamps or skips the access.  In the regular build
+// every check is the constant true and compiles away.
+#ifdef FP2_DEBUG
+__device__ __forceinline__ bool debug_check(bool ok, int32_t* status) {
+    if (!ok) atomicOr(status, (int32_t)FP2_STATUS_BOUNDS);
+    return ok;
+}
+#define FP2_CHECK(cond, status) ::fp2::debug_check((cond), (status))
+#else
+#define FP2_CHECK(cond, status) true
+#endif
+
 // A bounded wait gives up after this many nanoseconds (about a second).
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;
 

@@ -694,7 +694,8 @@ k_score_tc(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap tm_
                 const float* col = dots + (ri * G) * (kScoreKeys + 1) + jj;
                 float best = col[0];
                 for (int hl = 1; hl < G; ++hl) best = fmaxf(best, col[hl * (kScoreKeys + 1)]);
-                scores[(int64_t)i * (i + 1) / 2 + j] = best * inv_sqrt_d;
+                if (FP2_CHECK(P.tri_off[s] + (int64_t)i * (i + 1) / 2 + j < D.tri_total, P.status))
+                    scores[(int64_t)i * (i + 1) / 2 + j] = best * inv_sqrt_d;
             }
         }
         __syncthreads();   // the staged dots are read before the next tile's copies land
@@ -900,11 +901,20 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
                     tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + buf * kScoreKeys + 32 * cc, r);
                     tmem_ld_wait();
                     const int jb = kScoreKeys * c + 32 * cc;
+                    // max over the G heads (adjacent lanes), 32 columns at a time so
+                    // the shuffles of different columns overlap
+                    for (int o = 1; o < G; o <<= 1) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        float v = __uint_as_float(r[e]);
-                        for (int o = 1; o < G; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-                        if (row_ok && jb + e <= i) sc_row[jb + e] = v * inv_sqrt_d;
+                        for (int e = 0; e < 32; ++e)
+                            r[e] = __float_as_uint(fmaxf(__uint_as_float(r[e]),
+                                                         __shfl_xor_sync(0xffffffffu, __uint_as_float(r[e]), o)));
+                    }
+                    if (row_ok) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (jb + e <= i &&
+                                FP2_CHECK(sc_row + jb + e < W.scores + D.Hkv * D.tri_total, P.status))
+                                sc_row[jb + e] = __uint_as_float(r[e]) * inv_sqrt_d;
                     }
                 }
                 tc_fence_before();
@@ -930,16 +940,33 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
 // (warp-collective).
 template <int HD>
 __device__ double score64(const Dims& D, const WsPtrs& W, int64_t b_i, int64_t b_j, int g) {
+    constexpr int E = HD / 32;   // elements per lane
     const int lane = threadIdx.x & 31;
     const double* kp = W.kbar64 + (b_j * D.Hkv + g) * HD;
-    double best = -DBL_MAX;
-    for (int hl = 0; hl < D.G; ++hl) {
-        const double* qp = W.qbar64 + (b_i * D.Hq + (int64_t)g * D.G + hl) * HD;
-        double acc = 0.0;
+    const double* qp0 = W.qbar64 + (b_i * D.Hq + (int64_t)g * D.G) * HD;
+    double kv[E];
 #pragma unroll
-        for (int e = lane; e < HD; e += 32) acc = fma(qp[e], kp[e], acc);
-        acc = warp_sum_d(acc);
-        best = fmax(best, acc);
+    for (int e = 0; e < E; ++e) kv[e] = __ldg(kp + lane + 32 * e);
+    double best = -DBL_MAX;
+    // four heads at a time: their loads and reductions overlap
+    for (int h0 = 0; h0 < D.G; h0 += 4) {
+        double acc[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            acc[u] = 0.0;
+            if (h0 + u < D.G) {
+                const double* qp = qp0 + (int64_t)(h0 + u) * HD;
+#pragma unroll
+                for (int e = 0; e < E; ++e) acc[u] = fma(__ldg(qp + lane + 32 * e), kv[e], acc[u]);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (h0 + u < D.G) best = fmax(best, acc[u]);
     }
     return best / sqrt((double)HD);
 }
@@ -953,8 +980,10 @@ __device__ double score64(const Dims& D, const WsPtrs& W, int64_t b_i, int64_t b
 // with rel_err the scoring kernel's bound (kScoreTcRelErr).  Every block whose
 // score could be the row maximum and every block whose score lies within e_j of
 // tau * m is re-scored in float64.
-// Rows of up to 32 * kThrRegs blocks load their scores in one pass.
-constexpr int kThrRegs = 32;
+// The loads of a row are issued kThrBatch words (32 blocks each) at a time,
+// so a pass over a row of n blocks waits on about n / (32 kThrBatch) round
+// trips to L2 rather than n / 32.
+constexpr int kThrBatch = 8;
 
 // The decision of one row (warp-collective), given the largest lower bound
 // m_lo of its scores: the row maximum in float64 over every block whose upper
@@ -968,41 +997,61 @@ __device__ __forceinline__ void thr_decide(const Dims& D, const WsPtrs& W, const
                                            int& count) {
     double m = -DBL_MAX;
 #pragma unroll 1
-    for (int jb = 0; jb <= i; jb += 32) {
-        const int j = jb + lane;
-        const bool cand = j <= i && (double)__ldg(sc + j) + Cq * __ldg(kn + (int64_t)j * D.Hkv) >= m_lo;
-        uint32_t cb = __ballot_sync(0xffffffffu, cand);
-        while (cb) {
-            const int l = __ffs(cb) - 1;
-            cb &= cb - 1;
-            m = fmax(m, score64<HD>(D, W, bi, b0 + jb + l, g));
+    for (int jb = 0; jb <= i; jb += 32 * kThrBatch) {
+        float xs[kThrBatch], ks[kThrBatch];
+#pragma unroll
+        for (int u = 0; u < kThrBatch; ++u) {
+            const int j = jb + 32 * u + lane;
+            xs[u] = j <= i ? __ldg(sc + j) : 0.f;
+            ks[u] = j <= i ? __ldg(kn + (int64_t)j * D.Hkv) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kThrBatch; ++u) {
+            const int j = jb + 32 * u + lane;
+            uint32_t cb = __ballot_sync(0xffffffffu, j <= i && (double)xs[u] + Cq * ks[u] >= m_lo);
+            while (cb) {
+                const int l = __ffs(cb) - 1;
+                cb &= cb - 1;
+                m = fmax(m, score64<HD>(D, W, bi, b0 + jb + 32 * u + l, g));
+            }
         }
     }
     const double t = D.tau * m;
 #pragma unroll 1
-    for (int w = 0; 32 * w <= i; ++w) {
-        const int j = 32 * w + lane;
-        bool keep = false, unsure = false;
-        if (j <= i) {
-            if (j == 0 || j == i) {
-                keep = true;
-            } else {
-                const double e = Cq * __ldg(kn + (int64_t)j * D.Hkv);
-                const double x = (double)__ldg(sc + j);
-                if (x - e >= t) keep = true;
-                else if (!(x + e < t)) unsure = true;
+    for (int jb = 0; jb <= i; jb += 32 * kThrBatch) {
+        float xs[kThrBatch], ks[kThrBatch];
+#pragma unroll
+        for (int u = 0; u < kThrBatch; ++u) {
+            const int j = jb + 32 * u + lane;
+            xs[u] = j <= i ? __ldg(sc + j) : 0.f;
+            ks[u] = j <= i ? __ldg(kn + (int64_t)j * D.Hkv) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kThrBatch; ++u) {
+            if (jb + 32 * u > i) break;
+            const int j = jb + 32 * u + lane;
+            bool keep = false, unsure = false;
+            if (j <= i) {
+                if (j == 0 || j == i) {
+                    keep = true;
+                } else {
+                    const double e = Cq * ks[u];
+                    const double x = (double)xs[u];
+                    if (x - e >= t) keep = true;
+                    else if (!(x + e < t)) unsure = true;
+                }
             }
+            uint32_t ub = __ballot_sync(0xffffffffu, unsure);
+            while (ub) {
+                const int l = __ffs(ub) - 1;
+                ub &= ub - 1;
+                const double x64 = score64<HD>(D, W, bi, b0 + jb + 32 * u + l, g);
+                if (lane == l) keep = x64 >= t;
+            }
+            const uint32_t bits = __ballot_sync(0xffffffffu, keep);
+            if (lane == 0) mask[(jb >> 5) + u] = bits;
+            count += __popc(bits);
         }
-        uint32_t ub = __ballot_sync(0xffffffffu, unsure);
-        while (ub) {
-            const int l = __ffs(ub) - 1;
-            ub &= ub - 1;
-            const double x64 = score64<HD>(D, W, bi, b0 + 32 * w + l, g);
-            if (lane == l) keep = x64 >= t;
-        }
-        const uint32_t bits = __ballot_sync(0xffffffffu, keep);
-        if (lane == 0) mask[w] = bits;
-        count += __popc(bits);
     }
     for (int w = i / 32 + 1 + lane; w < D.mask_words; w += 32) mask[w] = 0u;
 }
@@ -1035,40 +1084,26 @@ __global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W,
             mask[w] = bits;
         }
         count = i + 1;
-    } else if (i < 32 * kThrRegs) {
-        // one pass of loads with every load of the row in flight at once (the
-        // row's scores and key norms, 32 per lane, in registers), then the two
-        // decision passes over the same lines from L1
-        const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
-        const double C = rel_err / sqrt((double)HD);
-        const double qn = W.qnorm[bi * D.Hkv + g];
-        const float* kn = W.knorm + (int64_t)b0 * D.Hkv + g;
-        float x[kThrRegs], kv[kThrRegs];
-#pragma unroll
-        for (int u = 0; u < kThrRegs; ++u) {
-            const int j = 32 * u + lane;
-            const bool in = j <= i;
-            x[u] = in ? __ldg(sc + j) : 0.f;
-            kv[u] = in ? __ldg(kn + (int64_t)j * D.Hkv) : 0.f;
-        }
-        // largest lower bound of any score
-        double m_lo = -DBL_MAX;
-#pragma unroll
-        for (int u = 0; u < kThrRegs; ++u)
-            if (32 * u + lane <= i) m_lo = fmax(m_lo, (double)x[u] - C * qn * kv[u]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m_lo = fmax(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o));
-        thr_decide<HD>(D, W, sc, kn, C * qn, m_lo, i, bi, b0, g, lane, mask, count);
     } else {
         const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
         const double C = rel_err / sqrt((double)HD);
         const double qn = W.qnorm[bi * D.Hkv + g];
         const float* kn = W.knorm + (int64_t)b0 * D.Hkv + g;
-        // largest lower bound of any score
+        // largest lower bound of any score (kThrBatch words of loads at a time)
         double m_lo = -DBL_MAX;
-#pragma unroll 8
-        for (int j = lane; j <= i; j += 32)
-            m_lo = fmax(m_lo, (double)__ldg(sc + j) - C * qn * __ldg(kn + (int64_t)j * D.Hkv));
+#pragma unroll 1
+        for (int jb = 0; jb <= i; jb += 32 * kThrBatch) {
+            float xs[kThrBatch], ks[kThrBatch];
+#pragma unroll
+            for (int u = 0; u < kThrBatch; ++u) {
+                const int j = jb + 32 * u + lane;
+                xs[u] = j <= i ? __ldg(sc + j) : 0.f;
+                ks[u] = j <= i ? __ldg(kn + (int64_t)j * D.Hkv) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kThrBatch; ++u)
+                if (jb + 32 * u + lane <= i) m_lo = fmax(m_lo, (double)xs[u] - C * qn * ks[u]);
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m_lo = fmax(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o));
         thr_decide<HD>(D, W, sc, kn, C * qn, m_lo, i, bi, b0, g, lane, mask, count);
@@ -1205,7 +1240,9 @@ __global__ void k_compact(Dims D, PlanPtrs P) {
     int32_t base = P.row_ptr[r];
     for (int w = 0; 32 * w <= i; ++w) {
         const uint32_t bits = mask[w];
-        if ((bits >> lane) & 1u) P.col_idx[base + __popc(bits & ((1u << lane) - 1u))] = 32 * w + lane;
+        const int32_t at = base + __popc(bits & ((1u << lane) - 1u));
+        if (((bits >> lane) & 1u) && FP2_CHECK(at >= 0 && at < D.nnz_cap, P.status))
+            P.col_idx[at] = 32 * w + lane;
         base += __popc(bits);
     }
 }

@@ -71,6 +71,9 @@ extern "C" {
 #define FP2_STATUS_BAD_SEQLENS 0x1u   /* cu_seqlens not consistent with the problem sizes */
 #define FP2_STATUS_BAD_PAGE 0x2u      /* a page id outside [0, num_pages)                 */
 #define FP2_STATUS_TIMEOUT 0x4u       /* a bounded wait inside a kernel ran out           */
+#define FP2_STATUS_BOUNDS 0x8u        /* an index check of the debug build (libfp2_debug.so,
+                                         built with FP2_DEBUG) failed; the access was
+                                         clamped or skipped                                */
 
 /* ---- element types -------------------------------------------------------- */
 #define FP2_DTYPE_BF16 0   /* bfloat16 Q, K, V                                     */

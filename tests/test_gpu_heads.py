@@ -90,7 +90,7 @@ def test_head_slices_equal_the_full_layer(name):
             scales = torch.zeros((NB, H), dtype=torch.float32, device="cuda")
             fb.fp2_quantize_fp8(prob, plan, src, which, codes, scales)
             codes_f = torch.zeros_like(codes)
-            scales_f = torch.zeros((NB, src.shape[1]), dtype=torch.float32, device="cuda")
+            scales_f = torch.zeros((NB, src.shape[-2]), dtype=torch.float32, device="cuda")
             fb.fp2_quantize_fp8(full.prob, full.plan_buf, src, which, codes_f, scales_f)
             assert torch.equal(scales, scales_f[:, hs:hs + H])
             # (the head axis is the second-to-last one, contiguous or paged)
