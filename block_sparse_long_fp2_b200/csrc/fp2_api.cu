@@ -208,6 +208,7 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     L.ws_knorm = w.take(sizeof(float) * (size_t)NB * d.Hkv);
     L.ws_scores = w.take(sizeof(float) * (size_t)d.nnz_cap);
     L.ws_counts = w.take(sizeof(int32_t) * (size_t)d.R);
+    L.ws_bounds = w.take(sizeof(double) * 2 * (size_t)d.R);
     pub.workspace_bytes = align_up(w.off, 256);
     pub.num_work_items = sd.n_items;
     pub.num_split_slots = sd.split_slots * d.Hkv;
@@ -261,6 +262,7 @@ WsPtrs ws_ptrs(const Layout& L, void* ws) {
     w.knorm = reinterpret_cast<float*>(b + L.ws_knorm);
     w.scores = reinterpret_cast<float*>(b + L.ws_scores);
     w.counts = reinterpret_cast<int32_t*>(b + L.ws_counts);
+    w.bounds = reinterpret_cast<double*>(b + L.ws_bounds);
     return w;
 }
 

@@ -57,15 +57,10 @@ constexpr int kMmaWarp = 9;     // issues every MMA; owns the tensor memory
 // the 227 KiB of shared memory a CTA may use (at most 8).
 constexpr int kMaxSmem = 232448;
 constexpr int kMaxSlots = 8;
-// e4m3: P goes from the softmax to the P.V product through shared memory, two
-// 128-row buffers per softmax warpgroup, each row one 128-byte swizzle atom.
-constexpr int kPTileBytes = kTileM * 128;
-constexpr int kNumPBufs = 4;
 template <int HD, int BLK, bool F8>
 constexpr int ring_slots() {
     const int elt = F8 ? 1 : 2;
-    const int p_bytes = F8 ? kNumPBufs * kPTileBytes : 0;
-    const int avail = (kMaxSmem - 512 - 1024 - 2 * kTileM * HD * elt - p_bytes) / (BLK * HD * elt);
+    const int avail = (kMaxSmem - 512 - 1024 - 2 * kTileM * HD * elt) / (BLK * HD * elt);
     return avail < kMaxSlots ? avail : kMaxSlots;
 }
 
@@ -89,8 +84,7 @@ struct Cfg {
     static constexpr int kQBytes = kTileM * kRowBytes;   // one 128-row query tile
     static constexpr int kSlotBytes = BLK * kRowBytes;   // one K or V tile
     static constexpr int kOffQ = 0;
-    static constexpr int kOffP = 2 * kQBytes;                       // e4m3 only
-    static constexpr int kOffSlot = kOffP + (F8 ? kNumPBufs * kPTileBytes : 0);
+    static constexpr int kOffSlot = 2 * kQBytes;
     static constexpr int kOffBar = kOffSlot + kSlots * kSlotBytes;
     static_assert(kSlots >= 3, "the K/V ring needs at least three slots");
     static constexpr int kSmemBytes = kOffBar + 512 + 1024;   // barriers + alignment slack
@@ -118,10 +112,6 @@ struct Bars {
     uint64_t kv_full[kMaxSlots], kv_empty[kMaxSlots];
     uint64_t s_full[2];
     uint64_t p_full[2];
-    // e4m3: S read into registers (its columns may be overwritten), P buffer b
-    // of warpgroup m written, and the P.V product that read it completed
-    uint64_t s_free[2];
-    uint64_t p8_full[2][2], p8_free[2][2];
     uint64_t o_full[2], o_free[2];
     uint64_t drain;
     uint32_t tmem_base;
@@ -962,350 +952,8 @@ __device__ void softmax_wg(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
     }
 }
 
-// ---------------------------------------------------------------------------
-// e4m3 MMA issuer: S released by the softmax before it computes P
-// ---------------------------------------------------------------------------
-//
-// In the e4m3 path the softmax reads the whole S row into registers and frees
-// the S columns at once (s_free), writes P into a shared-memory buffer (two per
-// warpgroup) and publishes it (p8_full).  So S_m(n+1) is issued as soon as the
-// softmax has read S_m(n), and runs while the softmax computes P_m(n): the
-// issue order per tile is S0(n+1), P0(n).V, S1(n+1), P1(n).V, and a
-// warpgroup's period is its softmax, not its softmax plus two MMAs.  P_m(n).V
-// commits to p8_free[m][n % 2] (the buffer may be rewritten; O_m holds P_m(n).V).
-template <int HD, int BLK>
-__device__ void mma_issuer_f8(const AttnParams& P, Bars& B, uint8_t* smem) {
-    using C = Cfg<HD, BLK, true>;
-    constexpr int kSlots = C::kSlots;
-    const uint32_t tb = B.tmem_base;
-    const uint32_t s_base = smem_u32(smem);
-    const uint64_t q_desc[2] = {smem_desc_sw128(s_base + C::kOffQ, 16, 1024),
-                                smem_desc_sw128(s_base + C::kOffQ + C::kQBytes, 16, 1024)};
-    const uint64_t k_desc0 = smem_desc_sw128(s_base + C::kOffSlot, 16, 1024);
-    const uint64_t v_desc0 = smem_desc_sw128(s_base + C::kOffSlot, C::kAtomKV, 1024);
-    const uint64_t p_desc0 = smem_desc_sw128(s_base + C::kOffP, 16, 1024);
-    const uint32_t t_s[2] = {tb + C::kColS0, tb + C::kColS1};
-    const uint32_t t_o[2] = {tb + C::kColO0, tb + C::kColO1};
-    uint32_t qcnt[2] = {0, 0}, scnt[2] = {0, 0}, pcnt[2] = {0, 0}, ocnt[2] = {0, 0};
-    RingPos ring{0, 0};
-
-    struct KPos {
-        RingPos k, lo;
-        bool two;
-    };
-    auto kdesc = [&](const RingPos& r) { return desc_add(k_desc0, r.slot * C::kSlotBytes); };
-    // S_m = Q_m K^T into S_m once the softmax has read the previous S_m
-    auto issue_sm = [&](int m, const KPos& kk) -> bool {
-        if (!mbar_wait(&B.kv_full[kk.k.slot], kk.k.use & 1, &B.abort, P.status)) return false;
-        if (kk.two && !mbar_wait(&B.kv_full[kk.lo.slot], kk.lo.use & 1, &B.abort, P.status))
-            return false;
-        if (!mbar_wait(&B.s_free[m], (scnt[m] & 1) ^ 1, &B.abort, P.status)) return false;
-        ++scnt[m];
-        tc_fence_after();
-        issue_s<HD, BLK, true>(t_s[m], q_desc[m], kdesc(kk.k));
-        if (kk.two) issue_s<HD, BLK, true>(t_s[m], q_desc[m], kdesc(kk.lo), true);
-        umma_commit(&B.s_full[m]);
-        return true;
-    };
-    auto release_k = [&](const KPos& kk) {
-        umma_commit(&B.kv_empty[kk.k.slot]);
-        if (kk.two) umma_commit(&B.kv_empty[kk.lo.slot]);
-    };
-    // O_m (+)= P_m V with P_m from its shared-memory buffer
-    auto issue_pv = [&](int m, const RingPos& v, bool first, bool last) -> bool {
-        const int buf = pcnt[m] & 1;
-        if (!mbar_wait(&B.kv_full[v.slot], v.use & 1, &B.abort, P.status)) return false;
-        if (!mbar_wait(&B.p8_full[m][buf], (pcnt[m] >> 1) & 1, &B.abort, P.status)) return false;
-        if (first && !mbar_wait(&B.o_free[m], (ocnt[m] & 1) ^ 1, &B.abort, P.status)) return false;
-        ++pcnt[m];
-        tc_fence_after();
-        const uint64_t a = desc_add(p_desc0, (2 * m + buf) * kPTileBytes);
-        const uint64_t b = desc_add(v_desc0, v.slot * C::kSlotBytes);
-#pragma unroll
-        for (int kk = 0; kk < BLK / C::kKStep; ++kk)
-            umma_f8(t_o[m], desc_add(a, kk * 32), desc_add(b, kk * C::kKStep * 128), C::kIdescO,
-                    (!first || kk > 0) ? 1u : 0u);
-        umma_commit(&B.p8_free[m][buf]);
-        if (last) {
-            umma_commit(&B.o_full[m]);
-            ++ocnt[m];
-        }
-        return true;
-    };
-
-    for (int64_t w = blockIdx.x; w < P.n_slots; w += gridDim.x) {
-        const int64_t o = sched_index(w, P.zigzag);
-        if (o >= P.n_items) continue;
-        const Item it = decode_item(P, o);
-        if (!it.ok) continue;
-        int n_tiles, n_real;
-        {
-            TileWalk<BLK> walk;
-            walk.init(P, it);
-            n_tiles = walk.count();
-            n_real = walk.n_kept - walk.t;   // tiles before the pseudo tiles
-        }
-        if (n_tiles == 0) continue;
-        auto take_tile = [&](int n, KPos& kk, RingPos& v) {
-            kk.k = ring_take<kSlots>(ring);
-            kk.two = n >= n_real;   // a pseudo tile: two e4m3 terms of the key means
-            if (kk.two) kk.lo = ring_take<kSlots>(ring);
-            v = ring_take<kSlots>(ring);
-        };
-        KPos kp;
-        RingPos vp;
-        take_tile(0, kp, vp);
-        if (!mbar_wait(&B.q_full[0], qcnt[0] & 1, &B.abort, P.status)) goto drain;
-        ++qcnt[0];
-        if (!issue_sm(0, kp)) goto drain;
-        if (it.has_m1) {
-            if (!mbar_wait(&B.q_full[1], qcnt[1] & 1, &B.abort, P.status)) goto drain;
-            ++qcnt[1];
-            if (!issue_sm(1, kp)) goto drain;
-        }
-        release_k(kp);
-        if (n_tiles == 1) {
-            umma_commit(&B.q_empty[0]);
-            if (it.has_m1) umma_commit(&B.q_empty[1]);
-        }
-        for (int n = 0; n < n_tiles; ++n) {
-            const bool first = n == 0, last = n == n_tiles - 1;
-            KPos kn;
-            RingPos vn;
-            if (!last) {
-                take_tile(n + 1, kn, vn);
-                if (!issue_sm(0, kn)) goto drain;   // S0(n+1)
-            }
-            if (!issue_pv(0, vp, first, last)) goto drain;   // P0(n).V
-            if (it.has_m1) {
-                if (!last && !issue_sm(1, kn)) goto drain;   // S1(n+1)
-                if (!issue_pv(1, vp, first, last)) goto drain;   // P1(n).V
-            }
-            umma_commit(&B.kv_empty[vp.slot]);
-            if (!last) {
-                release_k(kn);
-                if (n + 1 == n_tiles - 1) {
-                    umma_commit(&B.q_empty[0]);
-                    if (it.has_m1) umma_commit(&B.q_empty[1]);
-                }
-                kp = kn;
-                vp = vn;
-            }
-        }
-    }
-drain:
-    umma_commit(&B.drain);
-    mbar_wait_drain(&B.drain, 0, P.status);
-}
-
-// ---------------------------------------------------------------------------
-// e4m3 softmax warpgroup: the S row in registers, P through shared memory
-// ---------------------------------------------------------------------------
-
-// Byte offset of 16-byte chunk c of row r in a 128-byte-swizzled tile of
-// 128-byte rows (8-row groups of 1024 bytes, the layout TMA writes and the
-// MMA descriptors above read).
-__device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
-    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
-}
-
-template <int HD, int BLK, bool CHUNK>
-__device__ void softmax_wg_f8(const AttnParams& P, Bars& B, uint8_t* smem, int m) {
-    using C = Cfg<HD, BLK, true>;
-    constexpr int NC = BLK / 32;
-    constexpr float kHeadroom = C::kHeadroom;
-    const Dims& D = P.D;
-    const int q4 = (threadIdx.x >> 5) & 3;        // TMEM lane quarter of this warp
-    const int lane = threadIdx.x & 31;
-    const int prow = 32 * q4 + lane;              // row of the 128-row query tile
-    const uint32_t lane_off = static_cast<uint32_t>(32 * q4) << 16;
-    const uint32_t t_s = B.tmem_base + lane_off + (m == 0 ? C::kColS0 : C::kColS1);
-    const uint32_t t_o = B.tmem_base + lane_off + (m == 0 ? C::kColO0 : C::kColO1);
-    const uint32_t p_row0 = smem_u32(smem + C::kOffP);
-    const float scale = 1.4426950408889634f / sqrtf((float)HD);   // log2(e) / sqrt(d)
-    const float pseudo_bias = log2f((float)BLK);                   // ln n_j in log2 units
-    uint32_t scnt = 0, ocnt = 0, pn = 0;   // S tiles, items, P tiles of this warpgroup
-
-    for (int64_t w = blockIdx.x; w < P.n_slots; w += gridDim.x) {
-        const int64_t o = sched_index(w, P.zigzag);
-        if (o >= P.n_items) continue;
-        const Item it = decode_item(P, o);
-        if (!it.ok) continue;
-        if (m == 1 && !it.has_m1) continue;
-        TileWalk<BLK> walk;
-        walk.init(P, it);
-        if (walk.count() == 0) continue;   // a split without tiles
-        const int split_slot = it.S > 1 ? it.slot + it.k : -1;
-        const int mt = 2 * it.mp + m;
-        const int pr = kTileM * mt + prow;
-        const int hl = pr / BLK;
-        const int tok = pr % BLK;
-        const int h = it.g * D.G + hl;
-        const int pos = it.i * BLK + tok;
-        const int qoff = CHUNK ? P.q_off[it.s] : 0;
-        bool row_valid = pos < it.L && (!CHUNK || pos >= qoff);
-        const int64_t qtok = CHUNK ? (int64_t)P.cu_q[it.s] - qoff : it.tok0;
-        RowState st{-INFINITY, 0.f, t_o, false};
-        const float q_sc = __ldg(P.q_scale + (int64_t)(it.b0 + it.i) * D.Hq + h);
-        const float k_row = 448.0f / (256.0f * __ldg(P.vmax + (int64_t)it.s * D.Hkv + it.g));
-
-        int kind, j;
-        while (walk.next(kind, j)) {
-            const int64_t sb = (int64_t)it.b0 + (kind == kPseudo ? (int64_t)BLK * j : j);
-            const float* ks = kind == kPseudo ? P.kbar_scale : P.k_scale;
-            const float* vs = kind == kPseudo ? P.vbar_scale : P.v_scale;
-            const float tscale = scale * q_sc * __ldg(ks + sb * D.Hkv + it.g);
-            const float pfac = __ldg(vs + sb * D.Hkv + it.g) * k_row;
-            const float bias = kind == kPseudo ? pseudo_bias : 0.f;
-            if (!warp_wait(&B.s_full[m], scnt & 1, B, P.status)) return;
-            ++scnt;
-            tc_fence_after();
-            // the whole S row into registers, then S is free for the next tile
-            uint32_t r[BLK];
-#pragma unroll
-            for (int c = 0; c < NC; ++c) tmem_ld32(t_s + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * c));
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&B.s_free[m]);
-            const bool masked = kind != kFull;
-            uint32_t vb[NC];
-#pragma unroll
-            for (int c = 0; c < NC; ++c) vb[c] = masked ? col_bits(kind, tok, walk, j, c) : 0xFFFFFFFFu;
-            // row maximum of the tile (scaled logits, log2 units)
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < NC; ++c)
-                mx = fmaxf(mx, masked ? max32<true>(*reinterpret_cast<uint32_t(*)[32]>(r + 32 * c), vb[c])
-                                      : max32<false>(*reinterpret_cast<uint32_t(*)[32]>(r + 32 * c), vb[c]));
-            const float cm = fmaf(mx, tscale, bias);
-            const bool need = cm > st.m_ref + kHeadroom;
-            if (__any_sync(0xffffffffu, need)) {
-                // the reference moves: O must hold every P.V issued so far (the
-                // last one, P(pn - 1).V, completes on its buffer's barrier)
-                if (st.o_valid) {
-                    const uint32_t prev = pn - 1;
-                    if (!warp_wait(&B.p8_free[m][prev & 1], (prev >> 1) & 1, B, P.status)) return;
-                    tc_fence_after();
-                }
-                const float m_new = need ? cm : st.m_ref;
-                const float alpha = m_new > st.m_ref ? ex2_approx(st.m_ref - m_new) : 1.0f;
-                st.m_ref = fmaxf(st.m_ref, m_new);
-                st.l *= alpha;
-                if (st.o_valid) {
-#pragma unroll 1
-                    for (int c = 0; c < HD / 32; ++c) {
-                        uint32_t ro[32];
-                        tmem_ld32(st.t_o + 32 * c, ro);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * alpha);
-                        tmem_st32(st.t_o + 32 * c, ro);
-                    }
-                    tmem_st_wait();
-                }
-            }
-            // P' = 2^(s * scale + bias - m_ref + log2 pfac): e4m3 codes, 4 per word
-            const float shift = bias + __log2f(pfac) - st.m_ref;
-            const uint64_t scale2 = f2_pack(tscale, tscale), shift2 = f2_pack(shift, shift);
-            uint64_t sum2 = f2_pack(0.f, 0.f);
-            uint32_t pk[BLK / 4];
-#pragma unroll
-            for (int c = 0; c < NC; ++c) {
-#pragma unroll
-                for (int e = 0; e < 32; e += 4) {
-                    float pv[4];
-#pragma unroll
-                    for (int u = 0; u < 4; u += 2) {
-                        float s0 = __uint_as_float(r[32 * c + e + u]), s1 = __uint_as_float(r[32 * c + e + u + 1]);
-                        if (masked) {
-                            s0 = ((vb[c] >> (e + u)) & 1u) ? s0 : -INFINITY;
-                            s1 = ((vb[c] >> (e + u + 1)) & 1u) ? s1 : -INFINITY;
-                        }
-                        float x0, x1;
-                        f2_unpack(f2_fma(f2_pack(s0, s1), scale2, shift2), x0, x1);
-                        pv[u] = ex2_approx(x0);
-                        pv[u + 1] = ex2_approx(x1);
-                        sum2 = f2_add(sum2, f2_pack(pv[u], pv[u + 1]));
-                    }
-                    pk[(32 * c + e) / 4] = pack_e4m3x4(pv[0], pv[1], pv[2], pv[3]);
-                }
-            }
-            // into this warpgroup's P buffer pn % 2, once the P.V that read it
-            // two tiles ago has completed
-            const int buf = pn & 1;
-            if (pn >= 2 && !warp_wait(&B.p8_free[m][buf], ((pn >> 1) - 1) & 1, B, P.status)) return;
-            const uint32_t prow_addr = p_row0 + (2 * m + buf) * kPTileBytes;
-#pragma unroll
-            for (int c16 = 0; c16 < 8; ++c16) {
-                const uint32_t a = prow_addr + sw128_offset(prow, c16);
-                if (c16 < BLK / 16)
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * c16]),
-                                 "r"(pk[4 * c16 + 1]), "r"(pk[4 * c16 + 2]), "r"(pk[4 * c16 + 3])
-                                 : "memory");
-                else
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
-            }
-            fence_proxy_async_smem();   // the MMA reads P through the async proxy
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&B.p8_full[m][buf]);
-            ++pn;
-            float a, b;
-            f2_unpack(sum2, a, b);
-            st.l += (a + b) * __frcp_rn(pfac);
-            st.o_valid = true;
-        }
-
-        // epilogue: O / l as bf16, LSE = ln(l) + m_ref * ln 2; a split row
-        // writes its part's O / l in fp32 and log2(l) + m_ref to its slot
-        if (!warp_wait(&B.o_full[m], ocnt & 1, B, P.status)) return;
-        ++ocnt;
-        tc_fence_after();
-        const float inv_l = 1.0f / (st.l * k_row);
-        const bool split = split_slot >= 0;
-        const int64_t srow = (int64_t)split_slot * (D.G * BLK) + pr;
-        const int64_t orow = (qtok + pos) * D.Hq_str + h;
-        if (row_valid && !(split ? FP2_CHECK(srow < P.n_split_rows, P.status)
-                                 : FP2_CHECK(qtok + pos >= 0 && qtok + pos < P.Tq, P.status)))
-            row_valid = false;
-        char* dst = split ? reinterpret_cast<char*>(P.split_o + srow * HD)
-                          : reinterpret_cast<char*>(P.o + orow * HD);
-#pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
-            uint32_t ro[32];
-            tmem_ld32(t_o + 32 * c, ro);
-            tmem_ld_wait();
-            if (row_valid && split) {
-#pragma unroll
-                for (int e = 0; e < 32; e += 4)
-                    reinterpret_cast<float4*>(dst)[(32 * c + e) / 4] =
-                        make_float4(__uint_as_float(ro[e + 0]) * inv_l, __uint_as_float(ro[e + 1]) * inv_l,
-                                    __uint_as_float(ro[e + 2]) * inv_l, __uint_as_float(ro[e + 3]) * inv_l);
-            } else if (row_valid) {
-#pragma unroll
-                for (int e = 0; e < 32; e += 8) {
-                    uint4 v;
-                    v.x = pack_bf16x2(__uint_as_float(ro[e + 0]) * inv_l, __uint_as_float(ro[e + 1]) * inv_l);
-                    v.y = pack_bf16x2(__uint_as_float(ro[e + 2]) * inv_l, __uint_as_float(ro[e + 3]) * inv_l);
-                    v.z = pack_bf16x2(__uint_as_float(ro[e + 4]) * inv_l, __uint_as_float(ro[e + 5]) * inv_l);
-                    v.w = pack_bf16x2(__uint_as_float(ro[e + 6]) * inv_l, __uint_as_float(ro[e + 7]) * inv_l);
-                    reinterpret_cast<uint4*>(dst)[(32 * c + e) / 8] = v;
-                }
-            }
-        }
-        const float lse2 = st.m_ref + log2f(st.l);
-        if (row_valid && split) P.split_lse[srow] = lse2;
-        else if (row_valid) P.lse[(int64_t)h * (CHUNK ? P.Tq : D.T) + qtok + pos] = lse2 * 0.6931471805599453f;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B.o_free[m]);
-    }
-}
-
-// 320 threads x 200 registers fill the register file of an SM (one CTA per
-// SM): the e4m3 softmax holds a whole 128-column S row in registers.
 template <int HD, int BLK, bool F8, bool CHUNK>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kThreads, 1)
 k_attn(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap tm_q,
        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
        const __grid_constant__ CUtensorMap tm_kbar, const __grid_constant__ CUtensorMap tm_vbar,
@@ -1325,11 +973,6 @@ k_attn(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap
             mbar_init(&B.q_empty[m], 1);
             mbar_init(&B.s_full[m], 1);
             mbar_init(&B.p_full[m], kTileM / 32);
-            mbar_init(&B.s_free[m], kTileM / 32);
-            for (int b = 0; b < 2; ++b) {
-                mbar_init(&B.p8_full[m][b], kTileM / 32);
-                mbar_init(&B.p8_free[m][b], 1);
-            }
             mbar_init(&B.o_full[m], 1);
             mbar_init(&B.o_free[m], kTileM / 32);
         }
@@ -1356,17 +999,12 @@ k_attn(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap
     tc_fence_after();
 
     if (warp < 8) {
-        if constexpr (F8) softmax_wg_f8<HD, BLK, CHUNK>(P, B, smem, warp >> 2);
-        else softmax_wg<HD, BLK, F8, CHUNK>(P, B, smem, warp >> 2);
+        softmax_wg<HD, BLK, F8, CHUNK>(P, B, smem, warp >> 2);
     } else if (warp == kProducerWarp) {
         if (lane == 0) producer<HD, BLK, F8, CHUNK>(P, B, smem, &tm_q, &tm_k, &tm_v, &tm_kbar, &tm_vbar,
                                                     &tm_kbar_lo);
     } else {
-        if constexpr (F8) {
-            if (lane == 0) mma_issuer_f8<HD, BLK>(P, B, smem);
-        } else {
-            if (lane == 0) mma_issuer<HD, BLK, F8>(P, B, smem);
-        }
+        if (lane == 0) mma_issuer<HD, BLK, F8>(P, B, smem);
     }
     __syncwarp();
     tc_fence_before();

@@ -127,10 +127,12 @@ struct WsPtrs {
     float* kbar_tf;   // [NB, Hkv, d] the key means rounded to tf32 (stored as fp32)
     double* kbar64;   // [NB, Hkv, d]
     float* qnorm;     // [NB, Hkv]  max over the group's heads of |Qbar|_2 (rounded up)
-    float* knorm;     // [NB, Hkv]  |Kbar|_2 (rounded up)
+    float* knorm;     // [Hkv, NB]  |Kbar|_2 (rounded up), contiguous over a head's blocks
     float* scores;    // [Hkv, tri_total] fp32 block scores, row (s,g,i) at
                       //   g * tri_total + tri_off[s] + i (i + 1) / 2 + j
     int32_t* counts;  // [R] kept blocks per row
+    double* bounds;   // [R, 2] per row: the largest lower and upper bound of any
+                      //   score (sc_j -/+ its error bound), from the pipelined scorer
 };
 
 struct Layout {
@@ -142,7 +144,8 @@ struct Layout {
     size_t off_meta_valid, off_cu_blocks, off_block_seq, off_tri_off, off_group_cu, off_group_seq,
         off_tile_cu, off_vmax, off_sched, off_sched_cnt, off_sched_off, off_split_o, off_split_lse,
         off_slot_item, off_q_off;
-    size_t ws_qbar64, ws_qbar32, ws_kbar_tf, ws_kbar64, ws_qnorm, ws_knorm, ws_scores, ws_counts;
+    size_t ws_qbar64, ws_qbar32, ws_kbar_tf, ws_kbar64, ws_qnorm, ws_knorm, ws_scores, ws_counts,
+        ws_bounds;
 };
 
 // Validates the problem on the host and computes sizes and offsets.

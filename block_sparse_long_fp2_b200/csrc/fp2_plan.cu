@@ -147,6 +147,8 @@ __device__ void meta_maps(const Dims& D, const SchedDims& S, const int32_t* __re
 // Tq their total.
 __global__ void __launch_bounds__(kMetaThreads, 1) k_meta(Dims D, SchedDims S, const int32_t* __restrict__ cu_seqlens,
                        const int32_t* __restrict__ page_table, int64_t Tq, PlanPtrs P) {
+    // the next kernel may be launched early: it waits for this one first
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int32_t* __restrict__ cu_q = P.cu_q;
     __shared__ int s_valid;
     if (threadIdx.x == 0) {
@@ -505,7 +507,7 @@ k_pool(Dims D, SeqMap M, int64_t Tq, const int32_t* __restrict__ cu_seqlens,
         const int tph = d / 8;
         for (int o = tph / 2; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
         const bool lead = active && (vec % tph) == 0;
-        if (lead && which == 1) W.knorm[b * D.Hkv + head] = round_up_f(sqrt(sq));
+        if (lead && which == 1) W.knorm[(int64_t)head * D.NB + b] = round_up_f(sqrt(sq));
         // the largest over the G query heads of a kv-head: the group's heads
         // lie in this CTA (G d divides the CTA's 1024 columns)
         __shared__ double head_sq[kPoolThreads];
@@ -545,7 +547,7 @@ __global__ void k_norms(Dims D, PlanPtrs P, WsPtrs W) {
         qmax = fmax(qmax, qq);
     }
     if (lane == 0) {
-        W.knorm[wid] = round_up_f(sqrt(kk));
+        W.knorm[(int64_t)g * D.NB + b] = round_up_f(sqrt(kk));
         W.qnorm[wid] = round_up_f(sqrt(qmax));
     }
 }
@@ -765,7 +767,9 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
              const __grid_constant__ CUtensorMap tm_k) {
     using C = ScorePCfg<HD>;
     // runs beside k_quant_means (launched before it as its programmatic
-    // dependent) and completes only after it
+    // dependent) and completes only after it; the threshold after it may be
+    // launched early (it waits for this kernel before reading anything)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (!*P.meta_valid) {
         asm volatile("griddepcontrol.wait;" ::: "memory");
         return;
@@ -875,8 +879,12 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
             mbar_wait_drain(&drain, 0, P.status);
         }
     } else {
-        // epilogue warps 0-3: thread = query vector (block ri, head hl) of the item
+        // epilogue warps 0-3: thread = query vector (block ri, head hl) of the item;
+        // the block's first lane also keeps the row's largest lower and upper
+        // bound of any score, sc_j -/+ C |Qbar|max |Kbar_j| (the threshold's
+        // first pass, done here while the scores are in registers)
         const float inv_sqrt_d = 1.0f / sqrtf((float)HD);
+        const double C = kScoreTcRelErr / sqrt((double)HD);
         const int G = D.G;
         const int row = 32 * warp + lane;
         const int ri = row / G, hl = row % G;
@@ -887,6 +895,9 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
             const int i = it.i0 + ri;
             const bool row_ok = i < it.i1 && hl == 0;
             float* sc_row = W.scores + (int64_t)it.g * D.tri_total + P.tri_off[it.s] + (int64_t)i * (i + 1) / 2;
+            const float* kn = W.knorm + (int64_t)it.g * D.NB + it.b0;
+            const double Cq = row_ok ? C * (double)W.qnorm[(int64_t)(it.b0 + i) * D.Hkv + it.g] : 0.0;
+            double m_lo = -DBL_MAX, m_hi = -DBL_MAX;
             bool ok = true;
             for (int c = 0; c < it.n_chunks; ++c, ++an) {
                 const int buf = an & 1;
@@ -913,8 +924,13 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
                             if (jb + e <= i &&
-                                FP2_CHECK(sc_row + jb + e < W.scores + D.Hkv * D.tri_total, P.status))
-                                sc_row[jb + e] = __uint_as_float(r[e]) * inv_sqrt_d;
+                                FP2_CHECK(sc_row + jb + e < W.scores + D.Hkv * D.tri_total, P.status)) {
+                                const float x = __uint_as_float(r[e]) * inv_sqrt_d;
+                                sc_row[jb + e] = x;
+                                const double err = Cq * (double)__ldg(kn + jb + e);
+                                m_lo = fmax(m_lo, (double)x - err);
+                                m_hi = fmax(m_hi, (double)x + err);
+                            }
                     }
                 }
                 tc_fence_before();
@@ -924,6 +940,11 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
             if (!ok) {
                 abort_flag = 1;
                 break;
+            }
+            if (row_ok) {
+                const int64_t r = (int64_t)it.g * D.NB + it.b0 + i;
+                W.bounds[2 * r] = m_lo;
+                W.bounds[2 * r + 1] = m_hi;
             }
         }
     }
@@ -936,25 +957,28 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// float64 score of key block j for row (b_i, g): max over the group's heads
-// (warp-collective).
+// float64 score of a key block for a row: max over the group's G heads of
+// Qbar_h . Kbar / sqrt(d), from the float64 means (warp-collective).
+// qp0: Qbar64 of the row's first head (the G heads follow, HD apart); kp: Kbar64.
+// (Not inlined: it is called from several unrolled loops, and a re-score is
+// rare -- about two per row -- so one out-of-line copy keeps the threshold
+// kernel small.)
 template <int HD>
-__device__ double score64(const Dims& D, const WsPtrs& W, int64_t b_i, int64_t b_j, int g) {
+__device__ __noinline__ double score64(const double* __restrict__ qp0, const double* __restrict__ kp,
+                                       int G) {
     constexpr int E = HD / 32;   // elements per lane
     const int lane = threadIdx.x & 31;
-    const double* kp = W.kbar64 + (b_j * D.Hkv + g) * HD;
-    const double* qp0 = W.qbar64 + (b_i * D.Hq + (int64_t)g * D.G) * HD;
     double kv[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) kv[e] = __ldg(kp + lane + 32 * e);
     double best = -DBL_MAX;
     // four heads at a time: their loads and reductions overlap
-    for (int h0 = 0; h0 < D.G; h0 += 4) {
+    for (int h0 = 0; h0 < G; h0 += 4) {
         double acc[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             acc[u] = 0.0;
-            if (h0 + u < D.G) {
+            if (h0 + u < G) {
                 const double* qp = qp0 + (int64_t)(h0 + u) * HD;
 #pragma unroll
                 for (int e = 0; e < E; ++e) acc[u] = fma(__ldg(qp + lane + 32 * e), kv[e], acc[u]);
@@ -966,7 +990,7 @@ __device__ double score64(const Dims& D, const WsPtrs& W, int64_t b_i, int64_t b
             for (int u = 0; u < 4; ++u) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-            if (h0 + u < D.G) best = fmax(best, acc[u]);
+            if (h0 + u < G) best = fmax(best, acc[u]);
     }
     return best / sqrt((double)HD);
 }
@@ -983,7 +1007,7 @@ __device__ double score64(const Dims& D, const WsPtrs& W, int64_t b_i, int64_t b
 // The loads of a row are issued kThrBatch words (32 blocks each) at a time,
 // so a pass over a row of n blocks waits on about n / (32 kThrBatch) round
 // trips to L2 rather than n / 32.
-constexpr int kThrBatch = 8;
+constexpr int kThrBatch = 4;
 
 // The decision of one row (warp-collective), given the largest lower bound
 // m_lo of its scores: the row maximum in float64 over every block whose upper
@@ -995,6 +1019,7 @@ __device__ __forceinline__ void thr_decide(const Dims& D, const WsPtrs& W, const
                                            const float* kn, double Cq, double m_lo, int i,
                                            int64_t bi, int b0, int g, int lane, uint32_t* mask,
                                            int& count) {
+    const double* q64 = W.qbar64 + (bi * D.Hq + (int64_t)g * D.G) * HD;   // the row's first head
     double m = -DBL_MAX;
 #pragma unroll 1
     for (int jb = 0; jb <= i; jb += 32 * kThrBatch) {
@@ -1003,7 +1028,7 @@ __device__ __forceinline__ void thr_decide(const Dims& D, const WsPtrs& W, const
         for (int u = 0; u < kThrBatch; ++u) {
             const int j = jb + 32 * u + lane;
             xs[u] = j <= i ? __ldg(sc + j) : 0.f;
-            ks[u] = j <= i ? __ldg(kn + (int64_t)j * D.Hkv) : 0.f;
+            ks[u] = j <= i ? __ldg(kn + j) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < kThrBatch; ++u) {
@@ -1012,7 +1037,7 @@ __device__ __forceinline__ void thr_decide(const Dims& D, const WsPtrs& W, const
             while (cb) {
                 const int l = __ffs(cb) - 1;
                 cb &= cb - 1;
-                m = fmax(m, score64<HD>(D, W, bi, b0 + jb + 32 * u + l, g));
+                m = fmax(m, score64<HD>(q64, W.kbar64 + ((int64_t)(b0 + jb + 32 * u + l) * D.Hkv + g) * HD, D.G));
             }
         }
     }
@@ -1024,7 +1049,7 @@ __device__ __forceinline__ void thr_decide(const Dims& D, const WsPtrs& W, const
         for (int u = 0; u < kThrBatch; ++u) {
             const int j = jb + 32 * u + lane;
             xs[u] = j <= i ? __ldg(sc + j) : 0.f;
-            ks[u] = j <= i ? __ldg(kn + (int64_t)j * D.Hkv) : 0.f;
+            ks[u] = j <= i ? __ldg(kn + j) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < kThrBatch; ++u) {
@@ -1045,7 +1070,7 @@ __device__ __forceinline__ void thr_decide(const Dims& D, const WsPtrs& W, const
             while (ub) {
                 const int l = __ffs(ub) - 1;
                 ub &= ub - 1;
-                const double x64 = score64<HD>(D, W, bi, b0 + jb + 32 * u + l, g);
+                const double x64 = score64<HD>(q64, W.kbar64 + ((int64_t)(b0 + jb + 32 * u + l) * D.Hkv + g) * HD, D.G);
                 if (lane == l) keep = x64 >= t;
             }
             const uint32_t bits = __ballot_sync(0xffffffffu, keep);
@@ -1056,8 +1081,78 @@ __device__ __forceinline__ void thr_decide(const Dims& D, const WsPtrs& W, const
     for (int w = i / 32 + 1 + lane; w < D.mask_words; w += 32) mask[w] = 0u;
 }
 
+// One pass over a row of at most 1024 blocks whose score bounds the scorer
+// left in W.bounds: the exact maximum m lies in [m_lo, m_hi], so a block is
+// kept outright when sc - e >= tau m_hi, dropped outright when
+// sc + e < tau m_lo, and otherwise (a few per row, if any) decided once m is
+// known.  Candidates for the maximum (sc + e >= m_lo) are re-scored on the
+// way.  Lane l keeps the undecided bits of mask word l.
+template <int HD>
+__device__ __forceinline__ void thr_one_pass(const Dims& D, const WsPtrs& W, const float* sc,
+                                             const float* kn, double Cq, double m_lo, double m_hi,
+                                             int i, int64_t bi, int b0, int g, int lane, uint32_t* mask,
+                                             int& count) {
+    const double* q64 = W.qbar64 + (bi * D.Hq + (int64_t)g * D.G) * HD;   // the row's first head
+    const double t_lo = D.tau * m_lo, t_hi = D.tau * m_hi;
+    double m = -DBL_MAX;
+    uint32_t my_pending = 0, my_keep = 0;   // of mask word `lane`
+#pragma unroll 1
+    for (int jb = 0; jb <= i; jb += 32 * kThrBatch) {
+        float xs[kThrBatch], ks[kThrBatch];
+#pragma unroll
+        for (int u = 0; u < kThrBatch; ++u) {
+            const int j = jb + 32 * u + lane;
+            xs[u] = j <= i ? __ldg(sc + j) : 0.f;
+            ks[u] = j <= i ? __ldg(kn + j) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kThrBatch; ++u) {
+            if (jb + 32 * u > i) break;
+            const int j = jb + 32 * u + lane;
+            const int w = (jb >> 5) + u;
+            bool keep = false, pend = false, cand = false;
+            if (j <= i) {
+                const double x = (double)xs[u], e = Cq * ks[u];
+                cand = x + e >= m_lo;
+                if (j == 0 || j == i || x - e >= t_hi) keep = true;
+                else if (!(x + e < t_lo)) pend = true;
+            }
+            uint32_t cb = __ballot_sync(0xffffffffu, cand);
+            while (cb) {
+                const int l = __ffs(cb) - 1;
+                cb &= cb - 1;
+                m = fmax(m, score64<HD>(q64, W.kbar64 + ((int64_t)(b0 + 32 * w + l) * D.Hkv + g) * HD, D.G));
+            }
+            const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+            const uint32_t pb = __ballot_sync(0xffffffffu, pend);
+            if (lane == w) {
+                my_keep = kb;
+                my_pending = pb;
+            }
+        }
+    }
+    // the undecided blocks against the exact threshold
+    const double t = D.tau * m;
+    uint32_t any = __ballot_sync(0xffffffffu, my_pending != 0);
+    while (any) {
+        const int w = __ffs(any) - 1;
+        any &= any - 1;
+        uint32_t pb = __shfl_sync(0xffffffffu, my_pending, w);
+        while (pb) {
+            const int l = __ffs(pb) - 1;
+            pb &= pb - 1;
+            const double x64 = score64<HD>(q64, W.kbar64 + ((int64_t)(b0 + 32 * w + l) * D.Hkv + g) * HD, D.G);
+            if (lane == w && x64 >= t) my_keep |= 1u << l;
+        }
+    }
+    if (32 * lane <= i) mask[lane] = my_keep;
+    count += __reduce_add_sync(0xffffffffu, __popc(my_keep));
+    for (int w = i / 32 + 1 + lane; w < D.mask_words; w += 32) mask[w] = 0u;
+}
+
 template <int HD, bool CHUNK>
-__global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W, double rel_err) {
+__global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W, double rel_err,
+                                                   bool have_bounds) {
     // launched as a programmatic dependent: everything before it is complete
     // once the wait returns
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -1084,11 +1179,18 @@ __global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W,
             mask[w] = bits;
         }
         count = i + 1;
+    } else if (have_bounds && i < 32 * 32) {
+        const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
+        const double C = rel_err / sqrt((double)HD);
+        const double qn = W.qnorm[bi * D.Hkv + g];
+        const float* kn = W.knorm + (int64_t)g * D.NB + b0;   // contiguous in j
+        thr_one_pass<HD>(D, W, sc, kn, C * qn, W.bounds[2 * r], W.bounds[2 * r + 1], i, bi, b0, g, lane,
+                         mask, count);
     } else {
         const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
         const double C = rel_err / sqrt((double)HD);
         const double qn = W.qnorm[bi * D.Hkv + g];
-        const float* kn = W.knorm + (int64_t)b0 * D.Hkv + g;
+        const float* kn = W.knorm + (int64_t)g * D.NB + b0;   // contiguous in j
         // largest lower bound of any score (kThrBatch words of loads at a time)
         double m_lo = -DBL_MAX;
 #pragma unroll 1
@@ -1098,7 +1200,7 @@ __global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W,
             for (int u = 0; u < kThrBatch; ++u) {
                 const int j = jb + 32 * u + lane;
                 xs[u] = j <= i ? __ldg(sc + j) : 0.f;
-                ks[u] = j <= i ? __ldg(kn + (int64_t)j * D.Hkv) : 0.f;
+                ks[u] = j <= i ? __ldg(kn + j) : 0.f;
             }
 #pragma unroll
             for (int u = 0; u < kThrBatch; ++u)
@@ -1132,8 +1234,10 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
 constexpr int kQuantMeansThreads = 1024;
 
 __global__ void __launch_bounds__(kQuantMeansThreads) k_quant_means(Dims D, PlanPtrs P) {
-    // the scorer, launched next, may run beside this kernel (it needs nothing
-    // from it) and waits for it before it completes
+    // a programmatic dependent of k_meta (everything before is complete once
+    // the wait returns); the scorer, launched next, may run beside this kernel
+    // (it needs nothing from it) and waits for it before it completes
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (!*P.meta_valid) return;
     const int s = blockIdx.y;
@@ -1303,9 +1407,12 @@ int launch_score(const Dims& D, const PlanPtrs& P, const WsPtrs& W, cudaStream_t
         }
         if (rc != FP2_OK) return rc;
     }
+    // the pipelined scorer leaves each row's score bounds for the threshold
+    const bool bounds = D.tau > 0.0 && D.G <= 32 && (D.G & (D.G - 1)) == 0;
     const dim3 grid((unsigned)((D.R * 32 + 255) / 256));
-    if (P.cu_q) return launch_pdl(k_threshold<HD, true>, grid, dim3(256), 0, st, D, P, W, kScoreTcRelErr);
-    return launch_pdl(k_threshold<HD, false>, grid, dim3(256), 0, st, D, P, W, kScoreTcRelErr);
+    if (P.cu_q)
+        return launch_pdl(k_threshold<HD, true>, grid, dim3(256), 0, st, D, P, W, kScoreTcRelErr, bounds);
+    return launch_pdl(k_threshold<HD, false>, grid, dim3(256), 0, st, D, P, W, kScoreTcRelErr, bounds);
 }
 
 }  // namespace
@@ -1402,8 +1509,9 @@ int launch_plan(const Layout& L, const fp2_problem* p, const void* q, const void
         k_norms<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(D, P, W);
     }
     // e4m3 block means (needs the pool's K/V means only); the scorer runs beside it
-    k_quant_means<<<dim3((unsigned)((D.max_nb + D.B - 1) / D.B), D.n_seqs, D.Hkv), kQuantMeansThreads, 0,
-                    st>>>(D, P);
+    if (launch_pdl(k_quant_means, dim3((unsigned)((D.max_nb + D.B - 1) / D.B), D.n_seqs, D.Hkv),
+                   dim3(kQuantMeansThreads), 0, st, D, P) != FP2_OK)
+        return FP2_ERR_CUDA;
     int rc = D.d == 64 ? launch_score<64>(D, P, W, st) : launch_score<128>(D, P, W, st);
     if (rc != FP2_OK) return rc;
     if (launch_pdl(k_scan, dim3(1), dim3(kScanThreads), 0, st, D, P, W) != FP2_OK ||
