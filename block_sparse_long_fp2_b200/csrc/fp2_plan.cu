@@ -896,8 +896,12 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
             const bool row_ok = i < it.i1 && hl == 0;
             float* sc_row = W.scores + (int64_t)it.g * D.tri_total + P.tri_off[it.s] + (int64_t)i * (i + 1) / 2;
             const float* kn = W.knorm + (int64_t)it.g * D.NB + it.b0;
-            const double Cq = row_ok ? C * (double)W.qnorm[(int64_t)(it.b0 + i) * D.Hkv + it.g] : 0.0;
-            double m_lo = -DBL_MAX, m_hi = -DBL_MAX;
+            // fp32 bound coefficient, rounded up (the bounds below only need to
+            // enclose the float64 ones: they are widened before they are stored)
+            const float Cq = row_ok ? (float)(C * (double)W.qnorm[(int64_t)(it.b0 + i) * D.Hkv + it.g]) *
+                                          (1.0f + 1.0f / 1048576.0f)
+                                    : 0.f;
+            float m_lo = -FLT_MAX, m_hi = -FLT_MAX, e_max = 0.f;
             bool ok = true;
             for (int c = 0; c < it.n_chunks; ++c, ++an) {
                 const int buf = an & 1;
@@ -921,16 +925,21 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
                                                          __shfl_xor_sync(0xffffffffu, __uint_as_float(r[e]), o)));
                     }
                     if (row_ok) {
+                        float lo4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
+                        float hi4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
                             if (jb + e <= i &&
                                 FP2_CHECK(sc_row + jb + e < W.scores + D.Hkv * D.tri_total, P.status)) {
                                 const float x = __uint_as_float(r[e]) * inv_sqrt_d;
                                 sc_row[jb + e] = x;
-                                const double err = Cq * (double)__ldg(kn + jb + e);
-                                m_lo = fmax(m_lo, (double)x - err);
-                                m_hi = fmax(m_hi, (double)x + err);
+                                const float err = Cq * __ldg(kn + jb + e);
+                                e_max = fmaxf(e_max, err);
+                                lo4[e & 3] = fmaxf(lo4[e & 3], x - err);
+                                hi4[e & 3] = fmaxf(hi4[e & 3], x + err);
                             }
+                        m_lo = fmaxf(m_lo, fmaxf(fmaxf(lo4[0], lo4[1]), fmaxf(lo4[2], lo4[3])));
+                        m_hi = fmaxf(m_hi, fmaxf(fmaxf(hi4[0], hi4[1]), fmaxf(hi4[2], hi4[3])));
                     }
                 }
                 tc_fence_before();
@@ -942,9 +951,12 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
                 break;
             }
             if (row_ok) {
+                // widened by far more than the fp32 rounding of the terms above, so
+                // that [m_lo, m_hi] holds the row's float64 maximum
+                const double slack = ((double)fabsf(m_lo) + (double)fabsf(m_hi) + (double)e_max) * 0x1p-18 + 1e-30;
                 const int64_t r = (int64_t)it.g * D.NB + it.b0 + i;
-                W.bounds[2 * r] = m_lo;
-                W.bounds[2 * r + 1] = m_hi;
+                W.bounds[2 * r] = (double)m_lo - slack;
+                W.bounds[2 * r + 1] = (double)m_hi + slack;
             }
         }
     }
