@@ -197,6 +197,8 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     L.off_split_lse = c.take(sizeof(float) * split_rows);
     L.off_slot_item = c.take(sizeof(int32_t) * (size_t)sd.split_slots * d.Hkv);
     L.off_q_off = c.take(sizeof(int32_t) * n);
+    L.off_lb_ticket = c.take(sizeof(int32_t));
+    L.off_lb_flags = c.take(sizeof(unsigned long long) * (size_t)((d.R + kThrRows - 1) / kThrRows));
     pub.plan_bytes = align_up(c.off, 256);
 
     Carver w;
@@ -247,6 +249,8 @@ PlanPtrs plan_ptrs(const Layout& L, void* plan) {
     p.split_lse = reinterpret_cast<float*>(b + L.off_split_lse);
     p.slot_item = reinterpret_cast<int32_t*>(b + L.off_slot_item);
     p.q_off = reinterpret_cast<int32_t*>(b + L.off_q_off);
+    p.lb_ticket = reinterpret_cast<int32_t*>(b + L.off_lb_ticket);
+    p.lb_flags = reinterpret_cast<unsigned long long*>(b + L.off_lb_flags);
     p.cu_q = nullptr;
     return p;
 }

@@ -15,6 +15,8 @@ namespace fp2 {
 
 // Query rows of one PackGQA tile (M of one tcgen05 MMA).
 constexpr int kTileM = 128;
+// CSR rows per CTA of the threshold kernel (one warp per row).
+constexpr int kThrRows = 8;
 // Query vectors scored together by one CTA of the scoring kernel (MMA M).
 constexpr int kScoreQV = 128;
 // Key blocks scored together by one CTA of the scoring kernel (MMA N).
@@ -117,6 +119,10 @@ struct PlanPtrs {
     float* split_lse;      // [Hkv * split_slots, G * B]     its log2-sum-exp
     int32_t* slot_item;    // [Hkv * split_slots]  schedule index of the slot's row (split 0, pair 0)
     int32_t* q_off;        // [n]  position of the first query (L - Q for a chunk, else 0)
+    // the threshold kernel's single-pass CSR prefix sum (decoupled look-back):
+    // a CTA ticket counter and one flag word per CTA, zeroed by k_meta
+    int32_t* lb_ticket;    // [1]
+    unsigned long long* lb_flags;   // [ceil(R / kThrRows)]
     const int32_t* cu_q;   // caller's cu_q_seqlens for a chunked problem, else null (set per call)
 };
 
@@ -143,7 +149,7 @@ struct Layout {
     fp2_plan_layout pub;
     size_t off_meta_valid, off_cu_blocks, off_block_seq, off_tri_off, off_group_cu, off_group_seq,
         off_tile_cu, off_vmax, off_sched, off_sched_cnt, off_sched_off, off_split_o, off_split_lse,
-        off_slot_item, off_q_off;
+        off_slot_item, off_q_off, off_lb_ticket, off_lb_flags;
     size_t ws_qbar64, ws_qbar32, ws_kbar_tf, ws_kbar64, ws_qnorm, ws_knorm, ws_scores, ws_counts,
         ws_bounds;
 };

@@ -3,26 +3,28 @@
 // scores under PackGQA, max-based thresholding and the CSR block index.
 //
 // Kernels, in launch order:
-//   meta     one CTA: checks cu_seqlens (and a chunk's cu_q_seqlens),
-//            derives block / scoring-group maps, the chunk offsets and the
-//            attention kernel's work schedule.
 //   pool     HBM-bound: streams Q, K, V once with 16-byte coalesced loads and
 //            accumulates each block's sum in float64 (exact for bf16 inputs),
-//            writing Qbar (fp64 workspace) and Kbar/Vbar (fp32, bf16, fp64).
-//   norms    |Qbar|, |Kbar| per block and kv-head (for the score error bound).
-//   score    persistent, one CTA per SM over the tiles of the causal
-//            triangles (128 query vectors of a group of query blocks x 128 key
-//            blocks, one kv-head): tf32 tcgen05 MMAs of the means rounded to
-//            tf32 (exact products, fp32 sums), max over the group's heads, to
-//            a scratch array.
+//            writing Qbar (fp64 workspace) and Kbar/Vbar (fp32, bf16, fp64),
+//            and the norms |Qbar|, |Kbar| of the score error bound.  For up to
+//            64 sequences it takes the block map by value and runs first.
+//   meta     one CTA, a programmatic dependent of the pool (it runs beside the
+//            pool's last wave): checks cu_seqlens (and a chunk's
+//            cu_q_seqlens), derives block / scoring-group maps, the chunk
+//            offsets and the attention kernel's work schedule.
+//   (norms   |Qbar|, |Kbar| when the pool cannot: G query heads of a kv-head
+//            not within one pooling CTA.)
+//   quant_means  e4m3 codes of Kbar / Vbar with one scale per pseudo-tile
+//            chunk (used by the FP8 correction).
+//   score    persistent, one CTA per SM, beside quant_means: tf32 tcgen05 MMAs
+//            of the means rounded to tf32 (exact products, fp32 sums), max over
+//            the group's heads, to a scratch array; also each row's bounds of
+//            its largest score.
 //   threshold  one warp per row: the threshold decision.  A block whose
 //            score lies within the scores' error bound of the threshold, and
 //            every candidate for the row maximum, is re-scored in float64, so
-//            the kept set is the one float64 scores give.
-//   scan     row_ptr = exclusive prefix sum of kept counts.
-//   quant_means  e4m3 codes of Kbar / Vbar with one scale per pseudo-tile
-//            chunk (used by the FP8 correction).
-//   compact  col_idx from the kept-block bit masks, ascending per row.
+//            the kept set is the one float64 scores give; the CSR row pointers
+//            by a decoupled look-back over the rows before, then the column ids.
 #include <cfloat>
 #include <cstring>
 #include <cmath>
@@ -194,7 +196,13 @@ __global__ void __launch_bounds__(kMetaThreads, 1) k_meta(Dims D, SchedDims S, c
         s_valid = valid;
     }
     __syncthreads();
-    if (s_valid) meta_maps(D, S, cu_seqlens, page_table, P);
+    if (s_valid) {
+        // the threshold kernel's look-back state starts from zero
+        const int64_t n_lb = (D.R + kThrRows - 1) / kThrRows;
+        for (int64_t c = threadIdx.x; c < n_lb; c += blockDim.x) P.lb_flags[c] = 0ull;
+        if (threadIdx.x == 0) *P.lb_ticket = 0;
+        meta_maps(D, S, cu_seqlens, page_table, P);
+    }
     // k_meta may run beside the pooling kernel launched before it (which
     // needs none of its outputs); it completes only after that kernel, so
     // the kernels after it see both
@@ -761,7 +769,7 @@ __device__ __forceinline__ ScoreItem score_item(const Dims& D, const PlanPtrs& P
     return it;
 }
 
-template <int HD>
+template <int HD, int GQ>
 __global__ void __launch_bounds__(kScorePThreads, 1)
 k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap tm_q,
              const __grid_constant__ CUtensorMap tm_k) {
@@ -885,7 +893,7 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
         // first pass, done here while the scores are in registers)
         const float inv_sqrt_d = 1.0f / sqrtf((float)HD);
         const double C = kScoreTcRelErr / sqrt((double)HD);
-        const int G = D.G;
+        constexpr int G = GQ;   // query heads per kv-head (a power of two, at most 32)
         const int row = 32 * warp + lane;
         const int ri = row / G, hl = row % G;
         uint32_t an = 0;
@@ -893,7 +901,8 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
             const ScoreItem it = score_item(D, P, w, n_groups);
             if (it.n_chunks == 0) continue;
             const int i = it.i0 + ri;
-            const bool row_ok = i < it.i1 && hl == 0;
+            // the G lanes of a block share its columns: lane hl takes columns hl, hl + G, ...
+            const bool row_ok = i < it.i1;
             float* sc_row = W.scores + (int64_t)it.g * D.tri_total + P.tri_off[it.s] + (int64_t)i * (i + 1) / 2;
             const float* kn = W.knorm + (int64_t)it.g * D.NB + it.b0;
             // fp32 bound coefficient, rounded up (the bounds below only need to
@@ -918,6 +927,7 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
                     const int jb = kScoreKeys * c + 32 * cc;
                     // max over the G heads (adjacent lanes), 32 columns at a time so
                     // the shuffles of different columns overlap
+#pragma unroll
                     for (int o = 1; o < G; o <<= 1) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
@@ -928,16 +938,21 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
                         float lo4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
                         float hi4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (jb + e <= i &&
-                                FP2_CHECK(sc_row + jb + e < W.scores + D.Hkv * D.tri_total, P.status)) {
-                                const float x = __uint_as_float(r[e]) * inv_sqrt_d;
-                                sc_row[jb + e] = x;
-                                const float err = Cq * __ldg(kn + jb + e);
+                        for (int e0 = 0; e0 < 32; e0 += G) {
+                            // this lane's column of the G columns e0 .. e0 + G - 1
+                            uint32_t v = r[e0];
+#pragma unroll
+                            for (int u = 1; u < G; ++u) v = hl == u ? r[e0 + u] : v;
+                            const int col = jb + e0 + hl;
+                            if (col <= i && FP2_CHECK(sc_row + col < W.scores + D.Hkv * D.tri_total, P.status)) {
+                                const float x = __uint_as_float(v) * inv_sqrt_d;
+                                sc_row[col] = x;
+                                const float err = Cq * __ldg(kn + col);
                                 e_max = fmaxf(e_max, err);
-                                lo4[e & 3] = fmaxf(lo4[e & 3], x - err);
-                                hi4[e & 3] = fmaxf(hi4[e & 3], x + err);
+                                lo4[(e0 / G) & 3] = fmaxf(lo4[(e0 / G) & 3], x - err);
+                                hi4[(e0 / G) & 3] = fmaxf(hi4[(e0 / G) & 3], x + err);
                             }
+                        }
                         m_lo = fmaxf(m_lo, fmaxf(fmaxf(lo4[0], lo4[1]), fmaxf(lo4[2], lo4[3])));
                         m_hi = fmaxf(m_hi, fmaxf(fmaxf(hi4[0], hi4[1]), fmaxf(hi4[2], hi4[3])));
                     }
@@ -950,7 +965,14 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
                 abort_flag = 1;
                 break;
             }
-            if (row_ok) {
+            // the row's bounds over its G lanes' columns
+#pragma unroll
+            for (int o = 1; o < G; o <<= 1) {
+                m_lo = fmaxf(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o));
+                m_hi = fmaxf(m_hi, __shfl_xor_sync(0xffffffffu, m_hi, o));
+                e_max = fmaxf(e_max, __shfl_xor_sync(0xffffffffu, e_max, o));
+            }
+            if (row_ok && hl == 0) {
                 // widened by far more than the fp32 rounding of the terms above, so
                 // that [m_lo, m_hi] holds the row's float64 maximum
                 const double slack = ((double)fabsf(m_lo) + (double)fabsf(m_hi) + (double)e_max) * 0x1p-18 + 1e-30;
@@ -1162,67 +1184,142 @@ __device__ __forceinline__ void thr_one_pass(const Dims& D, const WsPtrs& W, con
     for (int w = i / 32 + 1 + lane; w < D.mask_words; w += 32) mask[w] = 0u;
 }
 
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Look-back flag words: the value in the low 62 bits, the kind in the top two.
+constexpr unsigned long long kLbAggregate = 1ull << 62;   // this CTA's rows only
+constexpr unsigned long long kLbPrefix = 2ull << 62;      // every row up to this CTA's last
+constexpr unsigned long long kLbValue = (1ull << 62) - 1;
+
+// The threshold, the CSR row pointers and the CSR column ids in one pass: one
+// warp per row decides its blocks (kept-mask words), the CTA's kThrRows rows
+// find their offset among all rows by a decoupled look-back over the CTAs
+// before them (a CTA takes its rows by a ticket, so every CTA it waits for
+// is running or done), then each warp writes its row's column ids.
 template <int HD, bool CHUNK>
-__global__ void __launch_bounds__(256) k_threshold(Dims D, PlanPtrs P, WsPtrs W, double rel_err,
-                                                   bool have_bounds) {
+__global__ void __launch_bounds__(kThrRows * 32) k_threshold(Dims D, PlanPtrs P, WsPtrs W, double rel_err,
+                                                             bool have_bounds) {
     // launched as a programmatic dependent: everything before it is complete
     // once the wait returns
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (!*P.meta_valid) return;
-    const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    __shared__ int s_ticket;
+    __shared__ int s_count[kThrRows];
+    __shared__ long long s_base;
+    if (threadIdx.x == 0) s_ticket = atomicAdd(P.lb_ticket, 1);
+    __syncthreads();
+    const int64_t cta = s_ticket;
+    const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    if (r >= D.R) return;
-    const int g = (int)(r / D.NB);
-    const int64_t bi = r % D.NB;
-    const int s = P.block_seq[bi];
-    const int b0 = P.cu_blocks[s];
-    const int i = (int)(bi - b0);
-    uint32_t* mask = P.kept_mask + r * D.mask_words;
-    int count = 0;
-    if (CHUNK && i < P.q_off[s] / D.B) {
-        // query block below a chunk: no row, nothing kept
-        for (int w = lane; w < D.mask_words; w += 32) mask[w] = 0u;
-    } else if (D.tau == 0.0) {
-        for (int w = lane; w < D.mask_words; w += 32) {
-            uint32_t bits = 0;
-            if (32 * w + 31 <= i) bits = 0xFFFFFFFFu;
-            else if (32 * w <= i) bits = (1u << (i - 32 * w + 1)) - 1u;
-            mask[w] = bits;
-        }
-        count = i + 1;
-    } else if (have_bounds && i < 32 * 32) {
-        const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
-        const double C = rel_err / sqrt((double)HD);
-        const double qn = W.qnorm[bi * D.Hkv + g];
-        const float* kn = W.knorm + (int64_t)g * D.NB + b0;   // contiguous in j
-        thr_one_pass<HD>(D, W, sc, kn, C * qn, W.bounds[2 * r], W.bounds[2 * r + 1], i, bi, b0, g, lane,
-                         mask, count);
-    } else {
-        const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
-        const double C = rel_err / sqrt((double)HD);
-        const double qn = W.qnorm[bi * D.Hkv + g];
-        const float* kn = W.knorm + (int64_t)g * D.NB + b0;   // contiguous in j
-        // largest lower bound of any score (kThrBatch words of loads at a time)
-        double m_lo = -DBL_MAX;
+    const int64_t r = cta * kThrRows + warp;
+    const bool have_row = r < D.R;
+    int count = 0, i = -1;
+    uint32_t* mask = nullptr;
+    if (have_row) {
+        const int g = (int)(r / D.NB);
+        const int64_t bi = r % D.NB;
+        const int s = P.block_seq[bi];
+        const int b0 = P.cu_blocks[s];
+        i = (int)(bi - b0);
+        mask = P.kept_mask + r * D.mask_words;
+        if (CHUNK && i < P.q_off[s] / D.B) {
+            // query block below a chunk: no row, nothing kept
+            for (int w = lane; w < D.mask_words; w += 32) mask[w] = 0u;
+            i = -1;
+        } else if (D.tau == 0.0) {
+            for (int w = lane; w < D.mask_words; w += 32) {
+                uint32_t bits = 0;
+                if (32 * w + 31 <= i) bits = 0xFFFFFFFFu;
+                else if (32 * w <= i) bits = (1u << (i - 32 * w + 1)) - 1u;
+                mask[w] = bits;
+            }
+            count = i + 1;
+        } else if (have_bounds && i < 32 * 32) {
+            const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
+            const double C = rel_err / sqrt((double)HD);
+            const double qn = W.qnorm[bi * D.Hkv + g];
+            const float* kn = W.knorm + (int64_t)g * D.NB + b0;   // contiguous in j
+            thr_one_pass<HD>(D, W, sc, kn, C * qn, W.bounds[2 * r], W.bounds[2 * r + 1], i, bi, b0, g,
+                             lane, mask, count);
+        } else {
+            const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
+            const double C = rel_err / sqrt((double)HD);
+            const double qn = W.qnorm[bi * D.Hkv + g];
+            const float* kn = W.knorm + (int64_t)g * D.NB + b0;   // contiguous in j
+            // largest lower bound of any score (kThrBatch words of loads at a time)
+            double m_lo = -DBL_MAX;
 #pragma unroll 1
-        for (int jb = 0; jb <= i; jb += 32 * kThrBatch) {
-            float xs[kThrBatch], ks[kThrBatch];
+            for (int jb = 0; jb <= i; jb += 32 * kThrBatch) {
+                float xs[kThrBatch], ks[kThrBatch];
 #pragma unroll
-            for (int u = 0; u < kThrBatch; ++u) {
-                const int j = jb + 32 * u + lane;
-                xs[u] = j <= i ? __ldg(sc + j) : 0.f;
-                ks[u] = j <= i ? __ldg(kn + j) : 0.f;
+                for (int u = 0; u < kThrBatch; ++u) {
+                    const int j = jb + 32 * u + lane;
+                    xs[u] = j <= i ? __ldg(sc + j) : 0.f;
+                    ks[u] = j <= i ? __ldg(kn + j) : 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < kThrBatch; ++u)
+                    if (jb + 32 * u + lane <= i) m_lo = fmax(m_lo, (double)xs[u] - C * qn * ks[u]);
             }
 #pragma unroll
-            for (int u = 0; u < kThrBatch; ++u)
-                if (jb + 32 * u + lane <= i) m_lo = fmax(m_lo, (double)xs[u] - C * qn * ks[u]);
+            for (int o = 16; o > 0; o >>= 1) m_lo = fmax(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o));
+            thr_decide<HD>(D, W, sc, kn, C * qn, m_lo, i, bi, b0, g, lane, mask, count);
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m_lo = fmax(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o));
-        thr_decide<HD>(D, W, sc, kn, C * qn, m_lo, i, bi, b0, g, lane, mask, count);
     }
-    if (lane == 0) W.counts[r] = count;
+    if (lane == 0) s_count[warp] = count;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        long long agg = 0;
+        for (int w = 0; w < kThrRows; ++w) agg += s_count[w];
+        long long excl = 0;
+        if (cta == 0) {
+            st_release_u64(P.lb_flags, kLbPrefix | (unsigned long long)agg);
+        } else {
+            st_release_u64(P.lb_flags + cta, kLbAggregate | (unsigned long long)agg);
+            // add the CTAs before this one until one that holds its prefix
+            int64_t p = cta - 1;
+            const uint64_t t0 = global_timer_ns();
+            while (p >= 0) {
+                const unsigned long long f = ld_acquire_u64(P.lb_flags + p);
+                if (f == 0ull) {
+                    if (global_timer_ns() - t0 > kWaitLimitNs) {   // never: the CTAs before are running
+                        atomicOr(P.status, (int32_t)FP2_STATUS_TIMEOUT);
+                        break;
+                    }
+                    continue;
+                }
+                excl += (long long)(f & kLbValue);
+                if (f & kLbPrefix) break;
+                --p;
+            }
+            st_release_u64(P.lb_flags + cta, kLbPrefix | (unsigned long long)(excl + agg));
+        }
+        s_base = excl;
+    }
+    __syncthreads();
+    if (have_row) {
+        long long base = s_base;
+        for (int w = 0; w < warp; ++w) base += s_count[w];
+        if (lane == 0) P.row_ptr[r] = (int32_t)base;
+        if (r == D.R - 1 && lane == 0) P.row_ptr[D.R] = (int32_t)(base + count);
+        // column ids from the mask words this warp wrote, ascending
+        __syncwarp();
+        int32_t at0 = (int32_t)base;
+        for (int w = 0; 32 * w <= i; ++w) {
+            const uint32_t bits = mask[w];
+            const int32_t at = at0 + __popc(bits & ((1u << lane) - 1u));
+            if (((bits >> lane) & 1u) && FP2_CHECK(at >= 0 && at < D.nnz_cap, P.status))
+                P.col_idx[at] = 32 * w + lane;
+            at0 += __popc(bits);
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1312,57 +1409,6 @@ __global__ void __launch_bounds__(kQuantMeansThreads) k_quant_means(Dims D, Plan
     }
 }
 
-// ---------------------------------------------------------------------------
-// scan: row_ptr = exclusive prefix sum of counts (one CTA)
-// ---------------------------------------------------------------------------
-
-constexpr int kScanThreads = 1024;
-
-__global__ void __launch_bounds__(kScanThreads) k_scan(Dims D, PlanPtrs P, WsPtrs W) {
-    asm volatile("griddepcontrol.wait;" ::: "memory");   // (a programmatic dependent)
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (!*P.meta_valid) return;
-    static_assert(kScanThreads == kMetaThreads, "block_excl_scan is sized for kMetaThreads");
-    const int64_t R = D.R;
-    const int64_t per = (R + kScanThreads - 1) / kScanThreads;
-    const int64_t lo = R < (int64_t)threadIdx.x * per ? R : (int64_t)threadIdx.x * per;
-    const int64_t hi = R < lo + per ? R : lo + per;
-    int64_t sum = 0;
-#pragma unroll 4
-    for (int64_t r = lo; r < hi; ++r) sum += W.counts[r];
-    int64_t total;
-    int64_t run = block_excl_scan(sum, &total);
-    for (int64_t r = lo; r < hi; ++r) {
-        P.row_ptr[r] = (int32_t)run;
-        run += W.counts[r];
-    }
-    if (threadIdx.x == 0) P.row_ptr[R] = (int32_t)total;
-}
-
-// ---------------------------------------------------------------------------
-// compact: one warp per row writes its kept block ids in ascending order
-// ---------------------------------------------------------------------------
-
-__global__ void k_compact(Dims D, PlanPtrs P) {
-    asm volatile("griddepcontrol.wait;" ::: "memory");   // (a programmatic dependent)
-    if (!*P.meta_valid) return;
-    const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (r >= D.R) return;
-    const int64_t b = r % D.NB;
-    const int s = P.block_seq[b];
-    const int i = (int)(b - P.cu_blocks[s]);
-    const uint32_t* mask = P.kept_mask + r * D.mask_words;
-    int32_t base = P.row_ptr[r];
-    for (int w = 0; 32 * w <= i; ++w) {
-        const uint32_t bits = mask[w];
-        const int32_t at = base + __popc(bits & ((1u << lane) - 1u));
-        if (((bits >> lane) & 1u) && FP2_CHECK(at >= 0 && at < D.nnz_cap, P.status))
-            P.col_idx[at] = 32 * w + lane;
-        base += __popc(bits);
-    }
-}
-
 // Launch with programmatic stream serialization: the kernel may begin before
 // the one before it in the stream completes; what it may read before its
 // griddepcontrol.wait is stated at each kernel.
@@ -1380,6 +1426,17 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? FP2_OK : FP2_ERR_CUDA;
+}
+
+template <int HD, int GQ>
+int launch_score_pipe(const Dims& D, const PlanPtrs& P, const WsPtrs& W, const CUtensorMap& tq,
+                      const CUtensorMap& tk, int grid, cudaStream_t st) {
+    const int smem = ScorePCfg<HD>::kSmem;
+    if (cudaFuncSetAttribute(k_score_pipe<HD, GQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+        return FP2_ERR_CUDA;
+    return launch_pdl(k_score_pipe<HD, GQ>, dim3(grid), dim3(kScorePThreads), (size_t)smem, st, D, P, W,
+                      tq, tk);
 }
 
 // Scores (tau > 0; launched right after k_quant_means, beside which it runs)
@@ -1401,13 +1458,16 @@ int launch_score(const Dims& D, const PlanPtrs& P, const WsPtrs& W, cudaStream_t
         int rc;
         if (D.G <= 32 && (D.G & (D.G - 1)) == 0) {
             // the G heads of a block are G aligned, adjacent lanes of one warp
-            const int smem = ScorePCfg<HD>::kSmem;
-            if (cudaFuncSetAttribute(k_score_pipe<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     smem) != cudaSuccess)
-                return FP2_ERR_CUDA;
             const int64_t items = (int64_t)D.n_groups_cap * D.Hkv;
             const int grid = (int)std::min<int64_t>(items, std::max(1, sm_count()));
-            rc = launch_pdl(k_score_pipe<HD>, dim3(grid), dim3(kScorePThreads), smem, st, D, P, W, tq, tk);
+            switch (D.G) {
+                case 1: rc = launch_score_pipe<HD, 1>(D, P, W, tq, tk, grid, st); break;
+                case 2: rc = launch_score_pipe<HD, 2>(D, P, W, tq, tk, grid, st); break;
+                case 4: rc = launch_score_pipe<HD, 4>(D, P, W, tq, tk, grid, st); break;
+                case 8: rc = launch_score_pipe<HD, 8>(D, P, W, tq, tk, grid, st); break;
+                case 16: rc = launch_score_pipe<HD, 16>(D, P, W, tq, tk, grid, st); break;
+                default: rc = launch_score_pipe<HD, 32>(D, P, W, tq, tk, grid, st); break;
+            }
         } else {
             const int smem = ScoreTcCfg<HD>::kSmem;
             if (cudaFuncSetAttribute(k_score_tc<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1421,10 +1481,12 @@ int launch_score(const Dims& D, const PlanPtrs& P, const WsPtrs& W, cudaStream_t
     }
     // the pipelined scorer leaves each row's score bounds for the threshold
     const bool bounds = D.tau > 0.0 && D.G <= 32 && (D.G & (D.G - 1)) == 0;
-    const dim3 grid((unsigned)((D.R * 32 + 255) / 256));
+    const dim3 grid((unsigned)((D.R + kThrRows - 1) / kThrRows));
     if (P.cu_q)
-        return launch_pdl(k_threshold<HD, true>, grid, dim3(256), 0, st, D, P, W, kScoreTcRelErr, bounds);
-    return launch_pdl(k_threshold<HD, false>, grid, dim3(256), 0, st, D, P, W, kScoreTcRelErr, bounds);
+        return launch_pdl(k_threshold<HD, true>, grid, dim3(kThrRows * 32), 0, st, D, P, W, kScoreTcRelErr,
+                          bounds);
+    return launch_pdl(k_threshold<HD, false>, grid, dim3(kThrRows * 32), 0, st, D, P, W, kScoreTcRelErr,
+                      bounds);
 }
 
 }  // namespace
@@ -1526,9 +1588,6 @@ int launch_plan(const Layout& L, const fp2_problem* p, const void* q, const void
         return FP2_ERR_CUDA;
     int rc = D.d == 64 ? launch_score<64>(D, P, W, st) : launch_score<128>(D, P, W, st);
     if (rc != FP2_OK) return rc;
-    if (launch_pdl(k_scan, dim3(1), dim3(kScanThreads), 0, st, D, P, W) != FP2_OK ||
-        launch_pdl(k_compact, dim3((unsigned)((D.R * 32 + 255) / 256)), dim3(256), 0, st, D, P) != FP2_OK)
-        return FP2_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? FP2_OK : FP2_ERR_CUDA;
 }
 
