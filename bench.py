@@ -62,12 +62,12 @@ def kept_tile_flop(wl) -> float:
 
 
 def plan_launches(wl, tau=None) -> int:
-    """Kernels fp2_plan launches: pool, meta, e4m3 means and threshold (with the
-    CSR); with tau > 0 the scorer, and the separate norms kernel when the G
-    query heads of a kv-head do not fall into one pooling CTA (1024 columns)."""
+    """Kernels fp2_plan launches: pool, meta, e4m3 means, threshold and CSR;
+    with tau > 0 the scorer, and the separate norms kernel when the G query
+    heads of a kv-head do not fall into one pooling CTA (1024 columns)."""
     tau = wl.tau if tau is None else tau
     G = wl.Hq // wl.Hkv
-    return 4 + (1 if tau > 0 else 0) + (1 if tau > 0 and 1024 % (G * wl.d) != 0 else 0)
+    return 5 + (1 if tau > 0 else 0) + (1 if tau > 0 and 1024 % (G * wl.d) != 0 else 0)
 
 
 def rank_slice(wl, world: int, rank: int):

@@ -197,8 +197,8 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     L.off_split_lse = c.take(sizeof(float) * split_rows);
     L.off_slot_item = c.take(sizeof(int32_t) * (size_t)sd.split_slots * d.Hkv);
     L.off_q_off = c.take(sizeof(int32_t) * n);
-    L.off_lb_ticket = c.take(sizeof(int32_t));
-    L.off_lb_flags = c.take(sizeof(unsigned long long) * (size_t)((d.R + kThrRows - 1) / kThrRows));
+    L.off_lb_ticket = c.take(2 * sizeof(int32_t));
+    L.off_lb_flags = c.take(sizeof(unsigned long long) * (size_t)((d.R + kCsrRows - 1) / kCsrRows));
     pub.plan_bytes = align_up(c.off, 256);
 
     Carver w;

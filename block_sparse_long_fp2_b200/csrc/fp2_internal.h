@@ -16,7 +16,8 @@ namespace fp2 {
 // Query rows of one PackGQA tile (M of one tcgen05 MMA).
 constexpr int kTileM = 128;
 // CSR rows per CTA of the threshold kernel (one warp per row).
-constexpr int kThrRows = 8;
+constexpr int kThrRows = 8;    // threshold: warps (rows in flight) per CTA
+constexpr int kCsrRows = 32;   // CSR: rows per CTA, one warp each
 // Query vectors scored together by one CTA of the scoring kernel (MMA M).
 constexpr int kScoreQV = 128;
 // Key blocks scored together by one CTA of the scoring kernel (MMA N).
@@ -121,8 +122,8 @@ struct PlanPtrs {
     int32_t* q_off;        // [n]  position of the first query (L - Q for a chunk, else 0)
     // the threshold kernel's single-pass CSR prefix sum (decoupled look-back):
     // a CTA ticket counter and one flag word per CTA, zeroed by k_meta
-    int32_t* lb_ticket;    // [1]
-    unsigned long long* lb_flags;   // [ceil(R / kThrRows)]
+    int32_t* lb_ticket;    // [2]: the threshold's next row, the CSR kernel's next CTA
+    unsigned long long* lb_flags;   // [ceil(R / kCsrRows)]
     const int32_t* cu_q;   // caller's cu_q_seqlens for a chunked problem, else null (set per call)
 };
 

@@ -20,11 +20,13 @@
 //            of the means rounded to tf32 (exact products, fp32 sums), max over
 //            the group's heads, to a scratch array; also each row's bounds of
 //            its largest score.
-//   threshold  one warp per row: the threshold decision.  A block whose
-//            score lies within the scores' error bound of the threshold, and
-//            every candidate for the row maximum, is re-scored in float64, so
-//            the kept set is the one float64 scores give; the CSR row pointers
-//            by a decoupled look-back over the rows before, then the column ids.
+//   threshold  one warp per row, rows taken longest first: the threshold
+//            decision.  A block whose score lies within the scores' error
+//            bound of the threshold, and every candidate for the row maximum,
+//            is re-scored in float64, so the kept set is the one float64
+//            scores give.
+//   csr      the CSR row pointers by a decoupled look-back over the rows
+//            before, then the column ids.
 #include <cfloat>
 #include <cstring>
 #include <cmath>
@@ -197,10 +199,10 @@ __global__ void __launch_bounds__(kMetaThreads, 1) k_meta(Dims D, SchedDims S, c
     }
     __syncthreads();
     if (s_valid) {
-        // the threshold kernel's look-back state starts from zero
-        const int64_t n_lb = (D.R + kThrRows - 1) / kThrRows;
+        // the threshold's row counter and the CSR kernel's look-back state start from zero
+        const int64_t n_lb = (D.R + kCsrRows - 1) / kCsrRows;
         for (int64_t c = threadIdx.x; c < n_lb; c += blockDim.x) P.lb_flags[c] = 0ull;
-        if (threadIdx.x == 0) *P.lb_ticket = 0;
+        if (threadIdx.x < 2) P.lb_ticket[threadIdx.x] = 0;
         meta_maps(D, S, cu_seqlens, page_table, P);
     }
     // k_meta may run beside the pooling kernel launched before it (which
@@ -1198,61 +1200,38 @@ constexpr unsigned long long kLbAggregate = 1ull << 62;   // this CTA's rows onl
 constexpr unsigned long long kLbPrefix = 2ull << 62;      // every row up to this CTA's last
 constexpr unsigned long long kLbValue = (1ull << 62) - 1;
 
-// The threshold, the CSR row pointers and the CSR column ids in one pass: one
-// warp per row decides its blocks (kept-mask words), the CTA's kThrRows rows
-// find their offset among all rows by a decoupled look-back over the CTAs
-// before them (a CTA takes its rows by a ticket, so every CTA it waits for
-// is running or done), then each warp writes its row's column ids.
+// The decision of row r (warp-collective): writes its kept-mask words and
+// returns its kept count.
 template <int HD, bool CHUNK>
-__global__ void __launch_bounds__(kThrRows * 32) k_threshold(Dims D, PlanPtrs P, WsPtrs W, double rel_err,
-                                                             bool have_bounds) {
-    // launched as a programmatic dependent: everything before it is complete
-    // once the wait returns
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (!*P.meta_valid) return;
-    __shared__ int s_ticket;
-    __shared__ int s_count[kThrRows];
-    __shared__ long long s_base;
-    if (threadIdx.x == 0) s_ticket = atomicAdd(P.lb_ticket, 1);
-    __syncthreads();
-    const int64_t cta = s_ticket;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int64_t r = cta * kThrRows + warp;
-    const bool have_row = r < D.R;
-    int count = 0, i = -1;
-    uint32_t* mask = nullptr;
-    if (have_row) {
-        const int g = (int)(r / D.NB);
-        const int64_t bi = r % D.NB;
-        const int s = P.block_seq[bi];
-        const int b0 = P.cu_blocks[s];
-        i = (int)(bi - b0);
-        mask = P.kept_mask + r * D.mask_words;
-        if (CHUNK && i < P.q_off[s] / D.B) {
-            // query block below a chunk: no row, nothing kept
-            for (int w = lane; w < D.mask_words; w += 32) mask[w] = 0u;
-            i = -1;
-        } else if (D.tau == 0.0) {
-            for (int w = lane; w < D.mask_words; w += 32) {
-                uint32_t bits = 0;
-                if (32 * w + 31 <= i) bits = 0xFFFFFFFFu;
-                else if (32 * w <= i) bits = (1u << (i - 32 * w + 1)) - 1u;
-                mask[w] = bits;
-            }
-            count = i + 1;
-        } else if (have_bounds && i < 32 * 32) {
-            const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
-            const double C = rel_err / sqrt((double)HD);
-            const double qn = W.qnorm[bi * D.Hkv + g];
-            const float* kn = W.knorm + (int64_t)g * D.NB + b0;   // contiguous in j
+__device__ __forceinline__ int thr_row(const Dims& D, const PlanPtrs& P, const WsPtrs& W, int64_t r,
+                                       int lane, double rel_err, bool have_bounds) {
+    const int g = (int)(r / D.NB);
+    const int64_t bi = r % D.NB;
+    const int s = P.block_seq[bi];
+    const int b0 = P.cu_blocks[s];
+    const int i = (int)(bi - b0);
+    uint32_t* mask = P.kept_mask + r * D.mask_words;
+    int count = 0;
+    if (CHUNK && i < P.q_off[s] / D.B) {
+        // query block below a chunk: no row, nothing kept
+        for (int w = lane; w < D.mask_words; w += 32) mask[w] = 0u;
+    } else if (D.tau == 0.0) {
+        for (int w = lane; w < D.mask_words; w += 32) {
+            uint32_t bits = 0;
+            if (32 * w + 31 <= i) bits = 0xFFFFFFFFu;
+            else if (32 * w <= i) bits = (1u << (i - 32 * w + 1)) - 1u;
+            mask[w] = bits;
+        }
+        count = i + 1;
+    } else {
+        const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
+        const double C = rel_err / sqrt((double)HD);
+        const double qn = W.qnorm[bi * D.Hkv + g];
+        const float* kn = W.knorm + (int64_t)g * D.NB + b0;   // contiguous in j
+        if (have_bounds && i < 32 * 32) {
             thr_one_pass<HD>(D, W, sc, kn, C * qn, W.bounds[2 * r], W.bounds[2 * r + 1], i, bi, b0, g,
                              lane, mask, count);
         } else {
-            const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
-            const double C = rel_err / sqrt((double)HD);
-            const double qn = W.qnorm[bi * D.Hkv + g];
-            const float* kn = W.knorm + (int64_t)g * D.NB + b0;   // contiguous in j
             // largest lower bound of any score (kThrBatch words of loads at a time)
             double m_lo = -DBL_MAX;
 #pragma unroll 1
@@ -1273,52 +1252,127 @@ __global__ void __launch_bounds__(kThrRows * 32) k_threshold(Dims D, PlanPtrs P,
             thr_decide<HD>(D, W, sc, kn, C * qn, m_lo, i, bi, b0, g, lane, mask, count);
         }
     }
+    return count;
+}
+
+// The threshold: each warp takes rows one at a time from a shared counter,
+// longest first (block index from the last down, every kv-head of a block
+// together), decides them and leaves the kept count in row_ptr[r];
+// k_csr turns the counts into offsets and writes the column ids.
+template <int HD, bool CHUNK>
+__global__ void __launch_bounds__(kThrRows * 32, 3) k_threshold(Dims D, PlanPtrs P, WsPtrs W, double rel_err,
+                                                             bool have_bounds) {
+    // launched as a programmatic dependent: everything before it is complete
+    // once the wait returns
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // k_csr may be launched now: it waits for this kernel to complete
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (!*P.meta_valid) return;
+    const int lane = threadIdx.x & 31;
+    for (;;) {
+        int t = 0;
+        if (lane == 0) t = atomicAdd(P.lb_ticket, 1);
+        t = __shfl_sync(0xffffffffu, t, 0);
+        if (t >= D.R) break;
+        const int64_t bi = D.NB - 1 - t / D.Hkv;
+        const int64_t r = (int64_t)(t % D.Hkv) * D.NB + bi;
+        const int count = thr_row<HD, CHUNK>(D, P, W, r, lane, rel_err, have_bounds);
+        if (lane == 0) P.row_ptr[r] = count;
+    }
+}
+
+// Sum over the lanes of a warp.
+__device__ __forceinline__ long long warp_sum_ll(long long v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// The CSR from the kept counts and mask words: CTA c (taken by a ticket, so
+// every CTA it waits for is running or done) holds rows kCsrRows c ..
+// kCsrRows (c + 1) - 1, one warp each.  The CTA's offset among all rows comes
+// from a decoupled look-back (warp 0 reads the flags of the 32 CTAs before the
+// window's top at once, and sums back to the nearest that holds its prefix);
+// then each warp writes its row's column ids, ascending.
+__global__ void __launch_bounds__(kCsrRows * 32) k_csr(Dims D, PlanPtrs P) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (!*P.meta_valid) return;
+    __shared__ int s_ticket;
+    __shared__ int s_count[kCsrRows];
+    __shared__ long long s_base;
+    if (threadIdx.x == 0) s_ticket = atomicAdd(P.lb_ticket + 1, 1);
+    __syncthreads();
+    const int64_t cta = s_ticket;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t r = cta * kCsrRows + warp;
+    const bool have_row = r < D.R;
+    const int count = have_row ? P.row_ptr[r] : 0;
     if (lane == 0) s_count[warp] = count;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        long long agg = 0;
-        for (int w = 0; w < kThrRows; ++w) agg += s_count[w];
+    if (warp == 0) {
+        const long long agg = warp_sum_ll(lane < kCsrRows ? s_count[lane] : 0);
         long long excl = 0;
         if (cta == 0) {
-            st_release_u64(P.lb_flags, kLbPrefix | (unsigned long long)agg);
+            if (lane == 0) st_release_u64(P.lb_flags, kLbPrefix | (unsigned long long)agg);
         } else {
-            st_release_u64(P.lb_flags + cta, kLbAggregate | (unsigned long long)agg);
-            // add the CTAs before this one until one that holds its prefix
-            int64_t p = cta - 1;
+            if (lane == 0) st_release_u64(P.lb_flags + cta, kLbAggregate | (unsigned long long)agg);
+            int64_t top = cta - 1;   // the window is CTAs top, top - 1, .. top - 31
             const uint64_t t0 = global_timer_ns();
-            while (p >= 0) {
-                const unsigned long long f = ld_acquire_u64(P.lb_flags + p);
-                if (f == 0ull) {
-                    if (global_timer_ns() - t0 > kWaitLimitNs) {   // never: the CTAs before are running
-                        atomicOr(P.status, (int32_t)FP2_STATUS_TIMEOUT);
+            for (;;) {
+                const int64_t p = top - lane;
+                // before CTA 0: an empty prefix
+                const unsigned long long f = p >= 0 ? ld_acquire_u64(P.lb_flags + p) : kLbPrefix;
+                if (__any_sync(0xffffffffu, f == 0ull)) {
+                    // (never: the CTAs before are running; the vote keeps the warp together)
+                    if (__any_sync(0xffffffffu, global_timer_ns() - t0 > kWaitLimitNs)) {
+                        if (lane == 0) atomicOr(P.status, (int32_t)FP2_STATUS_TIMEOUT);
                         break;
                     }
                     continue;
                 }
-                excl += (long long)(f & kLbValue);
-                if (f & kLbPrefix) break;
-                --p;
+                const uint32_t pm = __ballot_sync(0xffffffffu, (f & kLbPrefix) != 0ull);
+                const int stop = pm ? __ffs(pm) - 1 : 31;   // nearest CTA holding its prefix
+                excl += warp_sum_ll(lane <= stop ? (long long)(f & kLbValue) : 0);
+                if (pm) break;
+                top -= 32;
             }
-            st_release_u64(P.lb_flags + cta, kLbPrefix | (unsigned long long)(excl + agg));
+            if (lane == 0) st_release_u64(P.lb_flags + cta, kLbPrefix | (unsigned long long)(excl + agg));
         }
-        s_base = excl;
+        if (lane == 0) s_base = excl;
     }
     __syncthreads();
-    if (have_row) {
-        long long base = s_base;
-        for (int w = 0; w < warp; ++w) base += s_count[w];
-        if (lane == 0) P.row_ptr[r] = (int32_t)base;
-        if (r == D.R - 1 && lane == 0) P.row_ptr[D.R] = (int32_t)(base + count);
-        // column ids from the mask words this warp wrote, ascending
-        __syncwarp();
-        int32_t at0 = (int32_t)base;
-        for (int w = 0; 32 * w <= i; ++w) {
-            const uint32_t bits = mask[w];
-            const int32_t at = at0 + __popc(bits & ((1u << lane) - 1u));
-            if (((bits >> lane) & 1u) && FP2_CHECK(at >= 0 && at < D.nnz_cap, P.status))
-                P.col_idx[at] = 32 * w + lane;
-            at0 += __popc(bits);
+    if (!have_row) return;
+    long long base = s_base;
+    for (int w = 0; w < warp; ++w) base += s_count[w];
+    if (lane == 0) P.row_ptr[r] = (int32_t)base;
+    if (r == D.R - 1 && lane == 0) P.row_ptr[D.R] = (int32_t)(base + count);
+    if (count == 0) return;
+    const int64_t bi = r % D.NB;
+    const int i = (int)(bi - P.cu_blocks[P.block_seq[bi]]);
+    const uint32_t* mask = P.kept_mask + r * D.mask_words;
+    // 32 mask words at a time: lane l loads word w0 + l, the lanes' exclusive
+    // sums of the words' bit counts place each word's ids
+    long long at = base;
+    for (int w0 = 0; 32 * w0 <= i; w0 += 32) {
+        const int w = w0 + lane;
+        const uint32_t bits = 32 * w <= i ? mask[w] : 0u;
+        const int c = __popc(bits);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
         }
+        const int ex = incl - c;
+        const int nw = min(32, i / 32 + 1 - w0);
+        for (int u = 0; u < nw; ++u) {
+            const uint32_t b = __shfl_sync(0xffffffffu, bits, u);
+            const long long a = at + __shfl_sync(0xffffffffu, ex, u) + __popc(b & ((1u << lane) - 1u));
+            if (((b >> lane) & 1u) && FP2_CHECK(a >= 0 && a < D.nnz_cap, P.status))
+                P.col_idx[a] = 32 * (w0 + u) + lane;
+        }
+        at += __shfl_sync(0xffffffffu, incl, 31);
     }
 }
 
@@ -1481,12 +1535,19 @@ int launch_score(const Dims& D, const PlanPtrs& P, const WsPtrs& W, cudaStream_t
     }
     // the pipelined scorer leaves each row's score bounds for the threshold
     const bool bounds = D.tau > 0.0 && D.G <= 32 && (D.G & (D.G - 1)) == 0;
-    const dim3 grid((unsigned)((D.R + kThrRows - 1) / kThrRows));
-    if (P.cu_q)
-        return launch_pdl(k_threshold<HD, true>, grid, dim3(kThrRows * 32), 0, st, D, P, W, kScoreTcRelErr,
-                          bounds);
-    return launch_pdl(k_threshold<HD, false>, grid, dim3(kThrRows * 32), 0, st, D, P, W, kScoreTcRelErr,
-                      bounds);
+    // the threshold's CTAs take rows until none is left: as many CTAs as fit
+    // on the device at once
+    auto thr = P.cu_q ? k_threshold<HD, true> : k_threshold<HD, false>;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, thr, kThrRows * 32, 0) != cudaSuccess)
+        return FP2_ERR_CUDA;
+    const int64_t fit = (int64_t)std::max(1, per_sm) * std::max(1, sm_count());
+    const int64_t need = (D.R + kThrRows - 1) / kThrRows;
+    const dim3 grid((unsigned)std::min(fit, need));
+    int rc = launch_pdl(thr, grid, dim3(kThrRows * 32), 0, st, D, P, W, kScoreTcRelErr, bounds);
+    if (rc != FP2_OK) return rc;
+    return launch_pdl(k_csr, dim3((unsigned)((D.R + kCsrRows - 1) / kCsrRows)), dim3(kCsrRows * 32), 0, st,
+                      D, P);
 }
 
 }  // namespace
