@@ -197,8 +197,10 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     L.off_split_lse = c.take(sizeof(float) * split_rows);
     L.off_slot_item = c.take(sizeof(int32_t) * (size_t)sd.split_slots * d.Hkv);
     L.off_q_off = c.take(sizeof(int32_t) * n);
-    L.off_lb_ticket = c.take(2 * sizeof(int32_t));
-    L.off_lb_flags = c.take(sizeof(unsigned long long) * (size_t)((d.R + kCsrRows - 1) / kCsrRows));
+    L.off_thr_next = c.take(sizeof(int32_t));
+    L.off_csr_count = c.take(sizeof(int32_t) * (size_t)d.R);
+    L.off_csr_seg = c.take(sizeof(int32_t) * (size_t)((d.R + kCsrRows - 1) / kCsrRows));
+    L.off_csr_sup = c.take(sizeof(int32_t) * (size_t)((d.R + kCsrSup - 1) / kCsrSup));
     pub.plan_bytes = align_up(c.off, 256);
 
     Carver w;
@@ -207,9 +209,10 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     L.ws_kbar_tf = w.take(sizeof(float) * mean_elems);
     L.ws_kbar64 = w.take(sizeof(double) * mean_elems);
     L.ws_qnorm = w.take(sizeof(float) * (size_t)NB * d.Hkv);
+    L.ws_qres = w.take(sizeof(float) * (size_t)NB * d.Hkv);
     L.ws_knorm = w.take(sizeof(float) * (size_t)NB * d.Hkv);
+    L.ws_kres = w.take(sizeof(float) * (size_t)NB * d.Hkv);
     L.ws_scores = w.take(sizeof(float) * (size_t)d.nnz_cap);
-    L.ws_counts = w.take(sizeof(int32_t) * (size_t)d.R);
     L.ws_bounds = w.take(sizeof(double) * 2 * (size_t)d.R);
     pub.workspace_bytes = align_up(w.off, 256);
     pub.num_work_items = sd.n_items;
@@ -249,8 +252,10 @@ PlanPtrs plan_ptrs(const Layout& L, void* plan) {
     p.split_lse = reinterpret_cast<float*>(b + L.off_split_lse);
     p.slot_item = reinterpret_cast<int32_t*>(b + L.off_slot_item);
     p.q_off = reinterpret_cast<int32_t*>(b + L.off_q_off);
-    p.lb_ticket = reinterpret_cast<int32_t*>(b + L.off_lb_ticket);
-    p.lb_flags = reinterpret_cast<unsigned long long*>(b + L.off_lb_flags);
+    p.thr_next = reinterpret_cast<int32_t*>(b + L.off_thr_next);
+    p.csr_count = reinterpret_cast<int32_t*>(b + L.off_csr_count);
+    p.csr_seg = reinterpret_cast<int32_t*>(b + L.off_csr_seg);
+    p.csr_sup = reinterpret_cast<int32_t*>(b + L.off_csr_sup);
     p.cu_q = nullptr;
     return p;
 }
@@ -263,9 +268,10 @@ WsPtrs ws_ptrs(const Layout& L, void* ws) {
     w.kbar_tf = reinterpret_cast<float*>(b + L.ws_kbar_tf);
     w.kbar64 = reinterpret_cast<double*>(b + L.ws_kbar64);
     w.qnorm = reinterpret_cast<float*>(b + L.ws_qnorm);
+    w.qres = reinterpret_cast<float*>(b + L.ws_qres);
     w.knorm = reinterpret_cast<float*>(b + L.ws_knorm);
+    w.kres = reinterpret_cast<float*>(b + L.ws_kres);
     w.scores = reinterpret_cast<float*>(b + L.ws_scores);
-    w.counts = reinterpret_cast<int32_t*>(b + L.ws_counts);
     w.bounds = reinterpret_cast<double*>(b + L.ws_bounds);
     return w;
 }

@@ -17,7 +17,8 @@ namespace fp2 {
 constexpr int kTileM = 128;
 // CSR rows per CTA of the threshold kernel (one warp per row).
 constexpr int kThrRows = 8;    // threshold: warps (rows in flight) per CTA
-constexpr int kCsrRows = 32;   // CSR: rows per CTA, one warp each
+constexpr int kCsrRows = 32;     // CSR offsets: rows per segment
+constexpr int kCsrSup = 1024;    // rows per super-segment (kCsrRows segments)
 // Query vectors scored together by one CTA of the scoring kernel (MMA M).
 constexpr int kScoreQV = 128;
 // Key blocks scored together by one CTA of the scoring kernel (MMA N).
@@ -122,8 +123,10 @@ struct PlanPtrs {
     int32_t* q_off;        // [n]  position of the first query (L - Q for a chunk, else 0)
     // the threshold kernel's single-pass CSR prefix sum (decoupled look-back):
     // a CTA ticket counter and one flag word per CTA, zeroed by k_meta
-    int32_t* lb_ticket;    // [2]: the threshold's next row, the CSR kernel's next CTA
-    unsigned long long* lb_flags;   // [ceil(R / kCsrRows)]
+    int32_t* thr_next;     // [1]: the threshold's next row
+    int32_t* csr_count;    // [R]: kept blocks per row
+    int32_t* csr_seg;      // [ceil(R / kCsrRows)]: kept blocks per segment of kCsrRows rows
+    int32_t* csr_sup;      // [ceil(R / kCsrSup)]: kept blocks per super-segment of kCsrSup rows
     const int32_t* cu_q;   // caller's cu_q_seqlens for a chunked problem, else null (set per call)
 };
 
@@ -134,10 +137,11 @@ struct WsPtrs {
     float* kbar_tf;   // [NB, Hkv, d] the key means rounded to tf32 (stored as fp32)
     double* kbar64;   // [NB, Hkv, d]
     float* qnorm;     // [NB, Hkv]  max over the group's heads of |Qbar|_2 (rounded up)
+    float* qres;      // [NB, Hkv]  max over the group's heads of |Qbar - tf32(Qbar)|_2 (rounded up)
     float* knorm;     // [Hkv, NB]  |Kbar|_2 (rounded up), contiguous over a head's blocks
+    float* kres;      // [Hkv, NB]  |Kbar - tf32(Kbar)|_2 + c_d (|Kbar|_2 + that), rounded up
     float* scores;    // [Hkv, tri_total] fp32 block scores, row (s,g,i) at
                       //   g * tri_total + tri_off[s] + i (i + 1) / 2 + j
-    int32_t* counts;  // [R] kept blocks per row
     double* bounds;   // [R, 2] per row: the largest lower and upper bound of any
                       //   score (sc_j -/+ its error bound), from the pipelined scorer
 };
@@ -150,8 +154,8 @@ struct Layout {
     fp2_plan_layout pub;
     size_t off_meta_valid, off_cu_blocks, off_block_seq, off_tri_off, off_group_cu, off_group_seq,
         off_tile_cu, off_vmax, off_sched, off_sched_cnt, off_sched_off, off_split_o, off_split_lse,
-        off_slot_item, off_q_off, off_lb_ticket, off_lb_flags;
-    size_t ws_qbar64, ws_qbar32, ws_kbar_tf, ws_kbar64, ws_qnorm, ws_knorm, ws_scores, ws_counts,
+        off_slot_item, off_q_off, off_thr_next, off_csr_count, off_csr_seg, off_csr_sup;
+    size_t ws_qbar64, ws_qbar32, ws_kbar_tf, ws_kbar64, ws_qnorm, ws_qres, ws_knorm, ws_kres, ws_scores,
         ws_bounds;
 };
 

@@ -25,8 +25,8 @@
 //            bound of the threshold, and every candidate for the row maximum,
 //            is re-scored in float64, so the kept set is the one float64
 //            scores give.
-//   csr      the CSR row pointers by a decoupled look-back over the rows
-//            before, then the column ids.
+//   csr      the CSR row pointers (each warp adds up the kept counts of
+//            the rows before its row, by segments), then the column ids.
 #include <cfloat>
 #include <cstring>
 #include <cmath>
@@ -199,10 +199,11 @@ __global__ void __launch_bounds__(kMetaThreads, 1) k_meta(Dims D, SchedDims S, c
     }
     __syncthreads();
     if (s_valid) {
-        // the threshold's row counter and the CSR kernel's look-back state start from zero
-        const int64_t n_lb = (D.R + kCsrRows - 1) / kCsrRows;
-        for (int64_t c = threadIdx.x; c < n_lb; c += blockDim.x) P.lb_flags[c] = 0ull;
-        if (threadIdx.x < 2) P.lb_ticket[threadIdx.x] = 0;
+        // the threshold's row counter and the CSR segment counts start from zero
+        const int64_t n_seg = (D.R + kCsrRows - 1) / kCsrRows, n_sup = (D.R + kCsrSup - 1) / kCsrSup;
+        for (int64_t c = threadIdx.x; c < n_seg; c += blockDim.x) P.csr_seg[c] = 0;
+        for (int64_t c = threadIdx.x; c < n_sup; c += blockDim.x) P.csr_sup[c] = 0;
+        if (threadIdx.x == 0) *P.thr_next = 0;
         meta_maps(D, S, cu_seqlens, page_table, P);
     }
     // k_meta may run beside the pooling kernel launched before it (which
@@ -288,6 +289,24 @@ __device__ __forceinline__ float round_up_f(double x) {
     float f = (float)x;
     if ((double)f < x) f = nextafterf(f, FLT_MAX);
     return f * (1.0f + 1.0f / 1048576.0f);
+}
+
+// The error bound of a tensor-core score.  With q~ = tf32(Qbar_h) and
+// k~ = tf32(Kbar) the MMA's operands (exact products, fp32 sums), and the
+// score x = fl(fl(q~ . k~) / sqrt d):
+//   |Qbar_h . Kbar - q~ . k~| <= |Qbar_h - q~| |Kbar| + |q~| |Kbar - k~|   (Cauchy-Schwarz)
+//   |fl(q~ . k~) - q~ . k~|   <= d 2^-23 |q~| |k~|                          (fp32 sums)
+//   the division by sqrt d     <= 2^-22 |q~| |k~|                           (two roundings)
+// and |q~| <= |Qbar_h| + |Qbar_h - q~|, |k~| <= |Kbar| + |Kbar - k~|, so over
+// a row's G heads |x - Qbar . Kbar / sqrt d| <= A kn_j + B kr_j with
+//   A = max_h |Qbar_h - q~| / sqrt d,  B = (max_h |Qbar_h| + that) / sqrt d,
+//   kn_j = |Kbar_j|,  kr_j = |Kbar_j - k~_j| + c_d (|Kbar_j| + |Kbar_j - k~_j|),
+//   c_d = d 2^-23 + 2^-22.
+// The residual norms are those of the actual rounding, typically a few times
+// below the worst case 2^-11 |.|, which keeps the band of undecided blocks narrow.
+__device__ __forceinline__ float kres_bound(double kn, double kr, int d) {
+    const double c_d = (double)d * 0x1p-23 + 0x1p-22;
+    return round_up_f(kr + c_d * (kn + kr));
 }
 
 // Sequence of global block b, its block index i, and its token offsets.
@@ -509,25 +528,42 @@ k_pool(Dims D, SeqMap M, int64_t Tq, const int32_t* __restrict__ cu_seqlens,
         }
     }
     if (NORMS) {
-        // |mean|^2 of this thread's head: the d / 8 threads of a head are
-        // consecutive lanes of one warp (d / 8 in {8, 16})
-        double sq = 0.0;
+        // |mean|^2 and |mean - tf32(mean)|^2 of this thread's head: the d / 8
+        // threads of a head are consecutive lanes of one warp (d / 8 in {8, 16})
+        double sq = 0.0, rq = 0.0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) sq = fma(m[e], m[e], sq);
+        for (int e = 0; e < 8; ++e) {
+            sq = fma(m[e], m[e], sq);
+            const double rr = m[e] - (double)round_tf32((float)m[e]);
+            rq = fma(rr, rr, rq);
+        }
         const int tph = d / 8;
-        for (int o = tph / 2; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        for (int o = tph / 2; o > 0; o >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            rq += __shfl_xor_sync(0xffffffffu, rq, o);
+        }
         const bool lead = active && (vec % tph) == 0;
-        if (lead && which == 1) W.knorm[(int64_t)head * D.NB + b] = round_up_f(sqrt(sq));
+        if (lead && which == 1) {
+            W.knorm[(int64_t)head * D.NB + b] = round_up_f(sqrt(sq));
+            W.kres[(int64_t)head * D.NB + b] = kres_bound(sqrt(sq), sqrt(rq), d);
+        }
         // the largest over the G query heads of a kv-head: the group's heads
         // lie in this CTA (G d divides the CTA's 1024 columns)
-        __shared__ double head_sq[kPoolThreads];
+        __shared__ double head_sq[kPoolThreads], head_rq[kPoolThreads];
         const int hl = threadIdx.x / tph;   // head slot within the CTA
-        if (lead) head_sq[hl] = sq;
+        if (lead) {
+            head_sq[hl] = sq;
+            head_rq[hl] = rq;
+        }
         __syncthreads();
         if (lead && which == 0 && head % D.G == 0) {
-            double mx = 0.0;
-            for (int u = 0; u < D.G; ++u) mx = fmax(mx, head_sq[hl + u]);
+            double mx = 0.0, mr = 0.0;
+            for (int u = 0; u < D.G; ++u) {
+                mx = fmax(mx, head_sq[hl + u]);
+                mr = fmax(mr, head_rq[hl + u]);
+            }
             W.qnorm[b * D.Hkv + head / D.G] = round_up_f(sqrt(mx));
+            W.qres[b * D.Hkv + head / D.G] = round_up_f(sqrt(mr));
         }
     }
 }
@@ -544,21 +580,35 @@ __global__ void k_norms(Dims D, PlanPtrs P, WsPtrs W) {
     const int64_t b = wid / D.Hkv;
     const int g = (int)(wid % D.Hkv);
     const int d = D.d;
-    double kk = 0.0;
+    // |mean|^2 and |mean - tf32(mean)|^2 (tf32 of the fp32 mean, the scorer's operand)
+    double kk = 0.0, kr = 0.0;
     const double* kp = W.kbar64 + (b * D.Hkv + g) * d;
-    for (int e = lane; e < d; e += 32) kk += kp[e] * kp[e];
+    for (int e = lane; e < d; e += 32) {
+        kk += kp[e] * kp[e];
+        const double rr = kp[e] - (double)round_tf32((float)kp[e]);
+        kr += rr * rr;
+    }
     kk = warp_sum_d(kk);
-    double qmax = 0.0;
+    kr = warp_sum_d(kr);
+    double qmax = 0.0, rmax = 0.0;
     for (int hl = 0; hl < D.G; ++hl) {
         const double* qp = W.qbar64 + (b * D.Hq + (int64_t)g * D.G + hl) * d;
-        double qq = 0.0;
-        for (int e = lane; e < d; e += 32) qq += qp[e] * qp[e];
+        double qq = 0.0, qr = 0.0;
+        for (int e = lane; e < d; e += 32) {
+            qq += qp[e] * qp[e];
+            const double rr = qp[e] - (double)round_tf32((float)qp[e]);
+            qr += rr * rr;
+        }
         qq = warp_sum_d(qq);
+        qr = warp_sum_d(qr);
         qmax = fmax(qmax, qq);
+        rmax = fmax(rmax, qr);
     }
     if (lane == 0) {
         W.knorm[(int64_t)g * D.NB + b] = round_up_f(sqrt(kk));
+        W.kres[(int64_t)g * D.NB + b] = kres_bound(sqrt(kk), sqrt(kr), d);
         W.qnorm[wid] = round_up_f(sqrt(qmax));
+        W.qres[wid] = round_up_f(sqrt(rmax));
     }
 }
 
@@ -578,10 +628,10 @@ __global__ void k_norms(Dims D, PlanPtrs P, WsPtrs W) {
 // the products are exact and a dot product is within
 //   (2 * 2^-11 + d 2^-23) |Qbar| |Kbar|
 // of the one of the float64 means (tf32 rounding of both operands, fp32
-// accumulation); the threshold kernel is given 3 * 2^-10 (a factor of about
-// 2.8 of margin) and re-scores in float64 every block it cannot decide.
+// accumulation); the threshold kernel uses the tighter bound of kres_bound,
+// from the norms of the actual rounding residuals, and re-scores in float64
+// every block it cannot decide.
 constexpr int kScoreTcThreads = 160;  // warps 0-3: epilogue (TMEM lanes); warp 4: TMA + MMA
-constexpr double kScoreTcRelErr = 3.0 / 1024.0;
 
 template <int HD>
 struct ScoreTcCfg {
@@ -894,7 +944,7 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
         // bound of any score, sc_j -/+ C |Qbar|max |Kbar_j| (the threshold's
         // first pass, done here while the scores are in registers)
         const float inv_sqrt_d = 1.0f / sqrtf((float)HD);
-        const double C = kScoreTcRelErr / sqrt((double)HD);
+        const double inv_sqrt_d64 = 1.0 / sqrt((double)HD);
         constexpr int G = GQ;   // query heads per kv-head (a power of two, at most 32)
         const int row = 32 * warp + lane;
         const int ri = row / G, hl = row % G;
@@ -907,25 +957,48 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
             const bool row_ok = i < it.i1;
             float* sc_row = W.scores + (int64_t)it.g * D.tri_total + P.tri_off[it.s] + (int64_t)i * (i + 1) / 2;
             const float* kn = W.knorm + (int64_t)it.g * D.NB + it.b0;
-            // fp32 bound coefficient, rounded up (the bounds below only need to
-            // enclose the float64 ones: they are widened before they are stored)
-            const float Cq = row_ok ? (float)(C * (double)W.qnorm[(int64_t)(it.b0 + i) * D.Hkv + it.g]) *
-                                          (1.0f + 1.0f / 1048576.0f)
-                                    : 0.f;
+            const float* kr = W.kres + (int64_t)it.g * D.NB + it.b0;
+            // the row's bound coefficients A, B (see kres_bound), rounded up (the
+            // bounds below only need to enclose the float64 ones: they are
+            // widened before they are stored)
+            float A = 0.f, B = 0.f;
+            if (row_ok) {
+                const int64_t qi = (int64_t)(it.b0 + i) * D.Hkv + it.g;
+                const double qr = W.qres[qi];
+                A = round_up_f(qr * inv_sqrt_d64);
+                B = round_up_f(((double)W.qnorm[qi] + qr) * inv_sqrt_d64);
+            }
             float m_lo = -FLT_MAX, m_hi = -FLT_MAX, e_max = 0.f;
             bool ok = true;
             for (int c = 0; c < it.n_chunks; ++c, ++an) {
                 const int buf = an & 1;
+                // the chunk's key norms, lane l holding column 32 cc + l of each
+                // 32-column part (loaded before the wait, handed out by shuffles)
+                constexpr int NCC = kScoreKeys / 32;
+                float knr[NCC], krr[NCC];
+#pragma unroll
+                for (int cc = 0; cc < NCC; ++cc) {
+                    const int col = kScoreKeys * c + 32 * cc + lane;
+                    knr[cc] = col < it.nb ? __ldg(kn + col) : 0.f;
+                    krr[cc] = col < it.nb ? __ldg(kr + col) : 0.f;
+                }
                 if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (an >> 1) & 1, &abort_flag, P.status))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-#pragma unroll 1
-                for (int cc = 0; cc < kScoreKeys / 32; ++cc) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + buf * kScoreKeys + 32 * cc, r);
-                    tmem_ld_wait();
+                // all of the chunk's dot products at once; the accumulator is
+                // free for the MMAs two chunks on as soon as they are in registers
+                uint32_t r[NCC][32];
+#pragma unroll
+                for (int cc = 0; cc < NCC; ++cc)
+                    tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + buf * kScoreKeys + 32 * cc, r[cc]);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[buf]);
+#pragma unroll
+                for (int cc = 0; cc < NCC; ++cc) {
                     const int jb = kScoreKeys * c + 32 * cc;
                     // max over the G heads (adjacent lanes), 32 columns at a time so
                     // the shuffles of different columns overlap
@@ -933,35 +1006,33 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
                     for (int o = 1; o < G; o <<= 1) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
-                            r[e] = __float_as_uint(fmaxf(__uint_as_float(r[e]),
-                                                         __shfl_xor_sync(0xffffffffu, __uint_as_float(r[e]), o)));
+                            r[cc][e] = __float_as_uint(fmaxf(__uint_as_float(r[cc][e]),
+                                                             __shfl_xor_sync(0xffffffffu, __uint_as_float(r[cc][e]), o)));
                     }
-                    if (row_ok) {
-                        float lo4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
-                        float hi4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
+                    float lo4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
+                    float hi4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
 #pragma unroll
-                        for (int e0 = 0; e0 < 32; e0 += G) {
-                            // this lane's column of the G columns e0 .. e0 + G - 1
-                            uint32_t v = r[e0];
+                    for (int e0 = 0; e0 < 32; e0 += G) {
+                        // this lane's column of the G columns e0 .. e0 + G - 1
+                        uint32_t v = r[cc][e0];
 #pragma unroll
-                            for (int u = 1; u < G; ++u) v = hl == u ? r[e0 + u] : v;
-                            const int col = jb + e0 + hl;
-                            if (col <= i && FP2_CHECK(sc_row + col < W.scores + D.Hkv * D.tri_total, P.status)) {
-                                const float x = __uint_as_float(v) * inv_sqrt_d;
-                                sc_row[col] = x;
-                                const float err = Cq * __ldg(kn + col);
-                                e_max = fmaxf(e_max, err);
-                                lo4[(e0 / G) & 3] = fmaxf(lo4[(e0 / G) & 3], x - err);
-                                hi4[(e0 / G) & 3] = fmaxf(hi4[(e0 / G) & 3], x + err);
-                            }
+                        for (int u = 1; u < G; ++u) v = hl == u ? r[cc][e0 + u] : v;
+                        const float knv = __shfl_sync(0xffffffffu, knr[cc], e0 + hl);
+                        const float krv = __shfl_sync(0xffffffffu, krr[cc], e0 + hl);
+                        const int col = jb + e0 + hl;
+                        if (row_ok && col <= i &&
+                            FP2_CHECK(sc_row + col < W.scores + D.Hkv * D.tri_total, P.status)) {
+                            const float x = __uint_as_float(v) * inv_sqrt_d;
+                            sc_row[col] = x;
+                            const float err = fmaf(A, knv, B * krv);
+                            e_max = fmaxf(e_max, err);
+                            lo4[(e0 / G) & 3] = fmaxf(lo4[(e0 / G) & 3], x - err);
+                            hi4[(e0 / G) & 3] = fmaxf(hi4[(e0 / G) & 3], x + err);
                         }
-                        m_lo = fmaxf(m_lo, fmaxf(fmaxf(lo4[0], lo4[1]), fmaxf(lo4[2], lo4[3])));
-                        m_hi = fmaxf(m_hi, fmaxf(fmaxf(hi4[0], hi4[1]), fmaxf(hi4[2], hi4[3])));
                     }
+                    m_lo = fmaxf(m_lo, fmaxf(fmaxf(lo4[0], lo4[1]), fmaxf(lo4[2], lo4[3])));
+                    m_hi = fmaxf(m_hi, fmaxf(fmaxf(hi4[0], hi4[1]), fmaxf(hi4[2], hi4[3])));
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[buf]);
             }
             if (!ok) {
                 abort_flag = 1;
@@ -1035,41 +1106,49 @@ __device__ __noinline__ double score64(const double* __restrict__ qp0, const dou
 // threshold: one warp per row, decisions equal to the float64 ones
 // ---------------------------------------------------------------------------
 //
-// The score of a block differs from the exact one by at most
-//   e_j = rel_err max_h|Qbar_{i,h}| |Kbar_j| / sqrt(d)
-// with rel_err the scoring kernel's bound (kScoreTcRelErr).  Every block whose
-// score could be the row maximum and every block whose score lies within e_j of
-// tau * m is re-scored in float64.
+// The score of block j of a row differs from the exact one by at most
+//   e_j = A kn_j + B kr_j
+// (kres_bound: A, B per row from its query means, kn_j, kr_j per key block).
+// Every block whose score could be the row maximum and every block whose
+// score lies within e_j of tau * m is re-scored in float64.
 // The loads of a row are issued kThrBatch words (32 blocks each) at a time,
 // so a pass over a row of n blocks waits on about n / (32 kThrBatch) round
 // trips to L2 rather than n / 32.
 constexpr int kThrBatch = 4;
 
+// The error-bound terms of one row.
+struct RowBound {
+    const float* kn;   // |Kbar_j|, j = 0 .. i
+    const float* kr;   // kr_j
+    double A, B;
+    __device__ __forceinline__ double e(float knj, float krj) const { return A * knj + B * krj; }
+};
+
 // The decision of one row (warp-collective), given the largest lower bound
 // m_lo of its scores: the row maximum in float64 over every block whose upper
 // bound reaches m_lo, then keep / drop per block, re-scoring in float64 every
-// block within its bound Cq * |Kbar_j| of the threshold.  Writes the mask
-// words 0 .. i / 32 and zeroes the rest; adds the kept count to `count`.
+// block within its bound e_j of the threshold.  Writes the mask words
+// 0 .. i / 32 and zeroes the rest; adds the kept count to `count`.
 template <int HD>
 __device__ __forceinline__ void thr_decide(const Dims& D, const WsPtrs& W, const float* sc,
-                                           const float* kn, double Cq, double m_lo, int i,
-                                           int64_t bi, int b0, int g, int lane, uint32_t* mask,
-                                           int& count) {
+                                           const RowBound& rb, double m_lo, int i, int64_t bi, int b0,
+                                           int g, int lane, uint32_t* mask, int& count) {
     const double* q64 = W.qbar64 + (bi * D.Hq + (int64_t)g * D.G) * HD;   // the row's first head
     double m = -DBL_MAX;
 #pragma unroll 1
     for (int jb = 0; jb <= i; jb += 32 * kThrBatch) {
-        float xs[kThrBatch], ks[kThrBatch];
+        float xs[kThrBatch], ks[kThrBatch], rs[kThrBatch];
 #pragma unroll
         for (int u = 0; u < kThrBatch; ++u) {
             const int j = jb + 32 * u + lane;
             xs[u] = j <= i ? __ldg(sc + j) : 0.f;
-            ks[u] = j <= i ? __ldg(kn + j) : 0.f;
+            ks[u] = j <= i ? __ldg(rb.kn + j) : 0.f;
+            rs[u] = j <= i ? __ldg(rb.kr + j) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < kThrBatch; ++u) {
             const int j = jb + 32 * u + lane;
-            uint32_t cb = __ballot_sync(0xffffffffu, j <= i && (double)xs[u] + Cq * ks[u] >= m_lo);
+            uint32_t cb = __ballot_sync(0xffffffffu, j <= i && (double)xs[u] + rb.e(ks[u], rs[u]) >= m_lo);
             while (cb) {
                 const int l = __ffs(cb) - 1;
                 cb &= cb - 1;
@@ -1080,12 +1159,13 @@ __device__ __forceinline__ void thr_decide(const Dims& D, const WsPtrs& W, const
     const double t = D.tau * m;
 #pragma unroll 1
     for (int jb = 0; jb <= i; jb += 32 * kThrBatch) {
-        float xs[kThrBatch], ks[kThrBatch];
+        float xs[kThrBatch], ks[kThrBatch], rs[kThrBatch];
 #pragma unroll
         for (int u = 0; u < kThrBatch; ++u) {
             const int j = jb + 32 * u + lane;
             xs[u] = j <= i ? __ldg(sc + j) : 0.f;
-            ks[u] = j <= i ? __ldg(kn + j) : 0.f;
+            ks[u] = j <= i ? __ldg(rb.kn + j) : 0.f;
+            rs[u] = j <= i ? __ldg(rb.kr + j) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < kThrBatch; ++u) {
@@ -1096,7 +1176,7 @@ __device__ __forceinline__ void thr_decide(const Dims& D, const WsPtrs& W, const
                 if (j == 0 || j == i) {
                     keep = true;
                 } else {
-                    const double e = Cq * ks[u];
+                    const double e = rb.e(ks[u], rs[u]);
                     const double x = (double)xs[u];
                     if (x - e >= t) keep = true;
                     else if (!(x + e < t)) unsure = true;
@@ -1120,26 +1200,49 @@ __device__ __forceinline__ void thr_decide(const Dims& D, const WsPtrs& W, const
 // One pass over a row of at most 1024 blocks whose score bounds the scorer
 // left in W.bounds: the exact maximum m lies in [m_lo, m_hi], so a block is
 // kept outright when sc - e >= tau m_hi, dropped outright when
-// sc + e < tau m_lo, and otherwise (a few per row, if any) decided once m is
-// known.  Candidates for the maximum (sc + e >= m_lo) are re-scored on the
-// way.  Lane l keeps the undecided bits of mask word l.
+// sc + e < tau m_lo, and otherwise decided once m is known.  The tests run
+// in fp32 with every rounding directed against the outright decisions (e,
+// sc +/- e and the thresholds they meet rounded up or down as the test
+// needs), so a block decided outright is decided as the exact values decide
+// it.  The candidates for the maximum (sc + e >= m_lo) are marked on the way
+// and re-scored in float64 only when the row has an undecided block.  The
+// next 32 kThrBatch scores are loaded while a batch is classified.  Lane l
+// keeps the bits of mask word l.
 template <int HD>
 __device__ __forceinline__ void thr_one_pass(const Dims& D, const WsPtrs& W, const float* sc,
-                                             const float* kn, double Cq, double m_lo, double m_hi,
-                                             int i, int64_t bi, int b0, int g, int lane, uint32_t* mask,
+                                             const RowBound& rb, double m_lo, double m_hi, int i,
+                                             int64_t bi, int b0, int g, int lane, uint32_t* mask,
                                              int& count) {
     const double* q64 = W.qbar64 + (bi * D.Hq + (int64_t)g * D.G) * HD;   // the row's first head
-    const double t_lo = D.tau * m_lo, t_hi = D.tau * m_hi;
-    double m = -DBL_MAX;
-    uint32_t my_pending = 0, my_keep = 0;   // of mask word `lane`
+    const float a_f = __double2float_ru(rb.A), b_f = __double2float_ru(rb.B);
+    const float m_lo_f = __double2float_rd(m_lo);
+    const float t_lo_f = __double2float_rd(D.tau * m_lo);
+    const float t_hi_f = __double2float_ru(D.tau * m_hi);
+    uint32_t my_pending = 0, my_keep = 0, my_cand = 0;   // of mask word `lane`
+    float xn[kThrBatch], kq[kThrBatch], rq[kThrBatch];
+#pragma unroll
+    for (int u = 0; u < kThrBatch; ++u) {
+        const int j = 32 * u + lane;
+        xn[u] = j <= i ? __ldg(sc + j) : 0.f;
+        kq[u] = j <= i ? __ldg(rb.kn + j) : 0.f;
+        rq[u] = j <= i ? __ldg(rb.kr + j) : 0.f;
+    }
 #pragma unroll 1
     for (int jb = 0; jb <= i; jb += 32 * kThrBatch) {
-        float xs[kThrBatch], ks[kThrBatch];
+        float xs[kThrBatch], es[kThrBatch];
 #pragma unroll
         for (int u = 0; u < kThrBatch; ++u) {
-            const int j = jb + 32 * u + lane;
-            xs[u] = j <= i ? __ldg(sc + j) : 0.f;
-            ks[u] = j <= i ? __ldg(kn + j) : 0.f;
+            xs[u] = xn[u];
+            es[u] = __fmaf_ru(a_f, kq[u], __fmul_ru(b_f, rq[u]));   // >= e_j
+        }
+        if (jb + 32 * kThrBatch <= i) {
+#pragma unroll
+            for (int u = 0; u < kThrBatch; ++u) {
+                const int j = jb + 32 * kThrBatch + 32 * u + lane;
+                xn[u] = j <= i ? __ldg(sc + j) : 0.f;
+                kq[u] = j <= i ? __ldg(rb.kn + j) : 0.f;
+                rq[u] = j <= i ? __ldg(rb.kr + j) : 0.f;
+            }
         }
 #pragma unroll
         for (int u = 0; u < kThrBatch; ++u) {
@@ -1148,37 +1251,49 @@ __device__ __forceinline__ void thr_one_pass(const Dims& D, const WsPtrs& W, con
             const int w = (jb >> 5) + u;
             bool keep = false, pend = false, cand = false;
             if (j <= i) {
-                const double x = (double)xs[u], e = Cq * ks[u];
-                cand = x + e >= m_lo;
-                if (j == 0 || j == i || x - e >= t_hi) keep = true;
-                else if (!(x + e < t_lo)) pend = true;
+                const float hi = __fadd_ru(xs[u], es[u]);   // >= sc + e
+                const float lo = __fsub_rd(xs[u], es[u]);   // <= sc - e
+                cand = hi >= m_lo_f;
+                if (j == 0 || j == i || lo >= t_hi_f) keep = true;
+                else if (!(hi < t_lo_f)) pend = true;
             }
-            uint32_t cb = __ballot_sync(0xffffffffu, cand);
+            const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+            const uint32_t pb = __ballot_sync(0xffffffffu, pend);
+            const uint32_t cb = __ballot_sync(0xffffffffu, cand);
+            if (lane == w) {
+                my_keep = kb;
+                my_pending = pb;
+                my_cand = cb;
+            }
+        }
+    }
+    if (__any_sync(0xffffffffu, my_pending != 0)) {
+        // the exact maximum over the candidates, then the undecided blocks
+        // against the exact threshold
+        double m = -DBL_MAX;
+        uint32_t any = __ballot_sync(0xffffffffu, my_cand != 0);
+        while (any) {
+            const int w = __ffs(any) - 1;
+            any &= any - 1;
+            uint32_t cb = __shfl_sync(0xffffffffu, my_cand, w);
             while (cb) {
                 const int l = __ffs(cb) - 1;
                 cb &= cb - 1;
                 m = fmax(m, score64<HD>(q64, W.kbar64 + ((int64_t)(b0 + 32 * w + l) * D.Hkv + g) * HD, D.G));
             }
-            const uint32_t kb = __ballot_sync(0xffffffffu, keep);
-            const uint32_t pb = __ballot_sync(0xffffffffu, pend);
-            if (lane == w) {
-                my_keep = kb;
-                my_pending = pb;
-            }
         }
-    }
-    // the undecided blocks against the exact threshold
-    const double t = D.tau * m;
-    uint32_t any = __ballot_sync(0xffffffffu, my_pending != 0);
-    while (any) {
-        const int w = __ffs(any) - 1;
-        any &= any - 1;
-        uint32_t pb = __shfl_sync(0xffffffffu, my_pending, w);
-        while (pb) {
-            const int l = __ffs(pb) - 1;
-            pb &= pb - 1;
-            const double x64 = score64<HD>(q64, W.kbar64 + ((int64_t)(b0 + 32 * w + l) * D.Hkv + g) * HD, D.G);
-            if (lane == w && x64 >= t) my_keep |= 1u << l;
+        const double t = D.tau * m;
+        any = __ballot_sync(0xffffffffu, my_pending != 0);
+        while (any) {
+            const int w = __ffs(any) - 1;
+            any &= any - 1;
+            uint32_t pb = __shfl_sync(0xffffffffu, my_pending, w);
+            while (pb) {
+                const int l = __ffs(pb) - 1;
+                pb &= pb - 1;
+                const double x64 = score64<HD>(q64, W.kbar64 + ((int64_t)(b0 + 32 * w + l) * D.Hkv + g) * HD, D.G);
+                if (lane == w && x64 >= t) my_keep |= 1u << l;
+            }
         }
     }
     if (32 * lane <= i) mask[lane] = my_keep;
@@ -1186,25 +1301,11 @@ __device__ __forceinline__ void thr_one_pass(const Dims& D, const WsPtrs& W, con
     for (int w = i / 32 + 1 + lane; w < D.mask_words; w += 32) mask[w] = 0u;
 }
 
-__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
-    asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Look-back flag words: the value in the low 62 bits, the kind in the top two.
-constexpr unsigned long long kLbAggregate = 1ull << 62;   // this CTA's rows only
-constexpr unsigned long long kLbPrefix = 2ull << 62;      // every row up to this CTA's last
-constexpr unsigned long long kLbValue = (1ull << 62) - 1;
-
 // The decision of row r (warp-collective): writes its kept-mask words and
 // returns its kept count.
 template <int HD, bool CHUNK>
 __device__ __forceinline__ int thr_row(const Dims& D, const PlanPtrs& P, const WsPtrs& W, int64_t r,
-                                       int lane, double rel_err, bool have_bounds) {
+                                       int lane, bool have_bounds) {
     const int g = (int)(r / D.NB);
     const int64_t bi = r % D.NB;
     const int s = P.block_seq[bi];
@@ -1225,42 +1326,58 @@ __device__ __forceinline__ int thr_row(const Dims& D, const PlanPtrs& P, const W
         count = i + 1;
     } else {
         const float* sc = W.scores + (int64_t)g * D.tri_total + P.tri_off[s] + (int64_t)i * (i + 1) / 2;
-        const double C = rel_err / sqrt((double)HD);
-        const double qn = W.qnorm[bi * D.Hkv + g];
-        const float* kn = W.knorm + (int64_t)g * D.NB + b0;   // contiguous in j
+        const double inv_sqrt_d = 1.0 / sqrt((double)HD);
+        const double qr = W.qres[bi * D.Hkv + g];
+        RowBound rb;
+        rb.kn = W.knorm + (int64_t)g * D.NB + b0;   // contiguous in j
+        rb.kr = W.kres + (int64_t)g * D.NB + b0;
+        // (1 + 2^-20: far above the float64 rounding of the tests below)
+        rb.A = qr * inv_sqrt_d * (1.0 + 0x1p-20);
+        rb.B = ((double)W.qnorm[bi * D.Hkv + g] + qr) * inv_sqrt_d * (1.0 + 0x1p-20);
         if (have_bounds && i < 32 * 32) {
-            thr_one_pass<HD>(D, W, sc, kn, C * qn, W.bounds[2 * r], W.bounds[2 * r + 1], i, bi, b0, g,
-                             lane, mask, count);
+            thr_one_pass<HD>(D, W, sc, rb, W.bounds[2 * r], W.bounds[2 * r + 1], i, bi, b0, g, lane, mask,
+                             count);
         } else {
             // largest lower bound of any score (kThrBatch words of loads at a time)
             double m_lo = -DBL_MAX;
 #pragma unroll 1
             for (int jb = 0; jb <= i; jb += 32 * kThrBatch) {
-                float xs[kThrBatch], ks[kThrBatch];
+                float xs[kThrBatch], ks[kThrBatch], rs[kThrBatch];
 #pragma unroll
                 for (int u = 0; u < kThrBatch; ++u) {
                     const int j = jb + 32 * u + lane;
                     xs[u] = j <= i ? __ldg(sc + j) : 0.f;
-                    ks[u] = j <= i ? __ldg(kn + j) : 0.f;
+                    ks[u] = j <= i ? __ldg(rb.kn + j) : 0.f;
+                    rs[u] = j <= i ? __ldg(rb.kr + j) : 0.f;
                 }
 #pragma unroll
                 for (int u = 0; u < kThrBatch; ++u)
-                    if (jb + 32 * u + lane <= i) m_lo = fmax(m_lo, (double)xs[u] - C * qn * ks[u]);
+                    if (jb + 32 * u + lane <= i) m_lo = fmax(m_lo, (double)xs[u] - rb.e(ks[u], rs[u]));
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m_lo = fmax(m_lo, __shfl_xor_sync(0xffffffffu, m_lo, o));
-            thr_decide<HD>(D, W, sc, kn, C * qn, m_lo, i, bi, b0, g, lane, mask, count);
+            thr_decide<HD>(D, W, sc, rb, m_lo, i, bi, b0, g, lane, mask, count);
         }
     }
     return count;
 }
 
-// The threshold: each warp takes rows one at a time from a shared counter,
-// longest first (block index from the last down, every kv-head of a block
-// together), decides them and leaves the kept count in row_ptr[r];
-// k_csr turns the counts into offsets and writes the column ids.
+// Position o of the rows in the order "longest first" (block index from the
+// last down, every kv-head of a block together) that warp gw of nw takes as
+// its t-th row: passes of nw rows, odd passes from the other end, so that
+// every warp gets rows of about the same total length.
+__device__ __forceinline__ int64_t row_order(int64_t t, int64_t gw, int64_t nw) {
+    return t * nw + ((t & 1) ? nw - 1 - gw : gw);
+}
+
+// The threshold: each warp takes the next row "longest first" from a counter
+// (the rows' costs depend on how many blocks need re-scoring, so they are
+// handed out as warps free up), decides it, and leaves the row's kept count,
+// adding it to the counts of the row's segment (kCsrRows rows) and
+// super-segment (kCsrSup rows); k_csr turns the counts into offsets and
+// writes the column ids.
 template <int HD, bool CHUNK>
-__global__ void __launch_bounds__(kThrRows * 32, 3) k_threshold(Dims D, PlanPtrs P, WsPtrs W, double rel_err,
+__global__ void __launch_bounds__(kThrRows * 32, 2) k_threshold(Dims D, PlanPtrs P, WsPtrs W,
                                                              bool have_bounds) {
     // launched as a programmatic dependent: everything before it is complete
     // once the wait returns
@@ -1270,109 +1387,83 @@ __global__ void __launch_bounds__(kThrRows * 32, 3) k_threshold(Dims D, PlanPtrs
     if (!*P.meta_valid) return;
     const int lane = threadIdx.x & 31;
     for (;;) {
-        int t = 0;
-        if (lane == 0) t = atomicAdd(P.lb_ticket, 1);
-        t = __shfl_sync(0xffffffffu, t, 0);
-        if (t >= D.R) break;
-        const int64_t bi = D.NB - 1 - t / D.Hkv;
-        const int64_t r = (int64_t)(t % D.Hkv) * D.NB + bi;
-        const int count = thr_row<HD, CHUNK>(D, P, W, r, lane, rel_err, have_bounds);
-        if (lane == 0) P.row_ptr[r] = count;
+        int o = 0;
+        if (lane == 0) o = atomicAdd(P.thr_next, 1);
+        o = __shfl_sync(0xffffffffu, o, 0);
+        if (o >= D.R) break;
+        const int64_t bi = D.NB - 1 - o / D.Hkv;
+        const int64_t r = (int64_t)(o % D.Hkv) * D.NB + bi;
+        const int count = thr_row<HD, CHUNK>(D, P, W, r, lane, have_bounds);
+        if (lane == 0) {
+            P.csr_count[r] = count;
+            atomicAdd(P.csr_seg + r / kCsrRows, count);
+            atomicAdd(P.csr_sup + r / kCsrSup, count);
+        }
     }
 }
 
-// Sum over the lanes of a warp.
-__device__ __forceinline__ long long warp_sum_ll(long long v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-
-// The CSR from the kept counts and mask words: CTA c (taken by a ticket, so
-// every CTA it waits for is running or done) holds rows kCsrRows c ..
-// kCsrRows (c + 1) - 1, one warp each.  The CTA's offset among all rows comes
-// from a decoupled look-back (warp 0 reads the flags of the 32 CTAs before the
-// window's top at once, and sums back to the nearest that holds its prefix);
-// then each warp writes its row's column ids, ascending.
-__global__ void __launch_bounds__(kCsrRows * 32) k_csr(Dims D, PlanPtrs P) {
+// The CSR from the kept counts and mask words.  The warps take the rows in
+// row_order (which evens out their work); a row's offset is the kept count
+// of every row before it:
+// the super-segments before its own, the segments before it within its
+// super-segment, and the rows before it within its segment (at most
+// R / kCsrSup + 62 counts, added up by the warp's lanes).  Then the warp
+// writes the row pointer and the row's column ids, ascending.  No warp waits
+// on another.
+__global__ void __launch_bounds__(kThrRows * 32) k_csr(Dims D, PlanPtrs P) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (!*P.meta_valid) return;
-    __shared__ int s_ticket;
-    __shared__ int s_count[kCsrRows];
-    __shared__ long long s_base;
-    if (threadIdx.x == 0) s_ticket = atomicAdd(P.lb_ticket + 1, 1);
-    __syncthreads();
-    const int64_t cta = s_ticket;
-    const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t r = cta * kCsrRows + warp;
-    const bool have_row = r < D.R;
-    const int count = have_row ? P.row_ptr[r] : 0;
-    if (lane == 0) s_count[warp] = count;
-    __syncthreads();
-    if (warp == 0) {
-        const long long agg = warp_sum_ll(lane < kCsrRows ? s_count[lane] : 0);
-        long long excl = 0;
-        if (cta == 0) {
-            if (lane == 0) st_release_u64(P.lb_flags, kLbPrefix | (unsigned long long)agg);
-        } else {
-            if (lane == 0) st_release_u64(P.lb_flags + cta, kLbAggregate | (unsigned long long)agg);
-            int64_t top = cta - 1;   // the window is CTAs top, top - 1, .. top - 31
-            const uint64_t t0 = global_timer_ns();
-            for (;;) {
-                const int64_t p = top - lane;
-                // before CTA 0: an empty prefix
-                const unsigned long long f = p >= 0 ? ld_acquire_u64(P.lb_flags + p) : kLbPrefix;
-                if (__any_sync(0xffffffffu, f == 0ull)) {
-                    // (never: the CTAs before are running; the vote keeps the warp together)
-                    if (__any_sync(0xffffffffu, global_timer_ns() - t0 > kWaitLimitNs)) {
-                        if (lane == 0) atomicOr(P.status, (int32_t)FP2_STATUS_TIMEOUT);
-                        break;
-                    }
-                    continue;
-                }
-                const uint32_t pm = __ballot_sync(0xffffffffu, (f & kLbPrefix) != 0ull);
-                const int stop = pm ? __ffs(pm) - 1 : 31;   // nearest CTA holding its prefix
-                excl += warp_sum_ll(lane <= stop ? (long long)(f & kLbValue) : 0);
-                if (pm) break;
-                top -= 32;
-            }
-            if (lane == 0) st_release_u64(P.lb_flags + cta, kLbPrefix | (unsigned long long)(excl + agg));
+    const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    for (int64_t t = 0; ; ++t) {
+        const int64_t o = row_order(t, gw, nw);
+        if (o >= D.R) break;
+        const int64_t bi = D.NB - 1 - o / D.Hkv;
+        const int64_t r = (o % D.Hkv) * D.NB + bi;
+        const int64_t seg = r / kCsrRows, sup = r / kCsrSup;
+        long long part = 0;
+        for (int64_t q = lane; q < sup; q += 32) part += P.csr_sup[q];
+        {
+            const int64_t q = sup * (kCsrSup / kCsrRows) + lane;
+            if (q < seg) part += P.csr_seg[q];
+            const int64_t q2 = seg * kCsrRows + lane;
+            if (q2 < r) part += P.csr_count[q2];
         }
-        if (lane == 0) s_base = excl;
-    }
-    __syncthreads();
-    if (!have_row) return;
-    long long base = s_base;
-    for (int w = 0; w < warp; ++w) base += s_count[w];
-    if (lane == 0) P.row_ptr[r] = (int32_t)base;
-    if (r == D.R - 1 && lane == 0) P.row_ptr[D.R] = (int32_t)(base + count);
-    if (count == 0) return;
-    const int64_t bi = r % D.NB;
-    const int i = (int)(bi - P.cu_blocks[P.block_seq[bi]]);
-    const uint32_t* mask = P.kept_mask + r * D.mask_words;
-    // 32 mask words at a time: lane l loads word w0 + l, the lanes' exclusive
-    // sums of the words' bit counts place each word's ids
-    long long at = base;
-    for (int w0 = 0; 32 * w0 <= i; w0 += 32) {
-        const int w = w0 + lane;
-        const uint32_t bits = 32 * w <= i ? mask[w] : 0u;
-        const int c = __popc(bits);
-        int incl = c;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        const long long base = part;
+        const int count = P.csr_count[r];
+        if (lane == 0) P.row_ptr[r] = (int32_t)base;
+        if (r == D.R - 1 && lane == 0) P.row_ptr[D.R] = (int32_t)(base + count);
+        if (count == 0) continue;
+        const int i = (int)(bi - P.cu_blocks[P.block_seq[bi]]);
+        const uint32_t* mask = P.kept_mask + r * D.mask_words;
+        // 32 mask words at a time: lane l loads word w0 + l, the lanes' exclusive
+        // sums of the words' bit counts place each word's ids
+        // (positions fit in 32 bits: nnz_cap < 2^31)
+        int32_t* dst = P.col_idx + base;
+        const uint32_t below = (1u << lane) - 1u;
+        for (int w0 = 0; 32 * w0 <= i; w0 += 32) {
+            const int w = w0 + lane;
+            const uint32_t bits = 32 * w <= i ? mask[w] : 0u;
+            const int c = __popc(bits);
+            int incl = c;
+#pragma unroll
+            for (int o2 = 1; o2 < 32; o2 <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o2);
+                if (lane >= o2) incl += y;
+            }
+            const int ex = incl - c;
+            const int nwd = min(32, i / 32 + 1 - w0);
+            int id = 32 * w0 + lane;
+            for (int u = 0; u < nwd; ++u, id += 32) {
+                const uint32_t b = __shfl_sync(0xffffffffu, bits, u);
+                const int a = __shfl_sync(0xffffffffu, ex, u) + __popc(b & below);
+                if (((b >> lane) & 1u) && FP2_CHECK(base + a < D.nnz_cap, P.status)) dst[a] = id;
+            }
+            dst += __shfl_sync(0xffffffffu, incl, 31);
         }
-        const int ex = incl - c;
-        const int nw = min(32, i / 32 + 1 - w0);
-        for (int u = 0; u < nw; ++u) {
-            const uint32_t b = __shfl_sync(0xffffffffu, bits, u);
-            const long long a = at + __shfl_sync(0xffffffffu, ex, u) + __popc(b & ((1u << lane) - 1u));
-            if (((b >> lane) & 1u) && FP2_CHECK(a >= 0 && a < D.nnz_cap, P.status))
-                P.col_idx[a] = 32 * (w0 + u) + lane;
-        }
-        at += __shfl_sync(0xffffffffu, incl, 31);
     }
 }
 
@@ -1394,9 +1485,11 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
     return r;
 }
 
-constexpr int kQuantMeansThreads = 1024;
+// Small CTAs, so that they fit on an SM beside the scorer's (which runs at
+// the same time and holds most of an SM's shared memory and registers).
+constexpr int kQuantMeansThreads = 256;
 
-__global__ void __launch_bounds__(kQuantMeansThreads) k_quant_means(Dims D, PlanPtrs P) {
+__global__ void __launch_bounds__(kQuantMeansThreads, 4) k_quant_means(Dims D, PlanPtrs P) {
     // a programmatic dependent of k_meta (everything before is complete once
     // the wait returns); the scorer, launched next, may run beside this kernel
     // (it needs nothing from it) and waits for it before it completes
@@ -1412,6 +1505,7 @@ __global__ void __launch_bounds__(kQuantMeansThreads) k_quant_means(Dims D, Plan
     const int d = D.d;
     __shared__ float red[2][kQuantMeansThreads / 32];
     float mk = 0.f, mv = 0.f;
+#pragma unroll 8
     for (int idx = 4 * threadIdx.x; idx < nblk * d; idx += 4 * blockDim.x) {
         const int64_t off = ((b + idx / d) * D.Hkv + g) * d + idx % d;
         const float4 k4 = *reinterpret_cast<const float4*>(P.kbar + off);
@@ -1441,6 +1535,7 @@ __global__ void __launch_bounds__(kQuantMeansThreads) k_quant_means(Dims D, Plan
         P.kbar_scale[b * D.Hkv + g] = sk;
         P.vbar_scale[b * D.Hkv + g] = sv;
     }
+#pragma unroll 4
     for (int idx = 4 * threadIdx.x; idx < nblk * d; idx += 4 * blockDim.x) {
         const int64_t off = ((b + idx / d) * D.Hkv + g) * d + idx % d;
         const float4 k4 = *reinterpret_cast<const float4*>(P.kbar + off);
@@ -1544,10 +1639,13 @@ int launch_score(const Dims& D, const PlanPtrs& P, const WsPtrs& W, cudaStream_t
     const int64_t fit = (int64_t)std::max(1, per_sm) * std::max(1, sm_count());
     const int64_t need = (D.R + kThrRows - 1) / kThrRows;
     const dim3 grid((unsigned)std::min(fit, need));
-    int rc = launch_pdl(thr, grid, dim3(kThrRows * 32), 0, st, D, P, W, kScoreTcRelErr, bounds);
+    int rc = launch_pdl(thr, grid, dim3(kThrRows * 32), 0, st, D, P, W, bounds);
     if (rc != FP2_OK) return rc;
-    return launch_pdl(k_csr, dim3((unsigned)((D.R + kCsrRows - 1) / kCsrRows)), dim3(kCsrRows * 32), 0, st,
-                      D, P);
+    int csr_per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&csr_per_sm, k_csr, kThrRows * 32, 0) != cudaSuccess)
+        return FP2_ERR_CUDA;
+    const int64_t csr_fit = (int64_t)std::max(1, csr_per_sm) * std::max(1, sm_count());
+    return launch_pdl(k_csr, dim3((unsigned)std::min(csr_fit, need)), dim3(kThrRows * 32), 0, st, D, P);
 }
 
 }  // namespace
