@@ -62,12 +62,13 @@ def kept_tile_flop(wl) -> float:
 
 
 def plan_launches(wl, tau=None) -> int:
-    """Kernels fp2_plan launches: pool, meta, e4m3 means, threshold and CSR;
-    with tau > 0 the scorer, and the separate norms kernel when the G query
-    heads of a kv-head do not fall into one pooling CTA (1024 columns)."""
+    """Kernels fp2_plan launches: pool, meta, threshold (which also takes the
+    e4m3 means' chunk maxima) and CSR (which also writes their codes); with
+    tau > 0 the scorer, and the separate norms kernel when the G query heads of
+    a kv-head do not fall into one pooling CTA (1024 columns)."""
     tau = wl.tau if tau is None else tau
     G = wl.Hq // wl.Hkv
-    return 5 + (1 if tau > 0 else 0) + (1 if tau > 0 and 1024 % (G * wl.d) != 0 else 0)
+    return 4 + (1 if tau > 0 else 0) + (1 if tau > 0 and 1024 % (G * wl.d) != 0 else 0)
 
 
 def rank_slice(wl, world: int, rank: int):
@@ -248,7 +249,7 @@ def run_ours(args, rank, world, local_rank):
     total_ms = t0.elapsed_time(t1)
     plan_ms = [e[0].elapsed_time(e[1]) for e in ev]
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    # plan: meta, pool, [norms, score], threshold, quant_means, scan, compact; prefill: attn
+    # plan: pool, meta, [norms, score], threshold, csr; prefill: attn
     # (+ the split merge when the schedule splits rows)
     launches_per_step = plan_launches(wl) + 1 + (1 if lay.num_split_slots > 0 else 0)
 

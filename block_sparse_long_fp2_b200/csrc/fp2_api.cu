@@ -198,6 +198,7 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     L.off_slot_item = c.take(sizeof(int32_t) * (size_t)sd.split_slots * d.Hkv);
     L.off_q_off = c.take(sizeof(int32_t) * n);
     L.off_thr_next = c.take(sizeof(int32_t));
+    L.off_mean_amax = c.take(sizeof(uint32_t) * 2 * (size_t)NB * d.Hkv);
     L.off_csr_count = c.take(sizeof(int32_t) * (size_t)d.R);
     L.off_csr_seg = c.take(sizeof(int32_t) * (size_t)((d.R + kCsrRows - 1) / kCsrRows));
     L.off_csr_sup = c.take(sizeof(int32_t) * (size_t)((d.R + kCsrSup - 1) / kCsrSup));
@@ -253,6 +254,7 @@ PlanPtrs plan_ptrs(const Layout& L, void* plan) {
     p.slot_item = reinterpret_cast<int32_t*>(b + L.off_slot_item);
     p.q_off = reinterpret_cast<int32_t*>(b + L.off_q_off);
     p.thr_next = reinterpret_cast<int32_t*>(b + L.off_thr_next);
+    p.mean_amax = reinterpret_cast<uint32_t*>(b + L.off_mean_amax);
     p.csr_count = reinterpret_cast<int32_t*>(b + L.off_csr_count);
     p.csr_seg = reinterpret_cast<int32_t*>(b + L.off_csr_seg);
     p.csr_sup = reinterpret_cast<int32_t*>(b + L.off_csr_sup);

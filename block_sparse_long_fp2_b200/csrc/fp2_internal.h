@@ -123,7 +123,8 @@ struct PlanPtrs {
     int32_t* q_off;        // [n]  position of the first query (L - Q for a chunk, else 0)
     // the threshold kernel's single-pass CSR prefix sum (decoupled look-back):
     // a CTA ticket counter and one flag word per CTA, zeroed by k_meta
-    int32_t* thr_next;     // [1]: the threshold's next row
+    int32_t* thr_next;     // [1]: the threshold's next item
+    uint32_t* mean_amax;   // [NB, Hkv, 2]: absmax of the K / V means of the chunk starting at the block
     int32_t* csr_count;    // [R]: kept blocks per row
     int32_t* csr_seg;      // [ceil(R / kCsrRows)]: kept blocks per segment of kCsrRows rows
     int32_t* csr_sup;      // [ceil(R / kCsrSup)]: kept blocks per super-segment of kCsrSup rows
@@ -154,7 +155,7 @@ struct Layout {
     fp2_plan_layout pub;
     size_t off_meta_valid, off_cu_blocks, off_block_seq, off_tri_off, off_group_cu, off_group_seq,
         off_tile_cu, off_vmax, off_sched, off_sched_cnt, off_sched_off, off_split_o, off_split_lse,
-        off_slot_item, off_q_off, off_thr_next, off_csr_count, off_csr_seg, off_csr_sup;
+        off_slot_item, off_q_off, off_thr_next, off_mean_amax, off_csr_count, off_csr_seg, off_csr_sup;
     size_t ws_qbar64, ws_qbar32, ws_kbar_tf, ws_kbar64, ws_qnorm, ws_qres, ws_knorm, ws_kres, ws_scores,
         ws_bounds;
 };

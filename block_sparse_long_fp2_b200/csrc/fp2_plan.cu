@@ -14,19 +14,20 @@
 //            offsets and the attention kernel's work schedule.
 //   (norms   |Qbar|, |Kbar| when the pool cannot: G query heads of a kv-head
 //            not within one pooling CTA.)
-//   quant_means  e4m3 codes of Kbar / Vbar with one scale per pseudo-tile
-//            chunk (used by the FP8 correction).
-//   score    persistent, one CTA per SM, beside quant_means: tf32 tcgen05 MMAs
+//   score    persistent, one CTA per SM: tf32 tcgen05 MMAs
 //            of the means rounded to tf32 (exact products, fp32 sums), max over
 //            the group's heads, to a scratch array; also each row's bounds of
 //            its largest score.
 //   threshold  one warp per row, rows taken longest first: the threshold
 //            decision.  A block whose score lies within the scores' error
-//            bound of the threshold, and every candidate for the row maximum,
-//            is re-scored in float64, so the kept set is the one float64
-//            scores give.
+//            bound of the threshold, and an undecided row's candidates for
+//            its maximum, are re-scored in float64, so the kept set is the one
+//            float64 scores give.  Before the rows, its warps take the
+//            absolute maxima of the e4m3 block means' chunks (one scale per
+//            chunk of B blocks, a pseudo tile of the FP8 correction).
 //   csr      the CSR row pointers (each warp adds up the kept counts of
-//            the rows before its row, by segments), then the column ids.
+//            the rows before its row, by segments), then the column ids;
+//            after the rows, the e4m3 codes of the block means.
 #include <cfloat>
 #include <cstring>
 #include <cmath>
@@ -199,11 +200,13 @@ __global__ void __launch_bounds__(kMetaThreads, 1) k_meta(Dims D, SchedDims S, c
     }
     __syncthreads();
     if (s_valid) {
-        // the threshold's row counter and the CSR segment counts start from zero
+        // the threshold's item counter, the CSR segment counts and the e4m3
+        // means' chunk maxima start from zero
         const int64_t n_seg = (D.R + kCsrRows - 1) / kCsrRows, n_sup = (D.R + kCsrSup - 1) / kCsrSup;
         for (int64_t c = threadIdx.x; c < n_seg; c += blockDim.x) P.csr_seg[c] = 0;
         for (int64_t c = threadIdx.x; c < n_sup; c += blockDim.x) P.csr_sup[c] = 0;
         if (threadIdx.x == 0) *P.thr_next = 0;
+        for (int64_t c = threadIdx.x; c < 2 * D.NB * D.Hkv; c += blockDim.x) P.mean_amax[c] = 0u;
         meta_maps(D, S, cu_seqlens, page_table, P);
     }
     // k_meta may run beside the pooling kernel launched before it (which
@@ -647,12 +650,12 @@ __global__ void __launch_bounds__(kScoreTcThreads)
 k_score_tc(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap tm_q,
            const __grid_constant__ CUtensorMap tm_k) {
     using C = ScoreTcCfg<HD>;
-    // runs beside k_quant_means (launched before it as its programmatic
-    // dependent) and completes only after it
-    if (!*P.meta_valid) {
-        asm volatile("griddepcontrol.wait;" ::: "memory");
-        return;
-    }
+    // a programmatic dependent of the kernel before it: everything before is
+    // complete once the wait returns; the threshold after it may be launched
+    // early (it waits for this kernel before reading anything)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (!*P.meta_valid) return;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -769,7 +772,6 @@ k_score_tc(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap tm_
         tc_fence_after();
         tmem_dealloc(tmem, kScoreKeys);
     }
-    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Pipelined tensor-core scores (G a power of two, at most 32).  A persistent CTA per SM takes
@@ -826,14 +828,12 @@ __global__ void __launch_bounds__(kScorePThreads, 1)
 k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap tm_q,
              const __grid_constant__ CUtensorMap tm_k) {
     using C = ScorePCfg<HD>;
-    // runs beside k_quant_means (launched before it as its programmatic
-    // dependent) and completes only after it; the threshold after it may be
-    // launched early (it waits for this kernel before reading anything)
+    // a programmatic dependent of the kernel before it: everything before is
+    // complete once the wait returns; the threshold after it may be launched
+    // early (it waits for this kernel before reading anything)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (!*P.meta_valid) {
-        asm volatile("griddepcontrol.wait;" ::: "memory");
-        return;
-    }
+    if (!*P.meta_valid) return;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -1061,7 +1061,6 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
         tc_fence_after();
         tmem_dealloc(tmem, 2 * kScoreKeys);
     }
-    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // float64 score of a key block for a row: max over the group's G heads of
@@ -1100,6 +1099,104 @@ __device__ __noinline__ double score64(const double* __restrict__ qp0, const dou
             if (h0 + u < G) best = fmax(best, acc[u]);
     }
     return best / sqrt((double)HD);
+}
+
+// ---------------------------------------------------------------------------
+// e4m3 codes of the K / V block means for the FP8 correction
+// ---------------------------------------------------------------------------
+//
+// A chunk is the B consecutive blocks of a sequence that one pseudo-key tile
+// covers, so a pseudo tile needs a single scale per kv-head:
+// scale = absmax / 448 over the chunk's fp32 means (1 when all zero),
+// code = e4m3_rne_sat(mean / scale), both in fp32.  The key means get a second
+// e4m3 term, lo = e4m3_rne_sat(mean / scale - code), so that the pseudo-key
+// logits (one MMA over both terms) carry about 2^-8 relative error instead of
+// the 2^-4 of one e4m3 rounding.  Two steps ride on kernels that run anyway:
+// the threshold kernel's warps take the chunks' absolute maxima (one item per
+// block, atomicMax of the bits of a non-negative float into the chunk's slot),
+// the CSR kernel's warps then write the codes and scales (one item per block).
+
+__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// First block of the chunk that holds block b.
+__device__ __forceinline__ int64_t chunk_first(const Dims& D, const PlanPtrs& P, int64_t b) {
+    const int b0 = P.cu_blocks[P.block_seq[b]];
+    return b0 + (b - b0) / D.B * D.B;
+}
+
+// Warp-collective: the K and V means of block b, all kv-heads (Hkv d floats
+// each, lane l taking 4 consecutive floats of every 128), visited one float4
+// at a time with f(h, k4, v4, lead); the d / 4 lanes of a head form one
+// aligned group of lanes (d / 4 in {16, 32}), `lead` is its first lane.
+template <typename F>
+__device__ __forceinline__ void for_means(const Dims& D, const PlanPtrs& P, int64_t b, int lane, F f) {
+    const int d = D.d;
+    const int n4 = D.Hkv * d / 4;
+    const int lph = d / 4;
+    for (int f0 = 0; f0 < n4; f0 += 32) {
+        const int f4 = f0 + lane;
+        const bool in = f4 < n4;
+        const int64_t off = b * D.Hkv * d + 4 * (int64_t)f4;
+        const float4 k4 = in ? *reinterpret_cast<const float4*>(P.kbar + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 v4 = in ? *reinterpret_cast<const float4*>(P.vbar + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+        f(in ? 4 * f4 / d : -1, off, k4, v4, (lane % lph) == 0, lph);
+    }
+}
+
+__device__ __forceinline__ float absmax4(float4 x) {
+    return fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w)));
+}
+
+// Step 1 (a threshold-kernel item): block b's absolute maxima into its chunk's slots.
+__device__ __forceinline__ void means_absmax(const Dims& D, const PlanPtrs& P, int64_t b, int lane) {
+    const int64_t c0 = chunk_first(D, P, b);
+    for_means(D, P, b, lane, [&](int h, int64_t, float4 k4, float4 v4, bool lead, int lph) {
+        float mk = absmax4(k4), mv = absmax4(v4);
+        for (int o = lph / 2; o > 0; o >>= 1) {
+            mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, o));
+            mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, o));
+        }
+        if (lead && h >= 0) {
+            atomicMax(P.mean_amax + (c0 * D.Hkv + h) * 2, __float_as_uint(mk));
+            atomicMax(P.mean_amax + (c0 * D.Hkv + h) * 2 + 1, __float_as_uint(mv));
+        }
+    });
+}
+
+// Step 2 (a CSR-kernel item): block b's codes from its chunk's maxima; the
+// chunk's first block also writes the chunk's scales.
+__device__ __forceinline__ void means_codes(const Dims& D, const PlanPtrs& P, int64_t b, int lane) {
+    const int64_t c0 = chunk_first(D, P, b);
+    for_means(D, P, b, lane, [&](int h, int64_t off, float4 k4, float4 v4, bool lead, int) {
+        if (h < 0) return;
+        const float mk = __uint_as_float(P.mean_amax[(c0 * D.Hkv + h) * 2]);
+        const float mv = __uint_as_float(P.mean_amax[(c0 * D.Hkv + h) * 2 + 1]);
+        const float sk = mk > 0.f ? __fdiv_rn(mk, 448.0f) : 1.0f;
+        const float sv = mv > 0.f ? __fdiv_rn(mv, 448.0f) : 1.0f;
+        if (lead && b == c0) {
+            P.kbar_scale[b * D.Hkv + h] = sk;
+            P.vbar_scale[b * D.Hkv + h] = sv;
+        }
+        const float kq[4] = {__fdiv_rn(k4.x, sk), __fdiv_rn(k4.y, sk), __fdiv_rn(k4.z, sk),
+                             __fdiv_rn(k4.w, sk)};
+        const uint16_t h01 = e4m3x2(kq[0], kq[1]), h23 = e4m3x2(kq[2], kq[3]);
+        *reinterpret_cast<uint32_t*>(P.kbar8 + off) = (uint32_t)h01 | ((uint32_t)h23 << 16);
+        // second term: the residual of the quotient (exact in fp32, since the
+        // e4m3 value is within a factor 2 of it), rounded to e4m3 on its own
+        float hv[4];
+        unpack_e4m3x2(h01, hv[0], hv[1]);
+        unpack_e4m3x2(h23, hv[2], hv[3]);
+        *reinterpret_cast<uint32_t*>(P.kbar8lo + off) =
+            (uint32_t)e4m3x2(kq[0] - hv[0], kq[1] - hv[1]) |
+            ((uint32_t)e4m3x2(kq[2] - hv[2], kq[3] - hv[3]) << 16);
+        *reinterpret_cast<uint32_t*>(P.vbar8 + off) =
+            (uint32_t)e4m3x2(__fdiv_rn(v4.x, sv), __fdiv_rn(v4.y, sv)) |
+            ((uint32_t)e4m3x2(__fdiv_rn(v4.z, sv), __fdiv_rn(v4.w, sv)) << 16);
+    });
 }
 
 // ---------------------------------------------------------------------------
@@ -1370,10 +1467,11 @@ __device__ __forceinline__ int64_t row_order(int64_t t, int64_t gw, int64_t nw) 
     return t * nw + ((t & 1) ? nw - 1 - gw : gw);
 }
 
-// The threshold: each warp takes the next row "longest first" from a counter
-// (the rows' costs depend on how many blocks need re-scoring, so they are
-// handed out as warps free up), decides it, and leaves the row's kept count,
-// adding it to the counts of the row's segment (kCsrRows rows) and
+// The threshold: each warp takes the next item from a counter: first the
+// e4m3 means' chunk maxima of one block (NB short items), then the rows
+// "longest first" (their costs depend on how many blocks need re-scoring, so
+// they are handed out as warps free up).  A row's decision leaves its kept
+// count, added to the counts of the row's segment (kCsrRows rows) and
 // super-segment (kCsrSup rows); k_csr turns the counts into offsets and
 // writes the column ids.
 template <int HD, bool CHUNK>
@@ -1390,6 +1488,11 @@ __global__ void __launch_bounds__(kThrRows * 32, 2) k_threshold(Dims D, PlanPtrs
         int o = 0;
         if (lane == 0) o = atomicAdd(P.thr_next, 1);
         o = __shfl_sync(0xffffffffu, o, 0);
+        if (o < D.NB) {   // the first NB items: the e4m3 means' chunk maxima
+            means_absmax(D, P, o, lane);
+            continue;
+        }
+        o -= (int)D.NB;
         if (o >= D.R) break;
         const int64_t bi = D.NB - 1 - o / D.Hkv;
         const int64_t r = (int64_t)(o % D.Hkv) * D.NB + bi;
@@ -1402,9 +1505,10 @@ __global__ void __launch_bounds__(kThrRows * 32, 2) k_threshold(Dims D, PlanPtrs
     }
 }
 
-// The CSR from the kept counts and mask words.  The warps take the rows in
-// row_order (which evens out their work); a row's offset is the kept count
-// of every row before it:
+// The CSR from the kept counts and mask words, and after the rows the e4m3
+// means' codes (one item per block).  The warps take the items in row_order
+// (which evens out their work); a row's offset is the kept count of every
+// row before it:
 // the super-segments before its own, the segments before it within its
 // super-segment, and the rows before it within its segment (at most
 // R / kCsrSup + 62 counts, added up by the warp's lanes).  Then the warp
@@ -1418,7 +1522,11 @@ __global__ void __launch_bounds__(kThrRows * 32) k_csr(Dims D, PlanPtrs P) {
     const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     for (int64_t t = 0; ; ++t) {
         const int64_t o = row_order(t, gw, nw);
-        if (o >= D.R) break;
+        if (o >= D.R + D.NB) break;
+        if (o >= D.R) {   // after the rows: the e4m3 means' codes of one block
+            means_codes(D, P, o - D.R, lane);
+            continue;
+        }
         const int64_t bi = D.NB - 1 - o / D.Hkv;
         const int64_t r = (o % D.Hkv) * D.NB + bi;
         const int64_t seg = r / kCsrRows, sup = r / kCsrSup;
@@ -1467,97 +1575,6 @@ __global__ void __launch_bounds__(kThrRows * 32) k_csr(Dims D, PlanPtrs P) {
     }
 }
 
-// ---------------------------------------------------------------------------
-// quant_means: e4m3 codes of the K / V block means for the FP8 correction
-// ---------------------------------------------------------------------------
-//
-// One CTA per (chunk of B blocks of one sequence, kv-head): the chunk is the
-// set of blocks one pseudo-key tile covers, so a pseudo tile needs a single
-// scale.  scale = absmax / 448 over the chunk's fp32 means (1 when all zero),
-// code = e4m3_rne_sat(mean / scale), both in fp32.  The key means get a second
-// e4m3 term, lo = e4m3_rne_sat(mean / scale - code), so that the pseudo-key
-// logits (one MMA over both terms) carry about 2^-8 relative error instead of
-// the 2^-4 of one e4m3 rounding.
-
-__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-
-// Small CTAs, so that they fit on an SM beside the scorer's (which runs at
-// the same time and holds most of an SM's shared memory and registers).
-constexpr int kQuantMeansThreads = 256;
-
-__global__ void __launch_bounds__(kQuantMeansThreads, 4) k_quant_means(Dims D, PlanPtrs P) {
-    // a programmatic dependent of k_meta (everything before is complete once
-    // the wait returns); the scorer, launched next, may run beside this kernel
-    // (it needs nothing from it) and waits for it before it completes
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (!*P.meta_valid) return;
-    const int s = blockIdx.y;
-    const int g = blockIdx.z;
-    const int b0 = P.cu_blocks[s];
-    if ((int64_t)blockIdx.x * D.B >= P.cu_blocks[s + 1] - b0) return;   // past the sequence
-    const int64_t b = b0 + (int64_t)blockIdx.x * D.B;                       // first block of the chunk
-    const int nblk = min((int64_t)D.B, (int64_t)P.cu_blocks[s + 1] - b);
-    const int d = D.d;
-    __shared__ float red[2][kQuantMeansThreads / 32];
-    float mk = 0.f, mv = 0.f;
-#pragma unroll 8
-    for (int idx = 4 * threadIdx.x; idx < nblk * d; idx += 4 * blockDim.x) {
-        const int64_t off = ((b + idx / d) * D.Hkv + g) * d + idx % d;
-        const float4 k4 = *reinterpret_cast<const float4*>(P.kbar + off);
-        const float4 v4 = *reinterpret_cast<const float4*>(P.vbar + off);
-        mk = fmaxf(mk, fmaxf(fmaxf(fabsf(k4.x), fabsf(k4.y)), fmaxf(fabsf(k4.z), fabsf(k4.w))));
-        mv = fmaxf(mv, fmaxf(fmaxf(fabsf(v4.x), fabsf(v4.y)), fmaxf(fabsf(v4.z), fabsf(v4.w))));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, o));
-        mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, o));
-    }
-    if ((threadIdx.x & 31) == 0) {
-        red[0][threadIdx.x >> 5] = mk;
-        red[1][threadIdx.x >> 5] = mv;
-    }
-    __syncthreads();
-    mk = red[0][0];
-    mv = red[1][0];
-    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
-        mk = fmaxf(mk, red[0][w]);
-        mv = fmaxf(mv, red[1][w]);
-    }
-    const float sk = mk > 0.f ? __fdiv_rn(mk, 448.0f) : 1.0f;
-    const float sv = mv > 0.f ? __fdiv_rn(mv, 448.0f) : 1.0f;
-    if (threadIdx.x == 0) {
-        P.kbar_scale[b * D.Hkv + g] = sk;
-        P.vbar_scale[b * D.Hkv + g] = sv;
-    }
-#pragma unroll 4
-    for (int idx = 4 * threadIdx.x; idx < nblk * d; idx += 4 * blockDim.x) {
-        const int64_t off = ((b + idx / d) * D.Hkv + g) * d + idx % d;
-        const float4 k4 = *reinterpret_cast<const float4*>(P.kbar + off);
-        const float4 v4 = *reinterpret_cast<const float4*>(P.vbar + off);
-        const float kq[4] = {__fdiv_rn(k4.x, sk), __fdiv_rn(k4.y, sk), __fdiv_rn(k4.z, sk),
-                             __fdiv_rn(k4.w, sk)};
-        const uint16_t h01 = e4m3x2(kq[0], kq[1]), h23 = e4m3x2(kq[2], kq[3]);
-        *reinterpret_cast<uint32_t*>(P.kbar8 + off) = (uint32_t)h01 | ((uint32_t)h23 << 16);
-        // second term: the residual of the quotient (exact in fp32, since the
-        // e4m3 value is within a factor 2 of it), rounded to e4m3 on its own
-        float hv[4];
-        unpack_e4m3x2(h01, hv[0], hv[1]);
-        unpack_e4m3x2(h23, hv[2], hv[3]);
-        *reinterpret_cast<uint32_t*>(P.kbar8lo + off) =
-            (uint32_t)e4m3x2(kq[0] - hv[0], kq[1] - hv[1]) |
-            ((uint32_t)e4m3x2(kq[2] - hv[2], kq[3] - hv[3]) << 16);
-        *reinterpret_cast<uint32_t*>(P.vbar8 + off) =
-            (uint32_t)e4m3x2(__fdiv_rn(v4.x, sv), __fdiv_rn(v4.y, sv)) |
-            ((uint32_t)e4m3x2(__fdiv_rn(v4.z, sv), __fdiv_rn(v4.w, sv)) << 16);
-    }
-}
-
 // Launch with programmatic stream serialization: the kernel may begin before
 // the one before it in the stream completes; what it may read before its
 // griddepcontrol.wait is stated at each kernel.
@@ -1588,8 +1605,7 @@ int launch_score_pipe(const Dims& D, const PlanPtrs& P, const WsPtrs& W, const C
                       tq, tk);
 }
 
-// Scores (tau > 0; launched right after k_quant_means, beside which it runs)
-// and the threshold.
+// Scores (tau > 0), the threshold and the CSR.
 template <int HD>
 int launch_score(const Dims& D, const PlanPtrs& P, const WsPtrs& W, cudaStream_t st) {
     if (D.tau > 0.0) {
@@ -1637,7 +1653,7 @@ int launch_score(const Dims& D, const PlanPtrs& P, const WsPtrs& W, cudaStream_t
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, thr, kThrRows * 32, 0) != cudaSuccess)
         return FP2_ERR_CUDA;
     const int64_t fit = (int64_t)std::max(1, per_sm) * std::max(1, sm_count());
-    const int64_t need = (D.R + kThrRows - 1) / kThrRows;
+    const int64_t need = (D.R + D.NB + kThrRows - 1) / kThrRows;
     const dim3 grid((unsigned)std::min(fit, need));
     int rc = launch_pdl(thr, grid, dim3(kThrRows * 32), 0, st, D, P, W, bounds);
     if (rc != FP2_OK) return rc;
@@ -1741,10 +1757,6 @@ int launch_plan(const Layout& L, const fp2_problem* p, const void* q, const void
         const int64_t warps = D.NB * D.Hkv;
         k_norms<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(D, P, W);
     }
-    // e4m3 block means (needs the pool's K/V means only); the scorer runs beside it
-    if (launch_pdl(k_quant_means, dim3((unsigned)((D.max_nb + D.B - 1) / D.B), D.n_seqs, D.Hkv),
-                   dim3(kQuantMeansThreads), 0, st, D, P) != FP2_OK)
-        return FP2_ERR_CUDA;
     int rc = D.d == 64 ? launch_score<64>(D, P, W, st) : launch_score<128>(D, P, W, st);
     if (rc != FP2_OK) return rc;
     return cudaGetLastError() == cudaSuccess ? FP2_OK : FP2_ERR_CUDA;
