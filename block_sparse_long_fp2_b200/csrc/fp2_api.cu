@@ -211,8 +211,7 @@ int compute_layout(const fp2_problem* p, Layout* out) {
     L.ws_kbar64 = w.take(sizeof(double) * mean_elems);
     L.ws_qnorm = w.take(sizeof(float) * (size_t)NB * d.Hkv);
     L.ws_qres = w.take(sizeof(float) * (size_t)NB * d.Hkv);
-    L.ws_knorm = w.take(sizeof(float) * (size_t)NB * d.Hkv);
-    L.ws_kres = w.take(sizeof(float) * (size_t)NB * d.Hkv);
+    L.ws_kb2 = w.take(sizeof(float2) * (size_t)NB * d.Hkv);
     L.ws_scores = w.take(sizeof(float) * (size_t)d.nnz_cap);
     L.ws_bounds = w.take(sizeof(double) * 2 * (size_t)d.R);
     pub.workspace_bytes = align_up(w.off, 256);
@@ -271,8 +270,7 @@ WsPtrs ws_ptrs(const Layout& L, void* ws) {
     w.kbar64 = reinterpret_cast<double*>(b + L.ws_kbar64);
     w.qnorm = reinterpret_cast<float*>(b + L.ws_qnorm);
     w.qres = reinterpret_cast<float*>(b + L.ws_qres);
-    w.knorm = reinterpret_cast<float*>(b + L.ws_knorm);
-    w.kres = reinterpret_cast<float*>(b + L.ws_kres);
+    w.kb2 = reinterpret_cast<float2*>(b + L.ws_kb2);
     w.scores = reinterpret_cast<float*>(b + L.ws_scores);
     w.bounds = reinterpret_cast<double*>(b + L.ws_bounds);
     return w;

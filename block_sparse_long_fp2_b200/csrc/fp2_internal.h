@@ -139,8 +139,8 @@ struct WsPtrs {
     double* kbar64;   // [NB, Hkv, d]
     float* qnorm;     // [NB, Hkv]  max over the group's heads of |Qbar|_2 (rounded up)
     float* qres;      // [NB, Hkv]  max over the group's heads of |Qbar - tf32(Qbar)|_2 (rounded up)
-    float* knorm;     // [Hkv, NB]  |Kbar|_2 (rounded up), contiguous over a head's blocks
-    float* kres;      // [Hkv, NB]  |Kbar - tf32(Kbar)|_2 + c_d (|Kbar|_2 + that), rounded up
+    float2* kb2;      // [Hkv, NB]  (|Kbar|_2, |Kbar - tf32(Kbar)|_2 + c_d (|Kbar|_2 + that)),
+                      //   both rounded up, contiguous over a head's blocks
     float* scores;    // [Hkv, tri_total] fp32 block scores, row (s,g,i) at
                       //   g * tri_total + tri_off[s] + i (i + 1) / 2 + j
     double* bounds;   // [R, 2] per row: the largest lower and upper bound of any
@@ -156,7 +156,7 @@ struct Layout {
     size_t off_meta_valid, off_cu_blocks, off_block_seq, off_tri_off, off_group_cu, off_group_seq,
         off_tile_cu, off_vmax, off_sched, off_sched_cnt, off_sched_off, off_split_o, off_split_lse,
         off_slot_item, off_q_off, off_thr_next, off_mean_amax, off_csr_count, off_csr_seg, off_csr_sup;
-    size_t ws_qbar64, ws_qbar32, ws_kbar_tf, ws_kbar64, ws_qnorm, ws_qres, ws_knorm, ws_kres, ws_scores,
+    size_t ws_qbar64, ws_qbar32, ws_kbar_tf, ws_kbar64, ws_qnorm, ws_qres, ws_kb2, ws_scores,
         ws_bounds;
 };
 

@@ -27,7 +27,7 @@
 //            chunk of B blocks, a pseudo tile of the FP8 correction).
 //   csr      the CSR row pointers (each warp adds up the kept counts of
 //            the rows before its row, by segments), then the column ids;
-//            after the rows, the e4m3 codes of the block means.
+//            before the rows, the e4m3 codes of the block means.
 #include <cfloat>
 #include <cstring>
 #include <cmath>
@@ -547,8 +547,7 @@ k_pool(Dims D, SeqMap M, int64_t Tq, const int32_t* __restrict__ cu_seqlens,
         }
         const bool lead = active && (vec % tph) == 0;
         if (lead && which == 1) {
-            W.knorm[(int64_t)head * D.NB + b] = round_up_f(sqrt(sq));
-            W.kres[(int64_t)head * D.NB + b] = kres_bound(sqrt(sq), sqrt(rq), d);
+            W.kb2[(int64_t)head * D.NB + b] = make_float2(round_up_f(sqrt(sq)), kres_bound(sqrt(sq), sqrt(rq), d));
         }
         // the largest over the G query heads of a kv-head: the group's heads
         // lie in this CTA (G d divides the CTA's 1024 columns)
@@ -608,8 +607,7 @@ __global__ void k_norms(Dims D, PlanPtrs P, WsPtrs W) {
         rmax = fmax(rmax, qr);
     }
     if (lane == 0) {
-        W.knorm[(int64_t)g * D.NB + b] = round_up_f(sqrt(kk));
-        W.kres[(int64_t)g * D.NB + b] = kres_bound(sqrt(kk), sqrt(kr), d);
+        W.kb2[(int64_t)g * D.NB + b] = make_float2(round_up_f(sqrt(kk)), kres_bound(sqrt(kk), sqrt(kr), d));
         W.qnorm[wid] = round_up_f(sqrt(qmax));
         W.qres[wid] = round_up_f(sqrt(rmax));
     }
@@ -956,8 +954,7 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
             // the G lanes of a block share its columns: lane hl takes columns hl, hl + G, ...
             const bool row_ok = i < it.i1;
             float* sc_row = W.scores + (int64_t)it.g * D.tri_total + P.tri_off[it.s] + (int64_t)i * (i + 1) / 2;
-            const float* kn = W.knorm + (int64_t)it.g * D.NB + it.b0;
-            const float* kr = W.kres + (int64_t)it.g * D.NB + it.b0;
+            const float2* kb2 = W.kb2 + (int64_t)it.g * D.NB + it.b0;
             // the row's bound coefficients A, B (see kres_bound), rounded up (the
             // bounds below only need to enclose the float64 ones: they are
             // widened before they are stored)
@@ -979,8 +976,9 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
 #pragma unroll
                 for (int cc = 0; cc < NCC; ++cc) {
                     const int col = kScoreKeys * c + 32 * cc + lane;
-                    knr[cc] = col < it.nb ? __ldg(kn + col) : 0.f;
-                    krr[cc] = col < it.nb ? __ldg(kr + col) : 0.f;
+                    const float2 t2 = col < it.nb ? __ldg(kb2 + col) : make_float2(0.f, 0.f);
+                    knr[cc] = t2.x;
+                    krr[cc] = t2.y;
                 }
                 if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (an >> 1) & 1, &abort_flag, P.status))) {
                     ok = false;
@@ -1000,23 +998,31 @@ k_score_pipe(Dims D, PlanPtrs P, WsPtrs W, const __grid_constant__ CUtensorMap t
 #pragma unroll
                 for (int cc = 0; cc < NCC; ++cc) {
                     const int jb = kScoreKeys * c + 32 * cc;
-                    // max over the G heads (adjacent lanes), 32 columns at a time so
-                    // the shuffles of different columns overlap
+                    // max over the G heads (adjacent lanes) by halving exchanges: at
+                    // the step of bit b, lane hl keeps the columns whose bit b is
+                    // that of hl, sends its partner (lane ^ b) the others, and keeps
+                    // the max of each kept pair in the slot of the column with bit b
+                    // clear.  After the steps, slot e0 (a multiple of G) holds the
+                    // max for column e0 + hl: 32 - 32 / G shuffles, not 32 log2 G.
 #pragma unroll
-                    for (int o = 1; o < G; o <<= 1) {
+                    for (int b = G / 2; b >= 1; b >>= 1) {
+                        const bool up = (hl & b) != 0;
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            r[cc][e] = __float_as_uint(fmaxf(__uint_as_float(r[cc][e]),
-                                                             __shfl_xor_sync(0xffffffffu, __uint_as_float(r[cc][e]), o)));
+                        for (int c0 = 0; c0 < 32; ++c0) {
+                            // slots still in use have every bit of G above b clear
+                            if ((c0 & (G - 1) & ~(b - 1)) != 0) continue;
+                            const uint32_t lo = r[cc][c0], hi = r[cc][c0 | b];
+                            const uint32_t keep = up ? hi : lo, send = up ? lo : hi;
+                            const float got = __shfl_xor_sync(0xffffffffu, __uint_as_float(send), b);
+                            r[cc][c0] = __float_as_uint(fmaxf(__uint_as_float(keep), got));
+                        }
                     }
                     float lo4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
                     float hi4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
 #pragma unroll
                     for (int e0 = 0; e0 < 32; e0 += G) {
                         // this lane's column of the G columns e0 .. e0 + G - 1
-                        uint32_t v = r[cc][e0];
-#pragma unroll
-                        for (int u = 1; u < G; ++u) v = hl == u ? r[cc][e0 + u] : v;
+                        const uint32_t v = r[cc][e0];
                         const float knv = __shfl_sync(0xffffffffu, knr[cc], e0 + hl);
                         const float krv = __shfl_sync(0xffffffffu, krr[cc], e0 + hl);
                         const int col = jb + e0 + hl;
@@ -1215,8 +1221,7 @@ constexpr int kThrBatch = 4;
 
 // The error-bound terms of one row.
 struct RowBound {
-    const float* kn;   // |Kbar_j|, j = 0 .. i
-    const float* kr;   // kr_j
+    const float2* kb;  // (|Kbar_j|, kr_j), j = 0 .. i
     double A, B;
     __device__ __forceinline__ double e(float knj, float krj) const { return A * knj + B * krj; }
 };
@@ -1239,8 +1244,9 @@ __device__ __forceinline__ void thr_decide(const Dims& D, const WsPtrs& W, const
         for (int u = 0; u < kThrBatch; ++u) {
             const int j = jb + 32 * u + lane;
             xs[u] = j <= i ? __ldg(sc + j) : 0.f;
-            ks[u] = j <= i ? __ldg(rb.kn + j) : 0.f;
-            rs[u] = j <= i ? __ldg(rb.kr + j) : 0.f;
+            const float2 t2 = j <= i ? __ldg(rb.kb + j) : make_float2(0.f, 0.f);
+            ks[u] = t2.x;
+            rs[u] = t2.y;
         }
 #pragma unroll
         for (int u = 0; u < kThrBatch; ++u) {
@@ -1261,8 +1267,9 @@ __device__ __forceinline__ void thr_decide(const Dims& D, const WsPtrs& W, const
         for (int u = 0; u < kThrBatch; ++u) {
             const int j = jb + 32 * u + lane;
             xs[u] = j <= i ? __ldg(sc + j) : 0.f;
-            ks[u] = j <= i ? __ldg(rb.kn + j) : 0.f;
-            rs[u] = j <= i ? __ldg(rb.kr + j) : 0.f;
+            const float2 t2 = j <= i ? __ldg(rb.kb + j) : make_float2(0.f, 0.f);
+            ks[u] = t2.x;
+            rs[u] = t2.y;
         }
 #pragma unroll
         for (int u = 0; u < kThrBatch; ++u) {
@@ -1321,8 +1328,9 @@ __device__ __forceinline__ void thr_one_pass(const Dims& D, const WsPtrs& W, con
     for (int u = 0; u < kThrBatch; ++u) {
         const int j = 32 * u + lane;
         xn[u] = j <= i ? __ldg(sc + j) : 0.f;
-        kq[u] = j <= i ? __ldg(rb.kn + j) : 0.f;
-        rq[u] = j <= i ? __ldg(rb.kr + j) : 0.f;
+        const float2 t2 = j <= i ? __ldg(rb.kb + j) : make_float2(0.f, 0.f);
+        kq[u] = t2.x;
+        rq[u] = t2.y;
     }
 #pragma unroll 1
     for (int jb = 0; jb <= i; jb += 32 * kThrBatch) {
@@ -1337,8 +1345,9 @@ __device__ __forceinline__ void thr_one_pass(const Dims& D, const WsPtrs& W, con
             for (int u = 0; u < kThrBatch; ++u) {
                 const int j = jb + 32 * kThrBatch + 32 * u + lane;
                 xn[u] = j <= i ? __ldg(sc + j) : 0.f;
-                kq[u] = j <= i ? __ldg(rb.kn + j) : 0.f;
-                rq[u] = j <= i ? __ldg(rb.kr + j) : 0.f;
+                const float2 t2 = j <= i ? __ldg(rb.kb + j) : make_float2(0.f, 0.f);
+                kq[u] = t2.x;
+                rq[u] = t2.y;
             }
         }
 #pragma unroll
@@ -1426,8 +1435,7 @@ __device__ __forceinline__ int thr_row(const Dims& D, const PlanPtrs& P, const W
         const double inv_sqrt_d = 1.0 / sqrt((double)HD);
         const double qr = W.qres[bi * D.Hkv + g];
         RowBound rb;
-        rb.kn = W.knorm + (int64_t)g * D.NB + b0;   // contiguous in j
-        rb.kr = W.kres + (int64_t)g * D.NB + b0;
+        rb.kb = W.kb2 + (int64_t)g * D.NB + b0;   // contiguous in j
         // (1 + 2^-20: far above the float64 rounding of the tests below)
         rb.A = qr * inv_sqrt_d * (1.0 + 0x1p-20);
         rb.B = ((double)W.qnorm[bi * D.Hkv + g] + qr) * inv_sqrt_d * (1.0 + 0x1p-20);
@@ -1444,8 +1452,9 @@ __device__ __forceinline__ int thr_row(const Dims& D, const PlanPtrs& P, const W
                 for (int u = 0; u < kThrBatch; ++u) {
                     const int j = jb + 32 * u + lane;
                     xs[u] = j <= i ? __ldg(sc + j) : 0.f;
-                    ks[u] = j <= i ? __ldg(rb.kn + j) : 0.f;
-                    rs[u] = j <= i ? __ldg(rb.kr + j) : 0.f;
+                    const float2 t2 = j <= i ? __ldg(rb.kb + j) : make_float2(0.f, 0.f);
+                    ks[u] = t2.x;
+                    rs[u] = t2.y;
                 }
 #pragma unroll
                 for (int u = 0; u < kThrBatch; ++u)
@@ -1505,8 +1514,9 @@ __global__ void __launch_bounds__(kThrRows * 32, 2) k_threshold(Dims D, PlanPtrs
     }
 }
 
-// The CSR from the kept counts and mask words, and after the rows the e4m3
-// means' codes (one item per block).  The warps take the items in row_order
+// The CSR from the kept counts and mask words, and before the rows the e4m3
+// means' codes (one item per block: their dependent loads then overlap the
+// rows instead of forming the kernel's tail).  The warps take the items in row_order
 // (which evens out their work); a row's offset is the kept count of every
 // row before it:
 // the super-segments before its own, the segments before it within its
@@ -1521,12 +1531,13 @@ __global__ void __launch_bounds__(kThrRows * 32) k_csr(Dims D, PlanPtrs P) {
     const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
     const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     for (int64_t t = 0; ; ++t) {
-        const int64_t o = row_order(t, gw, nw);
+        int64_t o = row_order(t, gw, nw);
         if (o >= D.R + D.NB) break;
-        if (o >= D.R) {   // after the rows: the e4m3 means' codes of one block
-            means_codes(D, P, o - D.R, lane);
+        if (o < D.NB) {   // first: the e4m3 means' codes of one block
+            means_codes(D, P, o, lane);
             continue;
         }
+        o -= D.NB;
         const int64_t bi = D.NB - 1 - o / D.Hkv;
         const int64_t r = (o % D.Hkv) * D.NB + bi;
         const int64_t seg = r / kCsrRows, sup = r / kCsrSup;
